@@ -1,0 +1,315 @@
+"""CPU oracle for the fused mixture-of-experts FFN layer (com.microsoft::MoE, standard SwiGLU).
+
+TEST INFRASTRUCTURE.  Only the tests, the smoke entry point and the benchmark's
+CPU-baseline leg may import this module.  The product path (the CUDA library and
+its Python binding) never calls it, and it shares no code with that path.
+
+What it computes is the plain definition of the layer, in float64 with numpy,
+following the pages in their order:
+
+* "Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326" (onnxruntime/mobius
+  pull request), description and "Attribute set": activation_type swiglu with
+  activation_alpha = 1.0, activation_beta = 0.0, swiglu_limit = inf, i.e. standard
+  SwiGLU y = silu(gate) * up; swiglu_fusion = 1 (interleaved gate/up rows);
+  normalize_routing_weights = 1; k = top_k.
+* same page, "Weight layout": Hugging Face stores experts.gate_up_proj chunked as
+  [E, 2*inter, H], the first inter rows gate and the next inter rows up; the
+  fused op takes the interleaved layout, made by Reshape -> Transpose -> Reshape.
+* same page, "Fallback": the static per-expert unroll computes the same layer one
+  expert at a time; `moe_dense_masked` is that reading, used as a brute-force pin.
+* same page, "Changes": the fused op is wrapped in CastLike, so the output has the
+  input's dtype (the oracle reports float64; callers compare after widening).
+* "Contributing Gemma 4 support and ONNX export optimizations" (Hugging Face forum),
+  "Key Technical Contributions", ONNX tracing compatibility: inside
+  grouped_mm_experts_forward the per-expert token count is a bincount over the
+  chosen expert ids, followed by a grouped matmul over experts.
+
+Readings where the pages are silent (each is listed with its reason in the design
+notes of the repository):
+
+* router logits are hidden @ router_w^T (+ an optional per-expert bias added before
+  selection and softmax); no pre-norm or scale;
+* top-k picks the k largest logits in descending order, ties to the lower expert
+  index; the selection is taken in float32, the precision of the CUDA kernels'
+  logits, so that both sides decide in the same precision;
+* normalize_routing_weights = 1 means softmax over all E logits, keep the k chosen
+  probabilities, divide by their sum; with 0 the chosen probabilities are kept as is;
+* interleaved means row 2i = gate_i and row 2i+1 = up_i;
+* the stable permutation puts the (token, slot) pairs of expert e in ascending
+  token order, experts in ascending order.
+
+Parity pins for every function here live in tests/test_oracle_pins.py.  No
+function in this file is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import itertools
+from typing import Callable, Optional, Sequence, Union
+
+import numpy as np
+
+F64 = np.float64
+NEAR_TIE_GAP = 1e-5          # float32 logit gap below which a selection is ambiguous
+TIE_BOUNDARY = 1             # flag bit: k-th and (k+1)-th logits within the gap
+TIE_WITHIN = 2               # flag bit: two adjacent chosen logits within the gap
+
+ArrayOrGetter = Union[np.ndarray, Callable[[int], np.ndarray]]
+
+
+def _expert(w: ArrayOrGetter, e: int) -> np.ndarray:
+    return (w(e) if callable(w) else w[e]).astype(F64)
+
+
+# --------------------------------------------------------------------------- routing
+
+def router_logits(hidden, router_w, router_bias=None) -> np.ndarray:
+    """L[t, e] = sum_h hidden[t, h] * router_w[e, h] + router_bias[e], float64 [T, E]."""
+    L = np.asarray(hidden, dtype=F64) @ np.asarray(router_w, dtype=F64).T
+    if router_bias is not None:
+        L = L + np.asarray(router_bias, dtype=F64)[None, :]
+    return L
+
+
+def select_topk(L: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest logits per token, descending, ties to the lower index.
+
+    The comparison is made on the float32-rounded logits: the CUDA kernels decide in
+    float32, and the decision must be taken in the same precision on both sides.
+    """
+    L32 = np.asarray(L, dtype=F64).astype(np.float32)
+    T, E = L32.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    for t in range(T):
+        # a stable sort on the negated logits keeps equal logits in index order
+        order = np.argsort(-L32[t], kind="stable")
+        idx[t] = order[:k]
+    return idx
+
+
+def softmax_all(L: np.ndarray) -> np.ndarray:
+    """Softmax over the E experts of each token, float64."""
+    m = L.max(axis=1, keepdims=True)
+    z = np.exp(L - m)
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def routing_weights(L: np.ndarray, idx: np.ndarray, normalize: int) -> np.ndarray:
+    """Mixing weights of the chosen experts, float64 [T, k].
+
+    normalize_routing_weights = 1: softmax over all experts, keep the chosen k
+    probabilities, divide them by their sum.  0: keep the chosen probabilities.
+    """
+    p = softmax_all(np.asarray(L, dtype=F64))
+    chosen = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    if normalize:
+        chosen = chosen / chosen.sum(axis=1, keepdims=True)
+    return chosen
+
+
+def near_tie_flags(L: np.ndarray, k: int, gap: float = NEAR_TIE_GAP) -> np.ndarray:
+    """Per-token flags for ambiguous selections, computed on float32 logits.
+
+    TIE_BOUNDARY: the k-th and (k+1)-th largest logits differ by less than `gap`
+    (the chosen set may legitimately differ); TIE_WITHIN: two adjacent chosen logits
+    differ by less than `gap` (only the slot order may differ).
+    """
+    L32 = np.asarray(L, dtype=F64).astype(np.float32)
+    T, E = L32.shape
+    flags = np.zeros(T, dtype=np.int32)
+    for t in range(T):
+        s = np.sort(L32[t])[::-1]
+        if k < E and (s[k - 1] - s[k]) < gap:
+            flags[t] |= TIE_BOUNDARY
+        if k > 1 and np.any((s[: k - 1] - s[1:k]) < gap):
+            flags[t] |= TIE_WITHIN
+    return flags
+
+
+def valid_selections(L_row: np.ndarray, k: int, gap: float = NEAR_TIE_GAP):
+    """All k-sets a float32 selection may return when logits within `gap` are tied.
+
+    A set S is valid when no expert outside S beats a member of S by `gap` or more.
+    Each set is returned in the canonical slot order (descending float32 logit, ties
+    to the lower index).  The oracle's own choice is always the first entry.
+    """
+    L32 = np.asarray(L_row, dtype=F64).astype(np.float32)
+    E = L32.shape[0]
+    order = list(np.argsort(-L32, kind="stable"))
+    first = tuple(int(e) for e in order[:k])
+    if k == E:
+        return [first]
+    v_k, v_k1 = L32[order[k - 1]], L32[order[k]]
+    fixed = [e for e in order if L32[e] > v_k + gap]
+    band = [e for e in order if (v_k1 - gap) <= L32[e] <= (v_k + gap) and e not in fixed]
+    out = [first]
+    need = k - len(fixed)
+    if need <= 0 or len(band) > 12:
+        return out
+    for combo in itertools.combinations(band, need):
+        S = set(fixed) | set(combo)
+        inside = [L32[e] for e in S]
+        outside = [L32[e] for e in range(E) if e not in S]
+        if min(inside) > max(outside) - gap:
+            ordered = tuple(int(e) for e in order if e in S)
+            if ordered not in out:
+                out.append(ordered)
+    return out
+
+
+# ------------------------------------------------------------------ counts, permutation
+
+def expert_counts(idx: np.ndarray, E: int) -> np.ndarray:
+    """Tokens routed to each expert: a literal bincount over the flat expert ids."""
+    counts = [0] * E
+    for e in np.asarray(idx).ravel().tolist():
+        counts[e] += 1
+    return np.array(counts, dtype=np.int32)
+
+
+def exclusive_offsets(counts: np.ndarray) -> np.ndarray:
+    """offsets[e] = sum of counts[0..e-1]; offsets[E] = total.  int32 [E+1]."""
+    off = [0]
+    for c in np.asarray(counts).tolist():
+        off.append(off[-1] + c)
+    return np.array(off, dtype=np.int32)
+
+
+def stable_permutation(idx: np.ndarray, E: int):
+    """Group the (token, slot) pairs by expert, tokens ascending within an expert.
+
+    Returns (counts [E], offsets [E+1], perm_src [T*k], perm_dst [T*k]):
+    permuted row r holds token perm_src[r]; pair (t, j) lands in row perm_dst[t*k + j].
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    buckets = [[] for _ in range(E)]
+    for t in range(T):
+        for j in range(k):
+            buckets[int(idx[t, j])].append((t, j))
+    counts = expert_counts(idx, E)
+    offsets = exclusive_offsets(counts)
+    perm_src = np.empty(T * k, dtype=np.int32)
+    perm_dst = np.empty(T * k, dtype=np.int32)
+    r = 0
+    for e in range(E):
+        for (t, j) in buckets[e]:
+            perm_src[r] = t
+            perm_dst[t * k + j] = r
+            r += 1
+    return counts, offsets, perm_src, perm_dst
+
+
+def gather_rows(hidden, perm_src) -> np.ndarray:
+    """x_perm[r] = hidden[perm_src[r]] (a copy, same dtype)."""
+    return np.asarray(hidden)[np.asarray(perm_src, dtype=np.int64)]
+
+
+# ------------------------------------------------------------------------ experts
+
+def silu(g: np.ndarray) -> np.ndarray:
+    """silu(g) = g * sigmoid(g) = g / (1 + exp(-g))."""
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g))
+
+
+def swiglu(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """Standard SwiGLU: silu(gate) * up (alpha 1, beta 0, no clipping)."""
+    return silu(gate) * up
+
+
+def fc1_gate_up(fc1_e: np.ndarray, layout: str):
+    """Split one expert's fc1 [2I, H] into its gate rows and up rows, each [I, H]."""
+    if layout == "interleaved":
+        return fc1_e[0::2], fc1_e[1::2]
+    if layout == "chunked":
+        I = fc1_e.shape[0] // 2
+        return fc1_e[:I], fc1_e[I:]
+    raise ValueError(f"unknown fc1 layout {layout!r}")
+
+
+def expert_ffn(x_rows, fc1_e, fc2_e, layout: str = "interleaved") -> np.ndarray:
+    """One expert on rows x [n, H]: a = swiglu(x W_gate^T, x W_up^T); y = a fc2^T.  [n, H]."""
+    x = np.asarray(x_rows, dtype=F64)
+    w_gate, w_up = fc1_gate_up(np.asarray(fc1_e, dtype=F64), layout)
+    a = swiglu(x @ w_gate.T, x @ w_up.T)
+    return a @ np.asarray(fc2_e, dtype=F64).T
+
+
+def combine(y_perm, perm_dst, w, T: int, k: int) -> np.ndarray:
+    """out[t] = sum_j w[t, j] * y_perm[perm_dst[t*k + j]], float64 [T, H]."""
+    y = np.asarray(y_perm, dtype=F64)
+    out = np.zeros((T, y.shape[1]), dtype=F64)
+    for j in range(k):
+        rows = np.asarray(perm_dst, dtype=np.int64).reshape(T, k)[:, j]
+        out += np.asarray(w, dtype=F64)[:, j:j + 1] * y[rows]
+    return out
+
+
+# ------------------------------------------------------------------------ the layer
+
+def moe_forward(hidden, router_w, router_bias, fc1: ArrayOrGetter, fc2: ArrayOrGetter,
+                k: int, normalize: int, layout: str = "interleaved",
+                idx: Optional[np.ndarray] = None,
+                tokens: Optional[Sequence[int]] = None) -> dict:
+    """The fused MoE layer on the given tensors, float64.
+
+    `idx` forces the routing (its weights are still computed from the logits);
+    `tokens` restricts the expert evaluation to those tokens (routing is always over
+    all tokens) and the returned `out` then has one row per listed token.
+    Returns dict(logits, idx, w, out).
+    """
+    x = np.asarray(hidden)
+    T = x.shape[0]
+    L = router_logits(x, router_w, router_bias)
+    if idx is None:
+        idx = select_topk(L, k)
+    w = routing_weights(L, idx, normalize)
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    out = np.zeros((tok.size, x.shape[1]), dtype=F64)
+    if tok.size == 0:
+        return dict(logits=L, idx=idx, w=w, out=out)
+    sub_idx = idx[tok]
+    E = np.asarray(router_w).shape[0]
+    for e in range(E):
+        rows, slots = np.nonzero(sub_idx == e)
+        if rows.size == 0:
+            continue
+        y = expert_ffn(x[tok[rows]], _expert(fc1, e), _expert(fc2, e), layout)
+        out[rows] += w[tok[rows], slots][:, None] * y
+    return dict(logits=L, idx=idx, w=w, out=out)
+
+
+def moe_dense_masked(hidden, router_w, router_bias, fc1, fc2, k: int, normalize: int,
+                     layout: str = "interleaved") -> np.ndarray:
+    """Brute force: every expert on every token, weighted by the routing mask.
+
+    This is the static per-expert unroll of the fallback: expert e's output for all
+    tokens times the token's weight for e (zero where e was not chosen).
+    """
+    x = np.asarray(hidden)
+    T, H = x.shape
+    E = np.asarray(router_w).shape[0]
+    L = router_logits(x, router_w, router_bias)
+    idx = select_topk(L, k)
+    w = routing_weights(L, idx, normalize)
+    mask = np.zeros((T, E), dtype=F64)
+    for t in range(T):
+        for j in range(k):
+            mask[t, idx[t, j]] = w[t, j]
+    out = np.zeros((T, H), dtype=F64)
+    for e in range(E):
+        out += mask[:, e:e + 1] * expert_ffn(x, _expert(fc1, e), _expert(fc2, e), layout)
+    return out
+
+
+def chunked_to_interleaved(fc1_chunked: np.ndarray) -> np.ndarray:
+    """[E, 2I, H] chunked -> interleaved: dst[e, 2j+s] = src[e, s*I + j] for s in {0, 1}."""
+    src = np.asarray(fc1_chunked)
+    E, two_i, H = src.shape
+    I = two_i // 2
+    dst = np.empty_like(src)
+    for j in range(I):
+        for s in (0, 1):
+            dst[:, 2 * j + s, :] = src[:, s * I + j, :]
+    return dst

@@ -1,0 +1,408 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself: each pin is a hand-derived value
+(tests/golden/micro_cases.txt), a closed form, an invariant, or an independent
+formulation through a different library routine (a stable sort, bincount,
+reshape/transpose, scipy's softmax).  The mutation tests at the end plant a
+plausible mistake in the oracle and check that some pin catches it.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import softmax as sp_softmax
+
+from golden_io import load_cases, shaped
+from oracle import moe_oracle as O
+from synth import WORKLOADS, Workload, make_inputs, round_to_bf16_bits, bf16_bits_to_f32
+
+CASES = load_cases()
+
+
+def small(T=24, H=32, E=6, k=2, I=16, dtype="f32", seed=3, bias=None, layout="interleaved"):
+    wl = Workload("pin", T=T, H=H, E=E, k=k, I=I, dtype=dtype, router_bias_std=bias,
+                  fc1_layout=layout, seed=seed)
+    return make_inputs(wl)
+
+
+def fwd(inp, k=None, normalize=1, layout="interleaved", **kw):
+    wl = inp.wl
+    return O.moe_forward(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                         inp.values("fc1"), inp.values("fc2"), wl.k if k is None else k,
+                         normalize, layout, **kw)
+
+
+# ------------------------------------------------------------------ golden cases
+
+def check_golden_values():
+    for name in ("single_expert", "normalize_off_two_experts", "chunked_gate_first"):
+        c = CASES[name]
+        s = shaped(c)
+        r = O.moe_forward(s["hidden"], s["router_w"], None, s["fc1"], s["fc2"], c["k"],
+                          c["normalize"], s["layout"])
+        np.testing.assert_array_equal(r["idx"].ravel(), c["idx"].astype(np.int32))
+        np.testing.assert_allclose(r["w"].ravel(), c["w"], rtol=1e-14, atol=0)
+        np.testing.assert_allclose(r["out"].ravel(), c["out"], rtol=1e-14, atol=1e-15)
+
+
+def check_golden_routing():
+    c = CASES["routing_rational"]
+    s = shaped(c)
+    L = O.router_logits(s["hidden"], s["router_w"])
+    idx = O.select_topk(L, c["k"])
+    np.testing.assert_array_equal(idx.ravel(), c["idx"])
+    np.testing.assert_allclose(O.routing_weights(L, idx, 1).ravel(), c["w"], rtol=1e-14)
+    np.testing.assert_allclose(O.routing_weights(L, idx, 0).ravel(), c["w_normalize_off"],
+                               rtol=1e-14)
+    c = CASES["exact_tie"]
+    s = shaped(c)
+    L = O.router_logits(s["hidden"], s["router_w"])
+    np.testing.assert_array_equal(O.select_topk(L, 1).ravel(), c["idx"])
+    np.testing.assert_array_equal(O.select_topk(L, 3).ravel(), c["idx_k3"])
+
+
+def test_golden_values():
+    check_golden_values()
+
+
+def test_golden_routing():
+    check_golden_routing()
+
+
+# --------------------------------------------------------------------- routing pins
+
+def check_topk_brute_force(seed=5):
+    inp = small(T=40, E=12, k=4, seed=seed)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    L32 = L.astype(np.float32)
+    idx = O.select_topk(L, 4)
+    for t in range(L.shape[0]):
+        ref = sorted(range(12), key=lambda e: (-float(L32[t, e]), e))[:4]
+        assert list(idx[t]) == ref
+
+
+def test_topk_matches_full_sort():
+    check_topk_brute_force()
+
+
+def test_topk_duplicate_router_rows_pick_lower_index():
+    inp = small(T=16, E=8, k=3, seed=11)
+    rw = inp.values("router_w").copy()
+    rw[5] = rw[2]          # experts 2 and 5 now always tie exactly
+    L = O.router_logits(inp.values("hidden"), rw)
+    idx = O.select_topk(L, 3)
+    for t in range(16):
+        row = list(idx[t])
+        if 5 in row:
+            assert 2 in row and row.index(2) < row.index(5)
+
+
+def test_k_equals_e_selects_all_in_sorted_order():
+    inp = small(T=10, E=5, k=5)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 5)
+    for t in range(10):
+        assert sorted(idx[t]) == list(range(5))
+        assert np.all(np.diff(L[t, idx[t]].astype(np.float32)) <= 0)
+
+
+def check_weights_sum_to_one():
+    inp = small(T=64, E=8, k=3, bias=0.5)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), inp["router_bias"])
+    w = O.routing_weights(L, O.select_topk(L, 3), 1)
+    assert np.max(np.abs(w.sum(axis=1) - 1.0)) <= 1e-12
+
+
+def test_weights_sum_to_one():
+    check_weights_sum_to_one()
+
+
+def test_normalized_weights_equal_softmax_over_chosen():
+    # softmax over all, keep k, renormalise == softmax over the chosen logits alone
+    inp = small(T=32, E=9, k=4)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 4)
+    w = O.routing_weights(L, idx, 1)
+    ref = sp_softmax(np.take_along_axis(L, idx.astype(np.int64), 1), axis=1)
+    np.testing.assert_allclose(w, ref, rtol=1e-13)
+
+
+def test_unnormalized_weights_are_full_softmax():
+    inp = small(T=32, E=9, k=4)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 4)
+    w = O.routing_weights(L, idx, 0)
+    ref = np.take_along_axis(sp_softmax(L, axis=1), idx.astype(np.int64), 1)
+    np.testing.assert_allclose(w, ref, rtol=1e-13)
+    assert np.all(w.sum(axis=1) < 1.0)
+
+
+def test_bias_is_added_before_selection():
+    inp = small(T=8, E=6, k=1)
+    bias = np.zeros(6, dtype=np.float32)
+    bias[4] = 1e3            # expert 4 must win every token
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), bias)
+    assert np.all(O.select_topk(L, 1) == 4)
+
+
+def test_near_tie_flags_and_alternatives():
+    # a gap of 4e-6 at the k/k+1 boundary is ambiguous; 1e-3 is not
+    L = np.array([[3.0, 1.0, 1.0 - 4e-6, -2.0], [3.0, 1.0, 0.999, -2.0]])
+    f = O.near_tie_flags(L, 2)
+    assert f[0] & O.TIE_BOUNDARY and not f[1] & O.TIE_BOUNDARY
+    alts = O.valid_selections(L[0], 2)
+    assert alts[0] == (0, 1) and (0, 2) in alts and len(alts) == 2
+    assert O.valid_selections(L[1], 2) == [(0, 1)]
+    Lw = np.array([[2.0, 2.0 - 3e-6, 0.0]])
+    assert O.near_tie_flags(Lw, 2)[0] == O.TIE_WITHIN
+
+
+# ------------------------------------------------------------- counts / permutation
+
+def test_counts_sum_and_match_bincount():
+    inp = small(T=50, E=7, k=3)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 3)
+    c = O.expert_counts(idx, 7)
+    assert c.sum() == 50 * 3
+    np.testing.assert_array_equal(c, np.bincount(idx.ravel(), minlength=7))
+
+
+def check_permutation(seed=7):
+    inp = small(T=50, E=7, k=3, seed=seed)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 3)
+    counts, offsets, src, dst = O.stable_permutation(idx, 7)
+    n = 150
+    # independent formulation: a stable argsort of the flat expert ids
+    order = np.argsort(idx.ravel(), kind="stable")
+    np.testing.assert_array_equal(src, order // 3)
+    ref_dst = np.empty(n, dtype=np.int64)
+    ref_dst[order] = np.arange(n)
+    np.testing.assert_array_equal(dst, ref_dst)
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(np.bincount(idx.ravel(), minlength=7))]))
+    assert sorted(dst.tolist()) == list(range(n))              # bijection
+    for t in range(50):
+        for j in range(3):
+            r = dst[t * 3 + j]
+            assert src[r] == t and offsets[idx[t, j]] <= r < offsets[idx[t, j] + 1]
+    for e in range(7):
+        seg = src[offsets[e]:offsets[e + 1]]
+        assert np.all(np.diff(seg) > 0)                          # stable: tokens ascending
+
+
+def test_permutation_properties():
+    check_permutation()
+
+
+def test_combine_of_permuted_rows_equals_layer():
+    inp = small(T=20, E=5, k=2)
+    r = fwd(inp)
+    counts, offsets, src, dst = O.stable_permutation(r["idx"], 5)
+    x_perm = O.gather_rows(inp.values("hidden"), src)
+    y_perm = np.zeros((x_perm.shape[0], inp.wl.H))
+    for e in range(5):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            y_perm[a:b] = O.expert_ffn(x_perm[a:b], inp.values("fc1")[e], inp.values("fc2")[e])
+    out = O.combine(y_perm, dst, r["w"], 20, 2)
+    np.testing.assert_allclose(out, r["out"], rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------ layout / values
+
+def check_chunked_equals_interleaved():
+    inp = small(T=12, E=4, k=2, I=8, layout="chunked")
+    chunked = inp.values("fc1")
+    E, two_i, H = chunked.shape
+    # the page's recipe: Reshape [E,2,I,H] -> Transpose [E,I,2,H] -> Reshape [E,2I,H]
+    recipe = chunked.reshape(E, 2, two_i // 2, H).transpose(0, 2, 1, 3).reshape(E, two_i, H)
+    conv = O.chunked_to_interleaved(chunked)
+    np.testing.assert_array_equal(conv, recipe)
+    a = fwd(inp, layout="chunked")["out"]
+    b = O.moe_forward(inp.values("hidden"), inp.values("router_w"), None, conv,
+                      inp.values("fc2"), 2, 1, "interleaved")["out"]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_chunked_equals_interleaved():
+    check_chunked_equals_interleaved()
+
+
+def check_dense_masked_equals_sparse(normalize=1):
+    inp = small(T=8, E=5, k=2, bias=0.3)
+    a = fwd(inp, normalize=normalize)["out"]
+    b = O.moe_dense_masked(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                           inp.values("fc1"), inp.values("fc2"), 2, normalize)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("normalize", [0, 1])
+def test_dense_masked_equals_sparse(normalize):
+    check_dense_masked_equals_sparse(normalize)
+
+
+def test_k_equals_e_is_softmax_weighted_sum_over_all_experts():
+    inp = small(T=6, E=4, k=4)
+    r = fwd(inp, k=4)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    p = sp_softmax(L, axis=1)
+    ref = sum(p[:, e:e + 1] * O.expert_ffn(inp.values("hidden"), inp.values("fc1")[e],
+                                           inp.values("fc2")[e]) for e in range(4))
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_zero_up_rows_give_zero():
+    inp = small()
+    fc1 = inp.values("fc1").copy()
+    fc1[:, 1::2, :] = 0.0
+    out = O.moe_forward(inp.values("hidden"), inp.values("router_w"), None, fc1,
+                        inp.values("fc2"), 2, 1)["out"]
+    assert np.all(out == 0.0)
+
+
+def test_zero_gate_rows_give_zero():
+    inp = small()
+    fc1 = inp.values("fc1").copy()
+    fc1[:, 0::2, :] = 0.0          # silu(0) = 0
+    out = O.moe_forward(inp.values("hidden"), inp.values("router_w"), None, fc1,
+                        inp.values("fc2"), 2, 1)["out"]
+    assert np.all(out == 0.0)
+
+
+def check_expert_ffn_scalar_loops():
+    # brute force with scalar loops on a tiny expert (orientation of every operand)
+    rng = np.random.default_rng(1)
+    H, I, n = 3, 2, 2
+    x = rng.standard_normal((n, H))
+    fc1 = rng.standard_normal((2 * I, H))
+    fc2 = rng.standard_normal((H, I))
+    y = O.expert_ffn(x, fc1, fc2)
+    for r in range(n):
+        for h in range(H):
+            acc = 0.0
+            for i in range(I):
+                g = sum(x[r, c] * fc1[2 * i, c] for c in range(H))
+                u = sum(x[r, c] * fc1[2 * i + 1, c] for c in range(H))
+                acc += fc2[h, i] * (g * (1.0 / (1.0 + math.exp(-g)))) * u
+            assert abs(acc - y[r, h]) <= 1e-12 * max(1.0, abs(acc))
+
+
+def test_expert_ffn_scalar_loops():
+    check_expert_ffn_scalar_loops()
+
+
+def test_sparse_evaluation_on_token_subset_matches_full():
+    inp = small(T=30, E=6, k=3)
+    full = fwd(inp)["out"]
+    sub = fwd(inp, tokens=[0, 7, 29])["out"]
+    # the BLAS may block a 3-row product differently from a 30-row one: rounding only
+    np.testing.assert_allclose(sub, full[[0, 7, 29]], rtol=1e-13, atol=1e-15)
+
+
+# ----------------------------------------------------------------------- inputs
+
+def test_bf16_rounding_is_nearest_even():
+    vals = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 2 ** -9,
+                     3.0e38], dtype=np.float32)
+    bits = round_to_bf16_bits(vals)
+    np.testing.assert_array_equal(bits, np.array([0x3F80, 0x3F80, 0x3F82, 0xC020, 0x3F80, 0x7F62],
+                                                 dtype=np.uint16))
+    np.testing.assert_array_equal(bf16_bits_to_f32(bits[:4]), np.array([1.0, 1.0, 1.0 + 2 ** -6, -2.5],
+                                                                        dtype=np.float32))
+
+
+def test_inputs_are_deterministic_and_seeded():
+    wl = Workload("d", T=5, H=16, E=3, k=2, I=8, dtype="bf16")
+    a, b = make_inputs(wl), make_inputs(wl)
+    for name in ("hidden", "router_w", "fc1", "fc2"):
+        np.testing.assert_array_equal(a[name], b[name])
+    c = make_inputs(wl, seed=1)
+    assert not np.array_equal(a["hidden"], c["hidden"])
+
+
+def test_batched_decode_workload_is_skewed():
+    # the workload asks for some experts with no token and some with more than 40
+    wl = WORKLOADS["batched_decode_bf16"]
+    inp = make_inputs(wl, weights=False)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), inp["router_bias"])
+    c = O.expert_counts(O.select_topk(L, wl.k), wl.E)
+    assert (c == 0).sum() >= 1 and (c > 40).sum() >= 1
+
+
+def test_outlier_rows():
+    wl = WORKLOADS["long_prefill_bf16"].with_(T=1000, H=64, E=4, k=2, I=64)
+    inp = make_inputs(wl, weights=False)
+    h = inp.values("hidden")
+    big = np.abs(h).max(axis=1) > 6.0
+    assert 0 < big.sum() <= 10
+
+
+# ---------------------------------------------------------------- mutation tests
+
+def _mut_drop_sigmoid(g):
+    return g
+
+
+def _mut_swap_gate_up(gate, up):
+    return O.silu(up) * gate
+
+
+def _mut_fc1_chunked_read(fc1_e, layout):
+    I = fc1_e.shape[0] // 2
+    return fc1_e[:I], fc1_e[I:]
+
+
+def _mut_ties_to_higher(L, k):
+    L32 = np.asarray(L).astype(np.float32)
+    out = np.empty((L32.shape[0], k), dtype=np.int32)
+    for t in range(L32.shape[0]):
+        order = sorted(range(L32.shape[1]), key=lambda e: (-float(L32[t, e]), -e))
+        out[t] = order[:k]
+    return out
+
+
+def _mut_no_renormalise(L, idx, normalize):
+    p = O.softmax_all(np.asarray(L, dtype=np.float64))
+    return np.take_along_axis(p, idx.astype(np.int64), axis=1)
+
+
+def _mut_unstable_perm(idx, E):
+    counts, offsets, src, dst = _real_perm(idx, E)
+    T, k = idx.shape
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        src[a:b] = src[a:b][::-1].copy()
+    for r, t in enumerate(src):
+        for j in range(k):
+            if idx[t, j] >= 0 and offsets[idx[t, j]] <= r < offsets[idx[t, j] + 1]:
+                dst[t * k + j] = r
+    return counts, offsets, src, dst
+
+
+_real_perm = O.stable_permutation
+
+MUTATIONS = [
+    ("silu", _mut_drop_sigmoid),
+    ("swiglu", _mut_swap_gate_up),
+    ("fc1_gate_up", _mut_fc1_chunked_read),
+    ("select_topk", _mut_ties_to_higher),
+    ("routing_weights", _mut_no_renormalise),
+    ("stable_permutation", _mut_unstable_perm),
+]
+
+PIN_CHECKS = [check_golden_values, check_golden_routing, check_topk_brute_force,
+              check_weights_sum_to_one, check_permutation, check_chunked_equals_interleaved,
+              check_dense_masked_equals_sparse, check_expert_ffn_scalar_loops]
+
+
+@pytest.mark.parametrize("name,mutant", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(monkeypatch, name, mutant):
+    monkeypatch.setattr(O, name, mutant)
+    caught = 0
+    for check in PIN_CHECKS:
+        try:
+            check()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin catches a mistake planted in {name}"
