@@ -1,0 +1,14 @@
+"""Fused mixture-of-experts FFN layer (com.microsoft::MoE with standard SwiGLU) for B200.
+
+The layer runs in the CUDA kernels of libmoe_b200.so (sm_100a), behind the C ABI
+declared in include/moe_b200.h; this package is the thin Python binding.
+"""
+from ._abi import MoEError, load as load_library  # noqa: F401
+from .ops import (alloc_workspace, combine, convert_chunked_to_interleaved,  # noqa: F401
+                  expert_ffn, forward, get_error, permute, route, set_stage_events,
+                  workspace_error_word, workspace_size)
+
+__all__ = ["forward", "route", "permute", "expert_ffn", "combine",
+           "convert_chunked_to_interleaved", "get_error", "set_stage_events",
+           "workspace_size", "alloc_workspace", "workspace_error_word", "load_library",
+           "MoEError"]

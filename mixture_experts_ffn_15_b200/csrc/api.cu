@@ -1,0 +1,387 @@
+// C ABI of the fused MoE FFN layer: argument checks, workspace layout and the
+// order of the launches.  Declarations and contracts: include/moe_b200.h.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe_b200.h"
+
+namespace moe {
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kNumStageEvents = 6;
+
+cudaEvent_t g_events[kNumStageEvents];
+bool g_events_on = false;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct Carver {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t r = off;
+        off = align_up(off + bytes);
+        return r;
+    }
+};
+
+struct FwdLayout {
+    size_t hdr, logits, idx, w, near, tile_counts, tile_base, counts, offsets, perm_src, perm_dst,
+        x_perm, act, y, total;
+};
+
+size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
+    const size_t es = elem_size(dt);
+    const size_t rows = static_cast<size_t>(T) * k;
+    const size_t nt = static_cast<size_t>(num_token_tiles(T));
+    Carver c;
+    FwdLayout L;
+    L.hdr = c.take(kAlign);   // [0] error word, [1] completion counter
+    L.logits = c.take(static_cast<size_t>(T) * E * 4);
+    L.idx = c.take(rows * 4);
+    L.w = c.take(rows * 4);
+    L.near = c.take(static_cast<size_t>(T) * 4);
+    L.tile_counts = c.take(nt * E * 4);
+    L.tile_base = c.take(nt * E * 4);
+    L.counts = c.take(static_cast<size_t>(E) * 4);
+    L.offsets = c.take(static_cast<size_t>(E + 1) * 4);
+    L.perm_src = c.take(rows * 4);
+    L.perm_dst = c.take(rows * 4);
+    L.x_perm = c.take(rows * H * es);
+    L.act = c.take(rows * I * es);
+    L.y = c.take(rows * H * es);
+    L.total = c.off;
+    return L;
+}
+
+struct PermLayout {
+    size_t hdr, tile_counts, tile_base, total;
+};
+
+PermLayout perm_layout(int T, int E) {
+    const size_t nt = static_cast<size_t>(num_token_tiles(T));
+    Carver c;
+    PermLayout L;
+    L.hdr = c.take(kAlign);
+    L.tile_counts = c.take(nt * E * 4);
+    L.tile_base = c.take(nt * E * 4);
+    L.total = c.off;
+    return L;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_dtype(moe_dtype dt) { return dt == MOE_F32 || dt == MOE_BF16; }
+
+// Sizes shared by the layer and the staged calls.
+bool valid_sizes(int T, int H, int E, int k) {
+    if (T < 0 || H <= 0 || E <= 0 || E > kMaxExperts || k < 1 || k > E) return false;
+    if (H % 8 != 0) return false;
+    if (static_cast<long long>(T) * k > (1LL << 30)) return false;
+    return true;
+}
+
+bool standard_swiglu(const moe_swiglu& a) {
+    return a.alpha == 1.0f && a.beta == 0.0f && isinf(a.limit) && a.limit > 0;
+}
+
+void record(int i, cudaStream_t s) {
+    if (g_events_on) cudaEventRecord(g_events[i], s);
+}
+
+#define MOE_CUDA(call)                                  \
+    do {                                                \
+        if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+size_t moe_workspace_size(int T, int H, int E, int k, int I, moe_dtype dt) {
+    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 != 0 || !valid_dtype(dt)) return 0;
+    return fwd_layout(T, H, E, k, I, dt).total;
+}
+
+size_t moe_permute_workspace_size(int T, int E) {
+    if (T < 0 || E <= 0 || E > kMaxExperts) return 0;
+    return perm_layout(T, E).total;
+}
+
+size_t moe_expert_ffn_workspace_size(int rows, int I, moe_dtype dt) {
+    if (rows < 0 || I <= 0 || !valid_dtype(dt)) return 0;
+    return align_up(static_cast<size_t>(rows) * I * elem_size(dt)) + kAlign;
+}
+
+int32_t* moe_workspace_error_word(void* workspace) { return static_cast<int32_t*>(workspace); }
+
+moe_status moe_set_stage_events(void* const* events, int n_events) {
+    if (events == nullptr) {
+        g_events_on = false;
+        return MOE_OK;
+    }
+    if (n_events != kNumStageEvents) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < kNumStageEvents; ++i) {
+        if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+        g_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_events_on = true;
+    return MOE_OK;
+}
+
+moe_status moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,
+                     int H, int E, int k, int normalize, moe_dtype dt, int32_t* topk_idx,
+                     float* topk_w, float* logits, int32_t* near_tie, void* stream) {
+    if (!valid_sizes(T, H, E, k) || !valid_dtype(dt)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!hidden || !router_w || !topk_idx || !topk_w || !logits) return MOE_ERR_INVALID_ARG;
+    if (!aligned(hidden, 16) || !aligned(router_w, 16) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4) || !aligned(logits, 16) || (router_bias && !aligned(router_bias, 4)) ||
+        (near_tie && !aligned(near_tie, 4)))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == MOE_BF16 && tc_router_supported(T, H, E))
+        MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, nullptr, s));
+    else
+        MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, dt == MOE_BF16, logits, s));
+    TopkHistArgs a;
+    a.logits = logits;
+    a.bias = router_bias;
+    a.logits_biased = router_bias ? logits : nullptr;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.normalize = normalize ? 1 : 0;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.near_tie = near_tie;
+    a.do_hist = false;
+    MOE_CUDA(launch_topk_hist(a, s));
+    return MOE_OK;
+}
+
+moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H, int E, int k,
+                       moe_dtype dt, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                       int32_t* perm_dst, void* x_perm, int32_t* err_word, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    if (!valid_sizes(T, H, E, k) || !valid_dtype(dt)) return MOE_ERR_INVALID_ARG;
+    if (!topk_idx || !counts || !offsets || !perm_src || !perm_dst || !err_word || !workspace)
+        return MOE_ERR_INVALID_ARG;
+    if ((hidden == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+    if ((hidden && !aligned(hidden, 16)) || (x_perm && !aligned(x_perm, 16)) ||
+        !aligned(workspace, kAlign))
+        return MOE_ERR_INVALID_ARG;
+    const PermLayout L = perm_layout(T, E);
+    if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* done = reinterpret_cast<int32_t*>(ws + L.hdr);
+    if (T == 0) {
+        MOE_CUDA(cudaMemsetAsync(counts, 0, static_cast<size_t>(E) * 4, s));
+        MOE_CUDA(cudaMemsetAsync(offsets, 0, static_cast<size_t>(E + 1) * 4, s));
+        return MOE_OK;
+    }
+    MOE_CUDA(cudaMemsetAsync(done, 0, 4, s));
+    TopkHistArgs a;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.topk_idx = const_cast<int32_t*>(topk_idx);
+    a.do_hist = true;
+    a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
+    a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
+    a.counts = counts;
+    a.offsets = offsets;
+    a.done = done;
+    a.err = err_word;
+    MOE_CUDA(launch_topk_hist(a, s));
+    MOE_CUDA(launch_scatter(topk_idx, a.tile_base, T, E, k, perm_src, perm_dst, err_word, s));
+    if (x_perm)
+        MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, T * k, H, static_cast<int>(elem_size(dt)),
+                               x_perm, s));
+    return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* fc1,
+                          const void* fc2, int rows, int H, int E, int I, moe_swiglu act,
+                          moe_dtype dt, void* y_perm, void* workspace, size_t ws_bytes,
+                          void* stream) {
+    if (rows < 0 || H <= 0 || H % 8 || I <= 0 || I % 8 || E <= 0 || E > kMaxExperts ||
+        !valid_dtype(dt))
+        return MOE_ERR_INVALID_ARG;
+    if (!standard_swiglu(act)) return MOE_ERR_UNSUPPORTED;
+    if (dt == MOE_BF16 && !tc_ffn_supported(H, I)) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!x_perm || !offsets || !fc1 || !fc2 || !y_perm || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_perm, 16) || !aligned(fc1, 16) || !aligned(fc2, 16) || !aligned(y_perm, 16) ||
+        !aligned(workspace, kAlign))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_expert_ffn_workspace_size(rows, I, dt)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* err = reinterpret_cast<int32_t*>(ws);   // scratch error word of this call
+    void* act_buf = ws + kAlign;
+    MOE_CUDA(cudaMemsetAsync(err, 0, 4, s));
+    if (dt == MOE_BF16)
+        MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
+                               nullptr));
+    else
+        MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
+                                     static_cast<const float*>(fc1), static_cast<const float*>(fc2),
+                                     rows, H, E, I, static_cast<float*>(act_buf),
+                                     static_cast<float*>(y_perm), s, nullptr));
+    return MOE_OK;
+}
+
+moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w, int T,
+                       int H, int k, moe_dtype dt, void* out, void* stream) {
+    if (T < 0 || H <= 0 || H % 8 || k < 1 || k > kMaxExperts || !valid_dtype(dt) ||
+        static_cast<long long>(T) * k > (1LL << 30))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !perm_dst || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(y_perm, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    MOE_CUDA(launch_combine(y_perm, perm_dst, topk_w, T, H, k, dt == MOE_BF16, out,
+                            static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
+                       const void* fc1, const void* fc2, int T, int H, int E, int k, int I,
+                       int normalize, moe_swiglu act, moe_dtype dt, void* out, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt)) return MOE_ERR_INVALID_ARG;
+    if (!standard_swiglu(act)) return MOE_ERR_UNSUPPORTED;
+    if (dt == MOE_BF16 && !tc_ffn_supported(H, I)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!hidden || !router_w || !fc1 || !fc2 || !out || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!aligned(hidden, 16) || !aligned(router_w, 16) || !aligned(fc1, 16) || !aligned(fc2, 16) ||
+        !aligned(out, 16) || !aligned(workspace, kAlign) ||
+        (router_bias && !aligned(router_bias, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const FwdLayout L = fwd_layout(T, H, E, k, I, dt);
+    if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* err = reinterpret_cast<int32_t*>(ws + L.hdr);
+    int32_t* done = err + 1;
+    float* logits = reinterpret_cast<float*>(ws + L.logits);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    float* w = reinterpret_cast<float*>(ws + L.w);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
+    int32_t* perm_dst = reinterpret_cast<int32_t*>(ws + L.perm_dst);
+    void* x_perm = ws + L.x_perm;
+    void* act_buf = ws + L.act;
+    void* y = ws + L.y;
+    const bool bf16 = dt == MOE_BF16;
+    const int rows = T * k;
+
+    MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, kAlign, s));
+    record(0, s);
+    // route: logits, then top-k + softmax + bincount + scan in one kernel
+    if (bf16 && tc_router_supported(T, H, E))
+        MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, err, s));
+    else
+        MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, bf16, logits, s));
+    TopkHistArgs a;
+    a.logits = logits;
+    a.bias = router_bias;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.normalize = normalize ? 1 : 0;
+    a.topk_idx = idx;
+    a.topk_w = w;
+    a.near_tie = reinterpret_cast<int32_t*>(ws + L.near);
+    a.do_hist = true;
+    a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
+    a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
+    a.counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    a.offsets = offsets;
+    a.done = done;
+    a.err = err;
+    MOE_CUDA(launch_topk_hist(a, s));
+    record(1, s);
+    // permute: stable placement, then the row gather
+    MOE_CUDA(launch_scatter(idx, a.tile_base, T, E, k, perm_src, perm_dst, err, s));
+    MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H, static_cast<int>(elem_size(dt)),
+                           x_perm, s));
+    record(2, s);
+    // experts: fc1 + SwiGLU, fc2
+    cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
+    if (bf16)
+        MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s, mid));
+    else
+        MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
+                                     static_cast<const float*>(fc1), static_cast<const float*>(fc2),
+                                     rows, H, E, I, static_cast<float*>(act_buf),
+                                     static_cast<float*>(y), s, mid));
+    record(4, s);
+    MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));
+    record(5, s);
+    return MOE_OK;
+}
+
+moe_status convert_chunked_to_interleaved(const void* src, void* dst, int E, int I, int H,
+                                          moe_dtype dt, void* stream) {
+    if (E <= 0 || I <= 0 || H <= 0 || H % 8 || !valid_dtype(dt)) return MOE_ERR_INVALID_ARG;
+    if (!src || !dst || !aligned(src, 16) || !aligned(dst, 16)) return MOE_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(E) * 2 * I * H * elem_size(dt);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(src), b = reinterpret_cast<uintptr_t>(dst);
+    if (a < b + bytes && b < a + bytes) return MOE_ERR_INVALID_ARG;   // overlap
+    MOE_CUDA(launch_convert(src, dst, E, I, H, static_cast<int>(elem_size(dt)),
+                            static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status moe_get_error(const int32_t* err_word, void* stream, int32_t* bits) {
+    if (!err_word) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    if (cudaMemcpyAsync(&v, err_word, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (bits) *bits = v;
+    if (v & MOE_DEVERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+    if (v) return MOE_ERR_DEVICE;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// Device helpers shared by the kernels of the fused MoE layer.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kErrBadExpert = 1;   // mirrors MOE_DEVERR_BAD_EXPERT
+constexpr int kErrTimeout = 2;     // mirrors MOE_DEVERR_TIMEOUT
+constexpr float kNearTieGap = 1e-5f;
+
+// Token tile of the histogram / scatter kernels.
+constexpr int kTileTokens = 128;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// 8 bf16 packed in 16 bytes -> 8 floats (exact).
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Two floats -> packed bf16x2 (round to nearest even), low half = a.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+
+// silu(g) * u in float32 (standard SwiGLU).
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+    return g / (1.0f + expf(-g)) * u;
+}
+
+}  // namespace moe

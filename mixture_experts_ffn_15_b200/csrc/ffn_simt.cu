@@ -1,0 +1,120 @@
+// float32 grouped expert FFN on plain FMA (no TF32, which would not meet a 1e-4
+// relative tolerance).  Same math as the tensor-core path:
+//   act[r, i] = silu(x_perm[r] . fc1[e, 2i]) * (x_perm[r] . fc1[e, 2i+1])
+//   y[r, h]   = act[r] . fc2[e, h]
+// for the rows r of expert e ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op -
+// #326", "Attribute set": standard SwiGLU, interleaved fc1).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int SBM = 32, SBN = 64, SBK = 32;
+
+// out[r, n] = A[r, :] . W[e, n, :] for the rows of each expert, 32 x 64 output tile
+// per unit; with SWIGLU the adjacent (gate, up) columns are fused into one act value.
+template <bool SWIGLU>
+__global__ void __launch_bounds__(256)
+simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __restrict__ W,
+                         int n_w, int K, const int32_t* __restrict__ offsets, int E, int rows,
+                         float* __restrict__ out, int ldo) {
+    __shared__ float sA[SBM][SBK + 1];
+    __shared__ float sW[SBN][SBK + 1];
+    __shared__ int s_off[kMaxExperts + 1];
+    __shared__ int s_pre[kMaxExperts + 1];
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        int prev = 0, pre = 0;
+        for (int e = 0; e <= E; ++e) {
+            int o = offsets[e];
+            o = o < prev ? prev : (o > rows ? rows : o);
+            s_off[e] = o;
+            prev = o;
+        }
+        for (int e = 0; e < E; ++e) {
+            s_pre[e] = pre;
+            pre += (s_off[e + 1] - s_off[e] + SBM - 1) / SBM;
+        }
+        s_pre[E] = pre;
+    }
+    __syncthreads();
+    const int NT = (n_w + SBN - 1) / SBN;
+    const int total = s_pre[E] * NT;
+    const int tx = tid & 15, ty = tid >> 4;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const int mt = u / NT, nt = u - (u / NT) * NT;
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_pre[mid] <= mt) lo = mid; else hi = mid - 1;
+        }
+        const int e = lo;
+        const int row0 = s_off[e] + (mt - s_pre[e]) * SBM;
+        const int nrows = min(SBM, s_off[e + 1] - row0);
+        const float* We = W + static_cast<size_t>(e) * n_w * K;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int k0 = 0; k0 < K; k0 += SBK) {
+            for (int i = tid; i < SBM * SBK; i += 256) {
+                const int r = i / SBK, c = i - (i / SBK) * SBK;
+                sA[r][c] = (r < nrows && k0 + c < K) ? A[static_cast<size_t>(row0 + r) * lda + k0 + c] : 0.f;
+            }
+            for (int i = tid; i < SBN * SBK; i += 256) {
+                const int n = i / SBK, c = i - (i / SBK) * SBK;
+                const int wn = nt * SBN + n;
+                sW[n][c] = (wn < n_w && k0 + c < K) ? We[static_cast<size_t>(wn) * K + k0 + c] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int c = 0; c < SBK; ++c) {
+                const float a0 = sA[ty * 2][c], a1 = sA[ty * 2 + 1][c];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float w = sW[tx * 4 + q][c];
+                    acc[0][q] = fmaf(a0, w, acc[0][q]);
+                    acc[1][q] = fmaf(a1, w, acc[1][q]);
+                }
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int r = ty * 2 + rr;
+            if (r >= nrows) continue;
+            float* o = out + static_cast<size_t>(row0 + r) * ldo;
+            const int n0 = nt * SBN + tx * 4;
+            if constexpr (SWIGLU) {
+                if (n0 + 1 < n_w) o[n0 / 2] = swiglu_f32(acc[rr][0], acc[rr][1]);
+                if (n0 + 3 < n_w) o[n0 / 2 + 1] = swiglu_f32(acc[rr][2], acc[rr][3]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (n0 + q < n_w) o[n0 + q] = acc[rr][q];
+            }
+        }
+    }
+}
+
+int simt_grid(int rows, int E, int n_w) {
+    const long long bound = (static_cast<long long>((rows + SBM - 1) / SBM) + E) * ((n_w + SBN - 1) / SBN);
+    const long long cap = static_cast<long long>(device_sm_count()) * 8;
+    return static_cast<int>(bound < cap ? bound : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
+                                const float* fc2, int rows, int H, int E, int I, float* act,
+                                float* y, cudaStream_t s, cudaEvent_t mid) {
+    if (rows <= 0) return cudaSuccess;
+    simt_grouped_gemm_kernel<true><<<simt_grid(rows, E, 2 * I), 256, 0, s>>>(
+        x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    if (mid) cudaEventRecord(mid, s);
+    simt_grouped_gemm_kernel<false><<<simt_grid(rows, E, H), 256, 0, s>>>(act, I, fc2, H, I,
+                                                                           offsets, E, rows, y, H);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

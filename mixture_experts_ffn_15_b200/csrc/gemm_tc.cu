@@ -1,0 +1,527 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// The grouped matmul of grouped_mm_experts_forward ("Contributing Gemma 4 support
+// and ONNX export optimizations", "Key Technical Contributions") runs, for every
+// expert e, over that expert's contiguous block of permuted rows:
+//   fc1 + SwiGLU: act[r, i] = silu(x[r] . fc1[e, 2i]) * (x[r] . fc1[e, 2i+1])
+//   fc2:          y[r, h]   = act[r] . fc2[e, h]
+// with standard SwiGLU and the interleaved fc1 layout of "Gemma 4 MoE: re-enable
+// fused com.microsoft::MoE op - #326", "Attribute set".  The router logits
+// (hidden . router_w^T) reuse the same kernel as a single group with a float32
+// epilogue.
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0     TMA producer: A and B tiles (64-wide K slices, 128-byte swizzle)
+//              into a ring of shared-memory stages, completion on mbarriers;
+//   warp 1     MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> f32) into one of
+//              two TMEM accumulators, tcgen05.commit frees stages / publishes tiles;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//              32*(w%4) .. +31), activation, bf16 pack, global stores.  The second
+//              accumulator lets the epilogue of one tile overlap the next mainloop.
+//
+// Two orientations of the same mainloop:
+//   token-M  (prefill):  M = 128 permuted rows, N = BN weight rows.  Tile map: for
+//            each expert, ceil(n_e / 128) row tiles x (n_out / BN) column tiles.
+//   weight-M (decode):   M = 128 weight rows, N = the expert's tokens (<= 64 per
+//            unit, loaded in 16-row boxes).  The weight tile streams from HBM once
+//            per unit; tokens are few, so this keeps every MMA 128 rows tall.
+// The tile map is rebuilt in every CTA from the device offsets (no host sync).
+//
+// Every wait is bounded (2 s); on expiry the CTA winds down, reports
+// MOE_DEVERR_TIMEOUT in the error word and still frees its TMEM.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;              // rows of A per tile (MMA M)
+constexpr int BK = 64;               // K per stage: one 128-byte row of bf16
+constexpr int kThreads = 192;
+constexpr int kTokChunk = 64;        // weight-M: tokens per unit
+constexpr int kBoxTok = 16;          // weight-M: token rows per TMA box
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+enum Mode : int { TOK_SWIGLU = 0, TOK_PLAIN = 1, TOK_F32 = 2, W_SWIGLU = 3, W_PLAIN = 4 };
+
+template <int MODE, int BN>
+struct Tr {
+    static constexpr bool kWeightM = (MODE == W_SWIGLU || MODE == W_PLAIN);
+    static constexpr int kBRows = kWeightM ? kTokChunk : BN;
+    static constexpr int kABytes = BM * BK * 2;
+    static constexpr int kBBytes = kBRows * BK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    static constexpr int kAccStride = kWeightM ? kTokChunk : 256;
+    static constexpr int kTmemCols = kWeightM ? 128 : 512;
+    static constexpr int kUnitRows = kWeightM ? kTokChunk : BM;
+    // barriers (2*stages + 4) + tmem slot + abort flag, then offsets and prefix
+    static constexpr int kMiscBytes = (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static_assert(kWeightM || (BN % 16 == 0 && BN >= 16 && BN <= 256), "UMMA N");
+};
+
+struct TcParams {
+    const int32_t* offsets;   // [E+1] device, or nullptr: one group of `rows` rows
+    int E;
+    int rows;                 // rows of the token matrix
+    int K;                    // reduction length (multiple of 64)
+    int n_out;                // weight rows per expert
+    void* out;
+    int ldo;                  // output row stride, elements
+    int32_t* err;
+};
+
+struct Unit {
+    int g;      // expert
+    int row0;   // first token row
+    int nrows;  // valid token rows (<= kUnitRows)
+    int sub;    // column tile (token-M) or weight row tile (weight-M) inside the expert
+};
+
+// s_off: sanitised offsets (clamped to [0, rows], non-decreasing); s_pre[g]: first
+// tile of group g; s_pre[G]: tile count.  Runs on one warp.
+__device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int unit_rows, int* s_off,
+                                               int* s_pre, int lane) {
+    constexpr int kPer = (kMaxExperts + 1 + 31) / 32;   // 9
+    const int per = (G + 1 + 31) / 32;
+    int v[kPer];
+    bool bad = false;
+    for (int q = 0; q < per; ++q) {
+        const int i = lane * per + q;
+        int raw = p.rows;
+        if (i <= G) raw = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows);
+        if (i == 0 && p.offsets && raw != 0) bad = true;
+        int c = raw < 0 ? 0 : (raw > p.rows ? p.rows : raw);
+        if (c != raw) bad = true;
+        v[q] = c;
+    }
+    for (int q = 1; q < per; ++q)
+        if (v[q] < v[q - 1]) {
+            bad = bad || (lane * per + q <= G);
+            v[q] = v[q - 1];
+        }
+    const int lmax = v[per - 1];
+    int inc = lmax;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc = max(inc, y);
+    }
+    int excl = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) excl = 0;
+    for (int q = 0; q < per; ++q) {
+        const int i = lane * per + q;
+        if (v[q] < excl && i <= G) bad = true;
+        const int c = max(v[q], excl);
+        if (i <= G) s_off[i] = c;
+    }
+    if (bad && p.offsets && p.err) atomicOr(p.err, kErrBadExpert);
+    __syncwarp();
+    const int per2 = (G + 31) / 32;
+    int cnt[kPer];
+    int lsum = 0;
+    for (int q = 0; q < per2; ++q) {
+        const int g = lane * per2 + q;
+        int c = 0;
+        if (g < G) c = (s_off[g + 1] - s_off[g] + unit_rows - 1) / unit_rows;
+        cnt[q] = c;
+        lsum += c;
+    }
+    int incl = lsum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    int run = incl - lsum;
+    for (int q = 0; q < per2; ++q) {
+        const int g = lane * per2 + q;
+        if (g < G) s_pre[g] = run;
+        run += cnt[q];
+    }
+    if (lane == 31) s_pre[G] = incl;
+}
+
+__device__ __forceinline__ Unit decode_unit(int u, int per_unit, int G, int unit_rows,
+                                            const int* s_off, const int* s_pre) {
+    const int tile = u / per_unit;
+    Unit t;
+    t.sub = u - tile * per_unit;
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    t.g = lo;
+    t.row0 = s_off[lo] + (tile - s_pre[lo]) * unit_rows;
+    t.nrows = min(unit_rows, s_off[lo + 1] - t.row0);
+    return t;
+}
+
+__device__ __forceinline__ float f32(uint32_t x) { return __uint_as_float(x); }
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcParams p) {
+    using C = Tr<MODE, BN>;
+    constexpr bool kW = C::kWeightM;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::kStages * C::kABytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* s_pre = s_off + (kMaxExperts + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.offsets ? p.E : 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) build_tile_map(p, G, C::kUnitRows, s_off, s_pre, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int per_unit = kW ? p.n_out / BM : p.n_out / BN;
+    const int num_units = s_pre[G] * per_unit;
+    const int nk = p.K / BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+                const int nl = kW ? (t.nrows + kBoxTok - 1) / kBoxTok : 0;
+                const uint32_t bytes =
+                    kW ? static_cast<uint32_t>(C::kABytes + nl * kBoxTok * BK * 2) : C::kStageBytes;
+                const int wrow = t.g * p.n_out + t.sub * (kW ? BM : BN);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, bytes);
+                    const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
+                    const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
+                    if constexpr (!kW) {
+                        tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
+                        tma_load_2d(b_dst, &tmB, fb, kb * BK, wrow);
+                    } else {
+                        tma_load_2d(a_dst, &tmA, fb, kb * BK, wrow);
+                        for (int l = 0; l < nl; ++l)
+                            tma_load_2d(b_dst + l * kBoxTok * BK * 2, &tmB, fb, kb * BK,
+                                        t.row0 + l * kBoxTok);
+                    }
+                    ++issued;
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag) {
+                // let the copies already in flight land before the CTA exits
+                int dummy = 0;
+                for (int s = 0; s < C::kStages; ++s) {
+                    if (issued <= s) break;
+                    const long long fills = (issued - 1 - s) / C::kStages + 1;
+                    mbar_wait(smem_u32(&full[s]), static_cast<uint32_t>((fills - 1) & 1),
+                              &dummy, kWaitLimitNs / 4);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
+                const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+                const int n_mma = kW ? ((t.nrows + 15) / 16) * 16 : BN;
+                const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                                  idesc, (kb | kk) != 0);
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&tfull[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;   // TMEM lane = row of the accumulator
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
+            const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
+            tc_fence_after();
+            const uint32_t tb =
+                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::kAccStride);
+            if constexpr (!kW) {
+                const bool valid = r < t.nrows;
+                const size_t orow = static_cast<size_t>(t.row0 + r);
+                const int col0 = t.sub * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v[32];
+                    const bool full32 = (c + 32 <= BN);
+                    if (full32) tmem_ld_32x32b_x32(tb + c, v);
+                    else tmem_ld_32x32b_x16(tb + c, v);
+                    tmem_wait_ld();
+                    if (!valid) continue;
+                    const int nv = full32 ? 32 : 16;
+                    if constexpr (MODE == TOK_SWIGLU) {
+                        float a[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            a[i] = (2 * i < nv) ? swiglu_f32(f32(v[2 * i]), f32(v[2 * i + 1])) : 0.f;
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                              orow * p.ldo + (col0 + c) / 2);
+                        dst[0] = pack_bf16x8(a);
+                        if (nv == 32) dst[1] = pack_bf16x8(a + 8);
+                    } else if constexpr (MODE == TOK_PLAIN) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                              orow * p.ldo + col0 + c);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (8 * q < nv) {
+                                float f[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) f[i] = f32(v[8 * q + i]);
+                                dst[q] = pack_bf16x8(f);
+                            }
+                        }
+                    } else {   // TOK_F32
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.out) +
+                                                              orow * p.ldo + col0 + c);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            if (4 * q < nv) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                }
+            } else {
+                const int wr = t.sub * BM + r;   // weight row inside the expert
+#pragma unroll 1
+                for (int c = 0; c < t.nrows; c += 16) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tb + c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int n = c + i;
+                        const float x = f32(v[i]);
+                        if constexpr (MODE == W_SWIGLU) {
+                            const float up = __shfl_xor_sync(0xffffffffu, x, 1);
+                            if (!(lane & 1) && n < t.nrows)
+                                static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(t.row0 + n) * p.ldo + (wr >> 1)] =
+                                    __float2bfloat16_rn(swiglu_f32(x, up));
+                        } else {
+                            if (n < t.nrows)
+                                static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(t.row0 + n) * p.ldo + wr] =
+                                    __float2bfloat16_rn(x);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 matrix [rows, K] row-major, boxes of 64 (K) x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || rows <= 0) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int bound,
+                       cudaStream_t s) {
+    using C = Tr<MODE, BN>;
+    auto kern = tc_gemm_kernel<MODE, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int grid = device_sm_count();
+    if (bound < grid) grid = bound;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kThreads, C::kSmemBytes, s>>>(a, b, p);
+    return cudaGetLastError();
+}
+
+int pick_bn(int n_out) {
+    const int cands[5] = {256, 192, 176, 128, 64};
+    for (int c : cands)
+        if (n_out % c == 0) return c;
+    return 0;
+}
+
+// One grouped GEMM: out = A(rows x K) . W_e^T over the experts' row blocks.
+cudaError_t grouped_gemm(bool swiglu, const void* act_in, int rows, int K, const void* w, int E,
+                         int n_out, const int32_t* offsets, void* out, int ldo, int32_t* err,
+                         cudaStream_t s) {
+    TcParams p{offsets, E, rows, K, n_out, out, ldo, err};
+    // Few rows per expert: put the weights on the MMA's M side (weight-M).
+    const bool weight_m = (n_out % BM == 0) && (static_cast<long long>(rows) <= 64LL * E);
+    CUtensorMap ma, mb;
+    if (weight_m) {
+        if (!make_map(&ma, w, static_cast<long long>(E) * n_out, K, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&mb, act_in, rows, K, kBoxTok)) return cudaErrorInvalidValue;
+        const long long bound = (static_cast<long long>((rows + kTokChunk - 1) / kTokChunk) + E) * (n_out / BM);
+        const int b = static_cast<int>(bound > (1 << 30) ? (1 << 30) : bound);
+        return swiglu ? launch_one<W_SWIGLU, 64>(ma, mb, p, b, s) : launch_one<W_PLAIN, 64>(ma, mb, p, b, s);
+    }
+    const int bn = pick_bn(n_out);
+    if (!make_map(&ma, act_in, rows, K, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, w, static_cast<long long>(E) * n_out, K, bn)) return cudaErrorInvalidValue;
+    const long long bound = (static_cast<long long>((rows + BM - 1) / BM) + E) * (n_out / bn);
+    const int b = static_cast<int>(bound > (1 << 30) ? (1 << 30) : bound);
+#define MOE_TOK_CASE(BNV)                                                          \
+    case BNV:                                                                      \
+        return swiglu ? launch_one<TOK_SWIGLU, BNV>(ma, mb, p, b, s)               \
+                      : launch_one<TOK_PLAIN, BNV>(ma, mb, p, b, s);
+    switch (bn) {
+        MOE_TOK_CASE(256)
+        MOE_TOK_CASE(192)
+        MOE_TOK_CASE(176)
+        MOE_TOK_CASE(128)
+        MOE_TOK_CASE(64)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MOE_TOK_CASE
+}
+
+}  // namespace
+
+bool tc_ffn_supported(int H, int I) { return H % 64 == 0 && I % 64 == 0 && H > 0 && I > 0; }
+
+bool tc_router_supported(int T, int H, int E) {
+    return T >= 512 && H % 64 == 0 && (E == 64 || E == 128 || E == 256);
+}
+
+cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
+                          const void* fc2, int rows, int H, int E, int I, void* act, void* y,
+                          int32_t* err, cudaStream_t s, cudaEvent_t mid) {
+    if (rows <= 0) return cudaSuccess;
+    cudaError_t e = grouped_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s);
+    if (e != cudaSuccess) return e;
+    if (mid) cudaEventRecord(mid, s);
+    return grouped_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
+}
+
+cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,
+                             float* logits, int32_t* err, cudaStream_t s) {
+    TcParams p{nullptr, 1, T, H, E, logits, E, err};
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
+    const int bound = (T + BM - 1) / BM;
+    switch (E) {
+        case 64: return launch_one<TOK_F32, 64>(ma, mb, p, bound, s);
+        case 128: return launch_one<TOK_F32, 128>(ma, mb, p, bound, s);
+        case 256: return launch_one<TOK_F32, 256>(ma, mb, p, bound, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,62 @@
+// Host-side launchers of the kernels (internal to the library, not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+int device_sm_count();
+
+// ---------------------------------------------------------------- route.cu
+cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, int T, int H,
+                                      int E, bool bf16, float* logits, cudaStream_t s);
+
+struct TopkHistArgs {
+    const float* logits = nullptr;   // [T, E] raw logits; nullptr: topk_idx is an input
+    const float* bias = nullptr;     // [E] or nullptr
+    float* logits_biased = nullptr;  // where to write logits + bias (nullptr: not written)
+    int T = 0, E = 0, k = 0, normalize = 1;
+    int32_t* topk_idx = nullptr;     // [T, k] out (or in when logits == nullptr)
+    float* topk_w = nullptr;         // [T, k] out
+    int32_t* near_tie = nullptr;     // [T] out or nullptr
+    bool do_hist = false;
+    int32_t* tile_counts = nullptr;  // [ntiles, E] scratch
+    int32_t* tile_base = nullptr;    // [ntiles, E] out: first permuted row of (tile, e)
+    int32_t* counts = nullptr;       // [E] out
+    int32_t* offsets = nullptr;      // [E + 1] out
+    int32_t* done = nullptr;         // completion counter, 0 on entry, 0 on exit
+    int32_t* err = nullptr;          // device error word
+};
+cudaError_t launch_topk_hist(const TopkHistArgs& a, cudaStream_t s);
+
+inline int num_token_tiles(int T) { return (T + 127) / 128; }
+
+// ---------------------------------------------------------------- permute.cu
+cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
+                           int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s);
+cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
+                          int E, int T, int rows_max, int H, int elem_bytes, void* x_perm,
+                          cudaStream_t s);
+
+// ---------------------------------------------------------------- combine.cu
+cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w,
+                           int T, int H, int k, bool bf16, void* out, cudaStream_t s);
+cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
+                           cudaStream_t s);
+
+// ---------------------------------------------------------------- ffn_simt.cu
+cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
+                                const float* fc2, int rows, int H, int E, int I, float* act,
+                                float* y, cudaStream_t s, cudaEvent_t mid);
+
+// ---------------------------------------------------------------- gemm_tc.cu
+bool tc_ffn_supported(int H, int I);
+bool tc_router_supported(int T, int H, int E);
+cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
+                          const void* fc2, int rows, int H, int E, int I, void* act, void* y,
+                          int32_t* err, cudaStream_t s, cudaEvent_t mid);
+cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,
+                             float* logits, int32_t* err, cudaStream_t s);
+
+}  // namespace moe

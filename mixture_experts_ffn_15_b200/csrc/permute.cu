@@ -1,0 +1,103 @@
+// Stable token permutation and row gather of the fused MoE layer.
+//
+// Pair (t, j) with expert e = topk_idx[t, j] goes to permuted row
+//   offsets[e] + #{t' < t : some slot of t' chose e}
+// i.e. the rows of an expert are contiguous and ordered by token (the grouped
+// matmul of grouped_mm_experts_forward, "Contributing Gemma 4 support and ONNX
+// export optimizations", "Key Technical Contributions").  Each 128-token tile knows
+// the first row of every expert from the histogram kernel; inside the tile the rank
+// of a token among the tile's tokens of the same expert is a population count over
+// a 128-bit membership mask held in shared memory, so the result is deterministic.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kScatterThreads = 512;
+constexpr int kMaskWords = kTileTokens / 32;
+
+__global__ void __launch_bounds__(kScatterThreads)
+scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ tile_base, int T,
+               int E, int k, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_dst,
+               int32_t* __restrict__ err) {
+    __shared__ uint32_t s_mask[kMaxExperts * kMaskWords];
+    const int tile = blockIdx.x;
+    const int t_begin = tile * kTileTokens;
+    const int nt = min(kTileTokens, T - t_begin);
+    for (int i = threadIdx.x; i < E * kMaskWords; i += kScatterThreads) s_mask[i] = 0;
+    __syncthreads();
+    const int npairs = nt * k;
+    const int32_t* ids = topk_idx + static_cast<size_t>(t_begin) * k;
+    for (int p = threadIdx.x; p < npairs; p += kScatterThreads) {
+        const int e = ids[p];
+        const int tl = p / k;
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+            const uint32_t bit = 1u << (tl & 31);
+            // the same expert twice in one token: reported, the ranks then collide
+            if (atomicOr(&s_mask[e * kMaskWords + (tl >> 5)], bit) & bit) atomicOr(err, kErrBadExpert);
+        }
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < npairs; p += kScatterThreads) {
+        const int e = ids[p];
+        const int tl = p / k;
+        int32_t row = -1;
+        if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+            const uint32_t* m = s_mask + e * kMaskWords;
+            const int w = tl >> 5;
+            int rank = __popc(m[w] & ((1u << (tl & 31)) - 1u));
+            for (int q = 0; q < w; ++q) rank += __popc(m[q]);
+            row = tile_base[static_cast<size_t>(tile) * E + e] + rank;
+            perm_src[row] = t_begin + tl;
+        }
+        perm_dst[static_cast<size_t>(t_begin) * k + p] = row;
+    }
+}
+
+// x_perm[r] = hidden[perm_src[r]] for r < offsets[E]; one warp per row, 16-byte
+// vectors.  A source index outside [0, T) (possible only after bad ids in the
+// staged API) writes a zero row instead of reading out of bounds.
+__global__ void __launch_bounds__(256)
+gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm_src,
+              const int32_t* __restrict__ offsets, int E, int T, int rows_max, int vec_per_row,
+              uint4* __restrict__ x_perm) {
+    const int rows = min(offsets[E], rows_max);
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+        const int src = perm_src[r];
+        uint4* dst = x_perm + static_cast<size_t>(r) * vec_per_row;
+        if (src < 0 || src >= T) {
+            for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        const uint4* s = hidden + static_cast<size_t>(src) * vec_per_row;
+        for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(s + v);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
+                           int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    scatter_kernel<<<num_token_tiles(T), kScatterThreads, 0, s>>>(topk_idx, tile_base, T, E, k,
+                                                                  perm_src, perm_dst, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
+                          int E, int T, int rows_max, int H, int elem_bytes, void* x_perm,
+                          cudaStream_t s) {
+    if (rows_max <= 0) return cudaSuccess;
+    const int vec = H * elem_bytes / 16;
+    int blocks = (rows_max + 7) / 8;
+    const int cap = device_sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    gather_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(hidden), perm_src, offsets, E,
+                                         T, rows_max, vec, static_cast<uint4*>(x_perm));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,206 @@
+"""Torch-facing wrappers of the C ABI.
+
+PyTorch provides device memory and streams only: every step of the layer runs in
+the CUDA kernels of libmoe_b200.so.  These functions check dtypes, devices, shapes
+and contiguity, allocate outputs and workspaces with torch when the caller does
+not pass them, and raise MoEError on any non-OK status.
+"""
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import STANDARD_SWIGLU, MoeSwiglu, check
+
+_DT = {torch.bfloat16: _abi.MOE_BF16, torch.float32: _abi.MOE_F32}
+
+
+def _lib():
+    return _abi.load()
+
+
+def _dtcode(t):
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32") from None
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _swiglu(alpha, beta, limit):
+    return MoeSwiglu(alpha, beta, limit)
+
+
+def workspace_size(T, H, E, k, I, dtype):
+    """Bytes of workspace moe_forward needs (0 for sizes it rejects)."""
+    return _lib().moe_workspace_size(T, H, E, k, I, _DT[dtype])
+
+
+def alloc_workspace(nbytes, device):
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out=None,
+            workspace=None, stream=None, swiglu=(1.0, 0.0, float("inf"))):
+    """The fused MoE layer: out[T, H] = sum_j w[t, j] * FFN_{idx[t, j]}(hidden[t])."""
+    _need(hidden, "hidden")
+    dt = hidden.dtype
+    T, H = hidden.shape
+    E = router_w.shape[0]
+    I = fc2.shape[2]
+    _need(router_w, "router_w", dt, (E, H))
+    _need(fc1, "fc1", dt, (E, 2 * I, H))
+    _need(fc2, "fc2", dt, (E, H, I))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    if out is None:
+        out = torch.empty_like(hidden)
+    _need(out, "out", dt, (T, H))
+    need = workspace_size(T, H, E, k, I, dt)
+    if workspace is None:
+        # invalid sizes give 0 bytes; the C call then reports them
+        workspace = alloc_workspace(max(need, 256), hidden.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = _lib().moe_forward(_ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(fc1), _ptr(fc2),
+                            T, H, E, k, I, int(bool(normalize)), _swiglu(*swiglu), _dtcode(hidden),
+                            _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    check(st, "moe_forward")
+    return out
+
+
+def workspace_error_word(workspace):
+    """The int32 error word at the start of a moe_forward workspace, as a tensor view."""
+    return workspace[:4].view(torch.int32)
+
+
+def route(hidden, router_w, k, normalize=True, router_bias=None, stream=None):
+    """Router logits, top-k (descending, ties to the lower index) and routing weights."""
+    _need(hidden, "hidden")
+    T, H = hidden.shape
+    E = router_w.shape[0]
+    _need(router_w, "router_w", hidden.dtype, (E, H))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    dev = hidden.device
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    near = torch.empty((T,), dtype=torch.int32, device=dev)
+    st = _lib().moe_route(_ptr(hidden), _ptr(router_w), _ptr(router_bias), T, H, E, k,
+                          int(bool(normalize)), _dtcode(hidden), _ptr(idx), _ptr(w), _ptr(logits),
+                          _ptr(near), _stream(stream))
+    check(st, "moe_route")
+    return dict(idx=idx, w=w, logits=logits, near_tie=near)
+
+
+def permute(topk_idx, E, hidden=None, err_word=None, stream=None):
+    """Bincount, offsets, stable permutation and (with hidden) the gathered rows."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    H = hidden.shape[1] if hidden is not None else 8
+    dt = _dtcode(hidden) if hidden is not None else _abi.MOE_BF16
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    perm_src = torch.full((T * k,), -1, dtype=torch.int32, device=dev)
+    perm_dst = torch.empty((T * k,), dtype=torch.int32, device=dev)
+    x_perm = None
+    if hidden is not None:
+        _need(hidden, "hidden")
+        x_perm = torch.empty((T * k, H), dtype=hidden.dtype, device=dev)
+    if err_word is None:
+        err_word = torch.zeros((1,), dtype=torch.int32, device=dev)
+    ws = alloc_workspace(_lib().moe_permute_workspace_size(T, E), dev)
+    st = _lib().moe_permute(_ptr(hidden), _ptr(topk_idx), T, H, E, k, dt, _ptr(counts),
+                            _ptr(offsets), _ptr(perm_src), _ptr(perm_dst), _ptr(x_perm),
+                            _ptr(err_word), _ptr(ws), ws.numel(), _stream(stream))
+    check(st, "moe_permute")
+    return dict(counts=counts, offsets=offsets, perm_src=perm_src, perm_dst=perm_dst,
+                x_perm=x_perm, err_word=err_word)
+
+
+def expert_ffn(x_perm, offsets, fc1, fc2, y_perm=None, stream=None,
+               swiglu=(1.0, 0.0, float("inf"))):
+    """y_perm[r] = fc2_e(silu(x fc1_gate^T) * (x fc1_up^T)) over each expert's rows."""
+    _need(x_perm, "x_perm")
+    rows, H = x_perm.shape
+    E, two_i, _ = fc1.shape
+    I = two_i // 2
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(fc1, "fc1", x_perm.dtype, (E, 2 * I, H))
+    _need(fc2, "fc2", x_perm.dtype, (E, H, I))
+    if y_perm is None:
+        y_perm = torch.zeros_like(x_perm)
+    dt = _dtcode(x_perm)
+    ws = alloc_workspace(_lib().moe_expert_ffn_workspace_size(rows, I, dt), x_perm.device)
+    st = _lib().moe_expert_ffn(_ptr(x_perm), _ptr(offsets), _ptr(fc1), _ptr(fc2), rows, H, E, I,
+                               _swiglu(*swiglu), dt, _ptr(y_perm), _ptr(ws), ws.numel(),
+                               _stream(stream))
+    check(st, "moe_expert_ffn")
+    return y_perm
+
+
+def combine(y_perm, perm_dst, topk_w, T, k, out=None, stream=None):
+    """out[t] = sum_j topk_w[t, j] * y_perm[perm_dst[t*k + j]] (float32 sum, slot order)."""
+    _need(y_perm, "y_perm")
+    H = y_perm.shape[1]
+    _need(perm_dst, "perm_dst", torch.int32)
+    _need(topk_w, "topk_w", torch.float32)
+    if out is None:
+        out = torch.empty((T, H), dtype=y_perm.dtype, device=y_perm.device)
+    st = _lib().moe_combine(_ptr(y_perm), _ptr(perm_dst), _ptr(topk_w), T, H, k, _dtcode(y_perm),
+                            _ptr(out), _stream(stream))
+    check(st, "moe_combine")
+    return out
+
+
+def convert_chunked_to_interleaved(src, dst=None, stream=None):
+    """[E, 2I, H] gate-rows-then-up-rows -> interleaved (row 2j gate_j, row 2j+1 up_j)."""
+    _need(src, "src")
+    E, two_i, H = src.shape
+    if dst is None:
+        dst = torch.empty_like(src)
+    _need(dst, "dst", src.dtype, src.shape)
+    st = _lib().convert_chunked_to_interleaved(_ptr(src), _ptr(dst), E, two_i // 2, H,
+                                               _dtcode(src), _stream(stream))
+    check(st, "convert_chunked_to_interleaved")
+    return dst
+
+
+def get_error(err_word, stream=None):
+    """(status, bits) of a device error word; synchronises the stream."""
+    bits = ctypes.c_int32(0)
+    st = _lib().moe_get_error(_ptr(err_word), _stream(stream), ctypes.byref(bits))
+    return st, bits.value
+
+
+def set_stage_events(events):
+    """Record 6 cudaEvent handles around the stages of every moe_forward (None: off)."""
+    lib = _lib()
+    if events is None:
+        check(lib.moe_set_stage_events(None, 0), "moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e) for e in events])
+    check(lib.moe_set_stage_events(arr, len(events)), "moe_set_stage_events")

@@ -1,0 +1,100 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/*.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from mixture_experts_ffn_15_b200 import _abi
+from mixture_experts_ffn_15_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    build()
+    return _abi.load()
+
+
+def declared_functions():
+    names = set()
+    for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(path).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        src = re.sub(r"#[^\n]*", " ", src)
+        for stmt in src.split(";"):
+            stmt = " ".join(stmt.split())
+            if not stmt or stmt.startswith("typedef") or "{" in stmt or "}" in stmt:
+                continue
+            m = re.match(r"^[\w\s\*]+?\b(\w+)\s*\(", stmt)
+            if m:
+                names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+              "convert_chunked_to_interleaved", "moe_workspace_size", "moe_get_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib()
+    missing = [n for n in sorted(declared_functions()) if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding declares the same set
+    assert set(_abi.SIGNATURES) == declared_functions()
+
+
+def test_status_strings_and_version():
+    lib = _lib()
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(2) == b"MOE_ERR_UNSUPPORTED"
+    assert lib.moe_version() >= 100
+
+
+def test_workspace_sizes():
+    lib = _lib()
+    assert lib.moe_workspace_size(4, 2816, 128, 8, 704, _abi.MOE_BF16) > 4 * 8 * (2 * 2816 + 704) * 2
+    assert lib.moe_workspace_size(4, 2816, 128, 300, 704, _abi.MOE_BF16) == 0     # k > E
+    assert lib.moe_workspace_size(4, 2816, 300, 8, 704, _abi.MOE_BF16) == 0       # E > 256
+    assert lib.moe_workspace_size(4, 2817, 128, 8, 704, _abi.MOE_BF16) == 0       # H % 8
+    assert lib.moe_workspace_size(4, 2816, 128, 8, 704, 7) == 0                   # dtype
+    a = lib.moe_workspace_size(100, 256, 8, 2, 128, _abi.MOE_BF16)
+    b = lib.moe_workspace_size(200, 256, 8, 2, 128, _abi.MOE_BF16)
+    assert b > a and a % 256 == 0
+    assert lib.moe_permute_workspace_size(1000, 64) >= 2 * 8 * 64 * 4
+
+
+def _fwd(lib, T=4, H=128, E=8, k=2, I=64, act=_abi.STANDARD_SWIGLU, dt=_abi.MOE_BF16, ptr=16):
+    p = ctypes.c_void_p(ptr)
+    return lib.moe_forward(p, p, None, p, p, T, H, E, k, I, 1, act, dt, p, ctypes.c_void_p(256),
+                           1 << 40, None)
+
+
+def test_host_validation_before_any_device_work():
+    lib = _lib()
+    assert _fwd(lib, k=9) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd(lib, T=-1) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd(lib, H=100) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd(lib, act=_abi.MoeSwiglu(1.702, 1.0, 7.0)) == _abi.MOE_ERR_UNSUPPORTED
+    assert _fwd(lib, H=72) == _abi.MOE_ERR_UNSUPPORTED      # bf16 needs H % 64 == 0
+    assert _fwd(lib, T=0) == _abi.MOE_OK                   # empty batch: nothing to do
+    assert _fwd(lib, ptr=18) == _abi.MOE_ERR_INVALID_ARG    # misaligned tensors
+    p = ctypes.c_void_p(4096)
+    assert lib.convert_chunked_to_interleaved(p, ctypes.c_void_p(4096 + 64), 2, 8, 64,
+                                              _abi.MOE_BF16, None) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_error(None, None, None) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_stage_events((ctypes.c_void_p * 2)(), 2) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_stage_events(None, 0) == _abi.MOE_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError, match="build"):
+        _abi.load()

@@ -1,0 +1,288 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Indices, counts and permutations are compared bit-exactly (near ties resolved
+through oracle-generated alternatives, see parity_util); values within the stated
+tolerances: bf16 |d| <= 1e-2 + 2e-2 |ref|, float32 |d| <= 1e-6 + 1e-4 |ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_15_b200 as moe
+from oracle import moe_oracle as O
+from parity_util import (W_ATOL, assert_close, device_inputs, from_dev, match_routing,
+                         sample_tokens, to_dev, tol)
+from synth import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def W(name, **kw):
+    base = dict(T=64, H=128, E=8, k=2, I=64, dtype="bf16", seed=1)
+    base.update(kw)
+    return Workload(name, **base)
+
+
+# Small cases: several tiles in every dimension with ragged tails, both orientations
+# of the tensor-core GEMM, every column-tile width, the float32 path and edge cases.
+CASES = [
+    W("f32_tiles", T=300, H=256, E=16, k=4, I=192, dtype="f32"),
+    W("f32_T1", T=1, H=64, E=4, k=2, I=32, dtype="f32"),
+    W("f32_normalize_off", T=70, H=64, E=6, k=3, I=32, dtype="f32", normalize=0),
+    W("bf16_tokenM_bn192", T=300, H=256, E=16, k=4, I=192),
+    W("bf16_tokenM_bn176", T=300, H=128, E=8, k=2, I=704),
+    W("bf16_tokenM_bias", T=520, H=192, E=8, k=2, I=64, router_bias_std=1.0),
+    W("bf16_weightM", T=40, H=256, E=16, k=4, I=192),
+    W("bf16_weightM_skew", T=100, H=256, E=8, k=2, I=128, router_bias_std=1.0),
+    W("bf16_router_tc", T=600, H=256, E=64, k=4, I=128),
+    W("bf16_k1", T=130, H=128, E=8, k=1, I=64),
+    W("bf16_k_eq_E", T=20, H=128, E=4, k=4, I=64),
+    W("bf16_T1", T=1, H=128, E=8, k=2, I=64),
+    W("bf16_normalize_off", T=90, H=128, E=8, k=3, I=64, normalize=0),
+]
+IDS = [c.name for c in CASES]
+
+
+def oracle_forward(inp, idx, tokens=None):
+    wl = inp.wl
+    layout = wl.fc1_layout
+    return O.moe_forward(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                         lambda e: inp.expert_values("fc1", e),
+                         lambda e: inp.expert_values("fc2", e), wl.k, wl.normalize, layout,
+                         idx=idx, tokens=tokens)
+
+
+def run_route(dev, wl):
+    return moe.route(dev["hidden"], dev["router_w"], wl.k, normalize=bool(wl.normalize),
+                     router_bias=dev["router_bias"])
+
+
+def check_routing(inp, r):
+    """GPU routing vs the oracle; returns (logits64, matched idx)."""
+    wl = inp.wl
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), inp["router_bias"])
+    gidx = from_dev(r["idx"]).astype(np.int64)
+    idx, _ = match_routing(L, gidx, wl.k)
+    np.testing.assert_array_equal(gidx, idx)
+    w_ref = O.routing_weights(L, idx, wl.normalize)
+    assert_close(from_dev(r["w"]), w_ref, W_ATOL, 0.0, "routing weights")
+    # the logits themselves: rigorous float32 summation bound, gamma_H * sum |x w|
+    H = wl.H
+    xw = np.abs(inp.values("hidden")).astype(np.float64) @ np.abs(inp.values("router_w")).astype(np.float64).T
+    u = 2.0 ** -24
+    bound = (H * u / (1 - H * u)) * xw + 1e-7
+    got = from_dev(r["logits"])
+    assert np.all(np.abs(got - L) <= bound), "router logits beyond the float32 summation bound"
+    return L, idx
+
+
+@pytest.mark.parametrize("wl", CASES, ids=IDS)
+def test_route(wl):
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    check_routing(inp, run_route(dev, wl))
+
+
+@pytest.mark.parametrize("wl", CASES, ids=IDS)
+def test_permute(wl):
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), inp["router_bias"])
+    idx = O.select_topk(L, wl.k)
+    p = moe.permute(torch.from_numpy(idx).cuda(), wl.E, hidden=dev["hidden"])
+    counts, offsets, src, dst = O.stable_permutation(idx, wl.E)
+    np.testing.assert_array_equal(from_dev(p["counts"]), counts)
+    np.testing.assert_array_equal(from_dev(p["offsets"]), offsets)
+    np.testing.assert_array_equal(from_dev(p["perm_src"]), src)
+    np.testing.assert_array_equal(from_dev(p["perm_dst"]), dst)
+    x_ref = O.gather_rows(inp["hidden"], src)
+    got = p["x_perm"].detach().cpu()
+    got = got.view(torch.int16).numpy().view(np.uint16) if got.dtype == torch.bfloat16 else got.numpy()
+    np.testing.assert_array_equal(got, x_ref)
+    st, bits = moe.get_error(p["err_word"])
+    assert st == 0 and bits == 0
+
+
+@pytest.mark.parametrize("wl", CASES, ids=IDS)
+def test_expert_ffn(wl):
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"), inp["router_bias"])
+    idx = O.select_topk(L, wl.k)
+    counts, offsets, src, dst = O.stable_permutation(idx, wl.E)
+    x_perm = O.gather_rows(inp["hidden"], src)
+    y = moe.expert_ffn(to_dev(x_perm, wl.dtype), torch.from_numpy(offsets).cuda(), dev["fc1"], dev["fc2"])
+    torch.cuda.synchronize()
+    xv = O.gather_rows(inp.values("hidden"), src)
+    y_ref = np.zeros((x_perm.shape[0], wl.H))
+    for e in range(wl.E):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            y_ref[a:b] = O.expert_ffn(xv[a:b], inp.expert_values("fc1", e), inp.expert_values("fc2", e))
+    atol, rtol = tol(wl.dtype, y_ref)
+    assert_close(from_dev(y), y_ref, atol, rtol, "y_perm")
+
+
+@pytest.mark.parametrize("wl", CASES, ids=IDS)
+def test_forward(wl):
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    out = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], wl.k,
+                      normalize=bool(wl.normalize), router_bias=dev["router_bias"])
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    ref = oracle_forward(inp, idx)["out"]
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} output")
+
+
+def test_combine_matches_oracle():
+    wl = W("comb", T=77, H=136, E=6, k=3, dtype="f32")
+    inp = make_inputs(wl)
+    L = O.router_logits(inp.values("hidden"), inp.values("router_w"))
+    idx = O.select_topk(L, 3)
+    w = O.routing_weights(L, idx, 1)
+    _, _, _, dst = O.stable_permutation(idx, 6)
+    y = np.random.default_rng(5).standard_normal((77 * 3, 136)).astype(np.float32)
+    got = moe.combine(torch.from_numpy(y).cuda(), torch.from_numpy(dst).cuda(),
+                      torch.from_numpy(w.astype(np.float32)).cuda(), 77, 3)
+    ref = O.combine(y, dst, w.astype(np.float32), 77, 3)
+    assert_close(from_dev(got), ref, 1e-6, 1e-5, "combine")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_convert_chunked_to_interleaved_bitexact(dtype):
+    wl = W("conv", E=5, I=96, H=64, dtype=dtype)
+    inp = make_inputs(wl)
+    src = inp["fc1"]
+    got = moe.convert_chunked_to_interleaved(to_dev(src, dtype)).cpu()
+    got = got.view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else got.numpy()
+    np.testing.assert_array_equal(got, O.chunked_to_interleaved(src))
+
+
+def test_forward_with_device_converted_weights_is_bitwise_equal():
+    wl = W("conv_fwd", T=200, H=128, E=8, k=2, I=128, fc1_layout="chunked")
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    fc1_dev = moe.convert_chunked_to_interleaved(dev["fc1"])
+    fc1_host = to_dev(O.chunked_to_interleaved(inp["fc1"]), "bf16")
+    a = moe.forward(dev["hidden"], dev["router_w"], fc1_dev, dev["fc2"], 2)
+    b = moe.forward(dev["hidden"], dev["router_w"], fc1_host, dev["fc2"], 2)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    # and the layer on chunked weights equals the oracle's chunked reading
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    ref = oracle_forward(inp, idx)["out"]
+    assert_close(from_dev(a), ref, 1e-2, 2e-2, "converted forward")
+
+
+def test_forward_is_deterministic():
+    wl = W("det", T=300, H=256, E=16, k=4, I=192)
+    dev = device_inputs(make_inputs(wl))
+    a = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], 4)
+    b = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], 4)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_exact_tie_goes_to_lower_index():
+    wl = W("tie", T=50, H=128, E=8, k=2)
+    inp = make_inputs(wl)
+    rw = inp["router_w"].copy()
+    rw[6] = rw[1]                       # experts 1 and 6 tie exactly for every token
+    r = moe.route(to_dev(inp["hidden"], "bf16"), to_dev(rw, "bf16"), 2)
+    idx = from_dev(r["idx"])
+    near = from_dev(r["near_tie"])
+    for t in range(50):
+        row = list(idx[t])
+        if 6 in row:
+            assert 1 in row and row.index(1) < row.index(6)
+            assert near[t] & 2            # the two tied experts are adjacent chosen slots
+        elif 1 in row:
+            assert near[t] & 1            # expert 6 ties the k-th choice at the boundary
+
+
+def test_zero_tokens_is_a_noop():
+    wl = W("empty", T=0)
+    H, E, I = 128, 8, 64
+    hidden = torch.empty((0, H), dtype=torch.bfloat16, device="cuda")
+    rw = torch.zeros((E, H), dtype=torch.bfloat16, device="cuda")
+    fc1 = torch.zeros((E, 2 * I, H), dtype=torch.bfloat16, device="cuda")
+    fc2 = torch.zeros((E, H, I), dtype=torch.bfloat16, device="cuda")
+    out = moe.forward(hidden, rw, fc1, fc2, 2)
+    assert out.shape == (0, H)
+    del wl
+
+
+def test_invalid_arguments_are_rejected():
+    H, E, I = 128, 8, 64
+    hidden = torch.zeros((4, H), dtype=torch.bfloat16, device="cuda")
+    rw = torch.zeros((E, H), dtype=torch.bfloat16, device="cuda")
+    fc1 = torch.zeros((E, 2 * I, H), dtype=torch.bfloat16, device="cuda")
+    fc2 = torch.zeros((E, H, I), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError, match="INVALID_ARG"):
+        moe.forward(hidden, rw, fc1, fc2, 9)                       # k > E
+    with pytest.raises(moe.MoEError, match="UNSUPPORTED"):
+        moe.forward(hidden, rw, fc1, fc2, 2, swiglu=(1.702, 1.0, 7.0))
+    bad = torch.zeros((4 * H + 8,), dtype=torch.bfloat16, device="cuda")[1:1 + 4 * H].view(4, H)
+    with pytest.raises(moe.MoEError, match="INVALID_ARG"):
+        moe.forward(bad, rw, fc1, fc2, 2)                          # misaligned hidden
+    # bf16 sizes without a tensor-core tiling are refused, not computed elsewhere
+    h2 = torch.zeros((4, 72), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError, match="UNSUPPORTED"):
+        moe.forward(h2, torch.zeros((E, 72), dtype=torch.bfloat16, device="cuda"),
+                    torch.zeros((E, 2 * I, 72), dtype=torch.bfloat16, device="cuda"),
+                    torch.zeros((E, 72, I), dtype=torch.bfloat16, device="cuda"), 2)
+
+
+def test_bad_expert_ids_are_reported_and_skipped():
+    E, T, k = 8, 40, 2
+    idx = np.stack([np.arange(T) % E, (np.arange(T) + 3) % E], axis=1).astype(np.int32)
+    idx[5, 1] = E          # out of range
+    idx[9, 0] = -2         # out of range
+    p = moe.permute(torch.from_numpy(idx).cuda(), E)
+    st, bits = moe.get_error(p["err_word"])
+    assert st == moe._abi.MOE_ERR_DEVICE and bits & moe._abi.MOE_DEVERR_BAD_EXPERT
+    good = idx.copy()
+    mask = (good < 0) | (good >= E)
+    counts = np.bincount(good[~mask], minlength=E)
+    np.testing.assert_array_equal(from_dev(p["counts"]), counts)
+    dst = from_dev(p["perm_dst"]).reshape(T, k)
+    assert dst[5, 1] == -1 and dst[9, 0] == -1
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+FULL = ["tiny_fp32", "decode_bf16", "batched_decode_bf16", "prefill_bf16", "long_prefill_bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload(name):
+    from synth import WORKLOADS, outlier_rows
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    fc1 = dev["fc1"]
+    if wl.fc1_layout == "chunked":
+        fc1 = moe.convert_chunked_to_interleaved(fc1)
+    out = moe.forward(dev["hidden"], dev["router_w"], fc1, dev["fc2"], wl.k,
+                      normalize=bool(wl.normalize), router_bias=dev["router_bias"])
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    # counts and permutation over all tokens, bit-exact
+    p = moe.permute(r["idx"], wl.E)
+    counts, offsets, src, dst = O.stable_permutation(idx, wl.E)
+    np.testing.assert_array_equal(from_dev(p["offsets"]), offsets)
+    np.testing.assert_array_equal(from_dev(p["perm_src"]), src)
+    np.testing.assert_array_equal(from_dev(p["perm_dst"]), dst)
+    # values: every token when the oracle is quick, else a seeded sample that holds
+    # the outlier rows and tokens of the least and most loaded experts
+    tokens = None
+    if wl.T > 256:
+        tokens = sample_tokens(wl.T, idx, wl.E, n=192, must=outlier_rows(wl, wl.seed)[:64])
+    ref = oracle_forward(inp, idx, tokens=tokens)["out"]
+    got = from_dev(out) if tokens is None else from_dev(out[torch.from_numpy(tokens).cuda()])
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(got, ref, atol, rtol, f"{name} output")
