@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the whole layer (route -> permute -> fc1 + SwiGLU -> fc2 ->
+combine) on one batch of synthetic tokens with the inputs resident in HBM.  The
+default workload is decode_bf16 (T=4, H=2816, E=128, k=8, I=704), the configuration
+the layer's headline metric is quoted on; --workload picks another row of
+synth.WORKLOADS.  Steps are replayed from CUDA graphs of S steps each; between
+reuses of a weight set, `--sets` - 1 other copies of the weights are streamed, so
+the touched weights never sit in L2 when a step starts.
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun, one rank per GPU) runs
+independent replicas: the layer has no exchange step on one GPU's batch, so there
+is no data-path collective; the barrier and the max-over-ranks timing are the only
+communication.  `--impl reference` times the CPU oracle (the reference arm of this
+build) on the host cores instead.
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s + TFLOP/s or HBM GB/s as fraction of roofline, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_STEPS = {"tiny_fp32": 2000, "decode_bf16": 6000, "batched_decode_bf16": 2000,
+                 "prefill_bf16": 400, "long_prefill_bf16": 100}
+GRAPH_STEPS = {"tiny_fp32": 20, "decode_bf16": 20, "batched_decode_bf16": 20,
+               "prefill_bf16": 4, "long_prefill_bf16": 2}
+HBM_BOUND = {"decode_bf16", "batched_decode_bf16", "tiny_fp32"}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_bf16")
+    ap.add_argument("--sets", type=int, default=None, help="rotating weight copies (L2)")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(1.0)
+
+    def mark(self, begin):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        # the rows of the timed region: the busiest (highest power) contiguous half
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return float("nan")
+        power = [num(r[3]) for r in rows]
+        thr = sorted(power)[len(power) // 2] if len(power) > 2 else -1
+        load = [r for r, p in zip(rows, power) if p >= thr] or rows
+        sm = sorted(num(r[1]) for r in load)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": num(load[0][2]), "reasons": reasons,
+                "samples": len(load), "power_w_max": max(num(r[3]) for r in load)}
+
+
+def algorithmic(wl, counts):
+    """Algorithmic bytes and FLOPs of one step (only the routed work, used experts once)."""
+    T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
+    es = 2 if wl.dtype == "bf16" else 4
+    rows = T * k
+    used = int(sum(1 for c in counts if c > 0))
+    fc1 = {"bytes": used * 2 * I * H * es + rows * H * es + rows * I * es,
+           "flops": 2.0 * rows * H * 2 * I}
+    fc2 = {"bytes": used * H * I * es + rows * I * es + rows * H * es,
+           "flops": 2.0 * rows * I * H}
+    layer = {"bytes": used * 3 * H * I * es + E * H * es + 2 * T * H * es
+             + 2 * rows * H * es + 2 * rows * I * es + 2 * rows * H * es,
+             "flops": float(T) * (6.0 * k * H * I + 2.0 * H * E)}
+    return used, fc1, fc2, layer
+
+
+def kernel_traffic(workload):
+    """DRAM bytes per fc1 launch from a committed ncu summary, if it matches the kernel."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    src = os.path.join(ROOT, "mixture_experts_ffn_15_b200", "csrc", "gemm_tc.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    e = table.get(workload)
+    if not e or e.get("source_sha") != sha:
+        return None
+    return e.get("bytes_per_launch")
+
+
+def device_tensor(a, dev):
+    """numpy storage array (uint16 bf16 bits or float32) -> torch tensor on `dev`."""
+    import numpy as np
+    import torch
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_cost(wl, inp, seconds):
+    """The CPU oracle, as it stands, on whole tokens of `wl` for about `seconds`.
+
+    Returns (tokens/s, threads, description of the sample)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import moe_oracle as O
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    x = inp.values("hidden")
+    rw = inp.values("router_w")
+    bias = inp["router_bias"]
+    fc1 = lambda e: inp.expert_values("fc1", e)
+    fc2 = lambda e: inp.expert_values("fc2", e)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        t = n % wl.T
+        r = O.moe_forward(x[t:t + 1], rw, bias, fc1, fc2, wl.k, wl.normalize, wl.fc1_layout)
+        assert np.isfinite(r["out"]).all()
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    return n / el, cores, (f"{n} whole tokens of the workload, one at a time (router logits, "
+                           f"top-k, {wl.k} expert FFNs, combine in float64), {el:.1f} s")
+
+
+def oracle_pair_step(wl, inp, state):
+    """One bounded reference step: routing of one token and one of its expert FFNs."""
+    import numpy as np
+
+    from oracle import moe_oracle as O
+    t = state["t"]
+    L = O.router_logits(inp.values("hidden")[t:t + 1], inp.values("router_w"), inp["router_bias"])
+    idx = O.select_topk(L, wl.k)
+    w = O.routing_weights(L, idx, wl.normalize)
+    j = state["j"]
+    e = int(idx[0, j])
+    y = O.expert_ffn(inp.values("hidden")[t:t + 1], inp.expert_values("fc1", e),
+                     inp.expert_values("fc2", e), wl.fc1_layout)
+    assert np.isfinite(w[0, j] * y).all()
+    state["j"] += 1
+    if state["j"] == wl.k:
+        state["j"] = 0
+        state["t"] = (t + 1) % wl.T
+
+
+def run_reference(args):
+    from synth import WORKLOADS, make_inputs
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(wl.name, 100)
+    from threadpoolctl import threadpool_info
+    cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    inp = make_inputs(wl)
+    state = {"t": 0, "j": 0}
+    for _ in range(args.warmup):
+        oracle_pair_step(wl, inp, state)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_pair_step(wl, inp, state)
+    el = time.perf_counter() - t0
+    value = (steps / wl.k) / el
+    sample = (f"each step: router logits + top-k of one token and one of its {wl.k} expert "
+              f"FFNs (1/{wl.k} token); {steps} steps in {el:.1f} s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, sets=1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, sets):
+    cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+           "normalize": wl.normalize, "seed": wl.seed, "fc1_layout_given": wl.fc1_layout}
+    if wl.router_bias_std is not None:
+        cfg["router_bias_std"] = wl.router_bias_std
+    if wl.outlier_frac:
+        cfg["outliers"] = f"{wl.outlier_frac:g} of rows x{wl.outlier_scale:g}"
+    cfg["l2"] = (f"{sets} rotating weight copies: {sets - 1} other copies stream between "
+                 "reuses of one (inputs larger than L2)" if sets > 1 else
+                 "per-step traffic larger than L2")
+    return cfg
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import mixture_experts_ffn_15_b200 as moe
+    from synth import WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    wl = WORKLOADS[args.workload]
+    S = GRAPH_STEPS.get(wl.name, 4)
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(wl.name, 100)
+    reps = max(1, math.ceil(steps / S))
+    steps = reps * S
+    warm_reps = max(1, math.ceil(args.warmup / S))
+    sets = args.sets if args.sets is not None else (4 if wl.name in HBM_BOUND else 1)
+
+    inp = make_inputs(wl)
+    hidden = device_tensor(inp["hidden"], dev)
+    router_w = device_tensor(inp["router_w"], dev)
+    bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).to(dev)
+    fc1 = device_tensor(inp["fc1"], dev)
+    if wl.fc1_layout == "chunked":
+        fc1 = moe.convert_chunked_to_interleaved(fc1)      # setup, as at session load
+    fc2 = device_tensor(inp["fc2"], dev)
+    fc1s = [fc1] + [fc1.clone() for _ in range(sets - 1)]
+    fc2s = [fc2] + [fc2.clone() for _ in range(sets - 1)]
+    out = torch.empty_like(hidden)
+    ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
+
+    # routing outside the timed region, for the byte accounting only
+    r = moe.route(hidden, router_w, wl.k, normalize=bool(wl.normalize), router_bias=bias)
+    p = moe.permute(r["idx"], wl.E)
+    counts = p["counts"].cpu().numpy()
+    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts)
+
+    stream = torch.cuda.Stream(device=dev)
+    call = lambda i: moe.forward(hidden, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+                                 normalize=bool(wl.normalize), router_bias=bias, out=out,
+                                 workspace=ws)
+    with torch.cuda.stream(stream):
+        for i in range(sets):
+            call(i)
+    torch.cuda.synchronize(dev)
+
+    # one graph of S steps; every step records its 6 stage events
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(S)]
+    for row in events:
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize(dev)
+    lib = moe.load_library()
+    n0 = lib.moe_kernel_launches()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(S):
+            moe.set_stage_events([ev.cuda_event for ev in events[i]])
+            call(i)
+        moe.set_stage_events(None)
+    launches_per_step = (lib.moe_kernel_launches() - n0) / S
+
+    with torch.cuda.stream(stream):
+        for _ in range(warm_reps):
+            graph.replay()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks.mark(True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark(False)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_step = ms_total / steps
+
+    # stage durations of the last replay (inside the timed region)
+    stage_names = ["route", "permute", "fc1_swiglu", "fc2", "combine"]
+    st = {n: 0.0 for n in stage_names}
+    for i in range(S):
+        for a, n in enumerate(stage_names):
+            st[n] += events[i][a].elapsed_time(events[i][a + 1]) / S
+    fc1_ms = max_over_ranks(st["fc1_swiglu"], world, dev)
+
+    peaks, peak_kind = load_peaks()
+    hbm = wl.name in HBM_BOUND
+    if hbm:
+        achieved = fc1_work["bytes"] / (fc1_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = fc1_work["flops"] / (fc1_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = "tc_gemm_kernel fc1+SwiGLU (" + ("weight rows on M" if wl.T * wl.k <= 64 * wl.E else "token rows on M") + ")"
+    roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if hbm else 'bf16_tflops, burst'})"
+    roof["algorithmic_per_launch"] = fc1_work["bytes"] if hbm else fc1_work["flops"]
+    roof["traffic"] = kernel_traffic(wl.name)
+
+    layer_s = ms_step * 1e-3
+    layer = {"GB/s": layer_work["bytes"] / layer_s / 1e9, "TFLOP/s": layer_work["flops"] / layer_s / 1e12,
+             "hbm_frac": layer_work["bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
+             "tensor_frac": layer_work["flops"] / layer_s / 1e12 / peaks["bf16_tflops"],
+             "experts_used": used, "algorithmic_bytes": layer_work["bytes"],
+             "algorithmic_flops": layer_work["flops"]}
+
+    # end to end through the public API: pinned host input -> device -> layer -> host
+    h_host = torch.empty(hidden.shape, dtype=hidden.dtype, pin_memory=True)
+    h_host.copy_(hidden)
+    o_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    d_in = torch.empty_like(hidden)
+    n_e2e = args.e2e_steps
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            d_in.copy_(h_host, non_blocking=True)
+            moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws)
+            o_host.copy_(out, non_blocking=True)
+            stream.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        t0 = time.perf_counter()
+        for i in range(n_e2e):
+            d_in.copy_(h_host, non_blocking=True)
+            moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws)
+            o_host.copy_(out, non_blocking=True)
+            stream.synchronize()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
+    e2e = {"value": wl.T * world * n_e2e / e2e_s, "unit": "tokens/s",
+           "h2d_bytes_per_step": h_host.numel() * h_host.element_size(),
+           "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "steps": n_e2e}
+
+    st_err, bits = moe.get_error(moe.workspace_error_word(ws), stream)
+    if st_err != 0:
+        raise SystemExit(f"device error word {bits} after the bench")
+
+    line = {
+        "metric": METRIC, "value": wl.T * world / ms_step * 1e3, "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": warm_reps * S, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
+                       graph_steps=S),
+        "roofline": roof, "layer": layer,
+        "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
+        "e2e": e2e, "clocks": clk,
+        "gpu_launches": int(round(launches_per_step * steps)),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

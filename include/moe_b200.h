@@ -185,6 +185,10 @@ const char* moe_status_string(moe_status s);
  * recording off.  The handles stay owned by the caller.  Process-wide setting. */
 moe_status moe_set_stage_events(void* const* events, int n_events);
 
+/* Number of kernel launches the library has issued in this process (host-side count,
+ * all devices).  A launch captured into a CUDA graph counts once, at capture. */
+unsigned long long moe_kernel_launches(void);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int moe_version(void);
 

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "moe_b200.h"
@@ -20,6 +22,20 @@ int device_sm_count() {
         cache[dev] = n;
     }
     return cache[dev];
+}
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n)); }
+
+void record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, s);
 }
 
 namespace {
@@ -104,7 +120,7 @@ bool standard_swiglu(const moe_swiglu& a) {
 }
 
 void record(int i, cudaStream_t s) {
-    if (g_events_on) cudaEventRecord(g_events[i], s);
+    if (g_events_on) record_event(g_events[i], s);
 }
 
 #define MOE_CUDA(call)                                  \
@@ -120,6 +136,8 @@ using namespace moe;
 extern "C" {
 
 int moe_version(void) { return 100; }
+
+unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 
 const char* moe_status_string(moe_status s) {
     switch (s) {

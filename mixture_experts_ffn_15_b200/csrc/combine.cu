@@ -99,6 +99,7 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
     else
         combine_kernel<false><<<blocks, threads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
                                                          rows_max, out);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -112,6 +113,7 @@ cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int 
     if (blocks > cap) blocks = cap;
     convert_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const uint4*>(src),
                                                              static_cast<uint4*>(dst), E, I, vec);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -109,11 +109,13 @@ cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, con
     if (rows <= 0) return cudaSuccess;
     simt_grouped_gemm_kernel<true><<<simt_grid(rows, E, 2 * I), 256, 0, s>>>(
         x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I);
+    count_launch();
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    if (mid) cudaEventRecord(mid, s);
+    if (mid) record_event(mid, s);
     simt_grouped_gemm_kernel<false><<<simt_grid(rows, E, H), 256, 0, s>>>(act, I, fc2, H, I,
                                                                            offsets, E, rows, y, H);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -438,13 +438,22 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParam
                        cudaStream_t s) {
     using C = Tr<MODE, BN>;
     auto kern = tc_gemm_kernel<MODE, BN>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
+    // once per device (outside any stream capture: the first call of every path
+    // runs eagerly before a graph is captured)
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     int grid = device_sm_count();
     if (bound < grid) grid = bound;
     if (grid <= 0) return cudaSuccess;
     kern<<<grid, kThreads, C::kSmemBytes, s>>>(a, b, p);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -505,7 +514,7 @@ cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void
     if (rows <= 0) return cudaSuccess;
     cudaError_t e = grouped_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s);
     if (e != cudaSuccess) return e;
-    if (mid) cudaEventRecord(mid, s);
+    if (mid) record_event(mid, s);
     return grouped_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
 }
 

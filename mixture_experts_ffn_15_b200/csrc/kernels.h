@@ -8,6 +8,13 @@ namespace moe {
 
 int device_sm_count();
 
+// Records `ev` on `s`; inside a stream capture the record becomes an external
+// event node, so that the event still times the replayed graph.
+void record_event(cudaEvent_t ev, cudaStream_t s);
+
+// Process-wide count of kernel launches issued by the library (host side).
+void count_launch(int n = 1);
+
 // ---------------------------------------------------------------- route.cu
 cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, int T, int H,
                                       int E, bool bf16, float* logits, cudaStream_t s);

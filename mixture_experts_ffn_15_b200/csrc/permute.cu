@@ -84,6 +84,7 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, in
     if (T <= 0) return cudaSuccess;
     scatter_kernel<<<num_token_tiles(T), kScatterThreads, 0, s>>>(topk_idx, tile_base, T, E, k,
                                                                   perm_src, perm_dst, err);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -97,6 +98,7 @@ cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int
     if (blocks > cap) blocks = cap;
     gather_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(hidden), perm_src, offsets, E,
                                          T, rows_max, vec, static_cast<uint4*>(x_perm));
+    count_launch();
     return cudaGetLastError();
 }
 

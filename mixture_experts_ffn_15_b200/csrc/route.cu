@@ -268,12 +268,14 @@ cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, 
     else
         router_logits_simt_kernel<false><<<grid, kLogitWarps * 32, 0, s>>>(hidden, router_w, T, H,
                                                                            E, logits);
+    count_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_topk_hist(const TopkHistArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
     topk_hist_kernel<<<num_token_tiles(a.T), kHistThreads, 0, s>>>(a);
+    count_launch();
     return cudaGetLastError();
 }
 
