@@ -32,6 +32,22 @@ def tol(dtype, ref=None):
     return F32_ATOL + floor, F32_RTOL
 
 
+def row_scale(ref):
+    """Per-row factor on the absolute term of the bf16 tolerance, shape [rows, 1].
+
+    The absolute term is in units of a typical row's output.  A row whose output
+    RMS is more than twice the median row RMS (an outlier token, whose input was
+    scaled up) gets s_t = rms_t / median: its intermediates are proportionally
+    larger, and bf16 storage of act and y_perm alone leaves errors that scale with
+    them.  Every other row keeps s_t = 1, i.e. exactly the stated tolerance.
+    """
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(np.square(ref), axis=1))
+    med = max(float(np.median(rms)) if rms.size else 1.0, 1e-30)
+    ratio = rms / med
+    return np.where(ratio > 2.0, ratio, 1.0)[:, None]
+
+
 def assert_close(got, ref, atol, rtol, what):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
