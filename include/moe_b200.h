@@ -159,6 +159,27 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
                        int normalize, moe_swiglu act, moe_dtype dt, void* out,
                        void* workspace, size_t ws_bytes, void* stream);
 
+/* The whole layer without a workspace argument, for callers that cannot allocate
+ * device memory while they run it (an engine plugin or a serving loop that forbids
+ * allocation after start-up, a plain C host with no allocator of its own).  The
+ * pages have no counterpart for this entry point.
+ *   Arguments as moe_forward, minus workspace and ws_bytes.  The scratch is a fixed
+ *   device array of MOE_STATIC_SCRATCH_BYTES inside the library, which every GPU
+ *   that loads the library holds until the process exits.  Sizes whose
+ *   moe_workspace_size(T, H, E, k, I, dt) exceeds MOE_STATIC_SCRATCH_BYTES (with
+ *   E = 128, k = 8, H = 2816, I = 704 in bf16: up to 82 tokens) are rejected with
+ *   MOE_ERR_INVALID_ARG before anything is enqueued; nothing is allocated, ever.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents (the parts
+ *   that must start at zero are cleared by every call): calls whose work can
+ *   overlap on the GPU, from two streams or two host threads, race on it. */
+#define MOE_STATIC_SCRATCH_BYTES (8u << 20)
+moe_status moe_forward_static(const void* hidden, const void* router_w, const float* router_bias,
+                              const void* fc1, const void* fc2, int T, int H, int E, int k, int I,
+                              int normalize, moe_swiglu act, moe_dtype dt, void* out,
+                              void* stream);
+
 /* Layout conversion of fc1 from the Hugging Face chunked layout ("Weight layout":
  * [E, 2*inter, H], the first inter rows gate, the next inter rows up) to the
  * interleaved layout of swiglu_fusion = 1:  dst[e, 2j+s, :] = src[e, s*I + j, :].
