@@ -206,6 +206,12 @@ const char* moe_status_string(moe_status s);
  * recording off.  The handles stay owned by the caller.  Process-wide setting. */
 moe_status moe_set_stage_events(void* const* events, int n_events);
 
+/* Which kernels moe_forward runs for these sizes, as bits: 1 single-CTA routing
+ * (T <= 512 and k <= 32), 2 fused decode FFN (fc1 + SwiGLU and fc2 in one launch,
+ * weight rows on the MMA's M side), 4 tensor-core router, 8 token-row grouped GEMMs,
+ * 16 float32 FMA FFN.  0 for invalid sizes.  Pure host arithmetic. */
+int moe_forward_path(int T, int H, int E, int k, int I, moe_dtype dt);
+
 /* Number of kernel launches the library has issued in this process (host-side count,
  * all devices).  A launch captured into a CUDA graph counts once, at capture. */
 unsigned long long moe_kernel_launches(void);

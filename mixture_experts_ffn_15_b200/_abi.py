@@ -35,6 +35,7 @@ SIGNATURES = {
     "moe_get_error": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_set_stage_events": (_i, [ctypes.POINTER(_vp), _i]),
+    "moe_forward_path": (_i, [_i, _i, _i, _i, _i, _i]),
     "moe_kernel_launches": (ctypes.c_ulonglong, []),
     "moe_version": (_i, []),
 }

@@ -20,8 +20,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["api.cu", "route.cu", "permute.cu", "combine.cu", "ffn_simt.cu", "gemm_tc.cu",
-           "static_scratch.cu"]
+SOURCES = ["api.cu", "route.cu", "route_small.cu", "permute.cu", "combine.cu", "ffn_simt.cu",
+           "gemm_tc.cu", "static_scratch.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -59,7 +59,7 @@ struct Carver {
 
 struct FwdLayout {
     size_t hdr, logits, idx, w, near, tile_counts, tile_base, counts, offsets, perm_src, perm_dst,
-        x_perm, act, y, total;
+        ctr, x_perm, act, y, total;
 };
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
@@ -81,6 +81,7 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     L.offsets = c.take(static_cast<size_t>(E + 1) * 4);
     L.perm_src = c.take(rows * 4);
     L.perm_dst = c.take(rows * 4);
+    L.ctr = c.take(static_cast<size_t>(decode_ffn_counters(static_cast<int>(rows), E)) * 4);
     L.x_perm = c.take(rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
@@ -117,6 +118,22 @@ bool valid_sizes(int T, int H, int E, int k) {
 
 bool standard_swiglu(const moe_swiglu& a) {
     return a.alpha == 1.0f && a.beta == 0.0f && isinf(a.limit) && a.limit > 0;
+}
+
+// Which kernels moe_forward runs for these sizes (bits of moe_forward_path).
+constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
+              kPathF32Ffn = 16;
+
+int forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
+    const bool bf16 = dt == MOE_BF16;
+    const int rows = T * k;
+    int path = 0;
+    if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) path |= kPathSmallRoute;
+    else if (bf16 && tc_router_supported(T, H, E)) path |= kPathTcRouter;
+    if (!bf16) path |= kPathF32Ffn;
+    else if ((path & kPathSmallRoute) && decode_ffn_supported(rows, E, H, I)) path |= kPathDecodeFfn;
+    else path |= kPathTokenGemm;
+    return path;
 }
 
 void record(int i, cudaStream_t s) {
@@ -163,7 +180,14 @@ size_t moe_permute_workspace_size(int T, int E) {
 
 size_t moe_expert_ffn_workspace_size(int rows, int I, moe_dtype dt) {
     if (rows < 0 || I <= 0 || !valid_dtype(dt)) return 0;
-    return align_up(static_cast<size_t>(rows) * I * elem_size(dt)) + kAlign;
+    // error word | activations [rows, I] | counters of the decode FFN (E <= 256)
+    return kAlign + align_up(static_cast<size_t>(rows) * I * elem_size(dt)) +
+           align_up(static_cast<size_t>(decode_ffn_counters(rows, kMaxExperts)) * 4);
+}
+
+int moe_forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
+    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt)) return 0;
+    return forward_path(T, H, E, k, I, dt);
 }
 
 int32_t* moe_workspace_error_word(void* workspace) { return static_cast<int32_t*>(workspace); }
@@ -274,15 +298,22 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     char* ws = static_cast<char*>(workspace);
     int32_t* err = reinterpret_cast<int32_t*>(ws);   // scratch error word of this call
     void* act_buf = ws + kAlign;
+    int32_t* ctr = reinterpret_cast<int32_t*>(ws + kAlign +
+                                              align_up(static_cast<size_t>(rows) * I * elem_size(dt)));
     MOE_CUDA(cudaMemsetAsync(err, 0, 4, s));
-    if (dt == MOE_BF16)
+    if (dt == MOE_BF16 && decode_ffn_supported(rows, E, H, I)) {
+        MOE_CUDA(cudaMemsetAsync(ctr, 0, static_cast<size_t>(decode_ffn_counters(rows, E)) * 4, s));
+        MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1, fc2, rows, H, E, I,
+                                   act_buf, y_perm, ctr, err, s));
+    } else if (dt == MOE_BF16) {
         MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
                                nullptr));
-    else
+    } else {
         MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                      static_cast<const float*>(fc1), static_cast<const float*>(fc2),
                                      rows, H, E, I, static_cast<float*>(act_buf),
                                      static_cast<float*>(y_perm), s, nullptr));
+    }
     return MOE_OK;
 }
 
@@ -331,46 +362,90 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     const bool bf16 = dt == MOE_BF16;
     const int rows = T * k;
 
-    MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, kAlign, s));
+    const int path = forward_path(T, H, E, k, I, dt);
+    int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
     record(0, s);
-    // route: logits, then top-k + softmax + bincount + scan in one kernel
-    if (bf16 && tc_router_supported(T, H, E))
-        MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, err, s));
-    else
-        MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, bf16, logits, s));
-    TopkHistArgs a;
-    a.logits = logits;
-    a.bias = router_bias;
-    a.T = T;
-    a.E = E;
-    a.k = k;
-    a.normalize = normalize ? 1 : 0;
-    a.topk_idx = idx;
-    a.topk_w = w;
-    a.near_tie = reinterpret_cast<int32_t*>(ws + L.near);
-    a.do_hist = true;
-    a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
-    a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
-    a.counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    a.offsets = offsets;
-    a.done = done;
-    a.err = err;
-    MOE_CUDA(launch_topk_hist(a, s));
-    record(1, s);
-    // permute: stable placement, then the row gather
-    MOE_CUDA(launch_scatter(idx, a.tile_base, T, E, k, perm_src, perm_dst, err, s));
-    MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H, static_cast<int>(elem_size(dt)),
-                           x_perm, s));
-    record(2, s);
-    // experts: fc1 + SwiGLU, fc2
-    cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
-    if (bf16)
-        MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s, mid));
-    else
-        MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
-                                     static_cast<const float*>(fc1), static_cast<const float*>(fc2),
-                                     rows, H, E, I, static_cast<float*>(act_buf),
-                                     static_cast<float*>(y), s, mid));
+    if (path & kPathSmallRoute) {
+        // logits on many CTAs (which also clear the header), then one CTA for top-k,
+        // bincount, scan and the stable permutation
+        MOE_CUDA(launch_router_logits_split(hidden, router_w, T, H, E, bf16, logits, err, s));
+        RouteSmallArgs a;
+        a.logits = logits;
+        a.bias = router_bias;
+        a.T = T;
+        a.E = E;
+        a.k = k;
+        a.normalize = normalize ? 1 : 0;
+        a.topk_idx = idx;
+        a.topk_w = w;
+        a.near_tie = near;
+        a.counts = counts;
+        a.offsets = offsets;
+        a.perm_src = perm_src;
+        a.perm_dst = perm_dst;
+        if (path & kPathDecodeFfn) {
+            a.zero_words = ctr;
+            a.n_zero = decode_ffn_counters(rows, E);
+        }
+        MOE_CUDA(launch_route_small(a, s));
+        record(1, s);
+    } else {
+        MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, kAlign, s));
+        // route: logits, then top-k + softmax + bincount + scan in one kernel
+        if (path & kPathTcRouter)
+            MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, err, s));
+        else
+            MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, bf16, logits, s));
+        TopkHistArgs a;
+        a.logits = logits;
+        a.bias = router_bias;
+        a.T = T;
+        a.E = E;
+        a.k = k;
+        a.normalize = normalize ? 1 : 0;
+        a.topk_idx = idx;
+        a.topk_w = w;
+        a.near_tie = near;
+        a.do_hist = true;
+        a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
+        a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
+        a.counts = counts;
+        a.offsets = offsets;
+        a.done = done;
+        a.err = err;
+        MOE_CUDA(launch_topk_hist(a, s));
+        record(1, s);
+        MOE_CUDA(launch_scatter(idx, a.tile_base, T, E, k, perm_src, perm_dst, err, s));
+    }
+    if (path & kPathDecodeFfn) {
+        // fc1 + SwiGLU and fc2 in one launch.  With at most 4 rows per expert on
+        // average, fc1 gathers its token rows straight from hidden (one TMA row box
+        // each); with more, the rows are gathered once into x_perm and loaded in
+        // 16-row boxes.
+        const bool tma_gather = rows <= 4 * E;
+        if (!tma_gather)
+            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
+                                   static_cast<int>(elem_size(dt)), x_perm, s));
+        record(2, s);
+        MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
+                                   T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err, s));
+        record(3, s);
+    } else {
+        MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
+                               static_cast<int>(elem_size(dt)), x_perm, s));
+        record(2, s);
+        cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
+        if (bf16)
+            MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s, mid));
+        else
+            MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
+                                         static_cast<const float*>(fc1),
+                                         static_cast<const float*>(fc2), rows, H, E, I,
+                                         static_cast<float*>(act_buf), static_cast<float*>(y), s,
+                                         mid));
+    }
     record(4, s);
     MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));
     record(5, s);

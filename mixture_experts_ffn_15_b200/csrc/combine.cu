@@ -15,49 +15,62 @@
 namespace moe {
 namespace {
 
+// Block (token group, column slab): 128 threads, one 16-byte vector of the output row
+// each; a block walks tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...  The k rows of
+// a token are loaded before they are summed (in slot order), so the loads overlap.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineUnroll = 8;
+
 template <bool BF16>
-__global__ void combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm_dst,
-                               const float* __restrict__ topk_w, int T, int H, int k,
-                               int rows_max, void* __restrict__ out) {
-    __shared__ int s_row[kMaxExperts];
-    __shared__ float s_w[kMaxExperts];
+__global__ void __launch_bounds__(kCombineThreads)
+combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm_dst,
+               const float* __restrict__ topk_w, int T, int H, int k, int rows_max,
+               void* __restrict__ out) {
     constexpr int VEC = BF16 ? 8 : 4;
     const int nvec = H / VEC;
+    const int v = blockIdx.y * kCombineThreads + threadIdx.x;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        __syncthreads();
-        for (int j = threadIdx.x; j < k; j += blockDim.x) {
-            const int r = perm_dst[static_cast<size_t>(t) * k + j];
-            s_row[j] = (r >= 0 && r < rows_max) ? r : -1;
-            s_w[j] = topk_w[static_cast<size_t>(t) * k + j];
-        }
-        __syncthreads();
-        for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-            float acc[VEC];
+        if (v >= nvec) continue;
+        float acc[VEC];
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
-            for (int j = 0; j < k; ++j) {
-                const int r = s_row[j];
-                if (r < 0) continue;
-                const float w = s_w[j];
-                float f[VEC];
-                if constexpr (BF16) {
-                    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(y_perm) +
-                                        static_cast<size_t>(r) * nvec + v),
-                                  f);
-                } else {
-                    const float4 q = __ldg(reinterpret_cast<const float4*>(y_perm) +
-                                           static_cast<size_t>(r) * nvec + v);
-                    f[0] = q.x; f[1] = q.y; f[2] = q.z; f[3] = q.w;
+        for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+        for (int j0 = 0; j0 < k; j0 += kCombineUnroll) {
+            float f[kCombineUnroll][VEC];
+            float w[kCombineUnroll];
+#pragma unroll
+            for (int jj = 0; jj < kCombineUnroll; ++jj) {
+                const int j = j0 + jj;
+                int r = -1;
+                w[jj] = 0.f;
+                if (j < k) {
+                    r = __ldg(perm_dst + static_cast<size_t>(t) * k + j);
+                    w[jj] = __ldg(topk_w + static_cast<size_t>(t) * k + j);
                 }
+                if (r < 0 || r >= rows_max) {
+                    w[jj] = 0.f;
 #pragma unroll
-                for (int i = 0; i < VEC; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+                    for (int i = 0; i < VEC; ++i) f[jj][i] = 0.f;
+                } else if constexpr (BF16) {
+                    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(y_perm) + static_cast<size_t>(r) * nvec + v),
+                                  f[jj]);
+                } else {
+                    const float4 q = __ldg(reinterpret_cast<const float4*>(y_perm) + static_cast<size_t>(r) * nvec + v);
+                    f[jj][0] = q.x; f[jj][1] = q.y; f[jj][2] = q.z; f[jj][3] = q.w;
+                }
             }
-            if constexpr (BF16) {
-                reinterpret_cast<uint4*>(out)[static_cast<size_t>(t) * nvec + v] = pack_bf16x8(acc);
-            } else {
-                reinterpret_cast<float4*>(out)[static_cast<size_t>(t) * nvec + v] =
-                    make_float4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll
+            for (int jj = 0; jj < kCombineUnroll; ++jj) {
+                if (j0 + jj < k) {
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) acc[i] = fmaf(w[jj], f[jj][i], acc[i]);
+                }
             }
+        }
+        if constexpr (BF16) {
+            reinterpret_cast<uint4*>(out)[static_cast<size_t>(t) * nvec + v] = pack_bf16x8(acc);
+        } else {
+            reinterpret_cast<float4*>(out)[static_cast<size_t>(t) * nvec + v] =
+                make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
     }
 }
@@ -86,19 +99,17 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
                            int T, int H, int k, bool bf16, void* out, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     const int nvec = H / (bf16 ? 8 : 4);
-    int threads = ((nvec + 31) / 32) * 32;
-    if (threads > 512) threads = 512;
-    if (threads < 64) threads = 64;
-    int blocks = T;
-    const int cap = device_sm_count() * 16;
-    if (blocks > cap) blocks = cap;
+    const int slabs = (nvec + kCombineThreads - 1) / kCombineThreads;
+    long long tok_blocks = (static_cast<long long>(device_sm_count()) * 16 + slabs - 1) / slabs;
+    if (tok_blocks > T) tok_blocks = T;
+    dim3 grid(static_cast<unsigned>(tok_blocks), static_cast<unsigned>(slabs));
     const int rows_max = T * k;
     if (bf16)
-        combine_kernel<true><<<blocks, threads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k, rows_max,
-                                                        out);
+        combine_kernel<true><<<grid, kCombineThreads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
+                                                              rows_max, out);
     else
-        combine_kernel<false><<<blocks, threads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
-                                                         rows_max, out);
+        combine_kernel<false><<<grid, kCombineThreads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
+                                                               rows_max, out);
     count_launch();
     return cudaGetLastError();
 }

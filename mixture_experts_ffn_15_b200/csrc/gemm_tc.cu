@@ -61,8 +61,9 @@ struct Tr {
     static constexpr int kAccStride = kWeightM ? kTokChunk : 256;
     static constexpr int kTmemCols = kWeightM ? 128 : 512;
     static constexpr int kUnitRows = kWeightM ? kTokChunk : BM;
-    // barriers (2*stages + 4) + tmem slot + abort flag, then offsets and prefix
-    static constexpr int kMiscBytes = (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4;
+    // barriers, tmem slot + abort flag, offsets, prefix, gather rows of one chunk
+    static constexpr int kMiscBytes =
+        (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 16 * 8 + 64;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     static_assert(kWeightM || (BN % 16 == 0 && BN >= 16 && BN <= 256), "UMMA N");
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams p) {
     using C = Tr<MODE, BN>;
-    constexpr bool kW = C::kWeightM;
+    static_assert(!C::kWeightM, "weight rows on M run in tc_ffn_decode_kernel");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -217,7 +218,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int per_unit = kW ? p.n_out / BM : p.n_out / BN;
+    const int per_unit = p.n_out / BN;
     const int num_units = s_pre[G] * per_unit;
     const int nk = p.K / BK;
 
@@ -229,25 +230,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             long long issued = 0;
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
                 const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
-                const int nl = kW ? (t.nrows + kBoxTok - 1) / kBoxTok : 0;
-                const uint32_t bytes =
-                    kW ? static_cast<uint32_t>(C::kABytes + nl * kBoxTok * BK * 2) : C::kStageBytes;
-                const int wrow = t.g * p.n_out + t.sub * (kW ? BM : BN);
+                const uint32_t bytes = C::kStageBytes;
+                const int wrow = t.g * p.n_out + t.sub * BN;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                     const uint32_t fb = smem_u32(&full[stage]);
                     mbar_arrive_expect_tx(fb, bytes);
                     const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
                     const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                    if constexpr (!kW) {
-                        tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
-                        tma_load_2d(b_dst, &tmB, fb, kb * BK, wrow);
-                    } else {
-                        tma_load_2d(a_dst, &tmA, fb, kb * BK, wrow);
-                        for (int l = 0; l < nl; ++l)
-                            tma_load_2d(b_dst + l * kBoxTok * BK * 2, &tmB, fb, kb * BK,
-                                        t.row0 + l * kBoxTok);
-                    }
+                    tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
+                    tma_load_2d(b_dst, &tmB, fb, kb * BK, wrow);
                     ++issued;
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -275,8 +267,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t acc_phase = 0;
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
                 const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
-                const int n_mma = kW ? ((t.nrows + 15) / 16) * 16 : BN;
-                const uint32_t idesc = idesc_bf16_f32(BM, n_mma);
+                const uint32_t idesc = idesc_bf16_f32(BM, BN);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
@@ -317,75 +308,409 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_fence_after();
             const uint32_t tb =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::kAccStride);
-            if constexpr (!kW) {
-                const bool valid = r < t.nrows;
-                const size_t orow = static_cast<size_t>(t.row0 + r);
-                const int col0 = t.sub * BN;
+            const bool valid = r < t.nrows;
+            const size_t orow = static_cast<size_t>(t.row0 + r);
+            const int col0 = t.sub * BN;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v[32];
-                    const bool full32 = (c + 32 <= BN);
-                    if (full32) tmem_ld_32x32b_x32(tb + c, v);
-                    else tmem_ld_32x32b_x16(tb + c, v);
-                    tmem_wait_ld();
-                    if (!valid) continue;
-                    const int nv = full32 ? 32 : 16;
-                    if constexpr (MODE == TOK_SWIGLU) {
-                        float a[16];
+            for (int c = 0; c < BN; c += 32) {
+                uint32_t v[32];
+                const bool full32 = (c + 32 <= BN);
+                if (full32) tmem_ld_32x32b_x32(tb + c, v);
+                else tmem_ld_32x32b_x16(tb + c, v);
+                tmem_wait_ld();
+                if (!valid) continue;
+                const int nv = full32 ? 32 : 16;
+                if constexpr (MODE == TOK_SWIGLU) {
+                    float a[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            a[i] = (2 * i < nv) ? swiglu_f32(f32(v[2 * i]), f32(v[2 * i + 1])) : 0.f;
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                              orow * p.ldo + (col0 + c) / 2);
-                        dst[0] = pack_bf16x8(a);
-                        if (nv == 32) dst[1] = pack_bf16x8(a + 8);
-                    } else if constexpr (MODE == TOK_PLAIN) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                              orow * p.ldo + col0 + c);
+                    for (int i = 0; i < 16; ++i)
+                        a[i] = (2 * i < nv) ? swiglu_f32(f32(v[2 * i]), f32(v[2 * i + 1])) : 0.f;
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                          orow * p.ldo + (col0 + c) / 2);
+                    dst[0] = pack_bf16x8(a);
+                    if (nv == 32) dst[1] = pack_bf16x8(a + 8);
+                } else if constexpr (MODE == TOK_PLAIN) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                          orow * p.ldo + col0 + c);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            if (8 * q < nv) {
-                                float f[8];
+                    for (int q = 0; q < 4; ++q) {
+                        if (8 * q < nv) {
+                            float f[8];
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) f[i] = f32(v[8 * q + i]);
-                                dst[q] = pack_bf16x8(f);
-                            }
-                        }
-                    } else {   // TOK_F32
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.out) +
-                                                              orow * p.ldo + col0 + c);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            if (4 * q < nv) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                    }
-                }
-            } else {
-                const int wr = t.sub * BM + r;   // weight row inside the expert
-#pragma unroll 1
-                for (int c = 0; c < t.nrows; c += 16) {
-                    uint32_t v[16];
-                    tmem_ld_32x32b_x16(tb + c, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = c + i;
-                        const float x = f32(v[i]);
-                        if constexpr (MODE == W_SWIGLU) {
-                            const float up = __shfl_xor_sync(0xffffffffu, x, 1);
-                            if (!(lane & 1) && n < t.nrows)
-                                static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(t.row0 + n) * p.ldo + (wr >> 1)] =
-                                    __float2bfloat16_rn(swiglu_f32(x, up));
-                        } else {
-                            if (n < t.nrows)
-                                static_cast<__nv_bfloat16*>(p.out)[static_cast<size_t>(t.row0 + n) * p.ldo + wr] =
-                                    __float2bfloat16_rn(x);
+                            for (int i = 0; i < 8; ++i) f[i] = f32(v[8 * q + i]);
+                            dst[q] = pack_bf16x8(f);
                         }
                     }
+                } else {   // TOK_F32
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.out) +
+                                                          orow * p.ldo + col0 + c);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (4 * q < nv) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------------------ decode FFN
+// fc1 + SwiGLU and fc2 for batches with few rows per expert, in ONE persistent
+// launch.  Both GEMMs put 128 weight rows on the MMA's M side and the expert's tokens
+// (a chunk of at most 64 permuted rows) on N, so every weight byte streams from HBM
+// once.  The unit list holds every fc1 unit (chunk x 128 rows of fc1) and then every
+// fc2 unit (chunk x 128 rows of fc2).  CTAs claim units in that order from a global
+// counter (the producer warp claims, a 4-slot ring in shared memory hands the unit to
+// the MMA and epilogue warps), so the large fc1 units go first and the small fc2 units
+// even out the end; every fc1 unit is claimed before any fc2 unit.  An fc2 unit needs the
+// activations of its chunk: each fc1 epilogue warp publishes its stores with a proxy
+// fence and a release increment of the chunk's counter, and the fc2 producer waits
+// (bounded) for 4 x (fc1 units per chunk) increments with an acquire load before
+// loading the activations with TMA.  The fc2 weights of a unit do not depend on fc1.
+// With GATHER, fc1's token rows come straight from `hidden` through perm_src (one TMA
+// box of one row each); otherwise from contiguous rows of x_perm (16-row boxes).
+// Every CTA of the grid (at most one per SM) is resident, so the waits always end.
+constexpr int kUnitRing = 4;
+
+struct DecodeParams {
+    const int32_t* offsets;   // [E+1]
+    const int32_t* perm_src;  // [rows] with GATHER, else nullptr
+    int E, rows, T, H, I;
+    __nv_bfloat16* act;       // [rows, I]
+    __nv_bfloat16* y;         // [rows, H]
+    int32_t* done;            // one counter per chunk, zero on entry
+    int32_t* sched;           // next unit to claim, zero on entry
+    int32_t* err;
+};
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ bool wait_count(const int32_t* ctr, int target, volatile int* abort) {
+    if (ld_acquire(ctr) >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (ld_acquire(ctr) >= target) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+struct DUnit {
+    int phase;   // 1: fc1 + SwiGLU, 2: fc2
+    int chunk;
+    int g, row0, nrows, mt;
+};
+
+__device__ __forceinline__ DUnit decode_dunit(int u, int U1, int MT1, int MT2, int G,
+                                              const int* s_off, const int* s_pre) {
+    DUnit d;
+    int v, MT;
+    if (u < U1) {
+        d.phase = 1;
+        v = u;
+        MT = MT1;
+    } else {
+        d.phase = 2;
+        v = u - U1;
+        MT = MT2;
+    }
+    d.chunk = v / MT;
+    d.mt = v - d.chunk * MT;
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= d.chunk) lo = mid; else hi = mid - 1;
+    }
+    d.g = lo;
+    d.row0 = s_off[lo] + (d.chunk - s_pre[lo]) * kTokChunk;
+    d.nrows = min(kTokChunk, s_off[lo + 1] - d.row0);
+    return d;
+}
+
+template <bool GATHER>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX,
+                     const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmAct,
+                     const DecodeParams p) {
+    using C = Tr<W_PLAIN, 64>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::kStages * C::kABytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* s_pre = s_off + (kMaxExperts + 1);
+    int* s_unit = s_pre + (kMaxExperts + 1);                        // [kUnitRing]
+    uint64_t* ufull = reinterpret_cast<uint64_t*>(s_unit + 2 * kUnitRing);   // 8-byte aligned
+    uint64_t* uempty = ufull + kUnitRing;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.E;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 4);
+        }
+        for (int q = 0; q < kUnitRing; ++q) {
+            mbar_init(smem_u32(&ufull[q]), 1);
+            mbar_init(smem_u32(&uempty[q]), 5);   // the MMA thread and 4 epilogue warps
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW1);
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW2);
+        tma_prefetch_desc(&tmAct);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 2) {
+        TcParams tp{p.offsets, p.E, p.rows, 0, 0, nullptr, 0, p.err};
+        build_tile_map(tp, G, kTokChunk, s_off, s_pre, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int MT1 = 2 * p.I / BM, MT2 = p.H / BM;
+    const int CH = s_pre[G];
+    const int U1 = CH * MT1;
+    const int U = U1 + CH * MT2;
+    const int nk1 = p.H / BK, nk2 = p.I / BK;
+    const int fc1_done = 4 * MT1;   // increments per chunk: 4 epilogue warps per fc1 unit
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // Lane 0 owns the barriers; every lane issues its share of the token rows.
+        int stage = 0;
+        uint32_t phase = 0;
+        long long issued = 0;
+        int slot = 0;
+        uint32_t uphase = 0;
+        for (;;) {
+            int u = U;
+            if (lane == 0) {
+                if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
+                    u = *abort_flag ? U : atomicAdd(p.sched, 1);
+                s_unit[slot] = u;
+                mbar_arrive(smem_u32(&ufull[slot]));
+            }
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (++slot == kUnitRing) {
+                slot = 0;
+                uphase ^= 1u;
+            }
+            if (u >= U) break;
+            const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
+            const bool f1 = d.phase == 1;
+            const int nk = f1 ? nk1 : nk2;
+            const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;
+            const int wrow = d.g * (f1 ? 2 * p.I : p.H) + d.mt * BM;
+            const int nl = (d.nrows + kBoxTok - 1) / kBoxTok;
+            uint32_t bbytes = static_cast<uint32_t>(nl * kBoxTok * BK * 2);
+            int src[2] = {0, 0};   // this lane's gathered token rows: lane, lane + 32
+            if (f1 && GATHER) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int i = lane + 32 * h;
+                    if (i < d.nrows) {
+                        int t = p.perm_src[d.row0 + i];
+                        if (t < 0 || t >= p.T) {
+                            atomicOr(p.err, kErrBadExpert);
+                            t = 0;
+                        }
+                        src[h] = t;
+                    }
+                }
+                bbytes = static_cast<uint32_t>(d.nrows * BK * 2);
+            }
+            if (!f1) {
+                bool ok = true;
+                if (lane == 0) ok = wait_count(&p.done[d.chunk], fc1_done, abort_flag);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                fence_proxy_async_global();
+            }
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (lane == 0) {
+                    ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
+                    if (ok) mbar_arrive_expect_tx(smem_u32(&full[stage]), C::kABytes + bbytes);
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                const uint32_t fb = smem_u32(&full[stage]);
+                const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
+                const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
+                if (lane == 0) tma_load_2d(a_dst, ma, fb, kb * BK, wrow);
+                if (f1 && GATHER) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int i = lane + 32 * h;
+                        if (i < d.nrows) tma_load_2d(b_dst + i * BK * 2, &tmX, fb, kb * BK, src[h]);
+                    }
+                } else if (lane < nl) {
+                    tma_load_2d(b_dst + lane * kBoxTok * BK * 2, f1 ? &tmX : &tmAct, fb, kb * BK,
+                                d.row0 + lane * kBoxTok);
+                }
+                ++issued;
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+        if (lane == 0 && *abort_flag) {
+            // let the copies already in flight land before the CTA exits
+            int dummy = 0;
+            for (int s2 = 0; s2 < C::kStages; ++s2) {
+                if (issued <= s2) break;
+                const long long fills = (issued - 1 - s2) / C::kStages + 1;
+                mbar_wait(smem_u32(&full[s2]), static_cast<uint32_t>((fills - 1) & 1), &dummy,
+                          kWaitLimitNs / 4);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            int slot = 0;
+            uint32_t uphase = 0;
+            for (;;) {
+                if (!mbar_wait(smem_u32(&ufull[slot]), uphase, abort_flag, kWaitLimitNs)) break;
+                const int u = s_unit[slot];
+                mbar_arrive(smem_u32(&uempty[slot]));
+                if (++slot == kUnitRing) {
+                    slot = 0;
+                    uphase ^= 1u;
+                }
+                if (u >= U) break;
+                const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
+                const int nk = d.phase == 1 ? nk1 : nk2;
+                const uint32_t idesc = idesc_bf16_f32(BM, ((d.nrows + 15) / 16) * 16);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                                  idesc, (kb | kk) != 0);
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&tfull[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int slot = 0;
+        uint32_t uphase = 0;
+        for (;;) {
+            const bool got = mbar_wait(smem_u32(&ufull[slot]), uphase, abort_flag, kWaitLimitNs);
+            const int u = got ? s_unit[slot] : U;
+            __syncwarp();
+            if (got && lane == 0) mbar_arrive(smem_u32(&uempty[slot]));
+            if (++slot == kUnitRing) {
+                slot = 0;
+                uphase ^= 1u;
+            }
+            if (u >= U) break;
+            const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
+            const bool f1 = d.phase == 1;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                static_cast<uint32_t>(acc * C::kAccStride);
+            const int wr = d.mt * BM + r;   // weight row inside the expert
+#pragma unroll 1
+            for (int c = 0; c < d.nrows; c += 16) {
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tb + c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int n = c + i;
+                    const float x = f32(v[i]);
+                    if (f1) {
+                        const float up = __shfl_xor_sync(0xffffffffu, x, 1);
+                        if (!(lane & 1) && n < d.nrows)
+                            p.act[static_cast<size_t>(d.row0 + n) * p.I + (wr >> 1)] =
+                                __float2bfloat16_rn(swiglu_f32(x, up));
+                    } else if (n < d.nrows) {
+                        p.y[static_cast<size_t>(d.row0 + n) * p.H + wr] = __float2bfloat16_rn(x);
+                    }
+                }
+            }
+            tc_fence_before();
+            if (f1) fence_proxy_async_global();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&tempty[acc]));
+                if (f1) {
+                    __threadfence();
+                    atomicAdd(&p.done[d.chunk], 1);
+                }
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
@@ -469,16 +794,7 @@ cudaError_t grouped_gemm(bool swiglu, const void* act_in, int rows, int K, const
                          int n_out, const int32_t* offsets, void* out, int ldo, int32_t* err,
                          cudaStream_t s) {
     TcParams p{offsets, E, rows, K, n_out, out, ldo, err};
-    // Few rows per expert: put the weights on the MMA's M side (weight-M).
-    const bool weight_m = (n_out % BM == 0) && (static_cast<long long>(rows) <= 64LL * E);
     CUtensorMap ma, mb;
-    if (weight_m) {
-        if (!make_map(&ma, w, static_cast<long long>(E) * n_out, K, BM)) return cudaErrorInvalidValue;
-        if (!make_map(&mb, act_in, rows, K, kBoxTok)) return cudaErrorInvalidValue;
-        const long long bound = (static_cast<long long>((rows + kTokChunk - 1) / kTokChunk) + E) * (n_out / BM);
-        const int b = static_cast<int>(bound > (1 << 30) ? (1 << 30) : bound);
-        return swiglu ? launch_one<W_SWIGLU, 64>(ma, mb, p, b, s) : launch_one<W_PLAIN, 64>(ma, mb, p, b, s);
-    }
     const int bn = pick_bn(n_out);
     if (!make_map(&ma, act_in, rows, K, BM)) return cudaErrorInvalidValue;
     if (!make_map(&mb, w, static_cast<long long>(E) * n_out, K, bn)) return cudaErrorInvalidValue;
@@ -500,6 +816,34 @@ cudaError_t grouped_gemm(bool swiglu, const void* act_in, int rows, int K, const
 #undef MOE_TOK_CASE
 }
 
+// Grid of a persistent decode FFN launch: every unit of both GEMMs, at most one CTA per SM.
+int decode_grid(int rows, int E, int H, int I) {
+    const long long units =
+        (static_cast<long long>((rows + kTokChunk - 1) / kTokChunk) + E) * (2 * I / BM + H / BM);
+    const int sms = device_sm_count();
+    return static_cast<int>(units < sms ? units : sms);
+}
+
+template <bool GATHER>
+cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& w2,
+                          const CUtensorMap& a, const DecodeParams& p, int grid, cudaStream_t s) {
+    using C = Tr<W_PLAIN, 64>;
+    auto kern = tc_ffn_decode_kernel<GATHER>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kThreads, C::kSmemBytes, s>>>(w1, x, w2, a, p);
+    count_launch();
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool tc_ffn_supported(int H, int I) { return H % 64 == 0 && I % 64 == 0 && H > 0 && I > 0; }
@@ -516,6 +860,35 @@ cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void
     if (e != cudaSuccess) return e;
     if (mid) record_event(mid, s);
     return grouped_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
+}
+
+bool decode_ffn_supported(int rows, int E, int H, int I) {
+    return tc_ffn_supported(H, I) && (2 * I) % BM == 0 && H % BM == 0 &&
+           static_cast<long long>(rows) <= static_cast<long long>(kTokChunk) * E;
+}
+
+// one completion counter per chunk, then the unit scheduler's counter
+int decode_ffn_counters(int rows, int E) { return (rows + kTokChunk - 1) / kTokChunk + E + 1; }
+
+cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
+                              const int32_t* offsets, const void* fc1, const void* fc2, int rows,
+                              int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
+                              cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    CUtensorMap w1, x, w2, a;
+    if (!make_map(&w1, fc1, static_cast<long long>(E) * 2 * I, H, BM)) return cudaErrorInvalidValue;
+    if (perm_src) {
+        if (!make_map(&x, tokens, T, H, 1)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_map(&x, tokens, rows, H, kBoxTok)) return cudaErrorInvalidValue;
+    }
+    if (!make_map(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
+    DecodeParams p{offsets, perm_src, E, rows, T, H, I, static_cast<__nv_bfloat16*>(act),
+                   static_cast<__nv_bfloat16*>(y), done, done + decode_ffn_counters(rows, E) - 1, err};
+    const int grid = decode_grid(rows, E, H, I);
+    return perm_src ? launch_decode<true>(w1, x, w2, a, p, grid, s)
+                    : launch_decode<false>(w1, x, w2, a, p, grid, s);
 }
 
 cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,

@@ -39,6 +39,30 @@ cudaError_t launch_topk_hist(const TopkHistArgs& a, cudaStream_t s);
 
 inline int num_token_tiles(int T) { return (T + 127) / 128; }
 
+// ---------------------------------------------------------------- route_small.cu
+constexpr int kRouteSmallMaxT = 512;   // one CTA routes and permutes the whole batch
+constexpr int kRouteSmallMaxK = 32;
+
+cudaError_t launch_router_logits_split(const void* hidden, const void* router_w, int T, int H,
+                                       int E, bool bf16, float* logits, int32_t* clear_words,
+                                       cudaStream_t s);
+
+struct RouteSmallArgs {
+    const float* logits = nullptr;   // [T, E]
+    const float* bias = nullptr;     // [E] or nullptr
+    int T = 0, E = 0, k = 0, normalize = 1;
+    int32_t* topk_idx = nullptr;     // [T, k]
+    float* topk_w = nullptr;         // [T, k]
+    int32_t* near_tie = nullptr;     // [T] or nullptr
+    int32_t* counts = nullptr;       // [E]
+    int32_t* offsets = nullptr;      // [E + 1]
+    int32_t* perm_src = nullptr;     // [T * k]
+    int32_t* perm_dst = nullptr;     // [T * k]
+    int32_t* zero_words = nullptr;   // cleared by the kernel (the decode FFN's counters)
+    int n_zero = 0;
+};
+cudaError_t launch_route_small(const RouteSmallArgs& a, cudaStream_t s);
+
 // ---------------------------------------------------------------- permute.cu
 cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
                            int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s);
@@ -65,5 +89,14 @@ cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void
                           int32_t* err, cudaStream_t s, cudaEvent_t mid);
 cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,
                              float* logits, int32_t* err, cudaStream_t s);
+
+// Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
+bool decode_ffn_supported(int rows, int E, int H, int I);
+int decode_ffn_counters(int rows, int E);   // int32 counters it needs, zero on entry
+// tokens: `hidden` [T, H] gathered through perm_src, or x_perm [rows, H] if perm_src is null
+cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
+                              const int32_t* offsets, const void* fc1, const void* fc2, int rows,
+                              int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
+                              cudaStream_t s);
 
 }  // namespace moe

@@ -98,3 +98,17 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(ImportError, match="build"):
         _abi.load()
+
+
+def test_forward_path_per_workload():
+    """moe_forward_path: which kernels run for each workload (host arithmetic only)."""
+    lib = _lib()
+    bf, f32 = _abi.MOE_BF16, _abi.MOE_F32
+    small, fused, tc_router, token, fma = 1, 2, 4, 8, 16
+    assert lib.moe_forward_path(64, 256, 8, 2, 128, f32) == small | fma
+    assert lib.moe_forward_path(4, 2816, 128, 8, 704, bf) == small | fused
+    assert lib.moe_forward_path(256, 2816, 128, 8, 704, bf) == small | fused
+    assert lib.moe_forward_path(8192, 2816, 128, 8, 704, bf) == tc_router | token
+    assert lib.moe_forward_path(32768, 4096, 64, 4, 1536, bf) == tc_router | token
+    assert lib.moe_forward_path(300, 128, 8, 2, 704, bf) == small | token   # > 64 rows per expert
+    assert lib.moe_forward_path(4, 2816, 128, 300, 704, bf) == 0
