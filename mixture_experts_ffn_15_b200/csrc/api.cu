@@ -304,7 +304,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     if (dt == MOE_BF16 && decode_ffn_supported(rows, E, H, I)) {
         MOE_CUDA(cudaMemsetAsync(ctr, 0, static_cast<size_t>(decode_ffn_counters(rows, E)) * 4, s));
         MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1, fc2, rows, H, E, I,
-                                   act_buf, y_perm, ctr, err, s));
+                                   act_buf, y_perm, ctr, err, nullptr, nullptr, 0, nullptr, s));
     } else if (dt == MOE_BF16) {
         MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
                                nullptr));
@@ -429,9 +429,14 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
             MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
                                    static_cast<int>(elem_size(dt)), x_perm, s));
         record(2, s);
+        // ... and the weighted combine, after every fc2 unit has published its rows
         MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
-                                   T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err, s));
+                                   T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err,
+                                   perm_dst, w, k, out, s));
         record(3, s);
+        record(4, s);
+        record(5, s);
+        return MOE_OK;
     } else {
         MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
                                static_cast<int>(elem_size(dt)), x_perm, s));

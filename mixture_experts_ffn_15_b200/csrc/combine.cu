@@ -9,6 +9,7 @@
 // chunked [E, 2I, H] (gate rows first, then up rows); the interleaved layout of
 // swiglu_fusion = 1 is the Reshape [E,2,I,H] -> Transpose [E,I,2,H] -> Reshape
 // [E,2I,H], i.e. dst row 2j+s of expert e is src row s*I+j.
+#include "combine.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,56 +20,34 @@ namespace {
 // each; a block walks tokens t = blockIdx.x, blockIdx.x + gridDim.x, ...  The k rows of
 // a token are loaded before they are summed (in slot order), so the loads overlap.
 constexpr int kCombineThreads = 128;
-constexpr int kCombineUnroll = 8;
 
 template <bool BF16>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm_dst,
                const float* __restrict__ topk_w, int T, int H, int k, int rows_max,
                void* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int VEC = BF16 ? 8 : 4;
     const int nvec = H / VEC;
     const int v = blockIdx.y * kCombineThreads + threadIdx.x;
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (v >= nvec) continue;
-        float acc[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
-        for (int j0 = 0; j0 < k; j0 += kCombineUnroll) {
-            float f[kCombineUnroll][VEC];
-            float w[kCombineUnroll];
-#pragma unroll
-            for (int jj = 0; jj < kCombineUnroll; ++jj) {
-                const int j = j0 + jj;
-                int r = -1;
-                w[jj] = 0.f;
-                if (j < k) {
-                    r = __ldg(perm_dst + static_cast<size_t>(t) * k + j);
-                    w[jj] = __ldg(topk_w + static_cast<size_t>(t) * k + j);
-                }
-                if (r < 0 || r >= rows_max) {
-                    w[jj] = 0.f;
-#pragma unroll
-                    for (int i = 0; i < VEC; ++i) f[jj][i] = 0.f;
-                } else if constexpr (BF16) {
-                    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(y_perm) + static_cast<size_t>(r) * nvec + v),
-                                  f[jj]);
-                } else {
-                    const float4 q = __ldg(reinterpret_cast<const float4*>(y_perm) + static_cast<size_t>(r) * nvec + v);
-                    f[jj][0] = q.x; f[jj][1] = q.y; f[jj][2] = q.z; f[jj][3] = q.w;
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < kCombineUnroll; ++jj) {
-                if (j0 + jj < k) {
-#pragma unroll
-                    for (int i = 0; i < VEC; ++i) acc[i] = fmaf(w[jj], f[jj][i], acc[i]);
-                }
-            }
-        }
         if constexpr (BF16) {
-            reinterpret_cast<uint4*>(out)[static_cast<size_t>(t) * nvec + v] = pack_bf16x8(acc);
+            reinterpret_cast<uint4*>(out)[static_cast<size_t>(t) * nvec + v] = combine_vec_bf16(
+                reinterpret_cast<const uint4*>(y_perm), nvec, perm_dst, topk_w, t, k, v, rows_max);
         } else {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < k; ++j) {
+                const int r = perm_dst[static_cast<size_t>(t) * k + j];
+                if (r < 0 || r >= rows_max) continue;
+                const float w = topk_w[static_cast<size_t>(t) * k + j];
+                const float4 q = __ldg(reinterpret_cast<const float4*>(y_perm) + static_cast<size_t>(r) * nvec + v);
+                acc[0] = fmaf(w, q.x, acc[0]);
+                acc[1] = fmaf(w, q.y, acc[1]);
+                acc[2] = fmaf(w, q.z, acc[2]);
+                acc[3] = fmaf(w, q.w, acc[3]);
+            }
             reinterpret_cast<float4*>(out)[static_cast<size_t>(t) * nvec + v] =
                 make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
@@ -78,6 +57,8 @@ combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm
 __global__ void __launch_bounds__(256)
 convert_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int E, int I,
                int vec_per_row) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const long long rows = static_cast<long long>(E) * 2 * I;
     const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
@@ -104,14 +85,10 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
     if (tok_blocks > T) tok_blocks = T;
     dim3 grid(static_cast<unsigned>(tok_blocks), static_cast<unsigned>(slabs));
     const int rows_max = T * k;
-    if (bf16)
-        combine_kernel<true><<<grid, kCombineThreads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
-                                                              rows_max, out);
-    else
-        combine_kernel<false><<<grid, kCombineThreads, 0, s>>>(y_perm, perm_dst, topk_w, T, H, k,
-                                                               rows_max, out);
-    count_launch();
-    return cudaGetLastError();
+    return bf16 ? launch_k(combine_kernel<true>, grid, dim3(kCombineThreads), 0, s, y_perm, perm_dst,
+                           topk_w, T, H, k, rows_max, out)
+                : launch_k(combine_kernel<false>, grid, dim3(kCombineThreads), 0, s, y_perm,
+                           perm_dst, topk_w, T, H, k, rows_max, out);
 }
 
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
@@ -122,10 +99,8 @@ cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int 
     long long blocks = (rows + 7) / 8;
     const long long cap = static_cast<long long>(device_sm_count()) * 16;
     if (blocks > cap) blocks = cap;
-    convert_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const uint4*>(src),
-                                                             static_cast<uint4*>(dst), E, I, vec);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(convert_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                    static_cast<const uint4*>(src), static_cast<uint4*>(dst), E, I, vec);
 }
 
 }  // namespace moe

@@ -42,6 +42,16 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* f) {
                       pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that it
+// may start while the previous kernel on the stream is still running; pdl_wait()
+// blocks until that kernel has completed and its memory is visible, so each kernel
+// calls it before its first global-memory access.  pdl_trigger() lets the next
+// kernel start its own prologue.  Both are no-ops for a plain launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // silu(g) * u in float32 (standard SwiGLU).
 __device__ __forceinline__ float swiglu_f32(float g, float u) {
     return g / (1.0f + expf(-g)) * u;

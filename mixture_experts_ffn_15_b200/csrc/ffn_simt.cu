@@ -24,6 +24,8 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_pre[kMaxExperts + 1];
     const int tid = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
     if (tid == 0) {
         int prev = 0, pre = 0;
         for (int e = 0; e <= E; ++e) {
@@ -107,16 +109,12 @@ cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, con
                                 const float* fc2, int rows, int H, int E, int I, float* act,
                                 float* y, cudaStream_t s, cudaEvent_t mid) {
     if (rows <= 0) return cudaSuccess;
-    simt_grouped_gemm_kernel<true><<<simt_grid(rows, E, 2 * I), 256, 0, s>>>(
-        x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I);
-    count_launch();
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_k(simt_grouped_gemm_kernel<true>, dim3(simt_grid(rows, E, 2 * I)),
+                               dim3(256), 0, s, x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I);
     if (err != cudaSuccess) return err;
     if (mid) record_event(mid, s);
-    simt_grouped_gemm_kernel<false><<<simt_grid(rows, E, H), 256, 0, s>>>(act, I, fc2, H, I,
-                                                                           offsets, E, rows, y, H);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(simt_grouped_gemm_kernel<false>, dim3(simt_grid(rows, E, H)), dim3(256), 0, s,
+                    static_cast<const float*>(act), I, fc2, H, I, offsets, E, rows, y, H);
 }
 
 }  // namespace moe

@@ -31,6 +31,7 @@
 // MOE_DEVERR_TIMEOUT in the error word and still frees its TMEM.
 #include <cuda.h>
 
+#include "combine.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -212,6 +213,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
+    // the prologue above touches no global memory; everything below may
+    pdl_wait();
+    pdl_trigger();
     if (warp == 2) build_tile_map(p, G, C::kUnitRows, s_off, s_pre, lane);
     tc_fence_before();
     __syncthreads();
@@ -381,6 +385,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // loading the activations with TMA.  The fc2 weights of a unit do not depend on fc1.
 // With GATHER, fc1's token rows come straight from `hidden` through perm_src (one TMA
 // box of one row each); otherwise from contiguous rows of x_perm (16-row boxes).
+// With `out`, the kernel also does the weighted combine: once every fc2 unit has
+// published its rows (a grid-wide count, acquire), the epilogue warps of all CTAs
+// split the output vectors among themselves, with the same arithmetic as
+// combine_kernel.
 // Every CTA of the grid (at most one per SM) is resident, so the waits always end.
 constexpr int kUnitRing = 4;
 
@@ -392,6 +400,12 @@ struct DecodeParams {
     __nv_bfloat16* y;         // [rows, H]
     int32_t* done;            // one counter per chunk, zero on entry
     int32_t* sched;           // next unit to claim, zero on entry
+    int32_t* fc2_done;        // published fc2 units (x 4 warps), zero on entry
+    // fused combine (out != nullptr): out[t] = sum_j topk_w[t, j] y[perm_dst[t*k + j]]
+    const int32_t* perm_dst;
+    const float* topk_w;
+    int k;
+    __nv_bfloat16* out;
     int32_t* err;
 };
 
@@ -502,6 +516,9 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
+    // the prologue above touches no global memory; everything below may
+    pdl_wait();
+    pdl_trigger();
     if (warp == 2) {
         TcParams tp{p.offsets, p.E, p.rows, 0, 0, nullptr, 0, p.err};
         build_tile_map(tp, G, kTokChunk, s_off, s_pre, lane);
@@ -706,13 +723,28 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(smem_u32(&tempty[acc]));
-                if (f1) {
-                    __threadfence();
-                    atomicAdd(&p.done[d.chunk], 1);
-                }
+                __threadfence();
+                atomicAdd(f1 ? &p.done[d.chunk] : p.fc2_done, 1);
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
+        }
+        if (p.out != nullptr) {
+            // ------------------------------------------------------------ combine
+            bool ok = true;
+            if (lane == 0) ok = wait_count(p.fc2_done, 4 * (U - U1), abort_flag);
+            if (__shfl_sync(0xffffffffu, ok, 0)) {
+                const int nvec = p.H / 8;
+                const long long total = static_cast<long long>(p.T) * nvec;
+                const int et = (warp - 2) * 32 + lane;   // 0..127
+                for (long long q = static_cast<long long>(blockIdx.x) * 128 + et; q < total;
+                     q += static_cast<long long>(gridDim.x) * 128) {
+                    const int t = static_cast<int>(q / nvec), v = static_cast<int>(q - static_cast<long long>(t) * nvec);
+                    reinterpret_cast<uint4*>(p.out)[q] =
+                        combine_vec_bf16(reinterpret_cast<const uint4*>(p.y), nvec, p.perm_dst,
+                                         p.topk_w, t, p.k, v, p.rows);
+                }
+            }
         }
     }
 
@@ -777,9 +809,7 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParam
     int grid = device_sm_count();
     if (bound < grid) grid = bound;
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, C::kSmemBytes, s>>>(a, b, p);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p);
 }
 
 int pick_bn(int n_out) {
@@ -839,9 +869,7 @@ cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUt
         attr_set[dev] = true;
     }
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, C::kSmemBytes, s>>>(w1, x, w2, a, p);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, w1, x, w2, a, p);
 }
 
 }  // namespace
@@ -867,12 +895,13 @@ bool decode_ffn_supported(int rows, int E, int H, int I) {
            static_cast<long long>(rows) <= static_cast<long long>(kTokChunk) * E;
 }
 
-// one completion counter per chunk, then the unit scheduler's counter
-int decode_ffn_counters(int rows, int E) { return (rows + kTokChunk - 1) / kTokChunk + E + 1; }
+// one completion counter per chunk, the unit scheduler's counter, the fc2 count
+int decode_ffn_counters(int rows, int E) { return (rows + kTokChunk - 1) / kTokChunk + E + 2; }
 
 cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
+                              const int32_t* perm_dst, const float* topk_w, int k, void* out,
                               cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
     CUtensorMap w1, x, w2, a;
@@ -884,8 +913,10 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     }
     if (!make_map(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
     if (!make_map(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
+    const int nctr = decode_ffn_counters(rows, E);
     DecodeParams p{offsets, perm_src, E, rows, T, H, I, static_cast<__nv_bfloat16*>(act),
-                   static_cast<__nv_bfloat16*>(y), done, done + decode_ffn_counters(rows, E) - 1, err};
+                   static_cast<__nv_bfloat16*>(y), done, done + nctr - 2, done + nctr - 1,
+                   perm_dst, topk_w, k, static_cast<__nv_bfloat16*>(out), err};
     const int grid = decode_grid(rows, E, H, I);
     return perm_src ? launch_decode<true>(w1, x, w2, a, p, grid, s)
                     : launch_decode<false>(w1, x, w2, a, p, grid, s);

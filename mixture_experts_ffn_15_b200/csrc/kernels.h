@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
 
 int device_sm_count();
@@ -14,6 +16,26 @@ void record_event(cudaEvent_t ev, cudaStream_t s);
 
 // Process-wide count of kernel launches issued by the library (host side).
 void count_launch(int n = 1);
+
+// Every kernel launch of the library: programmatic stream serialisation allowed, so
+// the kernel may begin while its predecessor on the stream finishes (it waits with
+// griddepcontrol.wait before touching memory), counted by count_launch().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- route.cu
 cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, int T, int H,
@@ -93,10 +115,12 @@ cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, in
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);
 int decode_ffn_counters(int rows, int E);   // int32 counters it needs, zero on entry
-// tokens: `hidden` [T, H] gathered through perm_src, or x_perm [rows, H] if perm_src is null
+// tokens: `hidden` [T, H] gathered through perm_src, or x_perm [rows, H] if perm_src is null.
+// With out != nullptr the launch also does the weighted combine into out [T, H].
 cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
+                              const int32_t* perm_dst, const float* topk_w, int k, void* out,
                               cudaStream_t s);
 
 }  // namespace moe

@@ -22,6 +22,8 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
                int E, int k, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_dst,
                int32_t* __restrict__ err) {
     __shared__ uint32_t s_mask[kMaxExperts * kMaskWords];
+    pdl_wait();
+    pdl_trigger();
     const int tile = blockIdx.x;
     const int t_begin = tile * kTileTokens;
     const int nt = min(kTileTokens, T - t_begin);
@@ -62,6 +64,8 @@ __global__ void __launch_bounds__(256)
 gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm_src,
               const int32_t* __restrict__ offsets, int E, int T, int rows_max, int vec_per_row,
               uint4* __restrict__ x_perm) {
+    pdl_wait();
+    pdl_trigger();
     const int rows = min(offsets[E], rows_max);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
@@ -82,10 +86,8 @@ gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm
 cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
                            int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    scatter_kernel<<<num_token_tiles(T), kScatterThreads, 0, s>>>(topk_idx, tile_base, T, E, k,
-                                                                  perm_src, perm_dst, err);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(scatter_kernel, dim3(num_token_tiles(T)), dim3(kScatterThreads), 0, s, topk_idx,
+                    tile_base, T, E, k, perm_src, perm_dst, err);
 }
 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
@@ -96,10 +98,8 @@ cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int
     int blocks = (rows_max + 7) / 8;
     const int cap = device_sm_count() * 8;
     if (blocks > cap) blocks = cap;
-    gather_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(hidden), perm_src, offsets, E,
-                                         T, rows_max, vec, static_cast<uint4*>(x_perm));
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(gather_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(hidden),
+                    perm_src, offsets, E, T, rows_max, vec, static_cast<uint4*>(x_perm));
 }
 
 }  // namespace moe

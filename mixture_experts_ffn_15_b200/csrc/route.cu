@@ -32,6 +32,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(kLogitWarps * 32)
 router_logits_simt_kernel(const void* __restrict__ hidden, const void* __restrict__ router_w,
                           int T, int H, int E, float* __restrict__ logits) {
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * kLogitWarps + warp;
     const int t0 = blockIdx.y * kLogitTokens;
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(kHistThreads) topk_hist_kernel(const TopkHistA
     __shared__ int s_strip[kHistThreads];
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_last;
+    pdl_wait();
+    pdl_trigger();
 
     const int tile = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -262,21 +266,15 @@ cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, 
                                       int E, bool bf16, float* logits, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     dim3 grid((E + kLogitWarps - 1) / kLogitWarps, (T + kLogitTokens - 1) / kLogitTokens);
-    if (bf16)
-        router_logits_simt_kernel<true><<<grid, kLogitWarps * 32, 0, s>>>(hidden, router_w, T, H,
-                                                                          E, logits);
-    else
-        router_logits_simt_kernel<false><<<grid, kLogitWarps * 32, 0, s>>>(hidden, router_w, T, H,
-                                                                           E, logits);
-    count_launch();
-    return cudaGetLastError();
+    return bf16 ? launch_k(router_logits_simt_kernel<true>, grid, dim3(kLogitWarps * 32), 0, s,
+                           hidden, router_w, T, H, E, logits)
+                : launch_k(router_logits_simt_kernel<false>, grid, dim3(kLogitWarps * 32), 0, s,
+                           hidden, router_w, T, H, E, logits);
 }
 
 cudaError_t launch_topk_hist(const TopkHistArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    topk_hist_kernel<<<num_token_tiles(a.T), kHistThreads, 0, s>>>(a);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(topk_hist_kernel, dim3(num_token_tiles(a.T)), dim3(kHistThreads), 0, s, a);
 }
 
 }  // namespace moe

@@ -33,6 +33,8 @@ router_logits_split_kernel(const void* __restrict__ hidden, const void* __restri
     const int e0 = blockIdx.x * EPB;
     const int t0 = blockIdx.y * kSplitTokens;
     const int nt = min(kSplitTokens, T - t0);
+    pdl_wait();
+    pdl_trigger();
     if (clear_words && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2)
         clear_words[threadIdx.x] = 0;
     float acc[EPB][kSplitTokens];
@@ -115,6 +117,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Rou
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, E = a.E, k = a.k;
     const int words = (T + 31) / 32;
+    pdl_wait();
+    pdl_trigger();
     for (int i = threadIdx.x; i < E * words; i += kSmallThreads) s_mask[i] = 0;
     for (int e = threadIdx.x; e < E; e += kSmallThreads) s_cnt[e] = 0;
     for (int i = threadIdx.x; i < a.n_zero; i += kSmallThreads) a.zero_words[i] = 0;
@@ -255,26 +259,21 @@ cudaError_t launch_router_logits_split(const void* hidden, const void* router_w,
     const bool small = T <= kSplitTokens;
     const int epb = small ? 1 : 4;
     dim3 grid((E + epb - 1) / epb, (T + kSplitTokens - 1) / kSplitTokens);
-    if (bf16) {
-        if (small)
-            router_logits_split_kernel<true, 1><<<grid, kSplitThreads, 0, s>>>(hidden, router_w, T, H, E, logits, clear_words);
-        else
-            router_logits_split_kernel<true, 4><<<grid, kSplitThreads, 0, s>>>(hidden, router_w, T, H, E, logits, clear_words);
-    } else {
-        if (small)
-            router_logits_split_kernel<false, 1><<<grid, kSplitThreads, 0, s>>>(hidden, router_w, T, H, E, logits, clear_words);
-        else
-            router_logits_split_kernel<false, 4><<<grid, kSplitThreads, 0, s>>>(hidden, router_w, T, H, E, logits, clear_words);
-    }
-    count_launch();
-    return cudaGetLastError();
+    const dim3 block(kSplitThreads);
+    if (bf16)
+        return small ? launch_k(router_logits_split_kernel<true, 1>, grid, block, 0, s, hidden,
+                                router_w, T, H, E, logits, clear_words)
+                     : launch_k(router_logits_split_kernel<true, 4>, grid, block, 0, s, hidden,
+                                router_w, T, H, E, logits, clear_words);
+    return small ? launch_k(router_logits_split_kernel<false, 1>, grid, block, 0, s, hidden,
+                            router_w, T, H, E, logits, clear_words)
+                 : launch_k(router_logits_split_kernel<false, 4>, grid, block, 0, s, hidden,
+                            router_w, T, H, E, logits, clear_words);
 }
 
 cudaError_t launch_route_small(const RouteSmallArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    route_small_kernel<<<1, kSmallThreads, 0, s>>>(a);
-    count_launch();
-    return cudaGetLastError();
+    return launch_k(route_small_kernel, dim3(1), dim3(kSmallThreads), 0, s, a);
 }
 
 }  // namespace moe
