@@ -72,8 +72,8 @@ typedef struct { float alpha, beta, limit; } moe_swiglu;
  * arithmetic, no CUDA call).  Returns 0 for invalid sizes. */
 size_t moe_workspace_size(int T, int H, int E, int k, int I, moe_dtype dt);
 
-/* Bytes of scratch that moe_permute needs (tile histograms and a completion
- * counter).  Returns 0 for invalid sizes. */
+/* Bytes of scratch that moe_permute needs (the expert counts of every 128-token
+ * tile).  Returns 0 for invalid sizes. */
 size_t moe_permute_workspace_size(int T, int E);
 
 /* Bytes of scratch that moe_expert_ffn needs (the activation rows [rows, I]). */

@@ -58,8 +58,8 @@ struct Carver {
 };
 
 struct FwdLayout {
-    size_t hdr, logits, idx, w, near, tile_counts, tile_base, counts, offsets, perm_src, perm_dst,
-        ctr, x_perm, act, y, total;
+    size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, ctr, x_perm,
+        act, y, total;
 };
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
@@ -70,18 +70,19 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     const size_t nt = static_cast<size_t>(num_token_tiles(T));
     Carver c;
     FwdLayout L;
-    L.hdr = c.take(kAlign);   // [0] error word, [1] completion counter
+    // the header, the decode FFN's counters and the tile counts come first: one memset
+    // clears them
+    L.hdr = c.take(kAlign);   // [0] error word
+    L.ctr = c.take(static_cast<size_t>(decode_ffn_counters(static_cast<int>(rows), E)) * 4);
+    L.tile_counts = c.take(nt * E * 4);
     L.logits = c.take(static_cast<size_t>(T) * E * 4);
     L.idx = c.take(rows * 4);
     L.w = c.take(rows * 4);
     L.near = c.take(static_cast<size_t>(T) * 4);
-    L.tile_counts = c.take(nt * E * 4);
-    L.tile_base = c.take(nt * E * 4);
     L.counts = c.take(static_cast<size_t>(E) * 4);
     L.offsets = c.take(static_cast<size_t>(E + 1) * 4);
     L.perm_src = c.take(rows * 4);
     L.perm_dst = c.take(rows * 4);
-    L.ctr = c.take(static_cast<size_t>(decode_ffn_counters(static_cast<int>(rows), E)) * 4);
     L.x_perm = c.take(rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
@@ -90,7 +91,7 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
 }
 
 struct PermLayout {
-    size_t hdr, tile_counts, tile_base, total;
+    size_t hdr, tile_counts, total;
 };
 
 PermLayout perm_layout(int T, int E) {
@@ -99,7 +100,6 @@ PermLayout perm_layout(int T, int E) {
     PermLayout L;
     L.hdr = c.take(kAlign);
     L.tile_counts = c.take(nt * E * 4);
-    L.tile_base = c.take(nt * E * 4);
     L.total = c.off;
     return L;
 }
@@ -123,15 +123,18 @@ bool standard_swiglu(const moe_swiglu& a) {
 // Which kernels moe_forward runs for these sizes (bits of moe_forward_path).
 constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
               kPathF32Ffn = 16;
+// Up to this many tokens a bf16 batch is routed by the split router + one CTA; above
+// it, by the tensor-core router with the routing in its epilogue.
+constexpr int kRouteSmallTcT = 16;
 
 int forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
     const bool bf16 = dt == MOE_BF16;
     const int rows = T * k;
     int path = 0;
-    if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) path |= kPathSmallRoute;
-    else if (bf16 && tc_router_supported(T, H, E)) path |= kPathTcRouter;
+    if (bf16 && T > kRouteSmallTcT && tc_route_supported(H, E, k)) path |= kPathTcRouter;
+    else if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) path |= kPathSmallRoute;
     if (!bf16) path |= kPathF32Ffn;
-    else if ((path & kPathSmallRoute) && decode_ffn_supported(rows, E, H, I)) path |= kPathDecodeFfn;
+    else if (decode_ffn_supported(rows, E, H, I)) path |= kPathDecodeFfn;
     else path |= kPathTokenGemm;
     return path;
 }
@@ -217,10 +220,12 @@ moe_status moe_route(const void* hidden, const void* router_w, const float* rout
         (near_tie && !aligned(near_tie, 4)))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dt == MOE_BF16 && tc_router_supported(T, H, E))
-        MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, nullptr, s));
-    else
-        MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, dt == MOE_BF16, logits, s));
+    if (dt == MOE_BF16 && T > kRouteSmallTcT && tc_route_supported(H, E, k))
+        return launch_route_tc(hidden, router_w, router_bias, T, H, E, k, normalize, topk_idx,
+                               topk_w, near_tie, logits, nullptr, nullptr, s) == cudaSuccess
+                   ? MOE_OK
+                   : MOE_ERR_CUDA;
+    MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, dt == MOE_BF16, logits, s));
     TopkHistArgs a;
     a.logits = logits;
     a.bias = router_bias;
@@ -232,7 +237,6 @@ moe_status moe_route(const void* hidden, const void* router_w, const float* rout
     a.topk_idx = topk_idx;
     a.topk_w = topk_w;
     a.near_tie = near_tie;
-    a.do_hist = false;
     MOE_CUDA(launch_topk_hist(a, s));
     return MOE_OK;
 }
@@ -252,27 +256,21 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
     if (ws_bytes < L.total) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
-    int32_t* done = reinterpret_cast<int32_t*>(ws + L.hdr);
     if (T == 0) {
         MOE_CUDA(cudaMemsetAsync(counts, 0, static_cast<size_t>(E) * 4, s));
         MOE_CUDA(cudaMemsetAsync(offsets, 0, static_cast<size_t>(E + 1) * 4, s));
         return MOE_OK;
     }
-    MOE_CUDA(cudaMemsetAsync(done, 0, 4, s));
     TopkHistArgs a;
     a.T = T;
     a.E = E;
     a.k = k;
     a.topk_idx = const_cast<int32_t*>(topk_idx);
-    a.do_hist = true;
     a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
-    a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
-    a.counts = counts;
-    a.offsets = offsets;
-    a.done = done;
     a.err = err_word;
     MOE_CUDA(launch_topk_hist(a, s));
-    MOE_CUDA(launch_scatter(topk_idx, a.tile_base, T, E, k, perm_src, perm_dst, err_word, s));
+    MOE_CUDA(launch_scatter(topk_idx, a.tile_counts, T, E, k, counts, offsets, perm_src, perm_dst,
+                            err_word, s));
     if (x_perm)
         MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, T * k, H, static_cast<int>(elem_size(dt)),
                                x_perm, s));
@@ -349,7 +347,6 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     int32_t* err = reinterpret_cast<int32_t*>(ws + L.hdr);
-    int32_t* done = err + 1;
     float* logits = reinterpret_cast<float*>(ws + L.logits);
     int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
     float* w = reinterpret_cast<float*>(ws + L.w);
@@ -392,32 +389,32 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         MOE_CUDA(launch_route_small(a, s));
         record(1, s);
     } else {
-        MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, kAlign, s));
-        // route: logits, then top-k + softmax + bincount + scan in one kernel
-        if (path & kPathTcRouter)
-            MOE_CUDA(launch_router_tc(hidden, router_w, T, H, E, logits, err, s));
-        else
+        // the header, the decode FFN's counters and the tile counts start at zero
+        MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, L.logits - L.hdr, s));
+        int32_t* tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
+        if (path & kPathTcRouter) {
+            // logits on the tensor cores, routing and per-tile bincount in the epilogue
+            MOE_CUDA(launch_route_tc(hidden, router_w, router_bias, T, H, E, k, normalize, idx, w,
+                                     near, nullptr, tile_counts, err, s));
+        } else {
             MOE_CUDA(launch_router_logits_simt(hidden, router_w, T, H, E, bf16, logits, s));
-        TopkHistArgs a;
-        a.logits = logits;
-        a.bias = router_bias;
-        a.T = T;
-        a.E = E;
-        a.k = k;
-        a.normalize = normalize ? 1 : 0;
-        a.topk_idx = idx;
-        a.topk_w = w;
-        a.near_tie = near;
-        a.do_hist = true;
-        a.tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
-        a.tile_base = reinterpret_cast<int32_t*>(ws + L.tile_base);
-        a.counts = counts;
-        a.offsets = offsets;
-        a.done = done;
-        a.err = err;
-        MOE_CUDA(launch_topk_hist(a, s));
+            TopkHistArgs a;
+            a.logits = logits;
+            a.bias = router_bias;
+            a.T = T;
+            a.E = E;
+            a.k = k;
+            a.normalize = normalize ? 1 : 0;
+            a.topk_idx = idx;
+            a.topk_w = w;
+            a.near_tie = near;
+            a.tile_counts = tile_counts;
+            a.err = err;
+            MOE_CUDA(launch_topk_hist(a, s));
+        }
         record(1, s);
-        MOE_CUDA(launch_scatter(idx, a.tile_base, T, E, k, perm_src, perm_dst, err, s));
+        MOE_CUDA(launch_scatter(idx, tile_counts, T, E, k, counts, offsets, perm_src, perm_dst,
+                                err, s));
     }
     if (path & kPathDecodeFfn) {
         // fc1 + SwiGLU and fc2 in one launch.  With at most 4 rows per expert on

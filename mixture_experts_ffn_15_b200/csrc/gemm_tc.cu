@@ -48,11 +48,13 @@ constexpr int kTokChunk = 64;        // weight-M: tokens per unit
 constexpr int kBoxTok = 16;          // weight-M: token rows per TMA box
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-enum Mode : int { TOK_SWIGLU = 0, TOK_PLAIN = 1, TOK_F32 = 2, W_SWIGLU = 3, W_PLAIN = 4 };
+// TOK_ROUTE: router logits with the routing itself in the epilogue (top-k, softmax,
+// near-tie flags, per-tile bincount).
+enum Mode : int { TOK_SWIGLU = 0, TOK_PLAIN = 1, W_PLAIN = 4, TOK_ROUTE = 5 };
 
 template <int MODE, int BN>
 struct Tr {
-    static constexpr bool kWeightM = (MODE == W_SWIGLU || MODE == W_PLAIN);
+    static constexpr bool kWeightM = (MODE == W_PLAIN);
     static constexpr int kBRows = kWeightM ? kTokChunk : BN;
     static constexpr int kABytes = BM * BK * 2;
     static constexpr int kBBytes = kBRows * BK * 2;
@@ -64,7 +66,8 @@ struct Tr {
     static constexpr int kUnitRows = kWeightM ? kTokChunk : BM;
     // barriers, tmem slot + abort flag, offsets, prefix, gather rows of one chunk
     static constexpr int kMiscBytes =
-        (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 16 * 8 + 64;
+        (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 16 * 8 + 64 +
+        (MODE == TOK_ROUTE ? 5 * kMaxExperts * 4 : 0);   // bias [E], counts [4][E]
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     static_assert(kWeightM || (BN % 16 == 0 && BN >= 16 && BN <= 256), "UMMA N");
@@ -79,6 +82,17 @@ struct TcParams {
     void* out;
     int ldo;                  // output row stride, elements
     int32_t* err;
+};
+
+// The routing half of TOK_ROUTE (n_out = number of experts).
+struct RouteParams {
+    const float* bias;        // [E] or nullptr
+    int k, normalize;
+    int32_t* topk_idx;        // [T, k]
+    float* topk_w;            // [T, k]
+    int32_t* near_tie;        // [T] or nullptr
+    float* logits;            // [T, E] or nullptr (logits + bias)
+    int32_t* tile_counts;     // [ceil(T / 128), E]
 };
 
 struct Unit {
@@ -170,10 +184,112 @@ __device__ __forceinline__ Unit decode_unit(int u, int per_unit, int G, int unit
 
 __device__ __forceinline__ float f32(uint32_t x) { return __uint_as_float(x); }
 
-template <int MODE, int BN>
+// Routing of one 128-token tile from its logits in TMEM (columns 0..E-1, thread =
+// token row).  Each thread keeps the KS = k+1 (or more) largest biased logits in a
+// register list sorted descending, inserting the experts in index order so that equal
+// logits keep the lower index first; then the softmax weights over the chosen k (or,
+// normalize = 0, over all E), the near-tie flags, and the tile's bincount: per warp in
+// shared memory (s_cnt is this warp's [E] slice), then added to tile_counts.
+template <int E, int KS>
+__device__ __forceinline__ void route_epilogue(uint32_t tb, bool valid, size_t row, int tile,
+                                               const RouteParams& rp, const float* s_bias,
+                                               int* s_cnt, int lane) {
+    const int k = rp.k;
+    float vals[KS];
+    int ids[KS];
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        vals[j] = -INFINITY;
+        ids[j] = -1;
+    }
+#pragma unroll 1
+    for (int c = 0; c < E; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tb + c, v);
+        tmem_wait_ld();
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = f32(v[i]) + s_bias[c + i];
+        if (valid && rp.logits) {
+            uint4* dst = reinterpret_cast<uint4*>(rp.logits + row * E + c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                dst[q] = make_uint4(__float_as_uint(x[4 * q]), __float_as_uint(x[4 * q + 1]),
+                                    __float_as_uint(x[4 * q + 2]), __float_as_uint(x[4 * q + 3]));
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float xv = x[i];
+            if (xv > vals[KS - 1]) {
+                const int e = c + i;
+#pragma unroll
+                for (int j = KS - 1; j >= 0; --j) {
+                    if (vals[j] < xv) {
+                        if (j == 0 || vals[j - 1] >= xv) {
+                            vals[j] = xv;
+                            ids[j] = e;
+                        } else {
+                            vals[j] = vals[j - 1];
+                            ids[j] = ids[j - 1];
+                        }
+                    }
+                }
+            }
+        }
+    }
+    // rows past the batch hold bias-only logits (their A rows were zero-filled): finite
+    const float vmax = vals[0];
+    float den = 0.f;
+    if (rp.normalize) {
+#pragma unroll
+        for (int j = 0; j < KS; ++j)
+            if (j < k) den += expf(vals[j] - vmax);
+    } else {
+        // softmax over all E: a second, warp-uniform pass over the logits in TMEM
+#pragma unroll 1
+        for (int c = 0; c < E; c += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tb + c, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) den += expf(f32(v[i]) + s_bias[c + i] - vmax);
+        }
+    }
+    if (valid) {
+        int flags = 0;
+        float kth = 0.f, next = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+            if (j < k) {
+                rp.topk_idx[row * k + j] = ids[j];
+                rp.topk_w[row * k + j] = expf(vals[j] - vmax) / den;
+                atomicAdd(&s_cnt[ids[j]], 1);
+                if (j + 1 < k && vals[j] - vals[j + 1] < kNearTieGap) flags |= 2;
+            }
+            if (j == k - 1) kth = vals[j];
+            if (j == k) next = vals[j];
+        }
+        if (k < E && kth - next < kNearTieGap) flags |= 1;
+        if (rp.near_tie) rp.near_tie[row] = flags;
+    }
+    // this warp's 32 rows: add its counts to the tile's (zeroed before the launch) and
+    // clear them for the next tile; warp-local, so a warp that gave up on a wait never
+    // holds the others at a barrier
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) {
+        const int c = s_cnt[e];
+        if (c) {
+            if (rp.tile_counts) atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + e], c);
+            s_cnt[e] = 0;
+        }
+    }
+    __syncwarp();
+}
+
+template <int MODE, int BN, int KS = 1>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const TcParams p) {
+               const TcParams p, const RouteParams rp) {
     using C = Tr<MODE, BN>;
     static_assert(!C::kWeightM, "weight rows on M run in tc_ffn_decode_kernel");
     extern __shared__ uint8_t smem_raw[];
@@ -189,6 +305,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
     int* s_pre = s_off + (kMaxExperts + 1);
+    float* s_bias = reinterpret_cast<float*>(s_pre + (kMaxExperts + 1));   // TOK_ROUTE
+    int* s_cnt = reinterpret_cast<int*>(s_bias + kMaxExperts);            // TOK_ROUTE
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.offsets ? p.E : 1;
@@ -217,6 +335,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     pdl_wait();
     pdl_trigger();
     if (warp == 2) build_tile_map(p, G, C::kUnitRows, s_off, s_pre, lane);
+    if constexpr (MODE == TOK_ROUTE) {
+        for (int e = threadIdx.x; e < BN; e += kThreads) s_bias[e] = rp.bias ? rp.bias[e] : 0.f;
+        for (int e = threadIdx.x; e < 4 * BN; e += kThreads) s_cnt[e] = 0;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -315,6 +437,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const bool valid = r < t.nrows;
             const size_t orow = static_cast<size_t>(t.row0 + r);
             const int col0 = t.sub * BN;
+            if constexpr (MODE == TOK_ROUTE) {
+                route_epilogue<BN, KS>(tb, valid, orow, t.row0 / BM, rp, s_bias,
+                                       s_cnt + quad * BN, lane);
+            } else {
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t v[32];
@@ -345,13 +471,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                             dst[q] = pack_bf16x8(f);
                         }
                     }
-                } else {   // TOK_F32
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.out) +
-                                                          orow * p.ldo + col0 + c);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        if (4 * q < nv) dst[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();
@@ -790,11 +911,11 @@ bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, int box_ro
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int KS = 1>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int bound,
-                       cudaStream_t s) {
+                       cudaStream_t s, const RouteParams& rp = RouteParams{}) {
     using C = Tr<MODE, BN>;
-    auto kern = tc_gemm_kernel<MODE, BN>;
+    auto kern = tc_gemm_kernel<MODE, BN, KS>;
     // once per device (outside any stream capture: the first call of every path
     // runs eagerly before a graph is captured)
     static bool attr_set[64] = {false};
@@ -809,7 +930,7 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParam
     int grid = device_sm_count();
     if (bound < grid) grid = bound;
     if (grid <= 0) return cudaSuccess;
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p);
+    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p, rp);
 }
 
 int pick_bn(int n_out) {
@@ -876,8 +997,34 @@ cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUt
 
 bool tc_ffn_supported(int H, int I) { return H % 64 == 0 && I % 64 == 0 && H > 0 && I > 0; }
 
-bool tc_router_supported(int T, int H, int E) {
-    return T >= 512 && H % 64 == 0 && (E == 64 || E == 128 || E == 256);
+bool tc_route_supported(int H, int E, int k) {
+    return H % 64 == 0 && (E == 64 || E == 128 || E == 256) && k >= 1 && k <= 32;
+}
+
+cudaError_t launch_route_tc(const void* hidden, const void* router_w, const float* bias, int T,
+                            int H, int E, int k, int normalize, int32_t* topk_idx, float* topk_w,
+                            int32_t* near_tie, float* logits, int32_t* tile_counts, int32_t* err,
+                            cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    TcParams p{nullptr, 1, T, H, E, nullptr, E, err};
+    RouteParams rp{bias, k, normalize ? 1 : 0, topk_idx, topk_w, near_tie, logits, tile_counts};
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
+    const int bound = (T + BM - 1) / BM;
+    const bool small_k = k <= 8;
+#define MOE_ROUTE_CASE(EV)                                                                   \
+    case EV:                                                                                 \
+        return small_k ? launch_one<TOK_ROUTE, EV, 9>(ma, mb, p, bound, s, rp)               \
+                       : launch_one<TOK_ROUTE, EV, 33>(ma, mb, p, bound, s, rp);
+    switch (E) {
+        MOE_ROUTE_CASE(64)
+        MOE_ROUTE_CASE(128)
+        MOE_ROUTE_CASE(256)
+        default:
+            return cudaErrorInvalidValue;
+    }
+#undef MOE_ROUTE_CASE
 }
 
 cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
@@ -920,21 +1067,6 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     const int grid = decode_grid(rows, E, H, I);
     return perm_src ? launch_decode<true>(w1, x, w2, a, p, grid, s)
                     : launch_decode<false>(w1, x, w2, a, p, grid, s);
-}
-
-cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,
-                             float* logits, int32_t* err, cudaStream_t s) {
-    TcParams p{nullptr, 1, T, H, E, logits, E, err};
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
-    const int bound = (T + BM - 1) / BM;
-    switch (E) {
-        case 64: return launch_one<TOK_F32, 64>(ma, mb, p, bound, s);
-        case 128: return launch_one<TOK_F32, 128>(ma, mb, p, bound, s);
-        case 256: return launch_one<TOK_F32, 256>(ma, mb, p, bound, s);
-        default: return cudaErrorInvalidValue;
-    }
 }
 
 }  // namespace moe

@@ -49,12 +49,7 @@ struct TopkHistArgs {
     int32_t* topk_idx = nullptr;     // [T, k] out (or in when logits == nullptr)
     float* topk_w = nullptr;         // [T, k] out
     int32_t* near_tie = nullptr;     // [T] out or nullptr
-    bool do_hist = false;
-    int32_t* tile_counts = nullptr;  // [ntiles, E] scratch
-    int32_t* tile_base = nullptr;    // [ntiles, E] out: first permuted row of (tile, e)
-    int32_t* counts = nullptr;       // [E] out
-    int32_t* offsets = nullptr;      // [E + 1] out
-    int32_t* done = nullptr;         // completion counter, 0 on entry, 0 on exit
+    int32_t* tile_counts = nullptr;  // [ntiles, E] out (nullptr: no histogram)
     int32_t* err = nullptr;          // device error word
 };
 cudaError_t launch_topk_hist(const TopkHistArgs& a, cudaStream_t s);
@@ -86,8 +81,10 @@ struct RouteSmallArgs {
 cudaError_t launch_route_small(const RouteSmallArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- permute.cu
-cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
-                           int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s);
+// counts [E], offsets [E+1], perm_src, perm_dst from topk_idx and the per-tile counts
+cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, int T, int E,
+                           int k, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                           int32_t* perm_dst, int32_t* err, cudaStream_t s);
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
                           int E, int T, int rows_max, int H, int elem_bytes, void* x_perm,
                           cudaStream_t s);
@@ -105,12 +102,16 @@ cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, con
 
 // ---------------------------------------------------------------- gemm_tc.cu
 bool tc_ffn_supported(int H, int I);
-bool tc_router_supported(int T, int H, int E);
 cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
                           const void* fc2, int rows, int H, int E, int I, void* act, void* y,
                           int32_t* err, cudaStream_t s, cudaEvent_t mid);
-cudaError_t launch_router_tc(const void* hidden, const void* router_w, int T, int H, int E,
-                             float* logits, int32_t* err, cudaStream_t s);
+// Router logits on the tensor cores with the routing in the epilogue: top-k, softmax
+// weights, near-tie flags and the per-128-token-tile bincount (logits optional).
+bool tc_route_supported(int H, int E, int k);
+cudaError_t launch_route_tc(const void* hidden, const void* router_w, const float* bias, int T,
+                            int H, int E, int k, int normalize, int32_t* topk_idx, float* topk_w,
+                            int32_t* near_tie, float* logits, int32_t* tile_counts, int32_t* err,
+                            cudaStream_t s);
 
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);

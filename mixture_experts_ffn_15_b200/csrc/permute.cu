@@ -4,10 +4,9 @@
 //   offsets[e] + #{t' < t : some slot of t' chose e}
 // i.e. the rows of an expert are contiguous and ordered by token (the grouped
 // matmul of grouped_mm_experts_forward, "Contributing Gemma 4 support and ONNX
-// export optimizations", "Key Technical Contributions").  Each 128-token tile knows
-// the first row of every expert from the histogram kernel; inside the tile the rank
-// of a token among the tile's tokens of the same expert is a population count over
-// a 128-bit membership mask held in shared memory, so the result is deterministic.
+// export optimizations", "Key Technical Contributions"), and the offsets are the
+// exclusive scan of the per-expert bincount.  The inputs are the per-128-token-tile
+// expert counts; the result is unique and deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -17,18 +16,86 @@ namespace {
 constexpr int kScatterThreads = 512;
 constexpr int kMaskWords = kTileTokens / 32;
 
+// One block per 128-token tile.  The block first turns the per-tile expert counts of
+// ALL tiles (tile_counts [ntiles, E], a few KB from L2) into what it needs: the
+// per-expert totals, their exclusive scan (the offsets; block 0 writes counts and
+// offsets) and, for its own tile, the first row of every expert:
+//   base[e] = offsets[e] + sum over earlier tiles of tile_counts[tile', e].
+// Every block does this small reduction itself, so no block waits for another.
+// Then the rank of a token among the tile's tokens of the same expert is a population
+// count over a 128-bit membership mask.
 __global__ void __launch_bounds__(kScatterThreads)
-scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ tile_base, int T,
-               int E, int k, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_dst,
+scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ tile_counts,
+               int T, int E, int k, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+               int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_dst,
                int32_t* __restrict__ err) {
     __shared__ uint32_t s_mask[kMaxExperts * kMaskWords];
+    __shared__ int s_tot[kScatterThreads];
+    __shared__ int s_before[kScatterThreads];
+    __shared__ int s_base[kMaxExperts];
     pdl_wait();
     pdl_trigger();
     const int tile = blockIdx.x;
+    const int ntiles = gridDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t_begin = tile * kTileTokens;
     const int nt = min(kTileTokens, T - t_begin);
     for (int i = threadIdx.x; i < E * kMaskWords; i += kScatterThreads) s_mask[i] = 0;
+
+    // ---- totals and earlier-tile sums per expert: thread (strip, e)
+    const int strips = kScatterThreads / E;   // E <= 256: at least 2
+    const int chunk = (ntiles + strips - 1) / strips;
+    const int st = threadIdx.x / E, e_own = threadIdx.x - st * E;
+    int tot = 0, before = 0;
+    if (st < strips) {
+        const int i0 = st * chunk, i1 = min(ntiles, i0 + chunk);
+#pragma unroll 8
+        for (int i = i0; i < i1; ++i) {
+            const int c = tile_counts[static_cast<size_t>(i) * E + e_own];
+            tot += c;
+            before += (i < tile) ? c : 0;
+        }
+    }
+    s_tot[threadIdx.x] = tot;
+    s_before[threadIdx.x] = before;
     __syncthreads();
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        int loc[kMaxExperts / 32];
+        int lsum = 0;
+        for (int q = 0; q < per; ++q) {
+            const int e = lane * per + q;
+            int t = 0;
+            if (e < E)
+                for (int ss = 0; ss < strips; ++ss) t += s_tot[ss * E + e];
+            loc[q] = t;
+            lsum += t;
+        }
+        int incl = lsum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        int run = incl - lsum;
+        for (int q = 0; q < per; ++q) {
+            const int e = lane * per + q;
+            if (e < E) {
+                int b = run;
+                for (int ss = 0; ss < strips; ++ss) b += s_before[ss * E + e];
+                s_base[e] = b;
+                if (tile == 0) {
+                    offsets[e] = run;
+                    counts[e] = loc[q];
+                }
+            }
+            run += loc[q];
+        }
+        if (tile == 0 && lane == 31) offsets[E] = incl;
+    }
+    __syncthreads();
+
+    // ---- membership masks, then ranks
     const int npairs = nt * k;
     const int32_t* ids = topk_idx + static_cast<size_t>(t_begin) * k;
     for (int p = threadIdx.x; p < npairs; p += kScatterThreads) {
@@ -50,7 +117,7 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
             const int w = tl >> 5;
             int rank = __popc(m[w] & ((1u << (tl & 31)) - 1u));
             for (int q = 0; q < w; ++q) rank += __popc(m[q]);
-            row = tile_base[static_cast<size_t>(tile) * E + e] + rank;
+            row = s_base[e] + rank;
             perm_src[row] = t_begin + tl;
         }
         perm_dst[static_cast<size_t>(t_begin) * k + p] = row;
@@ -83,11 +150,12 @@ gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm
 
 }  // namespace
 
-cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_base, int T, int E, int k,
-                           int32_t* perm_src, int32_t* perm_dst, int32_t* err, cudaStream_t s) {
+cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, int T, int E,
+                           int k, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                           int32_t* perm_dst, int32_t* err, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     return launch_k(scatter_kernel, dim3(num_token_tiles(T)), dim3(kScatterThreads), 0, s, topk_idx,
-                    tile_base, T, E, k, perm_src, perm_dst, err);
+                    tile_counts, T, E, k, counts, offsets, perm_src, perm_dst, err);
 }
 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,

@@ -9,10 +9,8 @@
 //
 // "Contributing Gemma 4 support and ONNX export optimizations", "Key Technical
 // Contributions": the per-expert token count is a bincount over the chosen ids.
-// topk_hist_kernel computes it per 128-token tile; the last tile to finish turns
-// the tile counts into the per-expert totals, the exclusive offsets and, per
-// (tile, expert), the first permuted row, which the scatter kernel uses to place
-// every (token, slot) pair stably.
+// topk_hist_kernel computes it per 128-token tile; the scatter kernel turns the
+// tile counts into totals, offsets and per-tile bases.
 #include <math.h>
 
 #include "common.cuh"
@@ -98,9 +96,6 @@ __global__ void __launch_bounds__(kHistThreads) topk_hist_kernel(const TopkHistA
     __shared__ float s_val[kHistWarps][kMaxExperts + 1];
     __shared__ int s_sel[kHistWarps][kMaxExperts + 1];
     __shared__ int s_cnt[kMaxExperts];
-    __shared__ int s_strip[kHistThreads];
-    __shared__ int s_off[kMaxExperts + 1];
-    __shared__ int s_last;
     pdl_wait();
     pdl_trigger();
 
@@ -181,7 +176,7 @@ __global__ void __launch_bounds__(kHistThreads) topk_hist_kernel(const TopkHistA
             __syncwarp();
         }
     }
-    if (!a.do_hist) return;
+    if (a.tile_counts == nullptr) return;
 
     // ---- phase B: bincount of this tile's expert ids
     __syncthreads();   // this block's topk_idx writes are visible to the block
@@ -199,65 +194,6 @@ __global__ void __launch_bounds__(kHistThreads) topk_hist_kernel(const TopkHistA
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += kHistThreads)
         a.tile_counts[static_cast<size_t>(tile) * E + e] = s_cnt[e];
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = (atomicAdd(a.done, 1) == static_cast<int>(gridDim.x) - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-
-    // ---- last tile: per-expert totals, offsets, first row of every (tile, expert)
-    const int ntiles = gridDim.x;
-    const int strips = kHistThreads / E;   // E <= 256, so at least 2
-    const int chunk = (ntiles + strips - 1) / strips;
-    const int s = threadIdx.x / E, e = threadIdx.x - (threadIdx.x / E) * E;
-    const bool active = s < strips;
-    const int i0 = s * chunk, i1 = min(ntiles, i0 + chunk);
-    int sum = 0;
-    if (active)
-        for (int i = i0; i < i1; ++i) sum += __ldcg(&a.tile_counts[static_cast<size_t>(i) * E + e]);
-    s_strip[threadIdx.x] = sum;
-    __syncthreads();
-    if (warp == 0) {
-        const int per = (E + 31) / 32;
-        int loc[kLanesVals];
-        int lsum = 0;
-        for (int q = 0; q < per; ++q) {
-            const int ee = lane * per + q;
-            int tot = 0;
-            if (ee < E)
-                for (int ss = 0; ss < strips; ++ss) tot += s_strip[ss * E + ee];
-            loc[q] = tot;
-            lsum += tot;
-        }
-        int incl = lsum;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += y;
-        }
-        int run = incl - lsum;
-        for (int q = 0; q < per; ++q) {
-            const int ee = lane * per + q;
-            if (ee < E) {
-                s_off[ee] = run;
-                a.offsets[ee] = run;
-                a.counts[ee] = loc[q];
-            }
-            run += loc[q];
-        }
-        if (lane == 31) a.offsets[E] = incl;
-    }
-    __syncthreads();
-    if (active) {
-        int run = s_off[e];
-        for (int ss = 0; ss < s; ++ss) run += s_strip[ss * E + e];
-        for (int i = i0; i < i1; ++i) {
-            a.tile_base[static_cast<size_t>(i) * E + e] = run;
-            run += __ldcg(&a.tile_counts[static_cast<size_t>(i) * E + e]);
-        }
-    }
-    if (threadIdx.x == 0) *a.done = 0;   // ready for the next call
 }
 
 }  // namespace

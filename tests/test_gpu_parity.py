@@ -35,6 +35,10 @@ CASES = [
     W("bf16_weightM", T=40, H=256, E=16, k=4, I=192),
     W("bf16_weightM_skew", T=100, H=256, E=8, k=2, I=128, router_bias_std=1.0),
     W("bf16_router_tc", T=600, H=256, E=64, k=4, I=128),
+    W("bf16_router_tc_k16_E256", T=150, H=128, E=256, k=16, I=64),
+    W("bf16_router_tc_norm0_bias", T=300, H=192, E=128, k=6, I=64, normalize=0,
+      router_bias_std=0.5),
+    W("bf16_router_tc_T17", T=17, H=64, E=64, k=8, I=64),
     W("bf16_k1", T=130, H=128, E=8, k=1, I=64),
     W("bf16_k_eq_E", T=20, H=128, E=4, k=4, I=64),
     W("bf16_T1", T=1, H=128, E=8, k=2, I=64),
