@@ -408,6 +408,11 @@ def run_ours(args):
     comb_bytes = wl.T * wl.k * wl.H * es + wl.T * wl.H * es
     dom = {"bytes": fc1_work["bytes"] + fc2_work["bytes"] + comb_bytes,
            "flops": fc1_work["flops"] + fc2_work["flops"]} if fused else fc1_work
+    one_launch = bool(path & 32)
+    if one_launch:
+        # ... and the routing: router weights and the token rows, the logits
+        dom = {"bytes": dom["bytes"] + wl.E * wl.H * es + wl.T * wl.H * es + wl.T * wl.E * 4,
+               "flops": dom["flops"] + 2.0 * wl.T * wl.H * wl.E}
 
     peaks, peak_kind = load_peaks()
     hbm = wl.name in HBM_BOUND
@@ -418,7 +423,9 @@ def run_ours(args):
         achieved = dom["flops"] / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = ("tc_ffn_decode_kernel (fc1 + SwiGLU, fc2 and combine, weight rows on M)" if fused else
+    roof["kernel"] = ("tc_ffn_decode_kernel<ROUTE> (routing, fc1 + SwiGLU, fc2 and combine, weight rows on M)"
+                      if one_launch else
+                      "tc_ffn_decode_kernel (fc1 + SwiGLU, fc2 and combine, weight rows on M)" if fused else
                       "tc_gemm_kernel<TOK_SWIGLU> (fc1 + SwiGLU, token rows on M)")
     roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if hbm else 'bf16_tflops, burst'})"
     roof["algorithmic_per_launch"] = dom["bytes"] if hbm else dom["flops"]

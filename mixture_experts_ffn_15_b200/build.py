@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["api.cu", "route.cu", "route_small.cu", "permute.cu", "combine.cu", "ffn_simt.cu",
            "gemm_tc.cu", "static_scratch.cu"]
-HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
+HEADERS = ["common.cuh", "sm100.cuh", "kernels.h", "combine.cuh", "topk_warp.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

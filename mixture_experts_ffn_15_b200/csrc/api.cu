@@ -122,7 +122,7 @@ bool standard_swiglu(const moe_swiglu& a) {
 
 // Which kernels moe_forward runs for these sizes (bits of moe_forward_path).
 constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
-              kPathF32Ffn = 16;
+              kPathF32Ffn = 16, kPathFusedRoute = 32;
 // Up to this many tokens a bf16 batch is routed by the split router + one CTA; above
 // it, by the tensor-core router with the routing in its epilogue.
 constexpr int kRouteSmallTcT = 16;
@@ -130,6 +130,8 @@ constexpr int kRouteSmallTcT = 16;
 int forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
     const bool bf16 = dt == MOE_BF16;
     const int rows = T * k;
+    // small bf16 batches: the whole layer in one launch
+    if (bf16 && fused_route_supported(T, H, E, k, I)) return kPathFusedRoute | kPathDecodeFfn;
     int path = 0;
     if (bf16 && T > kRouteSmallTcT && tc_route_supported(H, E, k)) path |= kPathTcRouter;
     else if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) path |= kPathSmallRoute;
@@ -364,6 +366,43 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
     record(0, s);
+    if (path & kPathFusedRoute) {
+        // the error word and the counters start at zero; then one launch: routing,
+        // fc1 + SwiGLU, fc2 and the weighted combine
+        MOE_CUDA(launch_clear(ws + L.hdr, L.tile_counts - L.hdr, s));
+        record(1, s);
+        record(2, s);
+        DecodeRoutedArgs a{};
+        a.hidden = hidden;
+        a.router_w = router_w;
+        a.bias = router_bias;
+        a.fc1 = fc1;
+        a.fc2 = fc2;
+        a.T = T;
+        a.H = H;
+        a.E = E;
+        a.k = k;
+        a.I = I;
+        a.normalize = normalize ? 1 : 0;
+        a.logits = logits;
+        a.topk_idx = idx;
+        a.topk_w = w;
+        a.near_tie = near;
+        a.counts = counts;
+        a.offsets = offsets;
+        a.perm_src = perm_src;
+        a.perm_dst = perm_dst;
+        a.act = act_buf;
+        a.y = y;
+        a.counters = ctr;
+        a.err = err;
+        a.out = out;
+        MOE_CUDA(launch_ffn_decode_routed(a, s));
+        record(3, s);
+        record(4, s);
+        record(5, s);
+        return MOE_OK;
+    }
     if (path & kPathSmallRoute) {
         // logits on many CTAs (which also clear the header), then one CTA for top-k,
         // bincount, scan and the stable permutation
@@ -390,7 +429,7 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         record(1, s);
     } else {
         // the header, the decode FFN's counters and the tile counts start at zero
-        MOE_CUDA(cudaMemsetAsync(ws + L.hdr, 0, L.logits - L.hdr, s));
+        MOE_CUDA(launch_clear(ws + L.hdr, L.logits - L.hdr, s));
         int32_t* tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
         if (path & kPathTcRouter) {
             // logits on the tensor cores, routing and per-tile bincount in the epilogue

@@ -74,7 +74,25 @@ convert_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int E, in
     }
 }
 
+// words[0 .. n) = 0 with 16-byte stores (n a multiple of 4, words 16-byte aligned).
+__global__ void __launch_bounds__(256) clear_kernel(uint4* __restrict__ words, int n4) {
+    pdl_wait();
+    pdl_trigger();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
+        words[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 }  // namespace
+
+cudaError_t launch_clear(void* words, size_t bytes, cudaStream_t s) {
+    if (bytes == 0) return cudaSuccess;
+    if ((bytes & 15) != 0 || (reinterpret_cast<uintptr_t>(words) & 15) != 0) return cudaErrorInvalidValue;
+    const long long n4 = static_cast<long long>(bytes / 16);
+    long long blocks = (n4 + 1023) / 1024;
+    if (blocks > device_sm_count()) blocks = device_sm_count();
+    return launch_k(clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                    static_cast<uint4*>(words), static_cast<int>(n4));
+}
 
 cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w,
                            int T, int H, int k, bool bf16, void* out, cudaStream_t s) {

@@ -35,6 +35,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "topk_warp.cuh"
 
 namespace moe {
 namespace {
@@ -103,15 +104,17 @@ struct Unit {
 };
 
 // s_off: sanitised offsets (clamped to [0, rows], non-decreasing); s_pre[g]: first
-// tile of group g; s_pre[G]: tile count.  Runs on one warp.
+// tile of group g; s_pre[G]: tile count.  Runs on one warp; lane l owns the kPer
+// consecutive entries l*kPer ..; every loop has a compile-time trip count, so the
+// per-lane arrays stay in registers.
 __device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int unit_rows, int* s_off,
                                                int* s_pre, int lane) {
     constexpr int kPer = (kMaxExperts + 1 + 31) / 32;   // 9
-    const int per = (G + 1 + 31) / 32;
     int v[kPer];
     bool bad = false;
-    for (int q = 0; q < per; ++q) {
-        const int i = lane * per + q;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int i = lane * kPer + q;
         int raw = p.rows;
         if (i <= G) raw = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows);
         if (i == 0 && p.offsets && raw != 0) bad = true;
@@ -119,13 +122,13 @@ __device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int uni
         if (c != raw) bad = true;
         v[q] = c;
     }
-    for (int q = 1; q < per; ++q)
+#pragma unroll
+    for (int q = 1; q < kPer; ++q)
         if (v[q] < v[q - 1]) {
-            bad = bad || (lane * per + q <= G);
+            bad = bad || (lane * kPer + q <= G);
             v[q] = v[q - 1];
         }
-    const int lmax = v[per - 1];
-    int inc = lmax;
+    int inc = v[kPer - 1];
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, inc, d);
@@ -133,21 +136,24 @@ __device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int uni
     }
     int excl = __shfl_up_sync(0xffffffffu, inc, 1);
     if (lane == 0) excl = 0;
-    for (int q = 0; q < per; ++q) {
-        const int i = lane * per + q;
-        if (v[q] < excl && i <= G) bad = true;
-        const int c = max(v[q], excl);
-        if (i <= G) s_off[i] = c;
-    }
-    if (bad && p.offsets && p.err) atomicOr(p.err, kErrBadExpert);
-    __syncwarp();
-    const int per2 = (G + 31) / 32;
+    // tiles of group g = lane*kPer + q: from the clamped offsets g and g + 1 (the
+    // latter is the next entry, or the first entry of the next lane)
+    const int first_next = __shfl_down_sync(0xffffffffu, max(v[0], excl), 1);
     int cnt[kPer];
     int lsum = 0;
-    for (int q = 0; q < per2; ++q) {
-        const int g = lane * per2 + q;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int i = lane * kPer + q;
+        if (v[q] < excl && i <= G) bad = true;
+        v[q] = max(v[q], excl);
+        if (i <= G) s_off[i] = v[q];
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int g = lane * kPer + q;
+        const int hi = (q + 1 < kPer) ? v[q + 1 < kPer ? q + 1 : q] : first_next;
         int c = 0;
-        if (g < G) c = (s_off[g + 1] - s_off[g] + unit_rows - 1) / unit_rows;
+        if (g < G) c = (hi - v[q] + unit_rows - 1) / unit_rows;
         cnt[q] = c;
         lsum += c;
     }
@@ -158,12 +164,14 @@ __device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int uni
         if (lane >= d) incl += y;
     }
     int run = incl - lsum;
-    for (int q = 0; q < per2; ++q) {
-        const int g = lane * per2 + q;
-        if (g < G) s_pre[g] = run;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int g = lane * kPer + q;
+        if (g <= G) s_pre[g] = run;   // g == G: the tile count
         run += cnt[q];
     }
-    if (lane == 31) s_pre[G] = incl;
+    if (bad && p.offsets && p.err) atomicOr(p.err, kErrBadExpert);
+    __syncwarp();
 }
 
 __device__ __forceinline__ Unit decode_unit(int u, int per_unit, int G, int unit_rows,
@@ -528,7 +536,30 @@ struct DecodeParams {
     int k;
     __nv_bfloat16* out;
     int32_t* err;
+    // ROUTE: the routing runs inside the launch (fields below); offsets, perm_src,
+    // perm_dst and topk_w above are then unused (the kernel keeps them in shared memory)
+    const void* hidden;       // [T, H]
+    const void* router_w;     // [E, H]
+    const float* bias;        // [E] or nullptr
+    int normalize;
+    float* logits;            // [T, E] scratch
+    int32_t* route_bar;       // grid-barrier arrivals, zero on entry
+    // the routing as the staged calls would return it, written by CTA 0
+    int32_t* r_topk_idx;      // [T, k]
+    float* r_topk_w;          // [T, k]
+    int32_t* r_near_tie;      // [T] or nullptr
+    int32_t* r_counts;        // [E]
+    int32_t* r_offsets;       // [E + 1]
+    int32_t* r_perm_src;      // [T k]
+    int32_t* r_perm_dst;      // [T k]
 };
+
+// Shared memory the in-kernel routing keeps for the whole launch (after the misc block).
+constexpr int kRouteSmemBytes =
+    4 * kFusedRouteMaxRows * 4 +                  // ids, weights, perm_dst, perm_src
+    kMaxExperts * 4 + (kMaxExperts + 4) * 4 +     // counts, offsets
+    kMaxExperts * (kFusedRouteMaxT / 32) * 4 +    // token masks per expert
+    (kThreads / 32) * 8 * 4;                      // partial dot products
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     int v;
@@ -586,7 +617,7 @@ __device__ __forceinline__ DUnit decode_dunit(int u, int U1, int MT1, int MT2, i
     return d;
 }
 
-template <bool GATHER>
+template <bool GATHER, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmAct,
@@ -608,6 +639,15 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     int* s_unit = s_pre + (kMaxExperts + 1);                        // [kUnitRing]
     uint64_t* ufull = reinterpret_cast<uint64_t*>(s_unit + 2 * kUnitRing);   // 8-byte aligned
     uint64_t* uempty = ufull + kUnitRing;
+    // ROUTE only: the routing of the whole batch, after the misc block
+    int* s_ridx = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kMiscBytes);
+    float* s_rw = reinterpret_cast<float*>(s_ridx + kFusedRouteMaxRows);
+    int* s_pdst = reinterpret_cast<int*>(s_rw + kFusedRouteMaxRows);
+    int* s_psrc = s_pdst + kFusedRouteMaxRows;
+    int* s_rcnt = s_psrc + kFusedRouteMaxRows;
+    int* s_roff = s_rcnt + kMaxExperts;
+    uint32_t* s_rmask = reinterpret_cast<uint32_t*>(s_roff + kMaxExperts + 4);
+    float* s_red = reinterpret_cast<float*>(s_rmask + kMaxExperts * (kFusedRouteMaxT / 32));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.E;
@@ -640,8 +680,177 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     // the prologue above touches no global memory; everything below may
     pdl_wait();
     pdl_trigger();
+    if constexpr (ROUTE) {
+        // ---------------------------------------------------------------- routing
+        // (1) router logits: CTA c takes experts c, c + grid, ...; its 192 threads
+        //     split H in 16-byte vectors (up to kR1Vec per thread and pass, all loads
+        //     issued before the first product, so a pass costs one memory latency),
+        //     8 tokens at a time; the partial sums are added warp by warp in a fixed
+        //     order.
+        constexpr int kR1Vec = 3;
+        const int T = p.T, E = p.E, k = p.k;
+        const int nv = p.H / 8;
+        const uint4* x4 = reinterpret_cast<const uint4*>(p.hidden);
+        const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+        for (int e = blockIdx.x; e < E; e += gridDim.x) {
+            const uint4* w4 = reinterpret_cast<const uint4*>(p.router_w) + static_cast<size_t>(e) * nv;
+#pragma unroll 1
+            for (int t0 = 0; t0 < T; t0 += 8) {
+                float acc[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+#pragma unroll 1
+                for (int v0 = threadIdx.x; v0 < nv; v0 += kR1Vec * kThreads) {
+                    uint4 wv[kR1Vec], xv[8][kR1Vec];
+#pragma unroll
+                    for (int j = 0; j < kR1Vec; ++j) {
+                        const int v = v0 + j * kThreads;
+                        wv[j] = v < nv ? __ldg(w4 + v) : zero4;
+#pragma unroll
+                        for (int t = 0; t < 8; ++t)
+                            xv[t][j] = (v < nv && t0 + t < T)
+                                           ? __ldg(x4 + static_cast<size_t>(t0 + t) * nv + v)
+                                           : zero4;
+                    }
+#pragma unroll
+                    for (int j = 0; j < kR1Vec; ++j) {
+                        float wf[8];
+                        unpack_bf16x8(wv[j], wf);
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            float xf[8];
+                            unpack_bf16x8(xv[t][j], xf);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[t] = fmaf(xf[i], wf[i], acc[t]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const float sum = warp_sum(acc[t]);
+                    if (lane == 0) s_red[warp * 8 + t] = sum;
+                }
+                __syncthreads();
+                if (threadIdx.x < 8 && t0 + static_cast<int>(threadIdx.x) < T) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kThreads / 32; ++w) sum += s_red[w * 8 + threadIdx.x];
+                    p.logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = sum;
+                }
+                __syncthreads();
+            }
+        }
+        // (2) grid-wide barrier: every CTA of the launch is resident (at most one per
+        //     SM), so the wait ends; it is bounded all the same (abort on expiry).
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(p.route_bar, 1);
+            wait_count(p.route_bar, static_cast<int>(gridDim.x), abort_flag);
+        }
+        __syncthreads();
+        // (3) every CTA selects, counts and places the whole batch itself (the same
+        //     arithmetic everywhere, so every CTA holds the same routing); the logits
+        //     are staged in the idle stage ring.
+        float* s_log = reinterpret_cast<float*>(sA);
+        {
+            // all loads first, then the shared-memory stores (one L2 latency)
+            constexpr int kR3Per = 8;
+            for (int i0 = threadIdx.x; i0 < T * E; i0 += kR3Per * kThreads) {
+                float lv[kR3Per];
+#pragma unroll
+                for (int j = 0; j < kR3Per; ++j) {
+                    const int i = i0 + j * kThreads;
+                    lv[j] = i < T * E ? __ldcg(p.logits + i) : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kR3Per; ++j) {
+                    const int i = i0 + j * kThreads;
+                    if (i < T * E) s_log[i] = lv[j];
+                }
+            }
+        }
+        const int words = (T + 31) / 32;
+        for (int i = threadIdx.x; i < E * words; i += kThreads) s_rmask[i] = 0;
+        for (int e = threadIdx.x; e < E; e += kThreads) s_rcnt[e] = 0;
+        __syncthreads();
+        const bool lead = blockIdx.x == 0;
+#pragma unroll 1
+        for (int t = warp; t < T; t += kThreads / 32) {
+            const WarpTopk r = warp_topk(s_log + t * E, p.bias, E, k, p.normalize, lane);
+            if (lane < k) {
+                s_ridx[t * k + lane] = r.idx;
+                s_rw[t * k + lane] = r.w;
+                if (static_cast<unsigned>(r.idx) < static_cast<unsigned>(E)) {
+                    atomicAdd(&s_rcnt[r.idx], 1);
+                    atomicOr(&s_rmask[r.idx * words + (t >> 5)], 1u << (t & 31));
+                }
+                if (lead) {
+                    p.r_topk_idx[t * k + lane] = r.idx;
+                    p.r_topk_w[t * k + lane] = r.w;
+                }
+            }
+            if (lead && lane == 0 && p.r_near_tie) p.r_near_tie[t] = r.flags;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            constexpr int per = kMaxExperts / 32;   // compile-time: loc[] stays in registers
+            int loc[per];
+            int lsum = 0;
+#pragma unroll
+            for (int q = 0; q < per; ++q) {
+                const int e = lane * per + q;
+                loc[q] = e < E ? s_rcnt[e] : 0;
+                lsum += loc[q];
+            }
+            int incl = lsum;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            int run = incl - lsum;
+#pragma unroll
+            for (int q = 0; q < per; ++q) {
+                const int e = lane * per + q;
+                if (e < E) {
+                    s_roff[e] = run;
+                    if (lead) {
+                        p.r_offsets[e] = run;
+                        p.r_counts[e] = loc[q];
+                    }
+                }
+                run += loc[q];
+            }
+            if (lane == 31) {
+                s_roff[E] = incl;
+                if (lead) p.r_offsets[E] = incl;
+            }
+        }
+        __syncthreads();
+        // stable placement: the rank of t among the tokens of its expert
+        for (int q = threadIdx.x; q < T * k; q += kThreads) {
+            const int e = s_ridx[q], t = q / k;
+            int row = -1;
+            if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+                const uint32_t* m = s_rmask + e * words;
+                const int w = t >> 5;
+                int rank = __popc(m[w] & ((1u << (t & 31)) - 1u));
+                for (int i = 0; i < w; ++i) rank += __popc(m[i]);
+                row = s_roff[e] + rank;
+                s_psrc[row] = t;
+                if (lead) p.r_perm_src[row] = t;
+            }
+            s_pdst[q] = row;
+            if (lead) p.r_perm_dst[q] = row;
+        }
+        // the stage ring is written by TMA from here on
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+    }
     if (warp == 2) {
-        TcParams tp{p.offsets, p.E, p.rows, 0, 0, nullptr, 0, p.err};
+        TcParams tp{ROUTE ? s_roff : p.offsets, p.E, p.rows, 0, 0, nullptr, 0, p.err};
         build_tile_map(tp, G, kTokChunk, s_off, s_pre, lane);
     }
     tc_fence_before();
@@ -691,7 +900,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 for (int h = 0; h < 2; ++h) {
                     const int i = lane + 32 * h;
                     if (i < d.nrows) {
-                        int t = p.perm_src[d.row0 + i];
+                        int t = ROUTE ? s_psrc[d.row0 + i] : p.perm_src[d.row0 + i];
                         if (t < 0 || t >= p.T) {
                             atomicOr(p.err, kErrBadExpert);
                             t = 0;
@@ -862,8 +1071,9 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                      q += static_cast<long long>(gridDim.x) * 128) {
                     const int t = static_cast<int>(q / nvec), v = static_cast<int>(q - static_cast<long long>(t) * nvec);
                     reinterpret_cast<uint4*>(p.out)[q] =
-                        combine_vec_bf16(reinterpret_cast<const uint4*>(p.y), nvec, p.perm_dst,
-                                         p.topk_w, t, p.k, v, p.rows);
+                        combine_vec_bf16(reinterpret_cast<const uint4*>(p.y), nvec,
+                                         ROUTE ? s_pdst : p.perm_dst, ROUTE ? s_rw : p.topk_w,
+                                         t, p.k, v, p.rows);
                 }
             }
         }
@@ -975,22 +1185,23 @@ int decode_grid(int rows, int E, int H, int I) {
     return static_cast<int>(units < sms ? units : sms);
 }
 
-template <bool GATHER>
+template <bool GATHER, bool ROUTE>
 cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& w2,
                           const CUtensorMap& a, const DecodeParams& p, int grid, cudaStream_t s) {
     using C = Tr<W_PLAIN, 64>;
-    auto kern = tc_ffn_decode_kernel<GATHER>;
+    constexpr int kSmem = C::kSmemBytes + (ROUTE ? kRouteSmemBytes : 0);
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+    auto kern = tc_ffn_decode_kernel<GATHER, ROUTE>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
     if (grid <= 0) return cudaSuccess;
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, w1, x, w2, a, p);
+    return launch_k(kern, dim3(grid), dim3(kThreads), kSmem, s, w1, x, w2, a, p);
 }
 
 }  // namespace
@@ -1042,8 +1253,14 @@ bool decode_ffn_supported(int rows, int E, int H, int I) {
            static_cast<long long>(rows) <= static_cast<long long>(kTokChunk) * E;
 }
 
-// one completion counter per chunk, the unit scheduler's counter, the fc2 count
-int decode_ffn_counters(int rows, int E) { return (rows + kTokChunk - 1) / kTokChunk + E + 2; }
+// one completion counter per chunk, the unit scheduler's counter, the fc2 count, the
+// routing barrier
+int decode_ffn_counters(int rows, int E) { return (rows + kTokChunk - 1) / kTokChunk + E + 3; }
+
+bool fused_route_supported(int T, int H, int E, int k, int I) {
+    return T >= 1 && T <= kFusedRouteMaxT && T * k <= kFusedRouteMaxRows && k >= 1 && k <= 32 &&
+           k <= E && E <= kMaxExperts && decode_ffn_supported(T * k, E, H, I);
+}
 
 cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
@@ -1061,12 +1278,68 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     if (!make_map(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
     if (!make_map(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, E);
-    DecodeParams p{offsets, perm_src, E, rows, T, H, I, static_cast<__nv_bfloat16*>(act),
-                   static_cast<__nv_bfloat16*>(y), done, done + nctr - 2, done + nctr - 1,
-                   perm_dst, topk_w, k, static_cast<__nv_bfloat16*>(out), err};
+    DecodeParams p{};
+    p.offsets = offsets;
+    p.perm_src = perm_src;
+    p.E = E;
+    p.rows = rows;
+    p.T = T;
+    p.H = H;
+    p.I = I;
+    p.act = static_cast<__nv_bfloat16*>(act);
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.done = done;
+    p.sched = done + nctr - 3;
+    p.fc2_done = done + nctr - 2;
+    p.perm_dst = perm_dst;
+    p.topk_w = topk_w;
+    p.k = k;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.err = err;
     const int grid = decode_grid(rows, E, H, I);
-    return perm_src ? launch_decode<true>(w1, x, w2, a, p, grid, s)
-                    : launch_decode<false>(w1, x, w2, a, p, grid, s);
+    return perm_src ? launch_decode<true, false>(w1, x, w2, a, p, grid, s)
+                    : launch_decode<false, false>(w1, x, w2, a, p, grid, s);
+}
+
+cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) {
+    const int rows = r.T * r.k;
+    if (rows <= 0) return cudaSuccess;
+    if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I)) return cudaErrorInvalidValue;
+    CUtensorMap w1, x, w2, a;
+    if (!make_map(&w1, r.fc1, static_cast<long long>(r.E) * 2 * r.I, r.H, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&x, r.hidden, r.T, r.H, 1)) return cudaErrorInvalidValue;
+    if (!make_map(&w2, r.fc2, static_cast<long long>(r.E) * r.H, r.I, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&a, r.act, rows, r.I, kBoxTok)) return cudaErrorInvalidValue;
+    const int nctr = decode_ffn_counters(rows, r.E);
+    DecodeParams p{};
+    p.E = r.E;
+    p.rows = rows;
+    p.T = r.T;
+    p.H = r.H;
+    p.I = r.I;
+    p.act = static_cast<__nv_bfloat16*>(r.act);
+    p.y = static_cast<__nv_bfloat16*>(r.y);
+    p.done = r.counters;
+    p.sched = r.counters + nctr - 3;
+    p.fc2_done = r.counters + nctr - 2;
+    p.route_bar = r.counters + nctr - 1;
+    p.k = r.k;
+    p.out = static_cast<__nv_bfloat16*>(r.out);
+    p.err = r.err;
+    p.hidden = r.hidden;
+    p.router_w = r.router_w;
+    p.bias = r.bias;
+    p.normalize = r.normalize ? 1 : 0;
+    p.logits = r.logits;
+    p.r_topk_idx = r.topk_idx;
+    p.r_topk_w = r.topk_w;
+    p.r_near_tie = r.near_tie;
+    p.r_counts = r.counts;
+    p.r_offsets = r.offsets;
+    p.r_perm_src = r.perm_src;
+    p.r_perm_dst = r.perm_dst;
+    const int grid = decode_grid(rows, r.E, r.H, r.I);
+    return launch_decode<true, true>(w1, x, w2, a, p, grid, s);
 }
 
 }  // namespace moe

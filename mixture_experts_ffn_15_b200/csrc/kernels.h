@@ -90,6 +90,9 @@ cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int
                           cudaStream_t s);
 
 // ---------------------------------------------------------------- combine.cu
+// Zeroes `bytes` (a multiple of 16, 16-byte aligned) with a kernel, so that the launch
+// overlaps the previous kernel on the stream (a memset node would not).
+cudaError_t launch_clear(void* words, size_t bytes, cudaStream_t s);
 cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w,
                            int T, int H, int k, bool bf16, void* out, cudaStream_t s);
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
@@ -118,6 +121,35 @@ bool decode_ffn_supported(int rows, int E, int H, int I);
 int decode_ffn_counters(int rows, int E);   // int32 counters it needs, zero on entry
 // tokens: `hidden` [T, H] gathered through perm_src, or x_perm [rows, H] if perm_src is null.
 // With out != nullptr the launch also does the weighted combine into out [T, H].
+// The same launch with the routing inside it (small batches): router logits on every
+// CTA for its experts, a grid-wide barrier, then every CTA selects, counts and permutes
+// the whole batch itself.  counters: decode_ffn_counters(T k, E) words, zero on entry.
+constexpr int kFusedRouteMaxT = 64;
+constexpr int kFusedRouteMaxRows = 512;
+bool fused_route_supported(int T, int H, int E, int k, int I);
+struct DecodeRoutedArgs {
+    const void* hidden;        // [T, H] bf16
+    const void* router_w;      // [E, H] bf16
+    const float* bias;         // [E] or nullptr
+    const void* fc1;           // [E, 2I, H] interleaved
+    const void* fc2;           // [E, H, I]
+    int T, H, E, k, I, normalize;
+    float* logits;             // [T, E] scratch
+    int32_t* topk_idx;         // [T, k] out
+    float* topk_w;             // [T, k] out
+    int32_t* near_tie;         // [T] out or nullptr
+    int32_t* counts;           // [E] out
+    int32_t* offsets;          // [E + 1] out
+    int32_t* perm_src;         // [T k] out
+    int32_t* perm_dst;         // [T k] out
+    void* act;                 // [T k, I] scratch
+    void* y;                   // [T k, H] scratch
+    int32_t* counters;         // zero on entry
+    int32_t* err;
+    void* out;                 // [T, H]
+};
+cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& a, cudaStream_t s);
+
 cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,

@@ -60,9 +60,10 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
     s_before[threadIdx.x] = before;
     __syncthreads();
     if (warp == 0) {
-        const int per = (E + 31) / 32;
-        int loc[kMaxExperts / 32];
+        constexpr int per = kMaxExperts / 32;   // compile-time: loc[] stays in registers
+        int loc[per];
         int lsum = 0;
+#pragma unroll
         for (int q = 0; q < per; ++q) {
             const int e = lane * per + q;
             int t = 0;
@@ -78,6 +79,7 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
             if (lane >= d) incl += y;
         }
         int run = incl - lsum;
+#pragma unroll
         for (int q = 0; q < per; ++q) {
             const int e = lane * per + q;
             if (e < E) {

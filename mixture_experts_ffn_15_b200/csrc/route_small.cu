@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "topk_warp.cuh"
 
 namespace moe {
 namespace {
@@ -99,16 +100,6 @@ router_logits_split_kernel(const void* __restrict__ hidden, const void* __restri
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallMaskWords = kRouteSmallMaxT / 32;             // 16
-constexpr int kVals = kMaxExperts / 32;
-
-// float -> unsigned with the same order (larger float, larger key)
-__device__ __forceinline__ uint32_t order_key(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_value(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
 
 __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const RouteSmallArgs a) {
     __shared__ uint32_t s_mask[kMaxExperts * kSmallMaskWords];
@@ -127,81 +118,28 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Rou
     // ---- top-k per token (one warp per token), weights, near-tie flags, bincount.
     // The token loop stays rolled: this kernel runs once per layer call with a cold
     // instruction cache, and unrolled copies of the body cost more to fetch than to run.
-    const int rounds = min(k + 1, E);
 #pragma unroll 1
     for (int t = warp; t < T; t += kSmallWarps) {
-        {
-            float v[kVals];
-#pragma unroll
-            for (int i = 0; i < kVals; ++i) {
-                const int e = lane + 32 * i;
-                float x = -INFINITY;
-                if (e < E) {
-                    x = a.logits[static_cast<size_t>(t) * E + e];
-                    if (a.bias) x += a.bias[e];
-                }
-                v[i] = x;
+        const WarpTopk r = warp_topk(a.logits + static_cast<size_t>(t) * E, a.bias, E, k,
+                                     a.normalize, lane);
+        if (lane < k) {
+            a.topk_idx[static_cast<size_t>(t) * k + lane] = r.idx;
+            a.topk_w[static_cast<size_t>(t) * k + lane] = r.w;
+            if (static_cast<unsigned>(r.idx) < static_cast<unsigned>(E)) {
+                atomicAdd(&s_cnt[r.idx], 1);
+                atomicOr(&s_mask[r.idx * words + (t >> 5)], 1u << (t & 31));
             }
-            uint32_t taken = 0;
-            float sel_v = -INFINITY, next_v = -INFINITY;
-            int sel_i = -1;
-            for (int r = 0; r < rounds; ++r) {
-                uint32_t bk = 0;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int i = 0; i < kVals; ++i) {
-                    const int e = lane + 32 * i;
-                    if (e < E && !((taken >> i) & 1u)) {
-                        const uint32_t kk = order_key(v[i]);
-                        if (kk > bk || (kk == bk && e < bi)) {
-                            bk = kk;
-                            bi = e;
-                        }
-                    }
-                }
-                const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-                const int wi = static_cast<int>(__reduce_min_sync(0xffffffffu, static_cast<uint32_t>(bk == m ? bi : 0x7fffffff)));
-                if (wi < E && (wi & 31) == lane) taken |= 1u << (wi >> 5);
-                const float wv = key_value(m);
-                if (r == lane) {
-                    sel_v = wv;
-                    sel_i = wi;
-                }
-                if (r == k) next_v = wv;
-            }
-            const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
-            const float num = (lane < k) ? expf(sel_v - vmax) : 0.f;
-            float part = num;
-            if (!a.normalize) {
-                part = 0.f;
-#pragma unroll
-                for (int i = 0; i < kVals; ++i)
-                    if (lane + 32 * i < E) part += expf(v[i] - vmax);
-            }
-            const float den = warp_sum(part);
-            const float prev_v = __shfl_down_sync(0xffffffffu, sel_v, 1);
-            const bool within = lane + 1 < k && (sel_v - prev_v) < kNearTieGap;
-            const float kth = __shfl_sync(0xffffffffu, sel_v, k - 1);
-            if (lane < k) {
-                a.topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
-                a.topk_w[static_cast<size_t>(t) * k + lane] = num / den;
-                if (static_cast<unsigned>(sel_i) < static_cast<unsigned>(E)) {
-                    atomicAdd(&s_cnt[sel_i], 1);
-                    atomicOr(&s_mask[sel_i * words + (t >> 5)], 1u << (t & 31));
-                }
-            }
-            const unsigned wb = __ballot_sync(0xffffffffu, within);
-            if (a.near_tie && lane == 0)
-                a.near_tie[t] = ((k < E && kth - next_v < kNearTieGap) ? 1 : 0) | (wb ? 2 : 0);
         }
+        if (a.near_tie && lane == 0) a.near_tie[t] = r.flags;
     }
     __syncthreads();
 
     // ---- exclusive scan of the counts (warp 0)
     if (warp == 0) {
-        const int per = (E + 31) / 32;
-        int loc[kVals];
+        constexpr int per = kMaxExperts / 32;   // compile-time: loc[] stays in registers
+        int loc[per];
         int lsum = 0;
+#pragma unroll
         for (int q = 0; q < per; ++q) {
             const int e = lane * per + q;
             loc[q] = e < E ? s_cnt[e] : 0;
@@ -214,6 +152,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Rou
             if (lane >= d) incl += y;
         }
         int run = incl - lsum;
+#pragma unroll
         for (int q = 0; q < per; ++q) {
             const int e = lane * per + q;
             if (e < E) {

@@ -104,11 +104,14 @@ def test_forward_path_per_workload():
     """moe_forward_path: which kernels run for each workload (host arithmetic only)."""
     lib = _lib()
     bf, f32 = _abi.MOE_BF16, _abi.MOE_F32
-    small, fused, tc_router, token, fma = 1, 2, 4, 8, 16
+    small, fused, tc_router, token, fma, one_launch = 1, 2, 4, 8, 16, 32
     assert lib.moe_forward_path(64, 256, 8, 2, 128, f32) == small | fma
-    assert lib.moe_forward_path(4, 2816, 128, 8, 704, bf) == small | fused
+    assert lib.moe_forward_path(4, 2816, 128, 8, 704, bf) == one_launch | fused
+    assert lib.moe_forward_path(64, 2816, 128, 8, 704, bf) == one_launch | fused
+    assert lib.moe_forward_path(65, 2816, 128, 8, 704, bf) == tc_router | fused
+    assert lib.moe_forward_path(16, 2816, 128, 8, 704, bf) == one_launch | fused
     assert lib.moe_forward_path(256, 2816, 128, 8, 704, bf) == tc_router | fused
-    assert lib.moe_forward_path(16, 2816, 128, 8, 704, bf) == small | fused
+    assert lib.moe_forward_path(16, 192, 8, 2, 704, bf) == small | token      # H % 128 != 0
     assert lib.moe_forward_path(8192, 2816, 128, 8, 704, bf) == tc_router | token
     assert lib.moe_forward_path(32768, 4096, 64, 4, 1536, bf) == tc_router | token
     assert lib.moe_forward_path(300, 128, 8, 2, 704, bf) == small | token   # > 64 rows per expert

@@ -39,6 +39,11 @@ CASES = [
     W("bf16_router_tc_norm0_bias", T=300, H=192, E=128, k=6, I=64, normalize=0,
       router_bias_std=0.5),
     W("bf16_router_tc_T17", T=17, H=64, E=64, k=8, I=64),
+    # the whole layer in one launch (routing inside the decode FFN)
+    W("bf16_onelaunch_T64_k8", T=64, H=256, E=64, k=8, I=128),
+    W("bf16_onelaunch_bias_norm0", T=33, H=128, E=128, k=6, I=64, normalize=0,
+      router_bias_std=0.5),
+    W("bf16_onelaunch_E256_k16", T=8, H=128, E=256, k=16, I=64),
     W("bf16_k1", T=130, H=128, E=8, k=1, I=64),
     W("bf16_k_eq_E", T=20, H=128, E=4, k=4, I=64),
     W("bf16_T1", T=1, H=128, E=8, k=2, I=64),
