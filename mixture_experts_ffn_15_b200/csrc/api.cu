@@ -306,8 +306,8 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
         MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1, fc2, rows, H, E, I,
                                    act_buf, y_perm, ctr, err, nullptr, nullptr, 0, nullptr, s));
     } else if (dt == MOE_BF16) {
-        MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
-                               nullptr));
+        MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
+                                 nullptr));
     } else {
         MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                      static_cast<const float*>(fc1), static_cast<const float*>(fc2),
@@ -479,7 +479,8 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         record(2, s);
         cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
         if (bf16)
-            MOE_CUDA(launch_ffn_tc(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s, mid));
+            MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
+                                     mid));
         else
             MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                          static_cast<const float*>(fc1),

@@ -1,0 +1,414 @@
+// Grouped expert GEMMs for large batches on CTA pairs (tcgen05 cta_group::2, sm_100a).
+//
+// The grouped matmul of grouped_mm_experts_forward ("Contributing Gemma 4 support
+// and ONNX export optimizations", "Key Technical Contributions") over each expert's
+// contiguous block of permuted rows, with standard SwiGLU on the interleaved fc1
+// ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", "Attribute set"):
+//   fc1 + SwiGLU: act[r, i] = silu(x[r] . fc1[e, 2i]) * (x[r] . fc1[e, 2i+1])
+//   fc2:          y[r, h]   = act[r] . fc2[e, h]
+//
+// Orientation: the expert's WEIGHT rows are the MMA's M side and its tokens the N
+// side.  A unit is (expert, tile of up to 256 tokens, tile of 256 weight rows); a
+// cluster of two CTAs runs it as one M = 256 MMA: each CTA loads its own 128 weight
+// rows and half of the tokens, and accumulates its 128 weight rows x all the tokens
+// in its tensor memory.  Per CTA and 64-wide K slice that is 32 KB from L2 for
+// 128 x 256 x 64 multiply-adds -- two thirds of what a single-CTA 128 x 256 tile
+// needs -- and the token side rounds up to 32 rows, not to a 128-row tile.
+//
+// Both GEMMs read contiguous token rows (x_perm, act) in one 128-row TMA box.  The
+// accumulator holds weight rows x tokens, so the epilogue transposes each warp's
+// 32 x 32 block through shared memory and writes every token row with 16-byte stores.
+//
+// Per CTA, 10 warps:
+//   warp 0     TMA producer (both CTAs): its CTA's weight and token slices into a
+//              6-stage ring; completion counted on the even CTA's barrier;
+//   warp 1     MMA issuer (even CTA only): tcgen05.mma.cta_group::2 into one of two
+//              accumulators; commits free the ring stage in both CTAs and publish
+//              the accumulator to both epilogues;
+//   warps 2-9  epilogue (both CTAs): tcgen05.ld of their 128 weight rows x the
+//              tokens, SwiGLU (fc1) or plain (fc2), a warp-private transpose in
+//              shared memory, 16-byte stores of token rows, then release the
+//              accumulator on the even CTA's barrier.
+// Units are statically strided over the pairs (both CTAs walk the same list), so no
+// cluster ever waits on another.  Every wait is bounded (2 s) and reports
+// MOE_DEVERR_TIMEOUT; both CTAs always reach the final cluster barrier.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tile_map.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+
+constexpr int kPThreads = 320;                // producer, MMA, 8 epilogue warps
+constexpr int kPWRows = 128;                  // weight rows per CTA (256 per pair)
+constexpr int kPBK = 64;                      // K per stage: one 128-byte row of bf16
+constexpr int kPTok = 256;                    // tokens per pair tile (<= 128 per CTA)
+constexpr int kPStages = 6;
+constexpr int kPABytes = kPWRows * kPBK * 2;  // 16 KB
+constexpr int kPBBytes = (kPTok / 2) * kPBK * 2;   // 16 KB
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPAccCols = 256;                // one accumulator: 256 fp32 columns
+constexpr int kPTmemCols = 512;
+constexpr int kPBox = kPTok / 2;              // token rows per TMA box: a CTA's whole half
+constexpr uint64_t kPWaitNs = 2000000000ull;
+constexpr int kPMiscBytes =
+    (2 * kPStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 64;
+constexpr int kPEpiWarpBytes = 32 * 64;      // per epilogue warp: 32 tokens x 32 rows bf16
+constexpr int kPEpiBytes = 8 * kPEpiWarpBytes;
+constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kPEpiBytes + kPMiscBytes;
+static_assert(kPSmemBytes <= 227 * 1024, "shared memory");
+
+struct PairParams {
+    const int32_t* offsets;   // [E+1] device
+    int E;
+    int rows;                 // permuted rows (T k)
+    int K;                    // reduction length (multiple of 64)
+    int n_out;                // weight rows per expert (2I or H)
+    __nv_bfloat16* out;       // [rows, ldo]
+    int ldo;                  // I (fc1) or H (fc2)
+    int32_t* err;
+};
+
+struct PUnit {
+    int g, row0, nrows, n, mt;   // expert, first token row, valid tokens, MMA N, weight tile
+};
+
+__device__ __forceinline__ PUnit pair_unit(int u, int MT, int G, const int* s_off, const int* s_pre) {
+    PUnit d;
+    const int tile = u / MT;
+    d.mt = u - tile * MT;
+    d.g = tile_group(tile, G, s_pre);
+    d.row0 = s_off[d.g] + (tile - s_pre[d.g]) * kPTok;
+    d.nrows = min(kPTok, s_off[d.g + 1] - d.row0);
+    d.n = ((d.nrows + 31) / 32) * 32;   // each CTA's half: a multiple of 16 rows (TMA boxes)
+    return d;
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kPThreads, 1)
+tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+               const PairParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kPStages * kPABytes;
+    uint8_t* sEpi = sB + kPStages * kPBBytes;   // [8 warps][32 tokens][64 bytes]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kPEpiBytes);
+    uint64_t* empty = full + kPStages;
+    uint64_t* tfull = empty + kPStages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
+    int* s_pre = s_off + (kMaxExperts + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool lead = rank == 0;
+    const int G = p.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);    // the even CTA's producer (expect_tx)
+            mbar_init(smem_u32(&empty[s]), 1);   // the pair MMA's commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 16); // 8 epilogue warps x 2 CTAs
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kPTmemCols);
+        tmem_relinquish_pair();
+    }
+    // the prologue above touches no global memory; everything below may
+    pdl_wait();
+    pdl_trigger();
+    if (warp == 2) build_group_tiles(p.offsets, p.rows, p.err, G, kPTok, s_off, s_pre, lane);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // both CTAs' barriers and tensor memory exist before any signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int MT = (p.n_out + 2 * kPWRows - 1) / (2 * kPWRows);
+    const int num_units = s_pre[G] * MT;
+    const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+    const int nk = p.K / kPBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
+            const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
+            const int half = d.n / 2;                     // token rows of this CTA
+            const int trow0 = d.row0 + static_cast<int>(rank) * half;
+            const int wrow = d.g * p.n_out + d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
+            // one box of 128 weight rows and one of 128 token rows per CTA (rows past
+            // the tile are loaded too, and ignored: one TMA instruction each)
+            const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (lane == 0) {
+                    ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kPWaitNs);
+                    if (ok && lead) mbar_arrive_expect_tx(smem_u32(&full[stage]), bytes);
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);   // the even CTA's
+                const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
+                const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
+                if (lane == 0) {
+                    tma_load_2d_pair(a_dst, &tmW, fb, kb * kPBK, wrow);
+                    tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
+                }
+                if (++stage == kPStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lead && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
+                const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
+                const uint32_t idesc = idesc_bf16_f32(2 * kPWRows, d.n);
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kPWaitNs)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPAccCols);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kPWaitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * kPABytes);
+                    const uint32_t b0 = smem_u32(sB + stage * kPBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kPBK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                       smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                    umma_commit_pair(smem_u32(&empty[stage]), 0x3);
+                    if (++stage == kPStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair(smem_u32(&tfull[acc]), 0x3);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        // warps 2..9: TMEM lane quadrant warp % 4 (hardware rule), and every other
+        // 32-token chunk of the tile
+        const int quad = warp & 3;
+        const int part = (warp - 2) >> 2;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        uint8_t* scr = sEpi + (warp - 2) * kPEpiWarpBytes;
+        for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
+            const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kPWaitNs)) break;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                static_cast<uint32_t>(acc * kPAccCols);
+            // this warp's 32 weight rows inside the expert: w0 .. w0+31 (all valid or none:
+            // n_out is a multiple of 32)
+            const int w0 = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows + quad * 32;
+            const bool wvalid = w0 < p.n_out;
+#pragma unroll 1
+            for (int c = part * 32; c < d.nrows; c += 64) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tb + c, v);
+                tmem_wait_ld();
+                // lane = weight row w0 + lane, v[i] = token c + i.  Transpose through the
+                // warp's scratch (row i = token c + i's outputs), then store whole token
+                // rows: each store instruction writes full 32-byte sectors.
+                if constexpr (SWIGLU) {
+                    // rows come in (gate, up) pairs: lanes 2j, 2j+1 hold gate_j, up_j.  For
+                    // tokens (i, i+1) one exchange gives the even lane (gate, up) of token i
+                    // and the odd lane those of token i+1: every lane computes one output.
+                    const bool odd = lane & 1;
+                    const int j = lane >> 1;   // output 0..15 of this warp: 32 bytes a token
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float mine_g = __uint_as_float(v[i]), mine_u = __uint_as_float(v[i + 1]);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_g : mine_u, 1);
+                        const float g = odd ? other : mine_g;          // gate of token i + odd
+                        const float u = odd ? mine_u : other;          // up of token i + odd
+                        const int tok = i + (odd ? 1 : 0);
+                        *reinterpret_cast<__nv_bfloat16*>(scr + tok * 32 + j * 2) =
+                            __float2bfloat16_rn(swiglu_fast(g, u));
+                    }
+                    __syncwarp();
+                    const int i0 = w0 >> 1;   // first output column of this warp
+#pragma unroll
+                    for (int pass = 0; pass < 2; ++pass) {
+                        const int tt = pass * 16 + (lane >> 1), q = lane & 1;
+                        if (wvalid && c + tt < d.nrows)
+                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + i0 + q * 8) =
+                                *reinterpret_cast<const uint4*>(scr + tt * 32 + q * 16);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        *reinterpret_cast<__nv_bfloat16*>(scr + i * 64 + lane * 2) =
+                            __float2bfloat16_rn(__uint_as_float(v[i]));
+                    __syncwarp();
+#pragma unroll
+                    for (int pass = 0; pass < 4; ++pass) {
+                        const int tt = pass * 8 + (lane >> 2), q = lane & 3;
+                        if (wvalid && c + tt < d.nrows)
+                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + w0 + q * 8) =
+                                *reinterpret_cast<const uint4*>(scr + tt * 64 + q * 16);
+                    }
+                }
+                __syncwarp();   // the scratch is rewritten by the next chunk
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    if (*abort_flag) {
+        // copies already issued may still land: give them time before the pair exits
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // no CTA leaves while its partner may still read its memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kPTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* q = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(q);
+    }
+    return fn;
+}
+
+// bf16 matrix [rows, K] row-major, boxes of 64 (K) x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || rows <= 0) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kPBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool SWIGLU>
+cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairParams& p,
+                        long long units, cudaStream_t s) {
+    auto kern = tc_pair_kernel<SWIGLU>;
+    // once per device (outside any stream capture: the first call of every path runs
+    // eagerly before a graph is captured): the shared-memory limit and the number of
+    // pairs that fit on the GPU at once
+    static int max_pairs[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = kPSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    if (max_pairs[dev] == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kPSmemBytes);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3(2 * (device_sm_count() / 2));
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        max_pairs[dev] = n > 0 ? n : 1;
+    }
+    long long pairs = units < max_pairs[dev] ? units : max_pairs[dev];
+    if (pairs <= 0) return cudaSuccess;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.numAttrs = 2;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, kern, w, x, p);
+}
+
+// One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
+// the experts' blocks) and w [E * n_out, K].
+cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
+                      const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s) {
+    CUtensorMap mw, mx;
+    if (!make_map(&mw, w, static_cast<long long>(E) * n_out, K, kPWRows)) return cudaErrorInvalidValue;
+    if (!make_map(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
+    PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err};
+    const long long units = (static_cast<long long>((rows + kPTok - 1) / kPTok) + E) *
+                            ((n_out + 2 * kPWRows - 1) / (2 * kPWRows));
+    return swiglu ? launch_pair<true>(mw, mx, p, units, s) : launch_pair<false>(mw, mx, p, units, s);
+}
+
+}  // namespace
+
+bool pair_ffn_supported(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0; }
+
+cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
+                            const void* fc2, int rows, int H, int E, int I, void* act, void* y,
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid) {
+    if (rows <= 0) return cudaSuccess;
+    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s);
+    if (e != cudaSuccess) return e;
+    if (mid) record_event(mid, s);
+    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
+}
+
+}  // namespace moe

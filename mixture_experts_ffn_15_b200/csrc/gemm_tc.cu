@@ -1,14 +1,17 @@
-// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+// Single-CTA tcgen05 kernels (sm_100a): the router GEMM with the routing in its
+// epilogue, and the decode FFN.
 //
-// The grouped matmul of grouped_mm_experts_forward ("Contributing Gemma 4 support
-// and ONNX export optimizations", "Key Technical Contributions") runs, for every
-// expert e, over that expert's contiguous block of permuted rows:
-//   fc1 + SwiGLU: act[r, i] = silu(x[r] . fc1[e, 2i]) * (x[r] . fc1[e, 2i+1])
-//   fc2:          y[r, h]   = act[r] . fc2[e, h]
-// with standard SwiGLU and the interleaved fc1 layout of "Gemma 4 MoE: re-enable
-// fused com.microsoft::MoE op - #326", "Attribute set".  The router logits
-// (hidden . router_w^T) reuse the same kernel as a single group with a float32
-// epilogue.
+// Router ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", "Attribute
+// set": k = top_k, normalize_routing_weights): logits[t, e] = hidden[t] . router_w[e]
+// (+ bias) for 128-token tiles on M and all E experts on N; the epilogue selects,
+// weighs and counts (per-tile bincount of "Contributing Gemma 4 support and ONNX
+// export optimizations", "Key Technical Contributions").
+//
+// Decode FFN: the grouped matmul of grouped_mm_experts_forward for batches with few
+// rows per expert, fc1 + SwiGLU and fc2 (standard SwiGLU, interleaved fc1) in one
+// persistent launch with 128 weight rows on M and the expert's tokens on N, so that
+// every weight byte streams from HBM once; optionally with the routing and the
+// weighted combine inside the same launch.
 //
 // One persistent CTA per SM, 6 warps:
 //   warp 0     TMA producer: A and B tiles (64-wide K slices, 128-byte swizzle)
@@ -16,16 +19,9 @@
 //   warp 1     MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> f32) into one of
 //              two TMEM accumulators, tcgen05.commit frees stages / publishes tiles;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//              32*(w%4) .. +31), activation, bf16 pack, global stores.  The second
-//              accumulator lets the epilogue of one tile overlap the next mainloop.
-//
-// Two orientations of the same mainloop:
-//   token-M  (prefill):  M = 128 permuted rows, N = BN weight rows.  Tile map: for
-//            each expert, ceil(n_e / 128) row tiles x (n_out / BN) column tiles.
-//   weight-M (decode):   M = 128 weight rows, N = the expert's tokens (<= 64 per
-//            unit, loaded in 16-row boxes).  The weight tile streams from HBM once
-//            per unit; tokens are few, so this keeps every MMA 128 rows tall.
-// The tile map is rebuilt in every CTA from the device offsets (no host sync).
+//              32*(w%4) .. +31).  The second accumulator lets the epilogue of one
+//              tile overlap the next mainloop.
+// Tile maps are rebuilt in every CTA from device offsets (no host sync).
 //
 // Every wait is bounded (2 s); on expiry the CTA winds down, reports
 // MOE_DEVERR_TIMEOUT in the error word and still frees its TMEM.
@@ -35,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tile_map.cuh"
 #include "topk_warp.cuh"
 
 namespace moe {
@@ -51,7 +48,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // TOK_ROUTE: router logits with the routing itself in the epilogue (top-k, softmax,
 // near-tie flags, per-tile bincount).
-enum Mode : int { TOK_SWIGLU = 0, TOK_PLAIN = 1, W_PLAIN = 4, TOK_ROUTE = 5 };
+enum Mode : int { W_PLAIN = 4, TOK_ROUTE = 5 };
 
 template <int MODE, int BN>
 struct Tr {
@@ -64,7 +61,6 @@ struct Tr {
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     static constexpr int kAccStride = kWeightM ? kTokChunk : 256;
     static constexpr int kTmemCols = kWeightM ? 128 : 512;
-    static constexpr int kUnitRows = kWeightM ? kTokChunk : BM;
     // barriers, tmem slot + abort flag, offsets, prefix, gather rows of one chunk
     static constexpr int kMiscBytes =
         (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 16 * 8 + 64 +
@@ -103,75 +99,9 @@ struct Unit {
     int sub;    // column tile (token-M) or weight row tile (weight-M) inside the expert
 };
 
-// s_off: sanitised offsets (clamped to [0, rows], non-decreasing); s_pre[g]: first
-// tile of group g; s_pre[G]: tile count.  Runs on one warp; lane l owns the kPer
-// consecutive entries l*kPer ..; every loop has a compile-time trip count, so the
-// per-lane arrays stay in registers.
 __device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int unit_rows, int* s_off,
                                                int* s_pre, int lane) {
-    constexpr int kPer = (kMaxExperts + 1 + 31) / 32;   // 9
-    int v[kPer];
-    bool bad = false;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const int i = lane * kPer + q;
-        int raw = p.rows;
-        if (i <= G) raw = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.rows);
-        if (i == 0 && p.offsets && raw != 0) bad = true;
-        int c = raw < 0 ? 0 : (raw > p.rows ? p.rows : raw);
-        if (c != raw) bad = true;
-        v[q] = c;
-    }
-#pragma unroll
-    for (int q = 1; q < kPer; ++q)
-        if (v[q] < v[q - 1]) {
-            bad = bad || (lane * kPer + q <= G);
-            v[q] = v[q - 1];
-        }
-    int inc = v[kPer - 1];
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, d);
-        if (lane >= d) inc = max(inc, y);
-    }
-    int excl = __shfl_up_sync(0xffffffffu, inc, 1);
-    if (lane == 0) excl = 0;
-    // tiles of group g = lane*kPer + q: from the clamped offsets g and g + 1 (the
-    // latter is the next entry, or the first entry of the next lane)
-    const int first_next = __shfl_down_sync(0xffffffffu, max(v[0], excl), 1);
-    int cnt[kPer];
-    int lsum = 0;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const int i = lane * kPer + q;
-        if (v[q] < excl && i <= G) bad = true;
-        v[q] = max(v[q], excl);
-        if (i <= G) s_off[i] = v[q];
-    }
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const int g = lane * kPer + q;
-        const int hi = (q + 1 < kPer) ? v[q + 1 < kPer ? q + 1 : q] : first_next;
-        int c = 0;
-        if (g < G) c = (hi - v[q] + unit_rows - 1) / unit_rows;
-        cnt[q] = c;
-        lsum += c;
-    }
-    int incl = lsum;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += y;
-    }
-    int run = incl - lsum;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const int g = lane * kPer + q;
-        if (g <= G) s_pre[g] = run;   // g == G: the tile count
-        run += cnt[q];
-    }
-    if (bad && p.offsets && p.err) atomicOr(p.err, kErrBadExpert);
-    __syncwarp();
+    build_group_tiles(p.offsets, p.rows, p.err, G, unit_rows, s_off, s_pre, lane);
 }
 
 __device__ __forceinline__ Unit decode_unit(int u, int per_unit, int G, int unit_rows,
@@ -342,7 +272,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // the prologue above touches no global memory; everything below may
     pdl_wait();
     pdl_trigger();
-    if (warp == 2) build_tile_map(p, G, C::kUnitRows, s_off, s_pre, lane);
+    if (warp == 2) build_tile_map(p, G, BM, s_off, s_pre, lane);
     if constexpr (MODE == TOK_ROUTE) {
         for (int e = threadIdx.x; e < BN; e += kThreads) s_bias[e] = rp.bias ? rp.bias[e] : 0.f;
         for (int e = threadIdx.x; e < 4 * BN; e += kThreads) s_cnt[e] = 0;
@@ -363,7 +293,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint32_t phase = 0;
             long long issued = 0;
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-                const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+                const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
                 const uint32_t bytes = C::kStageBytes;
                 const int wrow = t.g * p.n_out + t.sub * BN;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -400,7 +330,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-                const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+                const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
                 const uint32_t idesc = idesc_bf16_f32(BM, BN);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                 tc_fence_after();
@@ -437,51 +367,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-            const Unit t = decode_unit(u, per_unit, G, C::kUnitRows, s_off, s_pre);
+            const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
             tc_fence_after();
             const uint32_t tb =
                 tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::kAccStride);
             const bool valid = r < t.nrows;
             const size_t orow = static_cast<size_t>(t.row0 + r);
-            const int col0 = t.sub * BN;
-            if constexpr (MODE == TOK_ROUTE) {
-                route_epilogue<BN, KS>(tb, valid, orow, t.row0 / BM, rp, s_bias,
-                                       s_cnt + quad * BN, lane);
-            } else {
-#pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
-                uint32_t v[32];
-                const bool full32 = (c + 32 <= BN);
-                if (full32) tmem_ld_32x32b_x32(tb + c, v);
-                else tmem_ld_32x32b_x16(tb + c, v);
-                tmem_wait_ld();
-                if (!valid) continue;
-                const int nv = full32 ? 32 : 16;
-                if constexpr (MODE == TOK_SWIGLU) {
-                    float a[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        a[i] = (2 * i < nv) ? swiglu_f32(f32(v[2 * i]), f32(v[2 * i + 1])) : 0.f;
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                          orow * p.ldo + (col0 + c) / 2);
-                    dst[0] = pack_bf16x8(a);
-                    if (nv == 32) dst[1] = pack_bf16x8(a + 8);
-                } else if constexpr (MODE == TOK_PLAIN) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                          orow * p.ldo + col0 + c);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (8 * q < nv) {
-                            float f[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) f[i] = f32(v[8 * q + i]);
-                            dst[q] = pack_bf16x8(f);
-                        }
-                    }
-                }
-            }
-            }
+            route_epilogue<BN, KS>(tb, valid, orow, t.row0 / BM, rp, s_bias,
+                                   s_cnt + quad * BN, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
@@ -1143,40 +1037,6 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParam
     return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p, rp);
 }
 
-int pick_bn(int n_out) {
-    const int cands[5] = {256, 192, 176, 128, 64};
-    for (int c : cands)
-        if (n_out % c == 0) return c;
-    return 0;
-}
-
-// One grouped GEMM: out = A(rows x K) . W_e^T over the experts' row blocks.
-cudaError_t grouped_gemm(bool swiglu, const void* act_in, int rows, int K, const void* w, int E,
-                         int n_out, const int32_t* offsets, void* out, int ldo, int32_t* err,
-                         cudaStream_t s) {
-    TcParams p{offsets, E, rows, K, n_out, out, ldo, err};
-    CUtensorMap ma, mb;
-    const int bn = pick_bn(n_out);
-    if (!make_map(&ma, act_in, rows, K, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&mb, w, static_cast<long long>(E) * n_out, K, bn)) return cudaErrorInvalidValue;
-    const long long bound = (static_cast<long long>((rows + BM - 1) / BM) + E) * (n_out / bn);
-    const int b = static_cast<int>(bound > (1 << 30) ? (1 << 30) : bound);
-#define MOE_TOK_CASE(BNV)                                                          \
-    case BNV:                                                                      \
-        return swiglu ? launch_one<TOK_SWIGLU, BNV>(ma, mb, p, b, s)               \
-                      : launch_one<TOK_PLAIN, BNV>(ma, mb, p, b, s);
-    switch (bn) {
-        MOE_TOK_CASE(256)
-        MOE_TOK_CASE(192)
-        MOE_TOK_CASE(176)
-        MOE_TOK_CASE(128)
-        MOE_TOK_CASE(64)
-        default:
-            return cudaErrorInvalidValue;
-    }
-#undef MOE_TOK_CASE
-}
-
 // Grid of a persistent decode FFN launch: every unit of both GEMMs, at most one CTA per SM.
 int decode_grid(int rows, int E, int H, int I) {
     const long long units =
@@ -1236,16 +1096,6 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
             return cudaErrorInvalidValue;
     }
 #undef MOE_ROUTE_CASE
-}
-
-cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
-                          const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                          int32_t* err, cudaStream_t s, cudaEvent_t mid) {
-    if (rows <= 0) return cudaSuccess;
-    cudaError_t e = grouped_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s);
-    if (e != cudaSuccess) return e;
-    if (mid) record_event(mid, s);
-    return grouped_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
 }
 
 bool decode_ffn_supported(int rows, int E, int H, int I) {

@@ -105,9 +105,6 @@ cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, con
 
 // ---------------------------------------------------------------- gemm_tc.cu
 bool tc_ffn_supported(int H, int I);
-cudaError_t launch_ffn_tc(const void* x_perm, const int32_t* offsets, const void* fc1,
-                          const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                          int32_t* err, cudaStream_t s, cudaEvent_t mid);
 // Router logits on the tensor cores with the routing in the epilogue: top-k, softmax
 // weights, near-tie flags and the per-128-token-tile bincount (logits optional).
 bool tc_route_supported(int H, int E, int k);
@@ -115,6 +112,15 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
                             int H, int E, int k, int normalize, int32_t* topk_idx, float* topk_w,
                             int32_t* near_tie, float* logits, int32_t* tile_counts, int32_t* err,
                             cudaStream_t s);
+
+// ---------------------------------------------------------------- gemm_pair.cu
+// fc1 + SwiGLU and fc2 for large batches on CTA pairs (weight rows on M, M = 256 per
+// pair): x_perm [rows, H] -> act [rows, I] -> y [rows, H]; `mid` (optional) is
+// recorded between the two GEMMs.
+bool pair_ffn_supported(int H, int I);
+cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
+                            const void* fc2, int rows, int H, int E, int I, void* act, void* y,
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid);
 
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);
