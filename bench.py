@@ -158,19 +158,29 @@ def algorithmic(wl, counts):
     return used, fc1, fc2, layer
 
 
-def kernel_traffic(workload):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu summary, if the
-    summary was taken on the current source of the kernel."""
+def kernel_source(one_launch_or_decode):
+    """Source file of the dominant kernel: the decode FFN (gemm_tc.cu) or the CTA-pair
+    grouped GEMM (gemm_pair.cu)."""
+    name = "gemm_tc.cu" if one_launch_or_decode else "gemm_pair.cu"
+    return os.path.join(ROOT, "mixture_experts_ffn_15_b200", "csrc", name)
+
+
+def source_sha(path):
     import hashlib
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def kernel_traffic(workload, src):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary
+    (profiles/traffic.json), if that summary was taken on the current source of the
+    kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         table = json.load(f)
-    src = os.path.join(ROOT, "mixture_experts_ffn_15_b200", "csrc", "gemm_tc.cu")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     e = table.get(workload)
-    if not e or e.get("source_sha") != sha:
+    if not e or e.get("source_sha") != source_sha(src):
         return None
     return e.get("bytes_per_launch")
 
@@ -426,11 +436,11 @@ def run_ours(args):
     roof["kernel"] = ("tc_ffn_decode_kernel<ROUTE> (routing, fc1 + SwiGLU, fc2 and combine, weight rows on M)"
                       if one_launch else
                       "tc_ffn_decode_kernel (fc1 + SwiGLU, fc2 and combine, weight rows on M)" if fused else
-                      "tc_gemm_kernel<TOK_SWIGLU> (fc1 + SwiGLU, token rows on M)")
+                      "tc_pair_kernel<SWIGLU> (fc1 + SwiGLU on CTA pairs, weight rows on M)")
     roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if hbm else 'bf16_tflops, burst'})"
     roof["algorithmic_per_launch"] = dom["bytes"] if hbm else dom["flops"]
     roof["kernel_us"] = round(dom_ms * 1e3, 2)
-    roof["traffic"] = kernel_traffic(wl.name)
+    roof["traffic"] = kernel_traffic(wl.name, kernel_source(fused))
 
     layer_s = ms_step * 1e-3
     layer = {"GB/s": layer_work["bytes"] / layer_s / 1e9, "TFLOP/s": layer_work["flops"] / layer_s / 1e12,
