@@ -59,7 +59,8 @@ def workspace_size(T, H, E, k, I, dtype):
 
 
 def alloc_workspace(nbytes, device):
-    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+    """Device workspace, zero-filled (moe_forward wants zeros before its first call)."""
+    return torch.zeros(int(nbytes), dtype=torch.uint8, device=device)
 
 
 def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out=None,

@@ -207,6 +207,28 @@ def test_forward_is_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_shared_workspace_across_paths_and_repeated_calls():
+    """One zero-filled workspace reused by calls of every bf16 path, in an order that
+    makes each path start from what the others left behind (the one-launch decode
+    relies on the counters being left at zero): every output equals the output of a
+    call on a fresh workspace, bit for bit, and the error word stays clear."""
+    cases = [W("ws_decode", T=4, H=256, E=64, k=4, I=128),      # one launch
+             W("ws_batched", T=100, H=256, E=64, k=4, I=128),    # tensor-core router + decode FFN
+             W("ws_small", T=100, H=256, E=16, k=4, I=128),      # one-CTA router + decode FFN
+             W("ws_prefill", T=1100, H=256, E=64, k=4, I=128)]   # tensor-core router + CTA pairs
+    devs = [device_inputs(make_inputs(wl)) for wl in cases]
+    fresh = [moe.forward(d["hidden"], d["router_w"], d["fc1"], d["fc2"], wl.k)
+             for wl, d in zip(cases, devs)]
+    need = max(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, torch.bfloat16) for wl in cases)
+    ws = moe.alloc_workspace(need, torch.device("cuda"))
+    for i in [0, 0, 1, 0, 2, 0, 3, 0, 1, 3, 2, 0, 0]:
+        wl, d = cases[i], devs[i]
+        got = moe.forward(d["hidden"], d["router_w"], d["fc1"], d["fc2"], wl.k, workspace=ws)
+        st, bits = moe.get_error(moe.workspace_error_word(ws))
+        assert st == 0 and bits == 0, (wl.name, bits)
+        assert torch.equal(got.view(torch.int16), fresh[i].view(torch.int16)), wl.name
+
+
 def test_exact_tie_goes_to_lower_index():
     wl = W("tie", T=50, H=128, E=8, k=2)
     inp = make_inputs(wl)
