@@ -21,7 +21,7 @@ namespace {
 // a token are loaded before they are summed (in slot order), so the loads overlap.
 constexpr int kCombineThreads = 128;
 
-template <bool BF16>
+template <bool BF16, int KC, int P>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm_dst,
                const float* __restrict__ topk_w, int T, int H, int k, int rows_max,
@@ -31,12 +31,26 @@ combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm
     constexpr int VEC = BF16 ? 8 : 4;
     const int nvec = H / VEC;
     const int v = blockIdx.y * kCombineThreads + threadIdx.x;
+    if constexpr (BF16) {
+        // P tokens per pass (about 16 row loads in flight per thread)
+        if (v >= nvec) return;
+        const uint4* y = reinterpret_cast<const uint4*>(y_perm);
+        uint4* o = reinterpret_cast<uint4*>(out);
+        const int step = gridDim.x;
+        int t = blockIdx.x;
+        for (; t + (P - 1) * step < T; t += P * step) {
+            uint4 r[P];
+            combine_vecs_bf16<KC, P>(y, nvec, perm_dst, topk_w, t, step, k, v, rows_max, r);
+#pragma unroll
+            for (int p = 0; p < P; ++p) o[static_cast<size_t>(t + p * step) * nvec + v] = r[p];
+        }
+        for (; t < T; t += step)
+            o[static_cast<size_t>(t) * nvec + v] = combine_vec_bf16(y, nvec, perm_dst, topk_w, t, k, v, rows_max);
+        return;
+    }
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
         if (v >= nvec) continue;
-        if constexpr (BF16) {
-            reinterpret_cast<uint4*>(out)[static_cast<size_t>(t) * nvec + v] = combine_vec_bf16(
-                reinterpret_cast<const uint4*>(y_perm), nvec, perm_dst, topk_w, t, k, v, rows_max);
-        } else {
+        {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < k; ++j) {
                 const int r = perm_dst[static_cast<size_t>(t) * k + j];
@@ -103,10 +117,14 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
     if (tok_blocks > T) tok_blocks = T;
     dim3 grid(static_cast<unsigned>(tok_blocks), static_cast<unsigned>(slabs));
     const int rows_max = T * k;
-    return bf16 ? launch_k(combine_kernel<true>, grid, dim3(kCombineThreads), 0, s, y_perm, perm_dst,
-                           topk_w, T, H, k, rows_max, out)
-                : launch_k(combine_kernel<false>, grid, dim3(kCombineThreads), 0, s, y_perm,
-                           perm_dst, topk_w, T, H, k, rows_max, out);
+    if (!bf16)
+        return launch_k(combine_kernel<false, 1, 1>, grid, dim3(kCombineThreads), 0, s, y_perm,
+                        perm_dst, topk_w, T, H, k, rows_max, out);
+    if (k <= 4)
+        return launch_k(combine_kernel<true, 4, 4>, grid, dim3(kCombineThreads), 0, s, y_perm,
+                        perm_dst, topk_w, T, H, k, rows_max, out);
+    return launch_k(combine_kernel<true, 8, 2>, grid, dim3(kCombineThreads), 0, s, y_perm, perm_dst,
+                    topk_w, T, H, k, rows_max, out);
 }
 
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,

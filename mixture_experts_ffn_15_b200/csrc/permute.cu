@@ -145,8 +145,17 @@ gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm
             for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
             continue;
         }
+        // 8 loads in flight per lane before the stores
         const uint4* s = hidden + static_cast<size_t>(src) * vec_per_row;
-        for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(s + v);
+        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (v0 + 32 * q < vec_per_row) buf[q] = __ldg(s + v0 + 32 * q);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (v0 + 32 * q < vec_per_row) dst[v0 + 32 * q] = buf[q];
+        }
     }
 }
 

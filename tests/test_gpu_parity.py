@@ -142,6 +142,39 @@ def test_expert_ffn(wl):
     assert_close(from_dev(y), y_ref, atol, rtol, "y_perm")
 
 
+# Expert row counts at every tile edge of the grouped GEMMs: empty, single rows, the
+# 32-token rounding of a CTA-pair tile, the 64-token chunks of the decode FFN, the
+# 256-token pair tile and one past each; fc1's 2I = 384 rows are a pair tile of 256
+# plus a half tile, fc2's H = 256 rows one pair tile.
+EDGE_COUNTS = [0, 1, 31, 32, 33, 63, 64, 65, 255, 256, 257, 300, 0, 2]
+
+
+@pytest.mark.parametrize("scale", [1, 0], ids=["pair_tiles", "decode_chunks"])
+def test_expert_ffn_at_tile_edges(scale):
+    """moe_expert_ffn on offsets built from EDGE_COUNTS, against the oracle's expert
+    FFN row block by row block.  scale=1 gives 1359 rows over 14 experts (> 64 per
+    expert on average: the CTA-pair GEMMs); scale=0 keeps the counts <= 65 (the
+    decode FFN, weight rows on M)."""
+    counts = np.array(EDGE_COUNTS if scale else [min(c, 65) for c in EDGE_COUNTS], dtype=np.int64)
+    E = len(counts)
+    rows = int(counts.sum())
+    wl = W("edges", T=rows, H=256, E=E, k=1, I=192)
+    inp = make_inputs(wl)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    x = inp["hidden"]                      # the rows themselves stand for x_perm
+    y = moe.expert_ffn(to_dev(x, wl.dtype), torch.from_numpy(offsets).cuda(), to_dev(inp["fc1"], wl.dtype),
+                       to_dev(inp["fc2"], wl.dtype))
+    torch.cuda.synchronize()
+    xv = inp.values("hidden")
+    y_ref = np.zeros((rows, wl.H))
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        if b > a:
+            y_ref[a:b] = O.expert_ffn(xv[a:b], inp.expert_values("fc1", e), inp.expert_values("fc2", e))
+    atol, rtol = tol(wl.dtype, y_ref)
+    assert_close(from_dev(y), y_ref, atol * row_scale(y_ref), rtol, f"y_perm at tile edges (scale {scale})")
+
+
 @pytest.mark.parametrize("wl", CASES, ids=IDS)
 def test_forward(wl):
     inp = make_inputs(wl)
