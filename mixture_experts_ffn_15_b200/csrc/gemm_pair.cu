@@ -272,10 +272,20 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                                 *reinterpret_cast<const uint4*>(scr + tt * 32 + q * 16);
                     }
                 } else {
+                    // lanes 2j, 2j+1 hold rows 2j, 2j+1.  For tokens (i, i+1) one exchange
+                    // gives the even lane both rows of token i and the odd lane both rows
+                    // of token i+1: one 4-byte store each, a full 128-byte wavefront.
+                    const bool odd = lane & 1;
+                    const int j = lane >> 1;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        *reinterpret_cast<__nv_bfloat16*>(scr + i * 64 + lane * 2) =
-                            __float2bfloat16_rn(__uint_as_float(v[i]));
+                    for (int i = 0; i < 32; i += 2) {
+                        const float a0 = __uint_as_float(v[i]), a1 = __uint_as_float(v[i + 1]);
+                        const float other = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                        const float lo = odd ? other : a0;    // row 2j of token i + odd
+                        const float hi = odd ? a1 : other;    // row 2j+1 of token i + odd
+                        const int tok = i + (odd ? 1 : 0);
+                        *reinterpret_cast<uint32_t*>(scr + tok * 64 + j * 4) = pack_bf16x2(lo, hi);
+                    }
                     __syncwarp();
 #pragma unroll
                     for (int pass = 0; pass < 4; ++pass) {
