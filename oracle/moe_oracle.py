@@ -19,6 +19,11 @@ following the pages in their order:
   expert at a time; `moe_dense_masked` is that reading, used as a brute-force pin.
 * same page, "Changes": the fused op is wrapped in CastLike, so the output has the
   input's dtype (the oracle reports float64; callers compare after widening).
+* same page, "Attribute set" and description: the op takes activation_alpha,
+  activation_beta and swiglu_limit (GPT-OSS: 1.702, 1.0, 7.0 -- the "1.702
+  multiplier", the "+1 bias on the up branch" and the clipping); `swiglu` implements
+  the family, standard SwiGLU being (1, 0, inf); the op's optional fc1/fc2 expert
+  biases are added to the pre-activation gate/up values and to the output.
 * "Contributing Gemma 4 support and ONNX export optimizations" (Hugging Face forum),
   "Key Technical Contributions", ONNX tracing compatibility: inside
   grouped_mm_experts_forward the per-expert token count is a bincount over the
@@ -34,7 +39,12 @@ notes of the repository):
   logits, so that both sides decide in the same precision;
 * normalize_routing_weights = 1 means softmax over all E logits, keep the k chosen
   probabilities, divide by their sum; with 0 the chosen probabilities are kept as is;
-* interleaved means row 2i = gate_i and row 2i+1 = up_i;
+* interleaved means row 2i = gate_i and row 2i+1 = up_i (the fc1 bias follows the
+  same layout as the fc1 rows);
+* SwiGLU attributes: act = (up' + beta) * gate' * sigmoid(alpha * gate') with
+  gate' = min(gate, limit) and up' = clip(up, -limit, limit) -- the multiplier acts
+  inside the sigmoid, the bias on the up branch after its clipping, and the clipping
+  bounds the gate from above only (the pages name the clipping but not its form);
 * the stable permutation puts the (token, slot) pairs of expert e in ascending
   token order, experts in ascending order.
 
@@ -50,6 +60,8 @@ from typing import Callable, Optional, Sequence, Union
 import numpy as np
 
 F64 = np.float64
+STANDARD_SWIGLU = (1.0, 0.0, float("inf"))   # (activation_alpha, activation_beta, swiglu_limit)
+GPT_OSS_SWIGLU = (1.702, 1.0, 7.0)
 NEAR_TIE_GAP = 1e-5          # float32 logit gap below which a selection is ambiguous
 TIE_BOUNDARY = 1             # flag bit: k-th and (k+1)-th logits within the gap
 TIE_WITHIN = 2               # flag bit: two adjacent chosen logits within the gap
@@ -213,9 +225,22 @@ def silu(g: np.ndarray) -> np.ndarray:
         return g / (1.0 + np.exp(-g))
 
 
-def swiglu(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
-    """Standard SwiGLU: silu(gate) * up (alpha 1, beta 0, no clipping)."""
-    return silu(gate) * up
+def swiglu(gate: np.ndarray, up: np.ndarray, alpha: float = 1.0, beta: float = 0.0,
+           limit: float = float("inf")) -> np.ndarray:
+    """SwiGLU with the op's attributes: (up' + beta) * gate' * sigmoid(alpha * gate'),
+    gate' = min(gate, limit), up' = clip(up, -limit, limit).
+
+    The standard attributes (1, 0, inf) give silu(gate) * up.
+    """
+    if limit != float("inf"):
+        gate = np.minimum(gate, limit)
+        up = np.clip(up, -limit, limit)
+    if alpha == 1.0:
+        s = silu(gate)
+    else:
+        with np.errstate(over="ignore"):
+            s = gate / (1.0 + np.exp(-alpha * gate))
+    return s * (up + beta) if beta != 0.0 else s * up
 
 
 def fc1_gate_up(fc1_e: np.ndarray, layout: str):
@@ -228,12 +253,21 @@ def fc1_gate_up(fc1_e: np.ndarray, layout: str):
     raise ValueError(f"unknown fc1 layout {layout!r}")
 
 
-def expert_ffn(x_rows, fc1_e, fc2_e, layout: str = "interleaved") -> np.ndarray:
-    """One expert on rows x [n, H]: a = swiglu(x W_gate^T, x W_up^T); y = a fc2^T.  [n, H]."""
+def expert_ffn(x_rows, fc1_e, fc2_e, layout: str = "interleaved", act=STANDARD_SWIGLU,
+               fc1_bias_e=None, fc2_bias_e=None) -> np.ndarray:
+    """One expert on rows x [n, H]: gate = x W_gate^T (+ b_gate), up = x W_up^T (+ b_up),
+    a = swiglu(gate, up, *act), y = a fc2^T (+ b2).  [n, H]; biases in fc1's layout."""
     x = np.asarray(x_rows, dtype=F64)
     w_gate, w_up = fc1_gate_up(np.asarray(fc1_e, dtype=F64), layout)
-    a = swiglu(x @ w_gate.T, x @ w_up.T)
-    return a @ np.asarray(fc2_e, dtype=F64).T
+    gate, up = x @ w_gate.T, x @ w_up.T
+    if fc1_bias_e is not None:
+        b_gate, b_up = fc1_gate_up(np.asarray(fc1_bias_e, dtype=F64)[:, None], layout)
+        gate, up = gate + b_gate[:, 0], up + b_up[:, 0]
+    a = swiglu(gate, up, *act)
+    y = a @ np.asarray(fc2_e, dtype=F64).T
+    if fc2_bias_e is not None:
+        y = y + np.asarray(fc2_bias_e, dtype=F64)
+    return y
 
 
 def combine(y_perm, perm_dst, w, T: int, k: int) -> np.ndarray:
@@ -251,12 +285,15 @@ def combine(y_perm, perm_dst, w, T: int, k: int) -> np.ndarray:
 def moe_forward(hidden, router_w, router_bias, fc1: ArrayOrGetter, fc2: ArrayOrGetter,
                 k: int, normalize: int, layout: str = "interleaved",
                 idx: Optional[np.ndarray] = None,
-                tokens: Optional[Sequence[int]] = None) -> dict:
+                tokens: Optional[Sequence[int]] = None, act=STANDARD_SWIGLU,
+                fc1_bias: Optional[ArrayOrGetter] = None,
+                fc2_bias: Optional[ArrayOrGetter] = None) -> dict:
     """The fused MoE layer on the given tensors, float64.
 
     `idx` forces the routing (its weights are still computed from the logits);
     `tokens` restricts the expert evaluation to those tokens (routing is always over
-    all tokens) and the returned `out` then has one row per listed token.
+    all tokens) and the returned `out` then has one row per listed token.  `act` is
+    (alpha, beta, limit); fc1_bias [E, 2I] (fc1's layout) and fc2_bias [E, H] optional.
     Returns dict(logits, idx, w, out).
     """
     x = np.asarray(hidden)
@@ -275,13 +312,16 @@ def moe_forward(hidden, router_w, router_bias, fc1: ArrayOrGetter, fc2: ArrayOrG
         rows, slots = np.nonzero(sub_idx == e)
         if rows.size == 0:
             continue
-        y = expert_ffn(x[tok[rows]], _expert(fc1, e), _expert(fc2, e), layout)
+        y = expert_ffn(x[tok[rows]], _expert(fc1, e), _expert(fc2, e), layout, act,
+                       None if fc1_bias is None else _expert(fc1_bias, e),
+                       None if fc2_bias is None else _expert(fc2_bias, e))
         out[rows] += w[tok[rows], slots][:, None] * y
     return dict(logits=L, idx=idx, w=w, out=out)
 
 
 def moe_dense_masked(hidden, router_w, router_bias, fc1, fc2, k: int, normalize: int,
-                     layout: str = "interleaved") -> np.ndarray:
+                     layout: str = "interleaved", act=STANDARD_SWIGLU, fc1_bias=None,
+                     fc2_bias=None) -> np.ndarray:
     """Brute force: every expert on every token, weighted by the routing mask.
 
     This is the static per-expert unroll of the fallback: expert e's output for all
@@ -299,17 +339,21 @@ def moe_dense_masked(hidden, router_w, router_bias, fc1, fc2, k: int, normalize:
             mask[t, idx[t, j]] = w[t, j]
     out = np.zeros((T, H), dtype=F64)
     for e in range(E):
-        out += mask[:, e:e + 1] * expert_ffn(x, _expert(fc1, e), _expert(fc2, e), layout)
+        out += mask[:, e:e + 1] * expert_ffn(
+            x, _expert(fc1, e), _expert(fc2, e), layout, act,
+            None if fc1_bias is None else _expert(fc1_bias, e),
+            None if fc2_bias is None else _expert(fc2_bias, e))
     return out
 
 
 def chunked_to_interleaved(fc1_chunked: np.ndarray) -> np.ndarray:
-    """[E, 2I, H] chunked -> interleaved: dst[e, 2j+s] = src[e, s*I + j] for s in {0, 1}."""
+    """[E, 2I, H] chunked -> interleaved: dst[e, 2j+s] = src[e, s*I + j] for s in {0, 1}.
+    Also for a bias [E, 2I] (rows of one element)."""
     src = np.asarray(fc1_chunked)
-    E, two_i, H = src.shape
+    E, two_i = src.shape[:2]
     I = two_i // 2
     dst = np.empty_like(src)
     for j in range(I):
         for s in (0, 1):
-            dst[:, 2 * j + s, :] = src[:, s * I + j, :]
+            dst[:, 2 * j + s] = src[:, s * I + j]
     return dst

@@ -338,14 +338,150 @@ def test_outlier_rows():
     assert 0 < big.sum() <= 10
 
 
+# ------------------------------------------------- SwiGLU attributes, expert biases
+# "Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", "Attribute set":
+# activation_alpha (the GPT-OSS "1.702 multiplier"), activation_beta (the "+1 bias
+# on the up branch"), swiglu_limit (the clipping); and the op's optional expert
+# biases.  Closed forms chosen so that each plausible misplacement changes a value.
+
+ALPHAS = [1.0, 1.702, 0.5]
+
+
+def check_swiglu_closed_forms():
+    # gate = ln(3) / alpha makes sigmoid(alpha * gate) = 3/4 exactly (in real
+    # arithmetic): act = (up + beta) * gate * 3/4.  A multiplier outside the sigmoid,
+    # a bias on the gate or sigmoid(-x) all change the value.
+    for alpha in ALPHAS:
+        g = math.log(3.0) / alpha
+        for beta in (0.0, 1.0, -0.25):
+            for u in (0.0, 1.5, -2.0):
+                got = float(O.swiglu(np.array([g]), np.array([u]), alpha, beta, 7.0)[0])
+                want = (u + beta) * g * 0.75
+                assert abs(got - want) <= 1e-14 * max(1.0, abs(want)), (alpha, beta, u, got, want)
+    # a zero gate gives exactly zero whatever the other attributes
+    assert np.all(O.swiglu(np.zeros(3), np.array([1.0, -3.0, 9.0]), 1.702, 1.0, 7.0) == 0.0)
+    # the standard attributes reduce to silu(gate) * up with silu(x) = x / (1 + e^-x)
+    g = np.linspace(-6, 6, 25)
+    u = np.cos(g)
+    want = np.array([x / (1.0 + math.exp(-x)) * y for x, y in zip(g, u)])
+    np.testing.assert_allclose(O.swiglu(g, u, *O.STANDARD_SWIGLU), want, rtol=1e-15, atol=0)
+
+
+def check_swiglu_limit_saturation():
+    L = 7.0
+    alpha, beta = O.GPT_OSS_SWIGLU[0], O.GPT_OSS_SWIGLU[1]
+    f = lambda g, u: float(O.swiglu(np.array([g]), np.array([u]), alpha, beta, L)[0])
+    # gate above the limit saturates at the limit; the up branch saturates on both sides
+    assert f(9.0, 0.3) == f(L, 0.3) and f(1e6, -2.0) == f(L, -2.0)
+    assert f(1.2, 12.0) == f(1.2, L) and f(1.2, -12.0) == f(1.2, -L)
+    # the bias is added after the up branch is clipped: at up = -L, (up' + beta) = -L + beta
+    g = math.log(3.0) / alpha
+    assert abs(f(g, -20.0) - (-L + beta) * g * 0.75) <= 1e-13
+    # the gate is not clipped from below (a large negative gate keeps decaying)
+    assert abs(f(-9.0, 1.0)) < abs(f(-L, 1.0))
+    # no limit: nothing saturates
+    assert O.swiglu(np.array([30.0]), np.array([30.0]), 1.0, 0.0, float("inf"))[0] > 800.0
+
+
+def check_expert_biases_zero_input():
+    # Zero input rows: gate = b_gate, up = b_up, y = fc2 act(b_gate, b_up) + b2.  With
+    # b_gate = ln(3)/alpha the activation is (b_up + beta) * b_gate * 3/4 in closed form.
+    alpha, beta, L = O.GPT_OSS_SWIGLU
+    g = math.log(3.0) / alpha
+    H, I = 3, 2
+    fc1 = np.full((2 * I, H), 0.37)                 # irrelevant: x = 0
+    fc2 = np.array([[1.0, 2.0], [0.0, -1.0], [0.5, 0.25]])
+    b1 = np.array([g, 0.5, g, -1.5])                 # interleaved: gate0, up0, gate1, up1
+    b2 = np.array([0.1, -0.2, 0.3])
+    a = np.array([(0.5 + beta) * g * 0.75, (-1.5 + beta) * g * 0.75])
+    want = fc2 @ a + b2
+    y = O.expert_ffn(np.zeros((2, H)), fc1, fc2, "interleaved", (alpha, beta, L), b1, b2)
+    np.testing.assert_allclose(y, np.stack([want, want]), rtol=1e-14, atol=1e-15)
+    # the layer: two experts with equal router logits (zero input) share weight 1/2 each
+    fc1s = np.stack([fc1, fc1])
+    fc2s = np.stack([fc2, 2.0 * fc2])
+    b1s = np.stack([b1, b1])
+    b2s = np.stack([b2, -b2])
+    want_layer = 0.5 * (fc2 @ a + b2) + 0.5 * (2.0 * fc2 @ a - b2)
+    r = O.moe_forward(np.zeros((1, H)), np.ones((2, H)), None, fc1s, fc2s, 2, 1,
+                      act=(alpha, beta, L), fc1_bias=b1s, fc2_bias=b2s)
+    np.testing.assert_allclose(r["out"][0], want_layer, rtol=1e-14, atol=1e-15)
+
+
+def check_biased_chunked_equals_interleaved():
+    # fc1 and its bias given chunked equal the same interleaved by the page's recipe
+    inp = small(T=10, E=4, k=2, layout="chunked")
+    E, two_i = inp.values("fc1").shape[:2]
+    rng = np.random.default_rng(11)
+    b1 = rng.standard_normal((E, two_i))
+    b2 = rng.standard_normal((E, inp.wl.H))
+    act = O.GPT_OSS_SWIGLU
+    a = fwd(inp, layout="chunked", act=act, fc1_bias=b1, fc2_bias=b2)["out"]
+    b = O.moe_forward(inp.values("hidden"), inp.values("router_w"), None,
+                      O.chunked_to_interleaved(inp.values("fc1")), inp.values("fc2"), 2, 1,
+                      "interleaved", act=act, fc1_bias=O.chunked_to_interleaved(b1), fc2_bias=b2)["out"]
+    np.testing.assert_array_equal(a, b)
+    # and the dense per-expert unroll agrees with the sparse layer
+    d = O.moe_dense_masked(inp.values("hidden"), inp.values("router_w"), None,
+                           O.chunked_to_interleaved(inp.values("fc1")), inp.values("fc2"), 2, 1,
+                           "interleaved", act, O.chunked_to_interleaved(b1), b2)
+    np.testing.assert_allclose(b, d, rtol=1e-12, atol=1e-13)
+
+
+def test_swiglu_closed_forms():
+    check_swiglu_closed_forms()
+
+
+def test_swiglu_limit_saturation():
+    check_swiglu_limit_saturation()
+
+
+def test_expert_biases_zero_input():
+    check_expert_biases_zero_input()
+
+
+def test_biased_chunked_equals_interleaved():
+    check_biased_chunked_equals_interleaved()
+
+
 # ---------------------------------------------------------------- mutation tests
 
 def _mut_drop_sigmoid(g):
     return g
 
 
-def _mut_swap_gate_up(gate, up):
+def _mut_swap_gate_up(gate, up, *attrs):
     return O.silu(up) * gate
+
+
+def _mut_alpha_outside_sigmoid(gate, up, alpha=1.0, beta=0.0, limit=float("inf")):
+    return alpha * _real_swiglu(gate, up, 1.0, beta, limit)
+
+
+def _mut_beta_on_gate(gate, up, alpha=1.0, beta=0.0, limit=float("inf")):
+    return _real_swiglu(gate + beta, up, alpha, 0.0, limit)
+
+
+def _mut_clip_gate_both_sides(gate, up, alpha=1.0, beta=0.0, limit=float("inf")):
+    return _real_swiglu(np.clip(gate, -limit, limit), up, alpha, beta, limit)
+
+
+def _mut_beta_before_clip(gate, up, alpha=1.0, beta=0.0, limit=float("inf")):
+    return _real_swiglu(gate, up + beta, alpha, 0.0, limit)
+
+
+def _mut_fc2_bias_dropped(x_rows, fc1_e, fc2_e, layout="interleaved", act=O.STANDARD_SWIGLU,
+                          fc1_bias_e=None, fc2_bias_e=None):
+    return _real_expert_ffn(x_rows, fc1_e, fc2_e, layout, act, fc1_bias_e, None)
+
+
+def _mut_fc1_bias_chunked(x_rows, fc1_e, fc2_e, layout="interleaved", act=O.STANDARD_SWIGLU,
+                          fc1_bias_e=None, fc2_bias_e=None):
+    if fc1_bias_e is not None and layout == "interleaved":
+        b = np.asarray(fc1_bias_e)
+        I = b.shape[0] // 2
+        fc1_bias_e = np.stack([b[:I], b[I:]], axis=1).ravel()   # read as if chunked
+    return _real_expert_ffn(x_rows, fc1_e, fc2_e, layout, act, fc1_bias_e, fc2_bias_e)
 
 
 def _mut_fc1_chunked_read(fc1_e, layout):
@@ -381,10 +517,18 @@ def _mut_unstable_perm(idx, E):
 
 
 _real_perm = O.stable_permutation
+_real_swiglu = O.swiglu
+_real_expert_ffn = O.expert_ffn
 
 MUTATIONS = [
     ("silu", _mut_drop_sigmoid),
     ("swiglu", _mut_swap_gate_up),
+    ("swiglu", _mut_alpha_outside_sigmoid),
+    ("swiglu", _mut_beta_on_gate),
+    ("swiglu", _mut_clip_gate_both_sides),
+    ("swiglu", _mut_beta_before_clip),
+    ("expert_ffn", _mut_fc2_bias_dropped),
+    ("expert_ffn", _mut_fc1_bias_chunked),
     ("fc1_gate_up", _mut_fc1_chunked_read),
     ("select_topk", _mut_ties_to_higher),
     ("routing_weights", _mut_no_renormalise),
@@ -393,10 +537,12 @@ MUTATIONS = [
 
 PIN_CHECKS = [check_golden_values, check_golden_routing, check_topk_brute_force,
               check_weights_sum_to_one, check_permutation, check_chunked_equals_interleaved,
-              check_dense_masked_equals_sparse, check_expert_ffn_scalar_loops]
+              check_dense_masked_equals_sparse, check_expert_ffn_scalar_loops,
+              check_swiglu_closed_forms, check_swiglu_limit_saturation,
+              check_expert_biases_zero_input, check_biased_chunked_equals_interleaved]
 
 
-@pytest.mark.parametrize("name,mutant", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+@pytest.mark.parametrize("name,mutant", MUTATIONS, ids=[f"{m[0]}-{m[1].__name__}" for m in MUTATIONS])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(O, name, mutant)
     caught = 0
