@@ -58,8 +58,12 @@ typedef enum {
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
 /* SwiGLU attributes of the op ("Attribute set": activation_alpha, activation_beta,
- * swiglu_limit).  Standard SwiGLU is {1.0f, 0.0f, INFINITY}; any other value is
- * rejected with MOE_ERR_UNSUPPORTED. */
+ * swiglu_limit; the GPT-OSS values 1.702, 1.0, 7.0 are the page's "1.702 multiplier",
+ * "+1 bias on the up branch" and clipping).  With g and u the pre-activation gate and
+ * up values of one output:
+ *   act = (clip(u, -limit, limit) + beta) * min(g, limit) * sigmoid(alpha * min(g, limit))
+ * Standard SwiGLU {1.0f, 0.0f, INFINITY} is silu(g) * u.  alpha and beta must be
+ * finite and limit > 0 (INFINITY: no clipping), else MOE_ERR_INVALID_ARG. */
 typedef struct { float alpha, beta, limit; } moe_swiglu;
 
 /* Bits of the device error word. */
@@ -124,19 +128,22 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
                        int32_t* err_word, void* workspace, size_t ws_bytes, void* stream);
 
 /* Grouped expert FFN over permuted rows.
- * ("Attribute set": standard SwiGLU, interleaved fc1; grouped matmul of
+ * ("Attribute set": SwiGLU attributes, interleaved fc1; grouped matmul of
  * grouped_mm_experts_forward.)
  *   x_perm   [rows, H] dt; rows offsets[e] .. offsets[e+1]-1 belong to expert e
  *   offsets  [E+1] int32 (device), non-decreasing, offsets[0] = 0, offsets[E] <= rows
  *   fc1      [E, 2I, H] dt, interleaved: row 2i = gate_i, row 2i+1 = up_i
  *   fc2      [E, H, I] dt
- *   y_perm   [rows, H] dt out: y_perm[r] = fc2_e (silu(g) * u) for r's expert e;
+ *   fc1_bias [E, 2I] dt (interleaved like fc1's rows) or NULL; fc2_bias [E, H] dt or
+ *            NULL: the op's optional expert biases, added in float32 to the gate/up
+ *            values before the activation and to the output
+ *   y_perm   [rows, H] dt out: y_perm[r] = fc2_e act(g, u) + b2_e for r's expert e;
  *            rows at or beyond offsets[E] are not written
  *   workspace at least moe_expert_ffn_workspace_size(rows, I, dt) bytes. */
 moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* fc1,
-                          const void* fc2, int rows, int H, int E, int I, moe_swiglu act,
-                          moe_dtype dt, void* y_perm, void* workspace, size_t ws_bytes,
-                          void* stream);
+                          const void* fc2, const void* fc1_bias, const void* fc2_bias, int rows,
+                          int H, int E, int I, moe_swiglu act, moe_dtype dt, void* y_perm,
+                          void* workspace, size_t ws_bytes, void* stream);
 
 /* Weighted combine (un-permute).
  *   out[t, :] = sum_{j<k} topk_w[t, j] * y_perm[perm_dst[t*k + j], :], summed in
@@ -150,14 +157,16 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 /* The whole layer: route -> permute -> fc1 + SwiGLU -> fc2 -> combine, all on
  * `stream`, no host synchronisation.
  *   hidden [T, H], router_w [E, H], fc1 [E, 2I, H] interleaved, fc2 [E, H, I]: dt
+ *   fc1_bias [E, 2I], fc2_bias [E, H] dt or NULL (as in moe_expert_ffn)
  *   router_bias [E] float32 or NULL; out [T, H] dt
  *   workspace >= moe_workspace_size(T, H, E, k, I, dt) bytes, 256-byte aligned; it
  *   holds every intermediate, and its first word is the device error word.
  * T = 0 is a no-op returning MOE_OK. */
 moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
-                       const void* fc1, const void* fc2, int T, int H, int E, int k, int I,
-                       int normalize, moe_swiglu act, moe_dtype dt, void* out,
-                       void* workspace, size_t ws_bytes, void* stream);
+                       const void* fc1, const void* fc2, const void* fc1_bias,
+                       const void* fc2_bias, int T, int H, int E, int k, int I, int normalize,
+                       moe_swiglu act, moe_dtype dt, void* out, void* workspace, size_t ws_bytes,
+                       void* stream);
 
 /* The whole layer without a workspace argument, for callers that cannot allocate
  * device memory while they run it (an engine plugin or a serving loop that forbids
@@ -176,7 +185,8 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
  *   overlap on the GPU, from two streams or two host threads, race on it. */
 #define MOE_STATIC_SCRATCH_BYTES (8u << 20)
 moe_status moe_forward_static(const void* hidden, const void* router_w, const float* router_bias,
-                              const void* fc1, const void* fc2, int T, int H, int E, int k, int I,
+                              const void* fc1, const void* fc2, const void* fc1_bias,
+                              const void* fc2_bias, int T, int H, int E, int k, int I,
                               int normalize, moe_swiglu act, moe_dtype dt, void* out,
                               void* stream);
 

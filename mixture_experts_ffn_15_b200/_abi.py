@@ -14,6 +14,7 @@ class MoeSwiglu(ctypes.Structure):
 
 
 STANDARD_SWIGLU = MoeSwiglu(1.0, 0.0, float("inf"))
+GPT_OSS_SWIGLU = MoeSwiglu(1.702, 1.0, 7.0)
 
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
 
@@ -25,12 +26,13 @@ SIGNATURES = {
     "moe_workspace_error_word": (_vp, [_vp]),
     "moe_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, MoeSwiglu, _i, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, MoeSwiglu, _i, _vp, _vp,
+                            _sz, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
-    "moe_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, MoeSwiglu, _i, _vp, _vp,
-                         _sz, _vp]),
-    "moe_forward_static": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, MoeSwiglu, _i,
-                                _vp, _vp]),
+    "moe_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, MoeSwiglu, _i,
+                         _vp, _vp, _sz, _vp]),
+    "moe_forward_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                MoeSwiglu, _i, _vp, _vp]),
     "convert_chunked_to_interleaved": (_i, [_vp, _vp, _i, _i, _i, _i, _vp]),
     "moe_get_error": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),

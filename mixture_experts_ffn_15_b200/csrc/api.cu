@@ -120,6 +120,19 @@ bool standard_swiglu(const moe_swiglu& a) {
     return a.alpha == 1.0f && a.beta == 0.0f && isinf(a.limit) && a.limit > 0;
 }
 
+// Finite alpha and beta, a positive limit (+inf = no clipping).
+bool valid_swiglu(const moe_swiglu& a) {
+    return isfinite(a.alpha) && isfinite(a.beta) && !isnan(a.limit) && a.limit > 0.0f;
+}
+
+FfnEpilogue make_epilogue(const moe_swiglu& a, const void* fc1_bias, const void* fc2_bias) {
+    FfnEpilogue ep;
+    ep.act = SwigluAttr{a.alpha, a.beta, a.limit, standard_swiglu(a) ? 1 : 0};
+    ep.fc1_bias = fc1_bias;
+    ep.fc2_bias = fc2_bias;
+    return ep;
+}
+
 // Which kernels moe_forward runs for these sizes (bits of moe_forward_path).
 constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
               kPathF32Ffn = 16, kPathFusedRoute = 32;
@@ -157,7 +170,7 @@ using namespace moe;
 
 extern "C" {
 
-int moe_version(void) { return 100; }
+int moe_version(void) { return 200; }
 
 unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 
@@ -280,13 +293,14 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
 }
 
 moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* fc1,
-                          const void* fc2, int rows, int H, int E, int I, moe_swiglu act,
-                          moe_dtype dt, void* y_perm, void* workspace, size_t ws_bytes,
-                          void* stream) {
+                          const void* fc2, const void* fc1_bias, const void* fc2_bias, int rows,
+                          int H, int E, int I, moe_swiglu act, moe_dtype dt, void* y_perm,
+                          void* workspace, size_t ws_bytes, void* stream) {
     if (rows < 0 || H <= 0 || H % 8 || I <= 0 || I % 8 || E <= 0 || E > kMaxExperts ||
-        !valid_dtype(dt))
+        !valid_dtype(dt) || !valid_swiglu(act))
         return MOE_ERR_INVALID_ARG;
-    if (!standard_swiglu(act)) return MOE_ERR_UNSUPPORTED;
+    if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
+        return MOE_ERR_INVALID_ARG;
     if (dt == MOE_BF16 && !tc_ffn_supported(H, I)) return MOE_ERR_UNSUPPORTED;
     if (rows == 0) return MOE_OK;
     if (!x_perm || !offsets || !fc1 || !fc2 || !y_perm || !workspace) return MOE_ERR_INVALID_ARG;
@@ -301,18 +315,19 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + kAlign +
                                               align_up(static_cast<size_t>(rows) * I * elem_size(dt)));
     MOE_CUDA(cudaMemsetAsync(err, 0, 4, s));
+    const FfnEpilogue ep = make_epilogue(act, fc1_bias, fc2_bias);
     if (dt == MOE_BF16 && decode_ffn_supported(rows, E, H, I)) {
         MOE_CUDA(cudaMemsetAsync(ctr, 0, static_cast<size_t>(decode_ffn_counters(rows, E)) * 4, s));
         MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1, fc2, rows, H, E, I,
-                                   act_buf, y_perm, ctr, err, nullptr, nullptr, 0, nullptr, s));
+                                   act_buf, y_perm, ctr, err, nullptr, nullptr, 0, nullptr, s, ep));
     } else if (dt == MOE_BF16) {
         MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y_perm, err, s,
-                                 nullptr));
+                                 nullptr, ep));
     } else {
         MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                      static_cast<const float*>(fc1), static_cast<const float*>(fc2),
                                      rows, H, E, I, static_cast<float*>(act_buf),
-                                     static_cast<float*>(y_perm), s, nullptr));
+                                     static_cast<float*>(y_perm), s, nullptr, ep));
     }
     return MOE_OK;
 }
@@ -331,11 +346,13 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 }
 
 moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
-                       const void* fc1, const void* fc2, int T, int H, int E, int k, int I,
-                       int normalize, moe_swiglu act, moe_dtype dt, void* out, void* workspace,
-                       size_t ws_bytes, void* stream) {
-    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt)) return MOE_ERR_INVALID_ARG;
-    if (!standard_swiglu(act)) return MOE_ERR_UNSUPPORTED;
+                       const void* fc1, const void* fc2, const void* fc1_bias, const void* fc2_bias,
+                       int T, int H, int E, int k, int I, int normalize, moe_swiglu act,
+                       moe_dtype dt, void* out, void* workspace, size_t ws_bytes, void* stream) {
+    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt) || !valid_swiglu(act))
+        return MOE_ERR_INVALID_ARG;
+    if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
+        return MOE_ERR_INVALID_ARG;
     if (dt == MOE_BF16 && !tc_ffn_supported(H, I)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
     if (!hidden || !router_w || !fc1 || !fc2 || !out || !workspace) return MOE_ERR_INVALID_ARG;
@@ -362,6 +379,7 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     const int rows = T * k;
 
     const int path = forward_path(T, H, E, k, I, dt);
+    const FfnEpilogue ep = make_epilogue(act, fc1_bias, fc2_bias);
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
@@ -397,6 +415,7 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         a.counters = ctr;
         a.err = err;
         a.out = out;
+        a.ep = ep;
         MOE_CUDA(launch_ffn_decode_routed(a, s));
         record(3, s);
         record(4, s);
@@ -468,7 +487,7 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         // ... and the weighted combine, after every fc2 unit has published its rows
         MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
                                    T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err,
-                                   perm_dst, w, k, out, s));
+                                   perm_dst, w, k, out, s, ep));
         record(3, s);
         record(4, s);
         record(5, s);
@@ -480,13 +499,13 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
         if (bf16)
             MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
-                                     mid));
+                                     mid, ep));
         else
             MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                          static_cast<const float*>(fc1),
                                          static_cast<const float*>(fc2), rows, H, E, I,
                                          static_cast<float*>(act_buf), static_cast<float*>(y), s,
-                                         mid));
+                                         mid, ep));
     }
     record(4, s);
     MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));

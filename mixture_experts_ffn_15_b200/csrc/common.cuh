@@ -64,4 +64,35 @@ __device__ __forceinline__ float swiglu_fast(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// The op's SwiGLU attributes ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op -
+// #326", "Attribute set": activation_alpha, activation_beta, swiglu_limit):
+//   act = (clip(u, -limit, limit) + beta) * g' * sigmoid(alpha * g'),  g' = min(g, limit)
+// `standard` marks (1, 0, inf), which runs the plain silu(g) * u above.
+struct SwigluAttr {
+    float alpha, beta, limit;
+    int standard;
+};
+
+__device__ __forceinline__ float swiglu_attr(float g, float u, const SwigluAttr& a) {
+    if (a.standard) return swiglu_f32(g, u);
+    if (a.limit < INFINITY) {
+        g = fminf(g, a.limit);
+        u = fminf(fmaxf(u, -a.limit), a.limit);
+    }
+    return g / (1.0f + expf(-a.alpha * g)) * (u + a.beta);
+}
+
+__device__ __forceinline__ float swiglu_attr_fast(float g, float u, const SwigluAttr& a) {
+    if (a.standard) return swiglu_fast(g, u);
+    if (a.limit < INFINITY) {
+        g = fminf(g, a.limit);
+        u = fminf(fmaxf(u, -a.limit), a.limit);
+    }
+    return __fdividef(g, 1.0f + __expf(-a.alpha * g)) * (u + a.beta);
+}
+
+__device__ __forceinline__ float bf16_at(const __nv_bfloat16* p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+
 }  // namespace moe

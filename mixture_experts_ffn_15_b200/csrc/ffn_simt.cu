@@ -1,9 +1,9 @@
 // float32 grouped expert FFN on plain FMA (no TF32, which would not meet a 1e-4
 // relative tolerance).  Same math as the tensor-core path:
-//   act[r, i] = silu(x_perm[r] . fc1[e, 2i]) * (x_perm[r] . fc1[e, 2i+1])
-//   y[r, h]   = act[r] . fc2[e, h]
+//   act[r, i] = swiglu(x_perm[r] . fc1[e, 2i] + b1[e, 2i], x_perm[r] . fc1[e, 2i+1] + b1[e, 2i+1])
+//   y[r, h]   = act[r] . fc2[e, h] + b2[e, h]
 // for the rows r of expert e ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op -
-// #326", "Attribute set": standard SwiGLU, interleaved fc1).
+// #326", "Attribute set": SwiGLU attributes, interleaved fc1; the biases optional).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,7 +18,8 @@ template <bool SWIGLU>
 __global__ void __launch_bounds__(256)
 simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __restrict__ W,
                          int n_w, int K, const int32_t* __restrict__ offsets, int E, int rows,
-                         float* __restrict__ out, int ldo) {
+                         float* __restrict__ out, int ldo, const float* __restrict__ bias,
+                         SwigluAttr act) {
     __shared__ float sA[SBM][SBK + 1];
     __shared__ float sW[SBN][SBK + 1];
     __shared__ int s_off[kMaxExperts + 1];
@@ -79,15 +80,23 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
             }
             __syncthreads();
         }
+        const int n0 = nt * SBN + tx * 4;
+        if (bias != nullptr) {   // the expert's bias of each output column
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float b = n0 + q < n_w ? bias[static_cast<size_t>(e) * n_w + n0 + q] : 0.f;
+                acc[0][q] += b;
+                acc[1][q] += b;
+            }
+        }
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
             const int r = ty * 2 + rr;
             if (r >= nrows) continue;
             float* o = out + static_cast<size_t>(row0 + r) * ldo;
-            const int n0 = nt * SBN + tx * 4;
             if constexpr (SWIGLU) {
-                if (n0 + 1 < n_w) o[n0 / 2] = swiglu_f32(acc[rr][0], acc[rr][1]);
-                if (n0 + 3 < n_w) o[n0 / 2 + 1] = swiglu_f32(acc[rr][2], acc[rr][3]);
+                if (n0 + 1 < n_w) o[n0 / 2] = swiglu_attr(acc[rr][0], acc[rr][1], act);
+                if (n0 + 3 < n_w) o[n0 / 2 + 1] = swiglu_attr(acc[rr][2], acc[rr][3], act);
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -107,14 +116,16 @@ int simt_grid(int rows, int E, int n_w) {
 
 cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
                                 const float* fc2, int rows, int H, int E, int I, float* act,
-                                float* y, cudaStream_t s, cudaEvent_t mid) {
+                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep) {
     if (rows <= 0) return cudaSuccess;
     cudaError_t err = launch_k(simt_grouped_gemm_kernel<true>, dim3(simt_grid(rows, E, 2 * I)),
-                               dim3(256), 0, s, x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I);
+                               dim3(256), 0, s, x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I,
+                               static_cast<const float*>(ep.fc1_bias), ep.act);
     if (err != cudaSuccess) return err;
     if (mid) record_event(mid, s);
     return launch_k(simt_grouped_gemm_kernel<false>, dim3(simt_grid(rows, E, H)), dim3(256), 0, s,
-                    static_cast<const float*>(act), I, fc2, H, I, offsets, E, rows, y, H);
+                    static_cast<const float*>(act), I, fc2, H, I, offsets, E, rows, y, H,
+                    static_cast<const float*>(ep.fc2_bias), ep.act);
 }
 
 }  // namespace moe

@@ -4,8 +4,10 @@
 // and ONNX export optimizations", "Key Technical Contributions") over each expert's
 // contiguous block of permuted rows, with standard SwiGLU on the interleaved fc1
 // ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", "Attribute set"):
-//   fc1 + SwiGLU: act[r, i] = silu(x[r] . fc1[e, 2i]) * (x[r] . fc1[e, 2i+1])
-//   fc2:          y[r, h]   = act[r] . fc2[e, h]
+//   fc1 + SwiGLU: act[r, i] = swiglu(x[r] . fc1[e, 2i] + b1[e, 2i], x[r] . fc1[e, 2i+1] + b1[e, 2i+1])
+//   fc2:          y[r, h]   = act[r] . fc2[e, h] + b2[e, h]
+// (standard SwiGLU silu(g) * u, or the op's alpha/beta/limit attributes; the biases
+// optional)
 //
 // Orientation: the expert's WEIGHT rows are the MMA's M side and its tokens the N
 // side.  A unit is (expert, tile of up to 256 tokens, tile of 256 weight rows); a
@@ -72,6 +74,8 @@ struct PairParams {
     __nv_bfloat16* out;       // [rows, ldo]
     int ldo;                  // I (fc1) or H (fc2)
     int32_t* err;
+    SwigluAttr act;           // fc1: SwiGLU attributes
+    const __nv_bfloat16* bias;   // [E, n_out] bias of the weight rows, or nullptr
 };
 
 struct PUnit {
@@ -238,6 +242,10 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // n_out is a multiple of 32)
             const int w0 = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows + quad * 32;
             const bool wvalid = w0 < p.n_out;
+            // this lane's weight row's bias (fc1: interleaved rows, fc2: h)
+            const float bias = (p.bias && wvalid)
+                                   ? bf16_at(p.bias, static_cast<size_t>(d.g) * p.n_out + w0 + lane)
+                                   : 0.f;
 #pragma unroll 1
             for (int c = part * 32; c < d.nrows; c += 64) {
                 uint32_t v[32];
@@ -254,13 +262,14 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     const int j = lane >> 1;   // output 0..15 of this warp: 32 bytes a token
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
-                        const float mine_g = __uint_as_float(v[i]), mine_u = __uint_as_float(v[i + 1]);
+                        const float mine_g = __uint_as_float(v[i]) + bias;
+                        const float mine_u = __uint_as_float(v[i + 1]) + bias;
                         const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_g : mine_u, 1);
                         const float g = odd ? other : mine_g;          // gate of token i + odd
                         const float u = odd ? mine_u : other;          // up of token i + odd
                         const int tok = i + (odd ? 1 : 0);
                         *reinterpret_cast<__nv_bfloat16*>(scr + tok * 32 + j * 2) =
-                            __float2bfloat16_rn(swiglu_fast(g, u));
+                            __float2bfloat16_rn(swiglu_attr_fast(g, u, p.act));
                     }
                     __syncwarp();
                     const int i0 = w0 >> 1;   // first output column of this warp
@@ -279,7 +288,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     const int j = lane >> 1;
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
-                        const float a0 = __uint_as_float(v[i]), a1 = __uint_as_float(v[i + 1]);
+                        const float a0 = __uint_as_float(v[i]) + bias, a1 = __uint_as_float(v[i + 1]) + bias;
                         const float other = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
                         const float lo = odd ? other : a0;    // row 2j of token i + odd
                         const float hi = odd ? a1 : other;    // row 2j+1 of token i + odd
@@ -397,11 +406,13 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
 // One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
 // the experts' blocks) and w [E * n_out, K].
 cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
-                      const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s) {
+                      const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s,
+                      const SwigluAttr& act, const void* bias) {
     CUtensorMap mw, mx;
     if (!make_map(&mw, w, static_cast<long long>(E) * n_out, K, kPWRows)) return cudaErrorInvalidValue;
     if (!make_map(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
-    PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err};
+    PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, act,
+                 static_cast<const __nv_bfloat16*>(bias)};
     const long long units = (static_cast<long long>((rows + kPTok - 1) / kPTok) + E) *
                             ((n_out + 2 * kPWRows - 1) / (2 * kPWRows));
     return swiglu ? launch_pair<true>(mw, mx, p, units, s) : launch_pair<false>(mw, mx, p, units, s);
@@ -413,12 +424,13 @@ bool pair_ffn_supported(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && 
 
 cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid) {
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep) {
     if (rows <= 0) return cudaSuccess;
-    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s);
+    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s, ep.act,
+                              ep.fc1_bias);
     if (e != cudaSuccess) return e;
     if (mid) record_event(mid, s);
-    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s);
+    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s, ep.act, ep.fc2_bias);
 }
 
 }  // namespace moe

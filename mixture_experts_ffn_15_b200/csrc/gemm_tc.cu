@@ -430,6 +430,9 @@ struct DecodeParams {
     int k;
     __nv_bfloat16* out;
     int32_t* err;
+    SwigluAttr act_attr;            // SwiGLU attributes
+    const __nv_bfloat16* b1;        // [E, 2I] fc1 bias (interleaved rows) or nullptr
+    const __nv_bfloat16* b2;        // [E, H] fc2 bias or nullptr
     // ROUTE: the routing runs inside the launch (fields below); offsets, perm_src,
     // perm_dst and topk_w above are then unused (the kernel keeps them in shared memory)
     const void* hidden;       // [T, H]
@@ -923,6 +926,10 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                 static_cast<uint32_t>(acc * C::kAccStride);
             const int wr = d.mt * BM + r;   // weight row inside the expert
+            // this lane's weight row's bias (fc1 in interleaved row order, fc2 by h)
+            const __nv_bfloat16* bsrc = f1 ? p.b1 : p.b2;
+            const float bias =
+                bsrc ? bf16_at(bsrc, static_cast<size_t>(d.g) * (f1 ? 2 * p.I : p.H) + wr) : 0.f;
 #pragma unroll 1
             for (int c = 0; c < d.nrows; c += 16) {
                 uint32_t v[16];
@@ -931,12 +938,12 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int n = c + i;
-                    const float x = f32(v[i]);
+                    const float x = f32(v[i]) + bias;
                     if (f1) {
                         const float up = __shfl_xor_sync(0xffffffffu, x, 1);
                         if (!(lane & 1) && n < d.nrows)
                             p.act[static_cast<size_t>(d.row0 + n) * p.I + (wr >> 1)] =
-                                __float2bfloat16_rn(swiglu_f32(x, up));
+                                __float2bfloat16_rn(swiglu_attr(x, up, p.act_attr));
                     } else if (n < d.nrows) {
                         p.y[static_cast<size_t>(d.row0 + n) * p.H + wr] = __float2bfloat16_rn(x);
                     }
@@ -1116,7 +1123,7 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
                               const int32_t* perm_dst, const float* topk_w, int k, void* out,
-                              cudaStream_t s) {
+                              cudaStream_t s, const FfnEpilogue& ep) {
     if (rows <= 0) return cudaSuccess;
     CUtensorMap w1, x, w2, a;
     if (!make_map(&w1, fc1, static_cast<long long>(E) * 2 * I, H, BM)) return cudaErrorInvalidValue;
@@ -1146,6 +1153,9 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     p.k = k;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.err = err;
+    p.act_attr = ep.act;
+    p.b1 = static_cast<const __nv_bfloat16*>(ep.fc1_bias);
+    p.b2 = static_cast<const __nv_bfloat16*>(ep.fc2_bias);
     const int grid = decode_grid(rows, E, H, I);
     return perm_src ? launch_decode<true, false>(w1, x, w2, a, p, grid, s)
                     : launch_decode<false, false>(w1, x, w2, a, p, grid, s);
@@ -1176,6 +1186,9 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     p.k = r.k;
     p.out = static_cast<__nv_bfloat16*>(r.out);
     p.err = r.err;
+    p.act_attr = r.ep.act;
+    p.b1 = static_cast<const __nv_bfloat16*>(r.ep.fc1_bias);
+    p.b2 = static_cast<const __nv_bfloat16*>(r.ep.fc2_bias);
     p.hidden = r.hidden;
     p.router_w = r.router_w;
     p.bias = r.bias;

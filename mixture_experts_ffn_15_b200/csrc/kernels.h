@@ -2,9 +2,12 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <utility>
+
+#include "common.cuh"
 
 namespace moe {
 
@@ -98,10 +101,19 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
                            cudaStream_t s);
 
+// What the expert FFN kernels apply after each GEMM: the SwiGLU attributes and the
+// optional expert biases (fc1_bias [E, 2I] in fc1's interleaved row order, fc2_bias
+// [E, H]; the activation dtype; nullptr = none).
+struct FfnEpilogue {
+    SwigluAttr act{1.0f, 0.0f, INFINITY, 1};
+    const void* fc1_bias = nullptr;
+    const void* fc2_bias = nullptr;
+};
+
 // ---------------------------------------------------------------- ffn_simt.cu
 cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
                                 const float* fc2, int rows, int H, int E, int I, float* act,
-                                float* y, cudaStream_t s, cudaEvent_t mid);
+                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep);
 
 // ---------------------------------------------------------------- gemm_tc.cu
 bool tc_ffn_supported(int H, int I);
@@ -120,7 +132,7 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
 bool pair_ffn_supported(int H, int I);
 cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid);
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep);
 
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);
@@ -153,6 +165,7 @@ struct DecodeRoutedArgs {
     int32_t* counters;         // zero on entry
     int32_t* err;
     void* out;                 // [T, H]
+    FfnEpilogue ep;
 };
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& a, cudaStream_t s);
 
@@ -160,6 +173,6 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
                               const int32_t* perm_dst, const float* topk_w, int k, void* out,
-                              cudaStream_t s);
+                              cudaStream_t s, const FfnEpilogue& ep);
 
 }  // namespace moe

@@ -46,7 +46,8 @@ moe_status scratch_address(void** out) {
 
 extern "C" moe_status moe_forward_static(const void* hidden, const void* router_w,
                                          const float* router_bias, const void* fc1,
-                                         const void* fc2, int T, int H, int E, int k, int I,
+                                         const void* fc2, const void* fc1_bias,
+                                         const void* fc2_bias, int T, int H, int E, int k, int I,
                                          int normalize, moe_swiglu act, moe_dtype dt, void* out,
                                          void* stream) {
     const size_t need = moe_workspace_size(T, H, E, k, I, dt);
@@ -55,6 +56,7 @@ extern "C" moe_status moe_forward_static(const void* hidden, const void* router_
     void* scratch = nullptr;
     const moe_status st = scratch_address(&scratch);
     if (st != MOE_OK) return st;
-    return moe_forward(hidden, router_w, router_bias, fc1, fc2, T, H, E, k, I, normalize, act, dt,
-                       out, scratch, static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES), stream);
+    return moe_forward(hidden, router_w, router_bias, fc1, fc2, fc1_bias, fc2_bias, T, H, E, k, I,
+                       normalize, act, dt, out, scratch, static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES),
+                       stream);
 }

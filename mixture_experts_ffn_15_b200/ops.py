@@ -63,9 +63,20 @@ def alloc_workspace(nbytes, device):
     return torch.zeros(int(nbytes), dtype=torch.uint8, device=device)
 
 
+def _biases(fc1_bias, fc2_bias, dt, E, I, H):
+    if fc1_bias is not None:
+        _need(fc1_bias, "fc1_bias", dt, (E, 2 * I))
+    if fc2_bias is not None:
+        _need(fc2_bias, "fc2_bias", dt, (E, H))
+
+
 def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out=None,
-            workspace=None, stream=None, swiglu=(1.0, 0.0, float("inf"))):
-    """The fused MoE layer: out[T, H] = sum_j w[t, j] * FFN_{idx[t, j]}(hidden[t])."""
+            workspace=None, stream=None, swiglu=(1.0, 0.0, float("inf")), fc1_bias=None,
+            fc2_bias=None):
+    """The fused MoE layer: out[T, H] = sum_j w[t, j] * FFN_{idx[t, j]}(hidden[t]).
+
+    swiglu = (alpha, beta, limit) of the op; fc1_bias [E, 2I] (fc1's interleaved row
+    order) and fc2_bias [E, H] are the optional expert biases."""
     _need(hidden, "hidden")
     dt = hidden.dtype
     T, H = hidden.shape
@@ -76,6 +87,7 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
     _need(fc2, "fc2", dt, (E, H, I))
     if router_bias is not None:
         _need(router_bias, "router_bias", torch.float32, (E,))
+    _biases(fc1_bias, fc2_bias, dt, E, I, H)
     if out is None:
         out = torch.empty_like(hidden)
     _need(out, "out", dt, (T, H))
@@ -85,8 +97,9 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
         workspace = alloc_workspace(max(need, 256), hidden.device)
     _need(workspace, "workspace", torch.uint8)
     st = _lib().moe_forward(_ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(fc1), _ptr(fc2),
-                            T, H, E, k, I, int(bool(normalize)), _swiglu(*swiglu), _dtcode(hidden),
-                            _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+                            _ptr(fc1_bias), _ptr(fc2_bias), T, H, E, k, I, int(bool(normalize)),
+                            _swiglu(*swiglu), _dtcode(hidden), _ptr(out), _ptr(workspace),
+                            workspace.numel(), _stream(stream))
     check(st, "moe_forward")
     return out
 
@@ -143,8 +156,9 @@ def permute(topk_idx, E, hidden=None, err_word=None, stream=None):
 
 
 def expert_ffn(x_perm, offsets, fc1, fc2, y_perm=None, stream=None,
-               swiglu=(1.0, 0.0, float("inf"))):
-    """y_perm[r] = fc2_e(silu(x fc1_gate^T) * (x fc1_up^T)) over each expert's rows."""
+               swiglu=(1.0, 0.0, float("inf")), fc1_bias=None, fc2_bias=None):
+    """y_perm[r] = fc2_e act(x fc1_gate^T + b_gate, x fc1_up^T + b_up) + b2_e over each
+    expert's rows (act: SwiGLU with the op's (alpha, beta, limit))."""
     _need(x_perm, "x_perm")
     rows, H = x_perm.shape
     E, two_i, _ = fc1.shape
@@ -152,13 +166,14 @@ def expert_ffn(x_perm, offsets, fc1, fc2, y_perm=None, stream=None,
     _need(offsets, "offsets", torch.int32, (E + 1,))
     _need(fc1, "fc1", x_perm.dtype, (E, 2 * I, H))
     _need(fc2, "fc2", x_perm.dtype, (E, H, I))
+    _biases(fc1_bias, fc2_bias, x_perm.dtype, E, I, H)
     if y_perm is None:
         y_perm = torch.zeros_like(x_perm)
     dt = _dtcode(x_perm)
     ws = alloc_workspace(_lib().moe_expert_ffn_workspace_size(rows, I, dt), x_perm.device)
-    st = _lib().moe_expert_ffn(_ptr(x_perm), _ptr(offsets), _ptr(fc1), _ptr(fc2), rows, H, E, I,
-                               _swiglu(*swiglu), dt, _ptr(y_perm), _ptr(ws), ws.numel(),
-                               _stream(stream))
+    st = _lib().moe_expert_ffn(_ptr(x_perm), _ptr(offsets), _ptr(fc1), _ptr(fc2), _ptr(fc1_bias),
+                               _ptr(fc2_bias), rows, H, E, I, _swiglu(*swiglu), dt, _ptr(y_perm),
+                               _ptr(ws), ws.numel(), _stream(stream))
     check(st, "moe_expert_ffn")
     return y_perm
 

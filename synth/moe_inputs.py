@@ -38,6 +38,7 @@ import numpy as np
 
 # Stream identifiers: fixed forever, so that a seed always means the same tensors.
 _S_HIDDEN, _S_ROUTER, _S_BIAS, _S_FC1, _S_FC2, _S_OUTLIER = 1, 2, 3, 4, 5, 6
+_S_FC1_BIAS, _S_FC2_BIAS = 7, 8
 
 
 @dataclass(frozen=True)
@@ -173,3 +174,13 @@ def make_inputs(wl: Workload, seed: Optional[int] = None, weights: bool = True) 
         arrays["fc1"] = fc1
         arrays["fc2"] = fc2
     return MoEInputs(wl, arrays)
+
+
+def make_expert_biases(wl: Workload, std: float = 0.5, seed: Optional[int] = None):
+    """The op's optional expert biases for `wl`: fc1_bias [E, 2I] (in the row order of
+    the workload's fc1 layout) and fc2_bias [E, H], N(0, std), stored like the weights
+    (bf16 bits or float32)."""
+    s = wl.seed if seed is None else seed
+    b1 = _normal((s, _S_FC1_BIAS), (wl.E, 2 * wl.I), std)
+    b2 = _normal((s, _S_FC2_BIAS), (wl.E, wl.H), std)
+    return _store(b1, wl.dtype), _store(b2, wl.dtype)

@@ -139,3 +139,11 @@ def sample_tokens(T, idx, E, n=256, must=(), seed=123):
     extra = rng.choice(T, size=min(T, n), replace=False)
     picks.update(int(t) for t in extra)
     return np.array(sorted(picks), dtype=np.int64)
+
+
+def bf16_storage_bound(act, fc2_e, y):
+    """First-order bound on what storing act and y in bf16 (round to nearest, relative
+    error <= 2^-9 each) moves y = act fc2^T: 2^-9 (|act| |fc2|^T + |y|), per element.
+    act [n, I], fc2_e [H, I], y [n, H], all exact (float64)."""
+    u = 2.0 ** -9
+    return u * (np.abs(act) @ np.abs(fc2_e).T + np.abs(y))

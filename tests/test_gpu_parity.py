@@ -10,9 +10,9 @@ import torch
 
 import mixture_experts_ffn_15_b200 as moe
 from oracle import moe_oracle as O
-from parity_util import (W_ATOL, assert_close, device_inputs, from_dev, match_routing,
-                         row_scale, sample_tokens, to_dev, tol)
-from synth import Workload, make_inputs
+from parity_util import (W_ATOL, assert_close, bf16_storage_bound, device_inputs, from_dev,
+                         match_routing, row_scale, sample_tokens, to_dev, tol)
+from synth import Workload, bf16_bits_to_f32, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -191,6 +191,81 @@ def test_forward(wl):
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} output")
 
 
+# ------------------------------------------- SwiGLU attributes and expert biases
+# The op's activation_alpha / activation_beta / swiglu_limit ("Attribute set") and its
+# optional fc1/fc2 expert biases, on every path of moe_forward.  limit 1.0 clips most
+# gate and up values; the GPT-OSS values clip a few.
+ATTR_CASES = [
+    W("attr_one_launch", T=4, H=256, E=64, k=4, I=128),
+    W("attr_router_decode", T=100, H=256, E=64, k=4, I=128, router_bias_std=0.5),
+    W("attr_pairs", T=1100, H=256, E=64, k=4, I=192),
+    W("attr_f32", T=70, H=64, E=6, k=3, I=32, dtype="f32"),
+]
+ATTRS = [("gpt_oss", (1.702, 1.0, 7.0)), ("clip_heavy", (0.5, -0.25, 1.0))]
+
+
+@pytest.mark.parametrize("biased", [False, True], ids=["no_bias", "bias"])
+@pytest.mark.parametrize("attr", ATTRS, ids=[a[0] for a in ATTRS])
+@pytest.mark.parametrize("wl", ATTR_CASES, ids=[c.name for c in ATTR_CASES])
+def test_forward_swiglu_attributes_and_biases(wl, attr, biased):
+    from synth import make_expert_biases
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    act = attr[1]
+    b1 = b2 = None
+    db1 = db2 = None
+    if biased:
+        b1, b2 = make_expert_biases(wl)
+        db1, db2 = to_dev(b1, wl.dtype), to_dev(b2, wl.dtype)
+    out = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], wl.k,
+                      normalize=bool(wl.normalize), router_bias=dev["router_bias"], swiglu=act,
+                      fc1_bias=db1, fc2_bias=db2)
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    f = lambda a: None if a is None else (bf16_bits_to_f32(a) if a.dtype == np.uint16 else a)
+    ref = O.moe_forward(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                        lambda e: inp.expert_values("fc1", e), lambda e: inp.expert_values("fc2", e),
+                        wl.k, wl.normalize, wl.fc1_layout, idx=idx, act=act,
+                        fc1_bias=f(b1), fc2_bias=f(b2))["out"]
+    atol, rtol = tol(wl.dtype, ref)
+    if wl.dtype == "bf16":
+        atol = atol * row_scale(ref)
+    assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} {attr[0]} biased={biased}")
+
+
+def test_expert_ffn_attributes_and_biases_on_both_bf16_kernels():
+    """moe_expert_ffn with the GPT-OSS attributes and biases: few rows per expert (the
+    decode FFN) and many (the CTA pairs)."""
+    from synth import make_expert_biases
+    for rows_per_expert, name in ((6, "decode"), (300, "pairs")):
+        wl = W("attr_ffn_" + name, T=rows_per_expert * 8, H=256, E=8, k=1, I=128)
+        inp = make_inputs(wl)
+        b1, b2 = make_expert_biases(wl, seed=5)
+        offsets = (np.arange(wl.E + 1) * rows_per_expert).astype(np.int32)
+        act = (1.702, 1.0, 7.0)
+        y = moe.expert_ffn(to_dev(inp["hidden"], wl.dtype), torch.from_numpy(offsets).cuda(),
+                           to_dev(inp["fc1"], wl.dtype), to_dev(inp["fc2"], wl.dtype), swiglu=act,
+                           fc1_bias=to_dev(b1, wl.dtype), fc2_bias=to_dev(b2, wl.dtype))
+        torch.cuda.synchronize()
+        xv = inp.values("hidden")
+        y_ref = np.zeros((wl.T, wl.H))
+        bound = np.zeros((wl.T, wl.H))
+        for e in range(wl.E):
+            a, b = offsets[e], offsets[e + 1]
+            fc1_e, fc2_e = inp.expert_values("fc1", e), inp.expert_values("fc2", e)
+            b1_e, b2_e = bf16_bits_to_f32(b1[e]), bf16_bits_to_f32(b2[e])
+            y_ref[a:b] = O.expert_ffn(xv[a:b], fc1_e, fc2_e, "interleaved", act, b1_e, b2_e)
+            # the activations themselves, for the bound of their bf16 storage
+            g = xv[a:b].astype(np.float64) @ fc1_e[0::2].T.astype(np.float64) + b1_e[0::2]
+            u = xv[a:b].astype(np.float64) @ fc1_e[1::2].T.astype(np.float64) + b1_e[1::2]
+            bound[a:b] = bf16_storage_bound(O.swiglu(g, u, *act), fc2_e.astype(np.float64), y_ref[a:b])
+        # the beta on the up branch roughly doubles |act|, and with it the error of
+        # storing act in bf16: the stated tolerance plus that storage bound
+        atol, rtol = tol(wl.dtype, y_ref)
+        assert_close(from_dev(y), y_ref, atol * row_scale(y_ref) + bound, rtol, f"y_perm {name}")
+
+
 def test_combine_matches_oracle():
     wl = W("comb", T=77, H=136, E=6, k=3, dtype="f32")
     inp = make_inputs(wl)
@@ -299,8 +374,10 @@ def test_invalid_arguments_are_rejected():
     fc2 = torch.zeros((E, H, I), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(moe.MoEError, match="INVALID_ARG"):
         moe.forward(hidden, rw, fc1, fc2, 9)                       # k > E
-    with pytest.raises(moe.MoEError, match="UNSUPPORTED"):
-        moe.forward(hidden, rw, fc1, fc2, 2, swiglu=(1.702, 1.0, 7.0))
+    with pytest.raises(moe.MoEError, match="INVALID_ARG"):
+        moe.forward(hidden, rw, fc1, fc2, 2, swiglu=(float("nan"), 1.0, 7.0))   # alpha
+    with pytest.raises(moe.MoEError, match="INVALID_ARG"):
+        moe.forward(hidden, rw, fc1, fc2, 2, swiglu=(1.702, 1.0, -1.0))         # limit
     bad = torch.zeros((4 * H + 8,), dtype=torch.bfloat16, device="cuda")[1:1 + 4 * H].view(4, H)
     with pytest.raises(moe.MoEError, match="INVALID_ARG"):
         moe.forward(bad, rw, fc1, fc2, 2)                          # misaligned hidden
