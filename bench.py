@@ -37,6 +37,7 @@ DEFAULT_STEPS = {"tiny_fp32": 2000, "decode_bf16": 6000, "batched_decode_bf16": 
 GRAPH_STEPS = {"tiny_fp32": 20, "decode_bf16": 20, "batched_decode_bf16": 20,
                "prefill_bf16": 4, "long_prefill_bf16": 2}
 HBM_BOUND = {"decode_bf16", "batched_decode_bf16", "tiny_fp32"}
+SWIGLU_PRESETS = {"standard": (1.0, 0.0, float("inf")), "gpt_oss": (1.702, 1.0, 7.0)}
 
 
 def parse_args(argv=None):
@@ -50,6 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--swiglu", choices=list(SWIGLU_PRESETS), default="standard",
+                    help="SwiGLU attributes (alpha, beta, limit) of the op")
+    ap.add_argument("--expert-bias", action="store_true", help="with fc1/fc2 expert biases")
     return ap.parse_args(argv)
 
 
@@ -229,7 +233,7 @@ def oracle_cost(wl, inp, seconds):
                            f"top-k, {wl.k} expert FFNs, combine in float64), {el:.1f} s")
 
 
-def oracle_pair_step(wl, inp, state):
+def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None)):
     """One bounded reference step: routing of one token and one of its expert FFNs."""
     import numpy as np
 
@@ -240,8 +244,10 @@ def oracle_pair_step(wl, inp, state):
     w = O.routing_weights(L, idx, wl.normalize)
     j = state["j"]
     e = int(idx[0, j])
+    b1, b2 = biases
     y = O.expert_ffn(inp.values("hidden")[t:t + 1], inp.expert_values("fc1", e),
-                     inp.expert_values("fc2", e), wl.fc1_layout)
+                     inp.expert_values("fc2", e), wl.fc1_layout, act,
+                     None if b1 is None else b1[e], None if b2 is None else b2[e])
     assert np.isfinite(w[0, j] * y).all()
     state["j"] += 1
     if state["j"] == wl.k:
@@ -259,12 +265,19 @@ def run_reference(args):
     from threadpoolctl import threadpool_info
     cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     inp = make_inputs(wl)
+    act = SWIGLU_PRESETS[args.swiglu]
+    biases = (None, None)
+    if args.expert_bias:
+        from synth import bf16_bits_to_f32, make_expert_biases
+        nb1, nb2 = make_expert_biases(wl)
+        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
+        biases = (wide(nb1), wide(nb2))
     state = {"t": 0, "j": 0}
     for _ in range(args.warmup):
-        oracle_pair_step(wl, inp, state)
+        oracle_pair_step(wl, inp, state, act, biases)
     t0 = time.perf_counter()
     for _ in range(steps):
-        oracle_pair_step(wl, inp, state)
+        oracle_pair_step(wl, inp, state, act, biases)
     el = time.perf_counter() - t0
     value = (steps / wl.k) / el
     sample = (f"each step: router logits + top-k of one token and one of its {wl.k} expert "
@@ -276,7 +289,8 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(workload_config(wl, sets=4 if wl.name in HBM_BOUND else 1),
                        parallelism=f"replicas x{args.gpus}",
-                       graph_steps=GRAPH_STEPS.get(wl.name, 4)),
+                       graph_steps=GRAPH_STEPS.get(wl.name, 4), swiglu=list(act),
+                       expert_bias=bool(args.expert_bias)),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -335,6 +349,13 @@ def run_ours(args):
     fc2 = device_tensor(inp["fc2"], dev)
     fc1s = [fc1] + [fc1.clone() for _ in range(sets - 1)]
     fc2s = [fc2] + [fc2.clone() for _ in range(sets - 1)]
+    act = SWIGLU_PRESETS[args.swiglu]
+    b1 = b2 = None
+    if args.expert_bias:
+        from synth import make_expert_biases
+        nb1, nb2 = make_expert_biases(wl)
+        b1, b2 = device_tensor(nb1, dev), device_tensor(nb2, dev)
+    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2)
     out = torch.empty_like(hidden)
     ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
 
@@ -347,7 +368,7 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=dev)
     call = lambda i: moe.forward(hidden, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
                                  normalize=bool(wl.normalize), router_bias=bias, out=out,
-                                 workspace=ws)
+                                 workspace=ws, **ffn_kw)
     with torch.cuda.stream(stream):
         for i in range(sets):
             call(i)
@@ -466,7 +487,8 @@ def run_ours(args):
         for i in range(3):
             d_in.copy_(h_host, non_blocking=True)
             moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
-                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws)
+                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
+                        **ffn_kw)
             o_host.copy_(out, non_blocking=True)
             stream.synchronize()
         if world > 1:
@@ -475,7 +497,8 @@ def run_ours(args):
         for i in range(n_e2e):
             d_in.copy_(h_host, non_blocking=True)
             moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
-                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws)
+                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
+                        **ffn_kw)
             o_host.copy_(out, non_blocking=True)
             stream.synchronize()
         e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
@@ -493,7 +516,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
-                       graph_steps=S),
+                       graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias)),
         "roofline": roof, "layer": layer,
         "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
         "stages_note": "second timed region, same steps with stage events between kernels",

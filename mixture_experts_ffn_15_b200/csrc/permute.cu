@@ -152,9 +152,10 @@ gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 if (v0 + 32 * q < vec_per_row) buf[q] = __ldg(s + v0 + 32 * q);
+            // streaming stores: x_perm is larger than L2 and read back from HBM anyway
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                if (v0 + 32 * q < vec_per_row) dst[v0 + 32 * q] = buf[q];
+                if (v0 + 32 * q < vec_per_row) __stcs(dst + v0 + 32 * q, buf[q]);
         }
     }
 }
