@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--swiglu", choices=list(SWIGLU_PRESETS), default="standard",
                     help="SwiGLU attributes (alpha, beta, limit) of the op")
     ap.add_argument("--expert-bias", action="store_true", help="with fc1/fc2 expert biases")
+    ap.add_argument("--fc1-convert", action="store_true",
+                    help="convert chunked fc1 to the interleaved layout at set-up instead of "
+                         "reading it in place")
     return ap.parse_args(argv)
 
 
@@ -290,7 +293,8 @@ def run_reference(args):
         "config": dict(workload_config(wl, sets=4 if wl.name in HBM_BOUND else 1),
                        parallelism=f"replicas x{args.gpus}",
                        graph_steps=GRAPH_STEPS.get(wl.name, 4), swiglu=list(act),
-                       expert_bias=bool(args.expert_bias)),
+                       expert_bias=bool(args.expert_bias),
+                       fc1_layout_read="interleaved" if args.fc1_convert else wl.fc1_layout),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -344,8 +348,10 @@ def run_ours(args):
     router_w = device_tensor(inp["router_w"], dev)
     bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).to(dev)
     fc1 = device_tensor(inp["fc1"], dev)
-    if wl.fc1_layout == "chunked":
-        fc1 = moe.convert_chunked_to_interleaved(fc1)      # setup, as at session load
+    layout = wl.fc1_layout
+    if layout == "chunked" and args.fc1_convert:
+        fc1 = moe.convert_chunked_to_interleaved(fc1)      # set-up, as at session load
+        layout = "interleaved"
     fc2 = device_tensor(inp["fc2"], dev)
     fc1s = [fc1] + [fc1.clone() for _ in range(sets - 1)]
     fc2s = [fc2] + [fc2.clone() for _ in range(sets - 1)]
@@ -355,7 +361,7 @@ def run_ours(args):
         from synth import make_expert_biases
         nb1, nb2 = make_expert_biases(wl)
         b1, b2 = device_tensor(nb1, dev), device_tensor(nb2, dev)
-    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2)
+    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2, fc1_layout=layout)
     out = torch.empty_like(hidden)
     ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
 
@@ -516,7 +522,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
-                       graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias)),
+                       graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias),
+                       fc1_layout_read=layout),
         "roofline": roof, "layer": layer,
         "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
         "stages_note": "second timed region, same steps with stage events between kernels",

@@ -66,6 +66,16 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * finite and limit > 0 (INFINITY: no clipping), else MOE_ERR_INVALID_ARG. */
 typedef struct { float alpha, beta, limit; } moe_swiglu;
 
+/* Row layout of fc1 [E, 2I, H] ("Weight layout" of the pull request: the op's
+ * swiglu_fusion = 1 is the interleaved layout, which the ORT CPU kernel requires; the
+ * CUDA kernel it names accepts either, and so does every kernel here, reading the
+ * chunked layout in place with no conversion pass):
+ *   MOE_FC1_INTERLEAVED  row 2i = gate_i, row 2i+1 = up_i
+ *   MOE_FC1_CHUNKED      row i = gate_i, row I+i = up_i (Hugging Face gate_up_proj)
+ * fc1_bias [E, 2I], when given, is in the same layout.  Any other value is
+ * MOE_ERR_INVALID_ARG. */
+typedef enum { MOE_FC1_INTERLEAVED = 0, MOE_FC1_CHUNKED = 1 } moe_fc1_layout;
+
 /* Bits of the device error word. */
 #define MOE_DEVERR_BAD_EXPERT 1   /* an expert id outside [0, E) was skipped */
 #define MOE_DEVERR_TIMEOUT    2   /* a bounded wait inside a kernel gave up */
@@ -132,9 +142,10 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
  * grouped_mm_experts_forward.)
  *   x_perm   [rows, H] dt; rows offsets[e] .. offsets[e+1]-1 belong to expert e
  *   offsets  [E+1] int32 (device), non-decreasing, offsets[0] = 0, offsets[E] <= rows
- *   fc1      [E, 2I, H] dt, interleaved: row 2i = gate_i, row 2i+1 = up_i
+ *   fc1      [E, 2I, H] dt in fc1_layout (interleaved: row 2i = gate_i, row 2i+1 = up_i;
+ *            chunked: row i = gate_i, row I+i = up_i)
  *   fc2      [E, H, I] dt
- *   fc1_bias [E, 2I] dt (interleaved like fc1's rows) or NULL; fc2_bias [E, H] dt or
+ *   fc1_bias [E, 2I] dt (in fc1's layout) or NULL; fc2_bias [E, H] dt or
  *            NULL: the op's optional expert biases, added in float32 to the gate/up
  *            values before the activation and to the output
  *   y_perm   [rows, H] dt out: y_perm[r] = fc2_e act(g, u) + b2_e for r's expert e;
@@ -142,8 +153,9 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
  *   workspace at least moe_expert_ffn_workspace_size(rows, I, dt) bytes. */
 moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* fc1,
                           const void* fc2, const void* fc1_bias, const void* fc2_bias, int rows,
-                          int H, int E, int I, moe_swiglu act, moe_dtype dt, void* y_perm,
-                          void* workspace, size_t ws_bytes, void* stream);
+                          int H, int E, int I, moe_swiglu act, moe_fc1_layout fc1_layout,
+                          moe_dtype dt, void* y_perm, void* workspace, size_t ws_bytes,
+                          void* stream);
 
 /* Weighted combine (un-permute).
  *   out[t, :] = sum_{j<k} topk_w[t, j] * y_perm[perm_dst[t*k + j], :], summed in
@@ -156,7 +168,7 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 
 /* The whole layer: route -> permute -> fc1 + SwiGLU -> fc2 -> combine, all on
  * `stream`, no host synchronisation.
- *   hidden [T, H], router_w [E, H], fc1 [E, 2I, H] interleaved, fc2 [E, H, I]: dt
+ *   hidden [T, H], router_w [E, H], fc1 [E, 2I, H] in fc1_layout, fc2 [E, H, I]: dt
  *   fc1_bias [E, 2I], fc2_bias [E, H] dt or NULL (as in moe_expert_ffn)
  *   router_bias [E] float32 or NULL; out [T, H] dt
  *   workspace >= moe_workspace_size(T, H, E, k, I, dt) bytes, 256-byte aligned; it
@@ -165,8 +177,8 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
                        const void* fc1, const void* fc2, const void* fc1_bias,
                        const void* fc2_bias, int T, int H, int E, int k, int I, int normalize,
-                       moe_swiglu act, moe_dtype dt, void* out, void* workspace, size_t ws_bytes,
-                       void* stream);
+                       moe_swiglu act, moe_fc1_layout fc1_layout, moe_dtype dt, void* out,
+                       void* workspace, size_t ws_bytes, void* stream);
 
 /* The whole layer without a workspace argument, for callers that cannot allocate
  * device memory while they run it (an engine plugin or a serving loop that forbids
@@ -187,8 +199,8 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
 moe_status moe_forward_static(const void* hidden, const void* router_w, const float* router_bias,
                               const void* fc1, const void* fc2, const void* fc1_bias,
                               const void* fc2_bias, int T, int H, int E, int k, int I,
-                              int normalize, moe_swiglu act, moe_dtype dt, void* out,
-                              void* stream);
+                              int normalize, moe_swiglu act, moe_fc1_layout fc1_layout,
+                              moe_dtype dt, void* out, void* stream);
 
 /* Layout conversion of fc1 from the Hugging Face chunked layout ("Weight layout":
  * [E, 2*inter, H], the first inter rows gate, the next inter rows up) to the

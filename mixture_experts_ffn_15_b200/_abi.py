@@ -6,6 +6,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(6)
 MOE_F32, MOE_BF16 = 0, 1
+MOE_FC1_INTERLEAVED, MOE_FC1_CHUNKED = 0, 1
 MOE_DEVERR_BAD_EXPERT, MOE_DEVERR_TIMEOUT = 1, 2
 
 
@@ -26,13 +27,13 @@ SIGNATURES = {
     "moe_workspace_error_word": (_vp, [_vp]),
     "moe_route": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, MoeSwiglu, _i, _vp, _vp,
-                            _sz, _vp]),
+    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, MoeSwiglu, _i, _i, _vp,
+                            _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp]),
     "moe_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, MoeSwiglu, _i,
-                         _vp, _vp, _sz, _vp]),
+                         _i, _vp, _vp, _sz, _vp]),
     "moe_forward_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
-                                MoeSwiglu, _i, _vp, _vp]),
+                                MoeSwiglu, _i, _i, _vp, _vp]),
     "convert_chunked_to_interleaved": (_i, [_vp, _vp, _i, _i, _i, _i, _vp]),
     "moe_get_error": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),

@@ -22,7 +22,8 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["api.cu", "route.cu", "route_small.cu", "permute.cu", "combine.cu", "ffn_simt.cu",
            "gemm_tc.cu", "gemm_pair.cu", "static_scratch.cu"]
-HEADERS = ["common.cuh", "sm100.cuh", "kernels.h", "combine.cuh", "topk_warp.cuh", "tile_map.cuh"]
+HEADERS = ["common.cuh", "sm100.cuh", "kernels.h", "combine.cuh", "topk_warp.cuh", "tile_map.cuh",
+           "tmap.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

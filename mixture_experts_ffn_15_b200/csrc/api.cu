@@ -125,9 +125,13 @@ bool valid_swiglu(const moe_swiglu& a) {
     return isfinite(a.alpha) && isfinite(a.beta) && !isnan(a.limit) && a.limit > 0.0f;
 }
 
-FfnEpilogue make_epilogue(const moe_swiglu& a, const void* fc1_bias, const void* fc2_bias) {
-    FfnEpilogue ep;
+bool valid_layout(moe_fc1_layout l) { return l == MOE_FC1_INTERLEAVED || l == MOE_FC1_CHUNKED; }
+
+FfnAttrs make_ffn_attrs(const moe_swiglu& a, moe_fc1_layout layout, const void* fc1_bias,
+                        const void* fc2_bias) {
+    FfnAttrs ep;
     ep.act = SwigluAttr{a.alpha, a.beta, a.limit, standard_swiglu(a) ? 1 : 0};
+    ep.fc1_chunked = layout == MOE_FC1_CHUNKED;
     ep.fc1_bias = fc1_bias;
     ep.fc2_bias = fc2_bias;
     return ep;
@@ -170,7 +174,7 @@ using namespace moe;
 
 extern "C" {
 
-int moe_version(void) { return 200; }
+int moe_version(void) { return 210; }
 
 unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 
@@ -294,10 +298,11 @@ moe_status moe_permute(const void* hidden, const int32_t* topk_idx, int T, int H
 
 moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void* fc1,
                           const void* fc2, const void* fc1_bias, const void* fc2_bias, int rows,
-                          int H, int E, int I, moe_swiglu act, moe_dtype dt, void* y_perm,
-                          void* workspace, size_t ws_bytes, void* stream) {
+                          int H, int E, int I, moe_swiglu act, moe_fc1_layout fc1_layout,
+                          moe_dtype dt, void* y_perm, void* workspace, size_t ws_bytes,
+                          void* stream) {
     if (rows < 0 || H <= 0 || H % 8 || I <= 0 || I % 8 || E <= 0 || E > kMaxExperts ||
-        !valid_dtype(dt) || !valid_swiglu(act))
+        !valid_dtype(dt) || !valid_swiglu(act) || !valid_layout(fc1_layout))
         return MOE_ERR_INVALID_ARG;
     if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
         return MOE_ERR_INVALID_ARG;
@@ -315,7 +320,7 @@ moe_status moe_expert_ffn(const void* x_perm, const int32_t* offsets, const void
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + kAlign +
                                               align_up(static_cast<size_t>(rows) * I * elem_size(dt)));
     MOE_CUDA(cudaMemsetAsync(err, 0, 4, s));
-    const FfnEpilogue ep = make_epilogue(act, fc1_bias, fc2_bias);
+    const FfnAttrs ep = make_ffn_attrs(act, fc1_layout, fc1_bias, fc2_bias);
     if (dt == MOE_BF16 && decode_ffn_supported(rows, E, H, I)) {
         MOE_CUDA(cudaMemsetAsync(ctr, 0, static_cast<size_t>(decode_ffn_counters(rows, E)) * 4, s));
         MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1, fc2, rows, H, E, I,
@@ -348,8 +353,10 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
                        const void* fc1, const void* fc2, const void* fc1_bias, const void* fc2_bias,
                        int T, int H, int E, int k, int I, int normalize, moe_swiglu act,
-                       moe_dtype dt, void* out, void* workspace, size_t ws_bytes, void* stream) {
-    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt) || !valid_swiglu(act))
+                       moe_fc1_layout fc1_layout, moe_dtype dt, void* out, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt) || !valid_swiglu(act) ||
+        !valid_layout(fc1_layout))
         return MOE_ERR_INVALID_ARG;
     if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
         return MOE_ERR_INVALID_ARG;
@@ -379,7 +386,7 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     const int rows = T * k;
 
     const int path = forward_path(T, H, E, k, I, dt);
-    const FfnEpilogue ep = make_epilogue(act, fc1_bias, fc2_bias);
+    const FfnAttrs ep = make_ffn_attrs(act, fc1_layout, fc1_bias, fc2_bias);
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);

@@ -46,11 +46,9 @@ combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm
         }
         for (; t < T; t += step)
             o[static_cast<size_t>(t) * nvec + v] = combine_vec_bf16(y, nvec, perm_dst, topk_w, t, k, v, rows_max);
-        return;
-    }
-    for (int t = blockIdx.x; t < T; t += gridDim.x) {
-        if (v >= nvec) continue;
-        {
+    } else {
+        if (v >= nvec) return;
+        for (int t = blockIdx.x; t < T; t += gridDim.x) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             for (int j = 0; j < k; ++j) {
                 const int r = perm_dst[static_cast<size_t>(t) * k + j];

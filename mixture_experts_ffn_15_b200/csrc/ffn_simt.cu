@@ -1,9 +1,10 @@
 // float32 grouped expert FFN on plain FMA (no TF32, which would not meet a 1e-4
 // relative tolerance).  Same math as the tensor-core path:
-//   act[r, i] = swiglu(x_perm[r] . fc1[e, 2i] + b1[e, 2i], x_perm[r] . fc1[e, 2i+1] + b1[e, 2i+1])
+//   act[r, i] = swiglu(x_perm[r] . gate_i + b1[gate_i], x_perm[r] . up_i + b1[up_i])
 //   y[r, h]   = act[r] . fc2[e, h] + b2[e, h]
 // for the rows r of expert e ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op -
-// #326", "Attribute set": SwiGLU attributes, interleaved fc1; the biases optional).
+// #326", "Attribute set": SwiGLU attributes; the biases optional), gate_i and up_i the
+// fc1 rows of either layout ("Weight layout": interleaved 2i / 2i+1, or chunked i / I+i).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -13,13 +14,15 @@ namespace {
 constexpr int SBM = 32, SBN = 64, SBK = 32;
 
 // out[r, n] = A[r, :] . W[e, n, :] for the rows of each expert, 32 x 64 output tile
-// per unit; with SWIGLU the adjacent (gate, up) columns are fused into one act value.
+// per unit; with SWIGLU the adjacent (gate, up) columns are fused into one act value
+// (column n of W is fc1's interleaved row n, read from the chunked layout in place when
+// `chunked`).
 template <bool SWIGLU>
 __global__ void __launch_bounds__(256)
 simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __restrict__ W,
                          int n_w, int K, const int32_t* __restrict__ offsets, int E, int rows,
                          float* __restrict__ out, int ldo, const float* __restrict__ bias,
-                         SwigluAttr act) {
+                         SwigluAttr act, bool chunked) {
     __shared__ float sA[SBM][SBK + 1];
     __shared__ float sW[SBN][SBK + 1];
     __shared__ int s_off[kMaxExperts + 1];
@@ -65,7 +68,8 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
             for (int i = tid; i < SBN * SBK; i += 256) {
                 const int n = i / SBK, c = i - (i / SBK) * SBK;
                 const int wn = nt * SBN + n;
-                sW[n][c] = (wn < n_w && k0 + c < K) ? We[static_cast<size_t>(wn) * K + k0 + c] : 0.f;
+                const int wr = SWIGLU ? fc1_row(wn, n_w / 2, chunked) : wn;
+                sW[n][c] = (wn < n_w && k0 + c < K) ? We[static_cast<size_t>(wr) * K + k0 + c] : 0.f;
             }
             __syncthreads();
 #pragma unroll 8
@@ -84,7 +88,8 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
         if (bias != nullptr) {   // the expert's bias of each output column
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float b = n0 + q < n_w ? bias[static_cast<size_t>(e) * n_w + n0 + q] : 0.f;
+                const int bn = SWIGLU ? fc1_row(n0 + q, n_w / 2, chunked) : n0 + q;
+                const float b = n0 + q < n_w ? bias[static_cast<size_t>(e) * n_w + bn] : 0.f;
                 acc[0][q] += b;
                 acc[1][q] += b;
             }
@@ -116,16 +121,16 @@ int simt_grid(int rows, int E, int n_w) {
 
 cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
                                 const float* fc2, int rows, int H, int E, int I, float* act,
-                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep) {
+                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep) {
     if (rows <= 0) return cudaSuccess;
     cudaError_t err = launch_k(simt_grouped_gemm_kernel<true>, dim3(simt_grid(rows, E, 2 * I)),
                                dim3(256), 0, s, x_perm, H, fc1, 2 * I, H, offsets, E, rows, act, I,
-                               static_cast<const float*>(ep.fc1_bias), ep.act);
+                               static_cast<const float*>(ep.fc1_bias), ep.act, ep.fc1_chunked);
     if (err != cudaSuccess) return err;
     if (mid) record_event(mid, s);
     return launch_k(simt_grouped_gemm_kernel<false>, dim3(simt_grid(rows, E, H)), dim3(256), 0, s,
                     static_cast<const float*>(act), I, fc2, H, I, offsets, E, rows, y, H,
-                    static_cast<const float*>(ep.fc2_bias), ep.act);
+                    static_cast<const float*>(ep.fc2_bias), ep.act, false);
 }
 
 }  // namespace moe

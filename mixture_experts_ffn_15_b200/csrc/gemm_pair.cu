@@ -40,6 +40,7 @@
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tile_map.cuh"
+#include "tmap.cuh"
 
 namespace moe {
 namespace {
@@ -49,6 +50,7 @@ using namespace sm100;
 constexpr int kPThreads = 320;                // producer, MMA, 8 epilogue warps
 constexpr int kPWRows = 128;                  // weight rows per CTA (256 per pair)
 constexpr int kPBK = 64;                      // K per stage: one 128-byte row of bf16
+static_assert(kPBK == tmap::kBoxK, "TMA box width");
 constexpr int kPTok = 256;                    // tokens per pair tile (<= 128 per CTA)
 constexpr int kPStages = 6;
 constexpr int kPABytes = kPWRows * kPBK * 2;  // 16 KB
@@ -76,6 +78,7 @@ struct PairParams {
     int32_t* err;
     SwigluAttr act;           // fc1: SwiGLU attributes
     const __nv_bfloat16* bias;   // [E, n_out] bias of the weight rows, or nullptr
+    bool fc1_chunked;            // fc1 (SWIGLU): weights and bias in the chunked layout
 };
 
 struct PUnit {
@@ -160,7 +163,10 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
             const int half = d.n / 2;                     // token rows of this CTA
             const int trow0 = d.row0 + static_cast<int>(rank) * half;
-            const int wrow = d.g * p.n_out + d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
+            // first weight row of this CTA inside the expert (fc1: in interleaved order;
+            // the 4-D fc1 view reads it from either layout as rows of (gate, up) pairs)
+            const int w_in = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
+            const int wrow = d.g * p.n_out + w_in;
             // one box of 128 weight rows and one of 128 token rows per CTA (rows past
             // the tile are loaded too, and ignored: one TMA instruction each)
             const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
@@ -175,7 +181,10 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
                 if (lane == 0) {
-                    tma_load_2d_pair(a_dst, &tmW, fb, kb * kPBK, wrow);
+                    if constexpr (SWIGLU)
+                        tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
+                    else
+                        tma_load_2d_pair(a_dst, &tmW, fb, kb * kPBK, wrow);
                     tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
                 }
                 if (++stage == kPStages) {
@@ -242,9 +251,11 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // n_out is a multiple of 32)
             const int w0 = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows + quad * 32;
             const bool wvalid = w0 < p.n_out;
-            // this lane's weight row's bias (fc1: interleaved rows, fc2: h)
+            // this lane's weight row's bias (fc1: interleaved row w0 + lane in fc1's
+            // layout, fc2: h)
+            const int brow = SWIGLU ? fc1_row(w0 + lane, p.n_out / 2, p.fc1_chunked) : w0 + lane;
             const float bias = (p.bias && wvalid)
-                                   ? bf16_at(p.bias, static_cast<size_t>(d.g) * p.n_out + w0 + lane)
+                                   ? bf16_at(p.bias, static_cast<size_t>(d.g) * p.n_out + brow)
                                    : 0.f;
 #pragma unroll 1
             for (int c = part * 32; c < d.nrows; c += 64) {
@@ -331,37 +342,6 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 
 // ------------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* q = nullptr;
-        cudaDriverEntryPointQueryResult r;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) ==
-                cudaSuccess &&
-            r == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(q);
-    }
-    return fn;
-}
-
-// bf16 matrix [rows, K] row-major, boxes of 64 (K) x box_rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc || rows <= 0) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kPBK), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool SWIGLU>
 cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairParams& p,
                         long long units, cudaStream_t s) {
@@ -404,15 +384,18 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
 }
 
 // One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
-// the experts' blocks) and w [E * n_out, K].
+// the experts' blocks) and the weights w of E experts (fc1 as the 4-D pair view,
+// n_out = 2I rows per expert; fc2 [E * n_out, K]).
 cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
                       const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s,
-                      const SwigluAttr& act, const void* bias) {
+                      const FfnAttrs& at, const void* bias) {
     CUtensorMap mw, mx;
-    if (!make_map(&mw, w, static_cast<long long>(E) * n_out, K, kPWRows)) return cudaErrorInvalidValue;
-    if (!make_map(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
-    PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, act,
-                 static_cast<const __nv_bfloat16*>(bias)};
+    const bool ok_w = swiglu ? tmap::fc1_pairs(&mw, w, E, n_out / 2, K, kPWRows / 2, at.fc1_chunked)
+                             : tmap::matrix(&mw, w, static_cast<long long>(E) * n_out, K, kPWRows);
+    if (!ok_w) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
+    PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, at.act,
+                 static_cast<const __nv_bfloat16*>(bias), at.fc1_chunked};
     const long long units = (static_cast<long long>((rows + kPTok - 1) / kPTok) + E) *
                             ((n_out + 2 * kPWRows - 1) / (2 * kPWRows));
     return swiglu ? launch_pair<true>(mw, mx, p, units, s) : launch_pair<false>(mw, mx, p, units, s);
@@ -424,13 +407,13 @@ bool pair_ffn_supported(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && 
 
 cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep) {
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep) {
     if (rows <= 0) return cudaSuccess;
-    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s, ep.act,
+    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s, ep,
                               ep.fc1_bias);
     if (e != cudaSuccess) return e;
     if (mid) record_event(mid, s);
-    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s, ep.act, ep.fc2_bias);
+    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s, ep, ep.fc2_bias);
 }
 
 }  // namespace moe

@@ -32,6 +32,7 @@
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tile_map.cuh"
+#include "tmap.cuh"
 #include "topk_warp.cuh"
 
 namespace moe {
@@ -41,6 +42,7 @@ using namespace sm100;
 
 constexpr int BM = 128;              // rows of A per tile (MMA M)
 constexpr int BK = 64;               // K per stage: one 128-byte row of bf16
+static_assert(BK == tmap::kBoxK, "TMA box width");
 constexpr int kThreads = 192;
 constexpr int kTokChunk = 64;        // weight-M: tokens per unit
 constexpr int kBoxTok = 16;          // weight-M: token rows per TMA box
@@ -431,7 +433,8 @@ struct DecodeParams {
     __nv_bfloat16* out;
     int32_t* err;
     SwigluAttr act_attr;            // SwiGLU attributes
-    const __nv_bfloat16* b1;        // [E, 2I] fc1 bias (interleaved rows) or nullptr
+    const __nv_bfloat16* b1;        // [E, 2I] fc1 bias (fc1's layout) or nullptr
+    bool fc1_chunked;               // fc1 and b1 in the chunked layout
     const __nv_bfloat16* b2;        // [E, H] fc2 bias or nullptr
     // ROUTE: the routing runs inside the launch (fields below); offsets, perm_src,
     // perm_dst and topk_w above are then unused (the kernel keeps them in shared memory)
@@ -787,8 +790,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
             const bool f1 = d.phase == 1;
             const int nk = f1 ? nk1 : nk2;
-            const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;
-            const int wrow = d.g * (f1 ? 2 * p.I : p.H) + d.mt * BM;
+            const int wrow = d.g * p.H + d.mt * BM;   // fc2 weight row (fc1: 4-D pair view)
             const int nl = (d.nrows + kBoxTok - 1) / kBoxTok;
             uint32_t bbytes = static_cast<uint32_t>(nl * kBoxTok * BK * 2);
             int src[2] = {0, 0};   // this lane's gathered token rows: lane, lane + 32
@@ -823,7 +825,12 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const uint32_t fb = smem_u32(&full[stage]);
                 const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                if (lane == 0) tma_load_2d(a_dst, ma, fb, kb * BK, wrow);
+                if (lane == 0) {
+                    if (f1)
+                        tma_load_4d(a_dst, &tmW1, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
+                    else
+                        tma_load_2d(a_dst, &tmW2, fb, kb * BK, wrow);
+                }
                 if (f1 && GATHER) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -926,10 +933,12 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                 static_cast<uint32_t>(acc * C::kAccStride);
             const int wr = d.mt * BM + r;   // weight row inside the expert
-            // this lane's weight row's bias (fc1 in interleaved row order, fc2 by h)
+            // this lane's weight row's bias (fc1: interleaved row wr in fc1's layout, fc2: h)
             const __nv_bfloat16* bsrc = f1 ? p.b1 : p.b2;
             const float bias =
-                bsrc ? bf16_at(bsrc, static_cast<size_t>(d.g) * (f1 ? 2 * p.I : p.H) + wr) : 0.f;
+                bsrc ? bf16_at(bsrc, static_cast<size_t>(d.g) * (f1 ? 2 * p.I : p.H) +
+                                         (f1 ? fc1_row(wr, p.I, p.fc1_chunked) : wr))
+                     : 0.f;
 #pragma unroll 1
             for (int c = 0; c < d.nrows; c += 16) {
                 uint32_t v[16];
@@ -990,37 +999,6 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
 }
 
 // ------------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// bf16 matrix [rows, K] row-major, boxes of 64 (K) x box_rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, long long rows, int K, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc || rows <= 0) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int MODE, int BN, int KS = 1>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int bound,
@@ -1087,8 +1065,8 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
     TcParams p{nullptr, 1, T, H, E, nullptr, E, err};
     RouteParams rp{bias, k, normalize ? 1 : 0, topk_idx, topk_w, near_tie, logits, tile_counts};
     CUtensorMap ma, mb;
-    if (!make_map(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
     const int bound = (T + BM - 1) / BM;
     const bool small_k = k <= 8;
 #define MOE_ROUTE_CASE(EV)                                                                   \
@@ -1123,17 +1101,17 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
                               const int32_t* perm_dst, const float* topk_w, int k, void* out,
-                              cudaStream_t s, const FfnEpilogue& ep) {
+                              cudaStream_t s, const FfnAttrs& ep) {
     if (rows <= 0) return cudaSuccess;
     CUtensorMap w1, x, w2, a;
-    if (!make_map(&w1, fc1, static_cast<long long>(E) * 2 * I, H, BM)) return cudaErrorInvalidValue;
+    if (!tmap::fc1_pairs(&w1, fc1, E, I, H, BM / 2, ep.fc1_chunked)) return cudaErrorInvalidValue;
     if (perm_src) {
-        if (!make_map(&x, tokens, T, H, 1)) return cudaErrorInvalidValue;
+        if (!tmap::matrix(&x, tokens, T, H, 1)) return cudaErrorInvalidValue;
     } else {
-        if (!make_map(&x, tokens, rows, H, kBoxTok)) return cudaErrorInvalidValue;
+        if (!tmap::matrix(&x, tokens, rows, H, kBoxTok)) return cudaErrorInvalidValue;
     }
-    if (!make_map(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, E);
     DecodeParams p{};
     p.offsets = offsets;
@@ -1155,6 +1133,7 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     p.err = err;
     p.act_attr = ep.act;
     p.b1 = static_cast<const __nv_bfloat16*>(ep.fc1_bias);
+    p.fc1_chunked = ep.fc1_chunked;
     p.b2 = static_cast<const __nv_bfloat16*>(ep.fc2_bias);
     const int grid = decode_grid(rows, E, H, I);
     return perm_src ? launch_decode<true, false>(w1, x, w2, a, p, grid, s)
@@ -1166,10 +1145,11 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     if (rows <= 0) return cudaSuccess;
     if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I)) return cudaErrorInvalidValue;
     CUtensorMap w1, x, w2, a;
-    if (!make_map(&w1, r.fc1, static_cast<long long>(r.E) * 2 * r.I, r.H, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&x, r.hidden, r.T, r.H, 1)) return cudaErrorInvalidValue;
-    if (!make_map(&w2, r.fc2, static_cast<long long>(r.E) * r.H, r.I, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&a, r.act, rows, r.I, kBoxTok)) return cudaErrorInvalidValue;
+    if (!tmap::fc1_pairs(&w1, r.fc1, r.E, r.I, r.H, BM / 2, r.ep.fc1_chunked))
+        return cudaErrorInvalidValue;
+    if (!tmap::matrix(&x, r.hidden, r.T, r.H, 1)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&w2, r.fc2, static_cast<long long>(r.E) * r.H, r.I, BM)) return cudaErrorInvalidValue;
+    if (!tmap::matrix(&a, r.act, rows, r.I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, r.E);
     DecodeParams p{};
     p.E = r.E;
@@ -1188,6 +1168,7 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     p.err = r.err;
     p.act_attr = r.ep.act;
     p.b1 = static_cast<const __nv_bfloat16*>(r.ep.fc1_bias);
+    p.fc1_chunked = r.ep.fc1_chunked;
     p.b2 = static_cast<const __nv_bfloat16*>(r.ep.fc2_bias);
     p.hidden = r.hidden;
     p.router_w = r.router_w;

@@ -101,19 +101,31 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
                            cudaStream_t s);
 
-// What the expert FFN kernels apply after each GEMM: the SwiGLU attributes and the
-// optional expert biases (fc1_bias [E, 2I] in fc1's interleaved row order, fc2_bias
+// The op's attributes of the expert FFN: the SwiGLU attributes, the row layout of fc1
+// and the optional expert biases (fc1_bias [E, 2I] in fc1's row layout, fc2_bias
 // [E, H]; the activation dtype; nullptr = none).
-struct FfnEpilogue {
+//   fc1 interleaved: row 2i = gate_i, row 2i+1 = up_i;
+//   fc1 chunked:     row i = gate_i,  row I+i  = up_i (the Hugging Face layout).
+// Every kernel reads the chunked layout in place, as if it were interleaved: the
+// bf16 kernels through a 4-D TMA view (H, gate/up, i, e) whose gate/up stride is one
+// row for interleaved weights and I rows for chunked ones.
+struct FfnAttrs {
     SwigluAttr act{1.0f, 0.0f, INFINITY, 1};
+    bool fc1_chunked = false;
     const void* fc1_bias = nullptr;
     const void* fc2_bias = nullptr;
 };
 
+// Row of fc1 (or entry of fc1_bias) inside one expert that holds interleaved row j
+// (gate_{j/2} for even j, up_{j/2} for odd j) in the given layout.
+__host__ __device__ __forceinline__ int fc1_row(int j, int I, bool chunked) {
+    return chunked ? (j & 1) * I + (j >> 1) : j;
+}
+
 // ---------------------------------------------------------------- ffn_simt.cu
 cudaError_t launch_ffn_simt_f32(const float* x_perm, const int32_t* offsets, const float* fc1,
                                 const float* fc2, int rows, int H, int E, int I, float* act,
-                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep);
+                                float* y, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep);
 
 // ---------------------------------------------------------------- gemm_tc.cu
 bool tc_ffn_supported(int H, int I);
@@ -132,7 +144,7 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
 bool pair_ffn_supported(int H, int I);
 cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnEpilogue& ep);
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep);
 
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);
@@ -165,7 +177,7 @@ struct DecodeRoutedArgs {
     int32_t* counters;         // zero on entry
     int32_t* err;
     void* out;                 // [T, H]
-    FfnEpilogue ep;
+    FfnAttrs ep;
 };
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& a, cudaStream_t s);
 
@@ -173,6 +185,6 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
                               int H, int E, int I, void* act, void* y, int32_t* done, int32_t* err,
                               const int32_t* perm_dst, const float* topk_w, int k, void* out,
-                              cudaStream_t s, const FfnEpilogue& ep);
+                              cudaStream_t s, const FfnAttrs& ep);
 
 }  // namespace moe

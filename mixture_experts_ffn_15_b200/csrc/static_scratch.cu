@@ -48,7 +48,8 @@ extern "C" moe_status moe_forward_static(const void* hidden, const void* router_
                                          const float* router_bias, const void* fc1,
                                          const void* fc2, const void* fc1_bias,
                                          const void* fc2_bias, int T, int H, int E, int k, int I,
-                                         int normalize, moe_swiglu act, moe_dtype dt, void* out,
+                                         int normalize, moe_swiglu act,
+                                         moe_fc1_layout fc1_layout, moe_dtype dt, void* out,
                                          void* stream) {
     const size_t need = moe_workspace_size(T, H, E, k, I, dt);
     if (need == 0) return MOE_ERR_INVALID_ARG;                    // invalid sizes
@@ -57,6 +58,6 @@ extern "C" moe_status moe_forward_static(const void* hidden, const void* router_
     const moe_status st = scratch_address(&scratch);
     if (st != MOE_OK) return st;
     return moe_forward(hidden, router_w, router_bias, fc1, fc2, fc1_bias, fc2_bias, T, H, E, k, I,
-                       normalize, act, dt, out, scratch, static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES),
+                       normalize, act, fc1_layout, dt, out, scratch, static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES),
                        stream);
 }

@@ -53,6 +53,15 @@ def _swiglu(alpha, beta, limit):
     return MoeSwiglu(alpha, beta, limit)
 
 
+_LAYOUT = {"interleaved": 0, "chunked": 1}
+
+
+def _layout(fc1_layout):
+    if fc1_layout not in _LAYOUT:
+        raise ValueError(f"fc1_layout must be 'interleaved' or 'chunked', got {fc1_layout!r}")
+    return _LAYOUT[fc1_layout]
+
+
 def workspace_size(T, H, E, k, I, dtype):
     """Bytes of workspace moe_forward needs (0 for sizes it rejects)."""
     return _lib().moe_workspace_size(T, H, E, k, I, _DT[dtype])
@@ -72,11 +81,12 @@ def _biases(fc1_bias, fc2_bias, dt, E, I, H):
 
 def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out=None,
             workspace=None, stream=None, swiglu=(1.0, 0.0, float("inf")), fc1_bias=None,
-            fc2_bias=None):
+            fc2_bias=None, fc1_layout="interleaved"):
     """The fused MoE layer: out[T, H] = sum_j w[t, j] * FFN_{idx[t, j]}(hidden[t]).
 
-    swiglu = (alpha, beta, limit) of the op; fc1_bias [E, 2I] (fc1's interleaved row
-    order) and fc2_bias [E, H] are the optional expert biases."""
+    swiglu = (alpha, beta, limit) of the op; fc1_layout "interleaved" (rows 2i, 2i+1 =
+    gate_i, up_i) or "chunked" (rows i, I+i), read in place either way; fc1_bias
+    [E, 2I] (fc1's layout) and fc2_bias [E, H] are the optional expert biases."""
     _need(hidden, "hidden")
     dt = hidden.dtype
     T, H = hidden.shape
@@ -98,7 +108,8 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
     _need(workspace, "workspace", torch.uint8)
     st = _lib().moe_forward(_ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(fc1), _ptr(fc2),
                             _ptr(fc1_bias), _ptr(fc2_bias), T, H, E, k, I, int(bool(normalize)),
-                            _swiglu(*swiglu), _dtcode(hidden), _ptr(out), _ptr(workspace),
+                            _swiglu(*swiglu), _layout(fc1_layout), _dtcode(hidden), _ptr(out),
+                            _ptr(workspace),
                             workspace.numel(), _stream(stream))
     check(st, "moe_forward")
     return out
@@ -156,9 +167,11 @@ def permute(topk_idx, E, hidden=None, err_word=None, stream=None):
 
 
 def expert_ffn(x_perm, offsets, fc1, fc2, y_perm=None, stream=None,
-               swiglu=(1.0, 0.0, float("inf")), fc1_bias=None, fc2_bias=None):
+               swiglu=(1.0, 0.0, float("inf")), fc1_bias=None, fc2_bias=None,
+               fc1_layout="interleaved"):
     """y_perm[r] = fc2_e act(x fc1_gate^T + b_gate, x fc1_up^T + b_up) + b2_e over each
-    expert's rows (act: SwiGLU with the op's (alpha, beta, limit))."""
+    expert's rows (act: SwiGLU with the op's (alpha, beta, limit); fc1 and fc1_bias in
+    fc1_layout, "interleaved" or "chunked")."""
     _need(x_perm, "x_perm")
     rows, H = x_perm.shape
     E, two_i, _ = fc1.shape
@@ -172,7 +185,8 @@ def expert_ffn(x_perm, offsets, fc1, fc2, y_perm=None, stream=None,
     dt = _dtcode(x_perm)
     ws = alloc_workspace(_lib().moe_expert_ffn_workspace_size(rows, I, dt), x_perm.device)
     st = _lib().moe_expert_ffn(_ptr(x_perm), _ptr(offsets), _ptr(fc1), _ptr(fc2), _ptr(fc1_bias),
-                               _ptr(fc2_bias), rows, H, E, I, _swiglu(*swiglu), dt, _ptr(y_perm),
+                               _ptr(fc2_bias), rows, H, E, I, _swiglu(*swiglu),
+                               _layout(fc1_layout), dt, _ptr(y_perm),
                                _ptr(ws), ws.numel(), _stream(stream))
     check(st, "moe_expert_ffn")
     return y_perm

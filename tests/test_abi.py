@@ -70,10 +70,11 @@ def test_workspace_sizes():
     assert lib.moe_permute_workspace_size(1000, 64) >= 8 * 64 * 4   # per-tile counts
 
 
-def _fwd(lib, T=4, H=128, E=8, k=2, I=64, act=_abi.STANDARD_SWIGLU, dt=_abi.MOE_BF16, ptr=16):
+def _fwd(lib, T=4, H=128, E=8, k=2, I=64, act=_abi.STANDARD_SWIGLU, dt=_abi.MOE_BF16, ptr=16,
+         layout=_abi.MOE_FC1_INTERLEAVED):
     p = ctypes.c_void_p(ptr)
-    return lib.moe_forward(p, p, None, p, p, None, None, T, H, E, k, I, 1, act, dt, p, ctypes.c_void_p(256),
-                           1 << 40, None)
+    return lib.moe_forward(p, p, None, p, p, None, None, T, H, E, k, I, 1, act, layout, dt, p,
+                           ctypes.c_void_p(256), 1 << 40, None)
 
 
 def test_host_validation_before_any_device_work():
@@ -85,6 +86,9 @@ def test_host_validation_before_any_device_work():
     assert _fwd(lib, act=_abi.MoeSwiglu(nan, 1.0, 7.0)) == _abi.MOE_ERR_INVALID_ARG     # alpha
     assert _fwd(lib, act=_abi.MoeSwiglu(1.702, float("inf"), 7.0)) == _abi.MOE_ERR_INVALID_ARG
     assert _fwd(lib, act=_abi.MoeSwiglu(1.702, 1.0, 0.0)) == _abi.MOE_ERR_INVALID_ARG   # limit
+    assert _fwd(lib, layout=2) == _abi.MOE_ERR_INVALID_ARG  # no such fc1 layout
+    assert _fwd(lib, layout=-1) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd(lib, T=0, layout=_abi.MOE_FC1_CHUNKED) == _abi.MOE_OK
     assert _fwd(lib, H=72) == _abi.MOE_ERR_UNSUPPORTED      # bf16 needs H % 64 == 0
     assert _fwd(lib, T=0) == _abi.MOE_OK                   # empty batch: nothing to do
     assert _fwd(lib, ptr=18) == _abi.MOE_ERR_INVALID_ARG    # misaligned tensors

@@ -266,6 +266,84 @@ def test_expert_ffn_attributes_and_biases_on_both_bf16_kernels():
         assert_close(from_dev(y), y_ref, atol * row_scale(y_ref) + bound, rtol, f"y_perm {name}")
 
 
+# ------------------------------------------- fc1 in the chunked layout, read in place
+# "Weight layout": Hugging Face stores gate_up_proj chunked (gate rows, then up rows);
+# the op's CUDA kernel accepts either layout.  Every path reads the chunked weights
+# (and a chunked fc1 bias) where they are: the result must be bit for bit the result
+# on the same weights converted to the interleaved layout, and match the oracle's
+# chunked reading.
+LAYOUT_CASES = [
+    W("chunked_one_launch", T=4, H=256, E=64, k=4, I=128, fc1_layout="chunked"),
+    W("chunked_router_decode", T=100, H=256, E=64, k=4, I=192, fc1_layout="chunked"),
+    W("chunked_small_decode", T=100, H=256, E=16, k=4, I=128, fc1_layout="chunked"),
+    W("chunked_pairs", T=1100, H=256, E=64, k=4, I=192, fc1_layout="chunked"),
+    # 2I = 1408 rows: the last 256-row tile of each expert is half padding
+    W("chunked_pairs_half_tile", T=1100, H=128, E=8, k=2, I=704, fc1_layout="chunked"),
+    W("chunked_f32", T=70, H=64, E=6, k=3, I=32, dtype="f32", fc1_layout="chunked"),
+]
+
+
+def _bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+@pytest.mark.parametrize("biased", [False, True], ids=["standard", "gpt_oss_bias"])
+@pytest.mark.parametrize("wl", LAYOUT_CASES, ids=[c.name for c in LAYOUT_CASES])
+def test_forward_reads_chunked_fc1_in_place(wl, biased):
+    from synth import make_expert_biases
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    act = (1.702, 1.0, 7.0) if biased else (1.0, 0.0, float("inf"))
+    b1 = b2 = None
+    if biased:
+        b1, b2 = make_expert_biases(wl, seed=3)      # b1 read in fc1's (chunked) layout
+    d = lambda a: None if a is None else to_dev(a, wl.dtype)
+    kw = dict(normalize=bool(wl.normalize), router_bias=dev["router_bias"], swiglu=act)
+    out_c = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], wl.k,
+                        fc1_bias=d(b1), fc2_bias=d(b2), fc1_layout="chunked", **kw)
+    fc1_i = to_dev(O.chunked_to_interleaved(inp["fc1"]), wl.dtype)
+    b1_i = None if b1 is None else O.chunked_to_interleaved(b1)
+    out_i = moe.forward(dev["hidden"], dev["router_w"], fc1_i, dev["fc2"], wl.k,
+                        fc1_bias=d(b1_i), fc2_bias=d(b2), **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(out_c), _bits(out_i)), f"{wl.name}: chunked != interleaved"
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    f = lambda a: None if a is None else (bf16_bits_to_f32(a) if a.dtype == np.uint16 else a)
+    ref = O.moe_forward(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                        lambda e: inp.expert_values("fc1", e), lambda e: inp.expert_values("fc2", e),
+                        wl.k, wl.normalize, "chunked", idx=idx, act=act,
+                        fc1_bias=f(b1), fc2_bias=f(b2))["out"]
+    atol, rtol = tol(wl.dtype, ref)
+    if wl.dtype == "bf16":
+        atol = atol * row_scale(ref)
+    assert_close(from_dev(out_c), ref, atol, rtol, f"{wl.name} chunked biased={biased}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_expert_ffn_reads_chunked_fc1_in_place(dtype):
+    """moe_expert_ffn with chunked fc1 and fc1 bias: bit-equal to the interleaved call,
+    for few rows per expert (the decode FFN) and many (the CTA pairs)."""
+    from synth import make_expert_biases
+    for rows_per_expert, name in ((6, "decode"), (300, "pairs")):
+        wl = W("chunked_ffn_" + name, T=rows_per_expert * 8, H=256, E=8, k=1, I=192,
+               dtype=dtype, fc1_layout="chunked")
+        inp = make_inputs(wl)
+        b1, b2 = make_expert_biases(wl, seed=6)
+        offsets = torch.from_numpy((np.arange(wl.E + 1) * rows_per_expert).astype(np.int32)).cuda()
+        x = to_dev(inp["hidden"], dtype)
+        fc2, db2 = to_dev(inp["fc2"], dtype), to_dev(b2, dtype)
+        act = (1.702, 1.0, 7.0)
+        y_c = moe.expert_ffn(x, offsets, to_dev(inp["fc1"], dtype), fc2, swiglu=act,
+                             fc1_bias=to_dev(b1, dtype), fc2_bias=db2, fc1_layout="chunked")
+        y_i = moe.expert_ffn(x, offsets, to_dev(O.chunked_to_interleaved(inp["fc1"]), dtype), fc2,
+                             swiglu=act, fc1_bias=to_dev(O.chunked_to_interleaved(b1), dtype),
+                             fc2_bias=db2)
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(y_c), _bits(y_i)), name
+
+
 def test_combine_matches_oracle():
     wl = W("comb", T=77, H=136, E=6, k=3, dtype="f32")
     inp = make_inputs(wl)
@@ -417,10 +495,16 @@ def test_full_workload(name):
     inp = make_inputs(wl)
     dev = device_inputs(inp)
     fc1 = dev["fc1"]
-    if wl.fc1_layout == "chunked":
-        fc1 = moe.convert_chunked_to_interleaved(fc1)
     out = moe.forward(dev["hidden"], dev["router_w"], fc1, dev["fc2"], wl.k,
-                      normalize=bool(wl.normalize), router_bias=dev["router_bias"])
+                      normalize=bool(wl.normalize), router_bias=dev["router_bias"],
+                      fc1_layout=wl.fc1_layout)
+    if wl.fc1_layout == "chunked":
+        # the chunked weights read in place equal the layer on converted weights
+        conv = moe.forward(dev["hidden"], dev["router_w"], moe.convert_chunked_to_interleaved(fc1),
+                           dev["fc2"], wl.k, normalize=bool(wl.normalize),
+                           router_bias=dev["router_bias"])
+        assert torch.equal(out.view(torch.int16), conv.view(torch.int16))
+        del conv
     r = run_route(dev, wl)
     torch.cuda.synchronize()
     L, idx = check_routing(inp, r)

@@ -28,7 +28,8 @@ def _static_forward(dev, wl, out):
     return lib.moe_forward_static(p(dev["hidden"]), p(dev["router_w"]), p(dev["router_bias"]),
                                   p(dev["fc1"]), p(dev["fc2"]), None, None, wl.T, wl.H, wl.E,
                                   wl.k, wl.I,
-                                  wl.normalize, _abi.STANDARD_SWIGLU, _abi.MOE_BF16, p(out),
+                                  wl.normalize, _abi.STANDARD_SWIGLU, _abi.MOE_FC1_INTERLEAVED,
+                                  _abi.MOE_BF16, p(out),
                                   stream)
 
 
