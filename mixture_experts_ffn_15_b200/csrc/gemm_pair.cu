@@ -163,10 +163,9 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
             const int half = d.n / 2;                     // token rows of this CTA
             const int trow0 = d.row0 + static_cast<int>(rank) * half;
-            // first weight row of this CTA inside the expert (fc1: in interleaved order;
-            // the 4-D fc1 view reads it from either layout as rows of (gate, up) pairs)
+            // first weight row of this CTA inside the expert (fc1: in interleaved order),
+            // loaded through the (k, s, i, e) pair view of either weight tensor
             const int w_in = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
-            const int wrow = d.g * p.n_out + w_in;
             // one box of 128 weight rows and one of 128 token rows per CTA (rows past
             // the tile are loaded too, and ignored: one TMA instruction each)
             const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
@@ -181,10 +180,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
                 if (lane == 0) {
-                    if constexpr (SWIGLU)
-                        tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
-                    else
-                        tma_load_2d_pair(a_dst, &tmW, fb, kb * kPBK, wrow);
+                    tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
                     tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
                 }
                 if (++stage == kPStages) {
@@ -384,14 +380,14 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
 }
 
 // One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
-// the experts' blocks) and the weights w of E experts (fc1 as the 4-D pair view,
-// n_out = 2I rows per expert; fc2 [E * n_out, K]).
+// the experts' blocks) and the weights w [E, n_out, K] of E experts (both through the
+// 4-D pair view, which reads chunked fc1 in place).
 cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
                       const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s,
                       const FfnAttrs& at, const void* bias) {
     CUtensorMap mw, mx;
     const bool ok_w = swiglu ? tmap::fc1_pairs(&mw, w, E, n_out / 2, K, kPWRows / 2, at.fc1_chunked)
-                             : tmap::matrix(&mw, w, static_cast<long long>(E) * n_out, K, kPWRows);
+                             : tmap::plain_pairs(&mw, w, E, n_out, K, kPWRows / 2);
     if (!ok_w) return cudaErrorInvalidValue;
     if (!tmap::matrix(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
     PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, at.act,

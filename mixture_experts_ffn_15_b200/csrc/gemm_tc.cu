@@ -790,7 +790,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
             const bool f1 = d.phase == 1;
             const int nk = f1 ? nk1 : nk2;
-            const int wrow = d.g * p.H + d.mt * BM;   // fc2 weight row (fc1: 4-D pair view)
+            // both weight maps are (k, s, i, e) pair views: rows d.mt BM .. of expert d.g
+            const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;
             const int nl = (d.nrows + kBoxTok - 1) / kBoxTok;
             uint32_t bbytes = static_cast<uint32_t>(nl * kBoxTok * BK * 2);
             int src[2] = {0, 0};   // this lane's gathered token rows: lane, lane + 32
@@ -825,12 +826,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const uint32_t fb = smem_u32(&full[stage]);
                 const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                if (lane == 0) {
-                    if (f1)
-                        tma_load_4d(a_dst, &tmW1, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
-                    else
-                        tma_load_2d(a_dst, &tmW2, fb, kb * BK, wrow);
-                }
+                if (lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
                 if (f1 && GATHER) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -1110,7 +1106,7 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     } else {
         if (!tmap::matrix(&x, tokens, rows, H, kBoxTok)) return cudaErrorInvalidValue;
     }
-    if (!tmap::matrix(&w2, fc2, static_cast<long long>(E) * H, I, BM)) return cudaErrorInvalidValue;
+    if (!tmap::plain_pairs(&w2, fc2, E, H, I, BM / 2)) return cudaErrorInvalidValue;
     if (!tmap::matrix(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, E);
     DecodeParams p{};
@@ -1148,7 +1144,7 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     if (!tmap::fc1_pairs(&w1, r.fc1, r.E, r.I, r.H, BM / 2, r.ep.fc1_chunked))
         return cudaErrorInvalidValue;
     if (!tmap::matrix(&x, r.hidden, r.T, r.H, 1)) return cudaErrorInvalidValue;
-    if (!tmap::matrix(&w2, r.fc2, static_cast<long long>(r.E) * r.H, r.I, BM)) return cudaErrorInvalidValue;
+    if (!tmap::plain_pairs(&w2, r.fc2, r.E, r.H, r.I, BM / 2)) return cudaErrorInvalidValue;
     if (!tmap::matrix(&a, r.act, rows, r.I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, r.E);
     DecodeParams p{};

@@ -43,27 +43,43 @@ inline bool matrix(CUtensorMap* m, const void* ptr, long long rows, int K, int b
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fc1 [E, 2I, H] as the 4-D tensor (h, s, i, e) with element (h, s, i, e) = gate_i
-// (s = 0) or up_i (s = 1) of expert e at column h, whichever the layout stores it:
-//   interleaved: row 2i + s (s stride one row, i stride two rows);
-//   chunked:     row s I + i (s stride I rows, i stride one row).
-// A box of 64 (h) x 2 (s) x box_pairs (i) x 1 (e) lands in shared memory as
-// 2 box_pairs rows of 128 bytes in interleaved order (row 2i + s), whatever the
-// layout in memory; coordinates (k0, 0, i0, e).  Pairs i >= I read as zeros.
-inline bool fc1_pairs(CUtensorMap* m, const void* fc1, int E, int I, int H, int box_pairs,
-                      bool chunked) {
+// The weights of E experts, n = 2 n_pairs rows of K each per expert, as the 4-D tensor
+// (k, s, i, e): element (k, s, i, e) is column k of the expert's row s_stride s +
+// i_stride i.  A box of 64 (k) x 2 (s) x box_pairs (i) x 1 (e) lands in shared memory as
+// 2 box_pairs rows of 128 bytes in the order of the row index 2i + s, whatever the
+// layout in memory; coordinates (k0, 0, j0 / 2, e) for rows j0 .. of expert e.  Pairs
+// i >= n_pairs read as zeros.
+//   plain [E, n, K] (fc2; fc1 interleaved: row 2i = gate_i, 2i+1 = up_i):
+//       s_stride 1, i_stride 2
+//   fc1 chunked [E, 2I, K] (row i = gate_i, I+i = up_i): s_stride I, i_stride 1
+inline bool row_pairs(CUtensorMap* m, const void* w, int E, int n_pairs, int K, int box_pairs,
+                      long long s_stride, long long i_stride) {
     EncodeTiledFn enc = encode_fn();
-    if (!enc || E <= 0 || I <= 0) return false;
-    const cuuint64_t row = static_cast<cuuint64_t>(H) * 2;
-    cuuint64_t dims[4] = {static_cast<cuuint64_t>(H), 2, static_cast<cuuint64_t>(I),
+    if (!enc || E <= 0 || n_pairs <= 0) return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(K) * 2;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), 2, static_cast<cuuint64_t>(n_pairs),
                           static_cast<cuuint64_t>(E)};
-    cuuint64_t strides[3] = {chunked ? row * static_cast<cuuint64_t>(I) : row,
-                             chunked ? row : 2 * row, 2 * row * static_cast<cuuint64_t>(I)};
+    cuuint64_t strides[3] = {row * static_cast<cuuint64_t>(s_stride),
+                             row * static_cast<cuuint64_t>(i_stride),
+                             row * 2 * static_cast<cuuint64_t>(n_pairs)};
     cuuint32_t box[4] = {static_cast<cuuint32_t>(kBoxK), 2, static_cast<cuuint32_t>(box_pairs), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(fc1), dims, strides, box,
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fc1 [E, 2I, H] of either layout, read in interleaved row order (gate_i, up_i pairs).
+inline bool fc1_pairs(CUtensorMap* m, const void* fc1, int E, int I, int H, int box_pairs,
+                      bool chunked) {
+    return chunked ? row_pairs(m, fc1, E, I, H, box_pairs, I, 1)
+                   : row_pairs(m, fc1, E, I, H, box_pairs, 1, 2);
+}
+
+// A plain [E, n, K] weight tensor (n even) in the same 4-D form, so that one load
+// instruction serves both GEMMs of a kernel.
+inline bool plain_pairs(CUtensorMap* m, const void* w, int E, int n, int K, int box_pairs) {
+    return n % 2 == 0 && row_pairs(m, w, E, n / 2, K, box_pairs, 1, 2);
 }
 
 }  // namespace tmap
