@@ -25,7 +25,12 @@ following the pages in their order:
   the family, standard SwiGLU being (1, 0, inf); the op's optional fc1/fc2 expert
   biases are added to the pre-activation gate/up values and to the output.
 * "Contributing Gemma 4 support and ONNX export optimizations" (Hugging Face forum),
-  "Key Technical Contributions", ONNX tracing compatibility: inside
+  "Key Technical Contributions", RMSNorm formulation realignment: Gemma 4's norms are
+  Llama-style, the normalised activations multiplied by the weight (not by 1 +
+  weight as in Gemma 2); the Rust weight-loader page lists a pre-FFN norm among the
+  four norms of each layer.  `rms_norm` is that norm, `pre_ffn_norm` the layer's
+  input made from a residual activation by it.
+* same forum page, "Key Technical Contributions", ONNX tracing compatibility: inside
   grouped_mm_experts_forward the per-expert token count is a bincount over the
   chosen expert ids, followed by a grouped matmul over experts.
 
@@ -46,7 +51,11 @@ notes of the repository):
   inside the sigmoid, the bias on the up branch after its clipping, and the clipping
   bounds the gate from above only (the pages name the clipping but not its form);
 * the stable permutation puts the (token, slot) pairs of expert e in ascending
-  token order, experts in ascending order.
+  token order, experts in ascending order;
+* the RMSNorm is y = (x / sqrt(mean(x^2) + eps)) * weight evaluated in float64 and
+  rounded once to the storage dtype (round to nearest, ties to even): the pages fix
+  the formula, not its precision, and one rounding of the exact value is the plain
+  definition; eps is the caller's.
 
 Parity pins for every function here live in tests/test_oracle_pins.py.  No
 function in this file is "parity unpinned".
@@ -278,6 +287,37 @@ def combine(y_perm, perm_dst, w, T: int, k: int) -> np.ndarray:
         rows = np.asarray(perm_dst, dtype=np.int64).reshape(T, k)[:, j]
         out += np.asarray(w, dtype=F64)[:, j:j + 1] * y[rows]
     return out
+
+
+# ------------------------------------------------------------------------ pre-FFN norm
+
+def round_to_dtype(y, dtype: str) -> np.ndarray:
+    """float64 values rounded once to the storage dtype, round to nearest, ties to
+    even, returned as float64.  "f32": numpy's correctly rounded cast.  "bf16" (8
+    significant bits, float32's exponent range): y = m 2^e with m in [0.5, 1) from
+    frexp, m 2^8 rounded to an integer with ties to even (numpy's rint), scaled back
+    -- every step exact in float64.  Values here stay in bf16's normal range."""
+    y = np.asarray(y, dtype=F64)
+    if dtype == "f32":
+        return y.astype(np.float32).astype(F64)
+    if dtype != "bf16":
+        raise ValueError(f"unknown dtype {dtype!r}")
+    m, e = np.frexp(y)
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
+def rms_norm(x, weight, eps: float) -> np.ndarray:
+    """Llama-style RMSNorm of each row of x [T, H]: (x / sqrt(mean_h x^2 + eps)) * weight,
+    float64, unrounded."""
+    x = np.asarray(x, dtype=F64)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + F64(eps))
+    return (x * r) * np.asarray(weight, dtype=F64)[None, :]
+
+
+def pre_ffn_norm(x, weight, eps: float, dtype: str) -> np.ndarray:
+    """The layer's input made from the residual activation x by the pre-FFN norm: the
+    RMSNorm rounded to the storage dtype (float64 values of that dtype)."""
+    return round_to_dtype(rms_norm(x, weight, eps), dtype)
 
 
 # ------------------------------------------------------------------------ the layer

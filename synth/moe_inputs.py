@@ -38,7 +38,7 @@ import numpy as np
 
 # Stream identifiers: fixed forever, so that a seed always means the same tensors.
 _S_HIDDEN, _S_ROUTER, _S_BIAS, _S_FC1, _S_FC2, _S_OUTLIER = 1, 2, 3, 4, 5, 6
-_S_FC1_BIAS, _S_FC2_BIAS = 7, 8
+_S_FC1_BIAS, _S_FC2_BIAS, _S_NORM_W, _S_RESIDUAL = 7, 8, 9, 10
 
 
 @dataclass(frozen=True)
@@ -184,3 +184,14 @@ def make_expert_biases(wl: Workload, std: float = 0.5, seed: Optional[int] = Non
     b1 = _normal((s, _S_FC1_BIAS), (wl.E, 2 * wl.I), std)
     b2 = _normal((s, _S_FC2_BIAS), (wl.E, wl.H), std)
     return _store(b1, wl.dtype), _store(b2, wl.dtype)
+
+
+def make_pre_norm_inputs(wl: Workload, scale: float = 4.0, seed: Optional[int] = None):
+    """Inputs of the pre-FFN RMSNorm for `wl`: a residual-stream activation [T, H]
+    (N(0, scale), a scale other than 1 so that the normalisation shows) and the norm
+    weight [H] (N(1, 0.1): a trained Llama-style weight sits near one), both stored
+    like the workload's activations (bf16 bits or float32)."""
+    s = wl.seed if seed is None else seed
+    x = _normal((s, _S_RESIDUAL), (wl.T, wl.H), scale)
+    w = 1.0 + _normal((s, _S_NORM_W), (wl.H,), 0.1)
+    return _store(x, wl.dtype), _store(w.astype(np.float32), wl.dtype)

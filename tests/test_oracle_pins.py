@@ -300,6 +300,78 @@ def test_sparse_evaluation_on_token_subset_matches_full():
     np.testing.assert_allclose(sub, full[[0, 7, 29]], rtol=1e-13, atol=1e-15)
 
 
+# ------------------------------------------------------------------- pre-FFN RMSNorm
+
+def check_round_to_dtype():
+    # float32 values are exact in float64: rounding them to bf16 from float64 must give
+    # the generator's float32 -> bf16 round-to-nearest-even, bit for bit
+    rng = np.random.default_rng(11)
+    v = (rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000))).astype(np.float32)
+    got = O.round_to_dtype(v.astype(np.float64), "bf16")
+    np.testing.assert_array_equal(got, bf16_bits_to_f32(round_to_bf16_bits(v)).astype(np.float64))
+    # midpoints go to the even neighbour; anything above a midpoint goes up
+    y = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 1 + 2 ** -8 + 2 ** -40,
+                  2 - 2 ** -9, 0.375 + 2 ** -11])
+    np.testing.assert_array_equal(O.round_to_dtype(y, "bf16"),
+                                  [1.0, 1 + 2 ** -6, -1.0, 1 + 2 ** -7, 2.0, 0.375])
+    np.testing.assert_array_equal(O.round_to_dtype(np.array([1 + 2 ** -24, 1 + 3 * 2 ** -24]), "f32"),
+                                  [1.0, 1 + 2 ** -22])
+
+
+def check_rms_norm_closed_forms():
+    # a worked example: x = (3, 4), mean of squares 12.5
+    got = O.rms_norm(np.array([[3.0, 4.0]]), np.array([2.0, 0.5]), 0.0)
+    np.testing.assert_allclose(got, [[6 / np.sqrt(12.5), 2 / np.sqrt(12.5)]], rtol=1e-15)
+    # a constant row c: every output is c w / sqrt(c^2 + eps); with eps = c^2, w / sqrt(2)
+    w = np.linspace(0.5, 1.5, 16)
+    for c, eps in ((3.0, 0.0), (-0.25, 1e-6), (2.0, 4.0)):
+        got = O.rms_norm(np.full((1, 16), c), w, eps)
+        np.testing.assert_allclose(got[0], c * w / np.sqrt(c * c + eps), rtol=1e-14)
+    np.testing.assert_allclose(O.rms_norm(np.full((1, 4), 2.0), np.ones(4), 4.0), 2 ** -0.5, rtol=1e-15)
+    # with unit weight and no eps every row has mean square one, whatever its scale,
+    # and the weight multiplies column by column
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((5, 64)) * np.array([[0.01], [1], [7], [300], [1e-3]])
+    y1 = O.rms_norm(x, np.ones(64), 0.0)
+    np.testing.assert_allclose(np.mean(y1 * y1, axis=1), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(O.rms_norm(9.0 * x, np.ones(64), 0.0), y1, rtol=1e-13)
+    wv = rng.uniform(0.5, 2.0, 64)
+    np.testing.assert_allclose(O.rms_norm(x, wv, 0.0), y1 * wv, rtol=1e-14)
+    # a row of zeros stays zero
+    np.testing.assert_array_equal(O.rms_norm(np.zeros((1, 8)), np.ones(8), 1e-6), 0.0)
+
+
+def check_pre_ffn_norm_rounds_once():
+    # the layer's input is the norm rounded to bf16 once: inputs whose norm is exact in
+    # bf16 come through unchanged; otherwise it is the nearest bf16 value
+    x = np.full((1, 4), 2.0)                       # mean square 4: r = 1/2 exactly
+    w = np.array([1.0, 1.5, 0.75, 3.0])
+    np.testing.assert_array_equal(O.pre_ffn_norm(x, w, 0.0, "bf16"), [w])
+    x = np.full((1, 4), 3.0)                       # x r = 1: y = w = 1/3 -> 0.333984375 in bf16
+    np.testing.assert_array_equal(O.pre_ffn_norm(x, np.full(4, 1 / 3), 0.0, "bf16"),
+                                  np.full((1, 4), 0.333984375))
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((6, 48)) * 5
+    w = rng.uniform(0.8, 1.2, 48)
+    y = O.pre_ffn_norm(x, w, 1e-6, "bf16")
+    exact = O.rms_norm(x, w, 1e-6)
+    m, e = np.frexp(exact)
+    np.testing.assert_array_less(np.abs(y - exact), np.ldexp(1.0, e - 8) * 0.5 + 1e-300)
+    np.testing.assert_array_equal(O.round_to_dtype(y, "bf16"), y)   # already bf16 values
+
+
+def test_round_to_dtype():
+    check_round_to_dtype()
+
+
+def test_rms_norm_closed_forms():
+    check_rms_norm_closed_forms()
+
+
+def test_pre_ffn_norm_rounds_once():
+    check_pre_ffn_norm_rounds_once()
+
+
 # ----------------------------------------------------------------------- inputs
 
 def test_bf16_rounding_is_nearest_even():
@@ -516,6 +588,35 @@ def _mut_unstable_perm(idx, E):
     return counts, offsets, src, dst
 
 
+def _mut_gemma2_offset(x, weight, eps):
+    return _real_rms_norm(x, 1.0 + np.asarray(weight, dtype=np.float64), eps)
+
+
+def _mut_eps_outside_sqrt(x, weight, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.sqrt(np.mean(x * x, axis=1, keepdims=True)) + eps) * weight
+
+
+def _mut_sum_not_mean(x, weight, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.sum(x * x, axis=1, keepdims=True) + eps) * weight
+
+
+def _mut_round_half_up(y, dtype):
+    y = np.asarray(y, dtype=np.float64)
+    if dtype == "f32":
+        return y.astype(np.float32).astype(np.float64)
+    m, e = np.frexp(y)
+    return np.ldexp(np.floor(np.ldexp(m, 8) + 0.5), e - 8)
+
+
+def _mut_round_truncate(y, dtype):
+    y = np.asarray(y, dtype=np.float64)
+    m, e = np.frexp(y)
+    return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
+
+
+_real_rms_norm = O.rms_norm
 _real_perm = O.stable_permutation
 _real_swiglu = O.swiglu
 _real_expert_ffn = O.expert_ffn
@@ -533,13 +634,19 @@ MUTATIONS = [
     ("select_topk", _mut_ties_to_higher),
     ("routing_weights", _mut_no_renormalise),
     ("stable_permutation", _mut_unstable_perm),
+    ("rms_norm", _mut_gemma2_offset),
+    ("rms_norm", _mut_eps_outside_sqrt),
+    ("rms_norm", _mut_sum_not_mean),
+    ("round_to_dtype", _mut_round_half_up),
+    ("round_to_dtype", _mut_round_truncate),
 ]
 
 PIN_CHECKS = [check_golden_values, check_golden_routing, check_topk_brute_force,
               check_weights_sum_to_one, check_permutation, check_chunked_equals_interleaved,
               check_dense_masked_equals_sparse, check_expert_ffn_scalar_loops,
               check_swiglu_closed_forms, check_swiglu_limit_saturation,
-              check_expert_biases_zero_input, check_biased_chunked_equals_interleaved]
+              check_expert_biases_zero_input, check_biased_chunked_equals_interleaved,
+              check_round_to_dtype, check_rms_norm_closed_forms, check_pre_ffn_norm_rounds_once]
 
 
 @pytest.mark.parametrize("name,mutant", MUTATIONS, ids=[f"{m[0]}-{m[1].__name__}" for m in MUTATIONS])
