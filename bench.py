@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--swiglu", choices=list(SWIGLU_PRESETS), default="standard",
                     help="SwiGLU attributes (alpha, beta, limit) of the op")
     ap.add_argument("--expert-bias", action="store_true", help="with fc1/fc2 expert biases")
+    ap.add_argument("--pre-norm", action="store_true",
+                    help="the layer's input is a residual activation normalised by the pre-FFN "
+                         "RMSNorm inside the call")
     ap.add_argument("--fc1-convert", action="store_true",
                     help="convert chunked fc1 to the interleaved layout at set-up instead of "
                          "reading it in place")
@@ -154,8 +157,12 @@ class ClockSampler:
                 "samples": len(load), "power_w_max": max(num(r[3]) for r in load)}
 
 
-def algorithmic(wl, counts):
-    """Algorithmic bytes and FLOPs of one step (only the routed work, used experts once)."""
+NORM_EPS = 1e-6
+
+
+def algorithmic(wl, counts, pre_norm=False):
+    """Algorithmic bytes and FLOPs of one step (only the routed work, used experts once;
+    with the pre-FFN norm, its read of the residual and the weight and its write)."""
     T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
     es = 2 if wl.dtype == "bf16" else 4
     rows = T * k
@@ -167,6 +174,8 @@ def algorithmic(wl, counts):
     layer = {"bytes": used * 3 * H * I * es + E * H * es + 2 * T * H * es
              + 2 * rows * H * es + 2 * rows * I * es + 2 * rows * H * es,
              "flops": float(T) * (6.0 * k * H * I + 2.0 * H * E)}
+    if pre_norm:
+        layer["bytes"] += 2 * T * H * es + H * es
     return used, fc1, fc2, layer
 
 
@@ -208,8 +217,10 @@ def device_tensor(a, dev):
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_cost(wl, inp, seconds):
-    """The CPU oracle, as it stands, on whole tokens of `wl` for about `seconds`.
+def oracle_cost(wl, inp, seconds, pre=None):
+    """The CPU oracle, as it stands, on whole tokens of `wl` for about `seconds` (with
+    pre = (residual values, norm weight values), each token through the pre-FFN norm
+    first).
 
     Returns (tokens/s, threads, description of the sample)."""
     import numpy as np
@@ -226,7 +237,9 @@ def oracle_cost(wl, inp, seconds):
     n = 0
     while True:
         t = n % wl.T
-        r = O.moe_forward(x[t:t + 1], rw, bias, fc1, fc2, wl.k, wl.normalize, wl.fc1_layout)
+        xt = x[t:t + 1] if pre is None else O.pre_ffn_norm(pre[0][t:t + 1], pre[1], NORM_EPS,
+                                                           wl.dtype)
+        r = O.moe_forward(xt, rw, bias, fc1, fc2, wl.k, wl.normalize, wl.fc1_layout)
         assert np.isfinite(r["out"]).all()
         n += 1
         if time.perf_counter() - t0 >= seconds:
@@ -236,19 +249,22 @@ def oracle_cost(wl, inp, seconds):
                            f"top-k, {wl.k} expert FFNs, combine in float64), {el:.1f} s")
 
 
-def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None)):
-    """One bounded reference step: routing of one token and one of its expert FFNs."""
+def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None), pre=None):
+    """One bounded reference step: routing of one token and one of its expert FFNs (with
+    pre, the token's pre-FFN norm first)."""
     import numpy as np
 
     from oracle import moe_oracle as O
     t = state["t"]
-    L = O.router_logits(inp.values("hidden")[t:t + 1], inp.values("router_w"), inp["router_bias"])
+    xt = inp.values("hidden")[t:t + 1] if pre is None else \
+        O.pre_ffn_norm(pre[0][t:t + 1], pre[1], NORM_EPS, wl.dtype)
+    L = O.router_logits(xt, inp.values("router_w"), inp["router_bias"])
     idx = O.select_topk(L, wl.k)
     w = O.routing_weights(L, idx, wl.normalize)
     j = state["j"]
     e = int(idx[0, j])
     b1, b2 = biases
-    y = O.expert_ffn(inp.values("hidden")[t:t + 1], inp.expert_values("fc1", e),
+    y = O.expert_ffn(xt, inp.expert_values("fc1", e),
                      inp.expert_values("fc2", e), wl.fc1_layout, act,
                      None if b1 is None else b1[e], None if b2 is None else b2[e])
     assert np.isfinite(w[0, j] * y).all()
@@ -259,7 +275,7 @@ def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None,
 
 
 def run_reference(args):
-    from synth import WORKLOADS, make_inputs
+    from synth import WORKLOADS, bf16_bits_to_f32, make_inputs
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -270,17 +286,23 @@ def run_reference(args):
     inp = make_inputs(wl)
     act = SWIGLU_PRESETS[args.swiglu]
     biases = (None, None)
+    pre = None
+    if args.pre_norm:
+        from synth import make_pre_norm_inputs
+        px, pw = make_pre_norm_inputs(wl)
+        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
+        pre = (wide(px), wide(pw))
     if args.expert_bias:
-        from synth import bf16_bits_to_f32, make_expert_biases
+        from synth import make_expert_biases
         nb1, nb2 = make_expert_biases(wl)
         wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
         biases = (wide(nb1), wide(nb2))
     state = {"t": 0, "j": 0}
     for _ in range(args.warmup):
-        oracle_pair_step(wl, inp, state, act, biases)
+        oracle_pair_step(wl, inp, state, act, biases, pre)
     t0 = time.perf_counter()
     for _ in range(steps):
-        oracle_pair_step(wl, inp, state, act, biases)
+        oracle_pair_step(wl, inp, state, act, biases, pre)
     el = time.perf_counter() - t0
     value = (steps / wl.k) / el
     sample = (f"each step: router logits + top-k of one token and one of its {wl.k} expert "
@@ -293,7 +315,7 @@ def run_reference(args):
         "config": dict(workload_config(wl, sets=4 if wl.name in HBM_BOUND else 1),
                        parallelism=f"replicas x{args.gpus}",
                        graph_steps=GRAPH_STEPS.get(wl.name, 4), swiglu=list(act),
-                       expert_bias=bool(args.expert_bias),
+                       expert_bias=bool(args.expert_bias), pre_norm=bool(args.pre_norm),
                        fc1_layout_read="interleaved" if args.fc1_convert else wl.fc1_layout),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -345,6 +367,15 @@ def run_ours(args):
 
     inp = make_inputs(wl)
     hidden = device_tensor(inp["hidden"], dev)
+    norm_kw, pre = {}, None
+    if args.pre_norm:
+        # the input is a residual activation; the layer normalises it itself
+        from synth import bf16_bits_to_f32, make_pre_norm_inputs
+        px, pw = make_pre_norm_inputs(wl)
+        hidden = device_tensor(px, dev)
+        norm_kw = dict(norm_weight=device_tensor(pw, dev), norm_eps=NORM_EPS)
+        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
+        pre = (wide(px), wide(pw))
     router_w = device_tensor(inp["router_w"], dev)
     bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).to(dev)
     fc1 = device_tensor(inp["fc1"], dev)
@@ -361,15 +392,16 @@ def run_ours(args):
         from synth import make_expert_biases
         nb1, nb2 = make_expert_biases(wl)
         b1, b2 = device_tensor(nb1, dev), device_tensor(nb2, dev)
-    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2, fc1_layout=layout)
+    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2, fc1_layout=layout, **norm_kw)
     out = torch.empty_like(hidden)
     ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
 
     # routing outside the timed region, for the byte accounting only
-    r = moe.route(hidden, router_w, wl.k, normalize=bool(wl.normalize), router_bias=bias)
+    x_in = moe.rmsnorm(hidden, norm_kw["norm_weight"], NORM_EPS) if args.pre_norm else hidden
+    r = moe.route(x_in, router_w, wl.k, normalize=bool(wl.normalize), router_bias=bias)
     p = moe.permute(r["idx"], wl.E)
     counts = p["counts"].cpu().numpy()
-    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts)
+    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts, args.pre_norm)
 
     stream = torch.cuda.Stream(device=dev)
     call = lambda i: moe.forward(hidden, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
@@ -523,7 +555,7 @@ def run_ours(args):
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
                        graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias),
-                       fc1_layout_read=layout),
+                       pre_norm=bool(args.pre_norm), fc1_layout_read=layout),
         "roofline": roof, "layer": layer,
         "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
         "stages_note": "second timed region, same steps with stage events between kernels",
@@ -531,7 +563,7 @@ def run_ours(args):
         "gpu_launches": int(round(launches_per_step * steps)),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds)
+        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds, pre)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     if rank == 0:

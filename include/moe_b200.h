@@ -166,15 +166,32 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
 
 /* ------------------------------------------------------------------------ the layer */
 
-/* The whole layer: route -> permute -> fc1 + SwiGLU -> fc2 -> combine, all on
- * `stream`, no host synchronisation.
+/* Pre-FFN RMSNorm, the step in front of the layer ("Contributing Gemma 4 support and
+ * ONNX export optimizations", "Key Technical Contributions": Llama-style, the normed
+ * states times the weight, not times 1 + weight):
+ *   y[t, h] = (x[t, h] / sqrt(mean_h x[t, h]^2 + eps)) * weight[h]
+ * evaluated in float64 and rounded once to dt (to nearest, ties to even), so the
+ * result does not depend on the order of the sums.
+ *   x [T, H] dt, weight [H] dt, y [T, H] dt (may not overlap x); eps finite and
+ *   >= 0 (eps = 0 and an all-zero row give NaN, as the formula does).
+ * T = 0 is a no-op. */
+moe_status moe_rmsnorm(const void* x, const void* weight, int T, int H, float eps, moe_dtype dt,
+                       void* y, void* stream);
+
+/* The whole layer: [pre-FFN RMSNorm ->] route -> permute -> fc1 + SwiGLU -> fc2 ->
+ * combine, all on `stream`, no host synchronisation.
  *   hidden [T, H], router_w [E, H], fc1 [E, 2I, H] in fc1_layout, fc2 [E, H, I]: dt
+ *   norm_weight [H] dt or NULL: with a weight, `hidden` is the residual activation and
+ *            the layer runs on moe_rmsnorm(hidden, norm_weight, norm_eps), which it
+ *            computes into its workspace (the launch that clears the workspace header
+ *            does it: no extra launch); NULL: hidden is the layer's input as is
  *   fc1_bias [E, 2I], fc2_bias [E, H] dt or NULL (as in moe_expert_ffn)
  *   router_bias [E] float32 or NULL; out [T, H] dt
  *   workspace >= moe_workspace_size(T, H, E, k, I, dt) bytes, 256-byte aligned; it
  *   holds every intermediate, and its first word is the device error word.
  * T = 0 is a no-op returning MOE_OK. */
-moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
+moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_eps,
+                       const void* router_w, const float* router_bias,
                        const void* fc1, const void* fc2, const void* fc1_bias,
                        const void* fc2_bias, int T, int H, int E, int k, int I, int normalize,
                        moe_swiglu act, moe_fc1_layout fc1_layout, moe_dtype dt, void* out,
@@ -196,7 +213,8 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
  *   that must start at zero are cleared by every call): calls whose work can
  *   overlap on the GPU, from two streams or two host threads, race on it. */
 #define MOE_STATIC_SCRATCH_BYTES (8u << 20)
-moe_status moe_forward_static(const void* hidden, const void* router_w, const float* router_bias,
+moe_status moe_forward_static(const void* hidden, const void* norm_weight, float norm_eps,
+                              const void* router_w, const float* router_bias,
                               const void* fc1, const void* fc2, const void* fc1_bias,
                               const void* fc2_bias, int T, int H, int E, int k, int I,
                               int normalize, moe_swiglu act, moe_fc1_layout fc1_layout,

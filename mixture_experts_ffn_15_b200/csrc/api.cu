@@ -59,7 +59,7 @@ struct Carver {
 
 struct FwdLayout {
     size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, ctr, x_perm,
-        act, y, total;
+        act, y, xn, total;
 };
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
@@ -86,6 +86,7 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     L.x_perm = c.take(rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
+    L.xn = c.take(static_cast<size_t>(T) * H * es);   // the normalised input (pre-FFN norm)
     L.total = c.off;
     return L;
 }
@@ -126,6 +127,8 @@ bool valid_swiglu(const moe_swiglu& a) {
 }
 
 bool valid_layout(moe_fc1_layout l) { return l == MOE_FC1_INTERLEAVED || l == MOE_FC1_CHUNKED; }
+
+bool valid_eps(float eps) { return isfinite(eps) && eps >= 0.0f; }
 
 FfnAttrs make_ffn_attrs(const moe_swiglu& a, moe_fc1_layout layout, const void* fc1_bias,
                         const void* fc2_bias) {
@@ -350,14 +353,30 @@ moe_status moe_combine(const void* y_perm, const int32_t* perm_dst, const float*
     return MOE_OK;
 }
 
-moe_status moe_forward(const void* hidden, const void* router_w, const float* router_bias,
+moe_status moe_rmsnorm(const void* x, const void* weight, int T, int H, float eps, moe_dtype dt,
+                       void* y, void* stream) {
+    if (T < 0 || H <= 0 || H % 8 || !valid_dtype(dt) || !valid_eps(eps)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !weight || !y || !aligned(x, 16) || !aligned(weight, 16) || !aligned(y, 16))
+        return MOE_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(T) * H * elem_size(dt);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(x), b = reinterpret_cast<uintptr_t>(y);
+    if (a < b + bytes && b < a + bytes) return MOE_ERR_INVALID_ARG;   // overlap
+    MOE_CUDA(launch_rmsnorm(x, weight, T, H, eps, dt == MOE_BF16, y, nullptr, 0,
+                            static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
+
+moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_eps,
+                       const void* router_w, const float* router_bias,
                        const void* fc1, const void* fc2, const void* fc1_bias, const void* fc2_bias,
                        int T, int H, int E, int k, int I, int normalize, moe_swiglu act,
                        moe_fc1_layout fc1_layout, moe_dtype dt, void* out, void* workspace,
                        size_t ws_bytes, void* stream) {
     if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt) || !valid_swiglu(act) ||
-        !valid_layout(fc1_layout))
+        !valid_layout(fc1_layout) || (norm_weight && !valid_eps(norm_eps)))
         return MOE_ERR_INVALID_ARG;
+    if (norm_weight && !aligned(norm_weight, 16)) return MOE_ERR_INVALID_ARG;
     if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
         return MOE_ERR_INVALID_ARG;
     if (dt == MOE_BF16 && !tc_ffn_supported(H, I)) return MOE_ERR_UNSUPPORTED;
@@ -391,10 +410,21 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
     record(0, s);
+    // The first launch zeroes what must start at zero (the error word, the decode-FFN
+    // counters, the tile counts; the split router of the small-route path clears the
+    // header itself) and, with a norm weight, also writes the normalised input, which
+    // then replaces `hidden` everywhere below.
+    const size_t clear_end = (path & kPathFusedRoute) ? L.tile_counts
+                             : (path & kPathSmallRoute) ? L.hdr : L.logits;
+    if (norm_weight) {
+        MOE_CUDA(launch_rmsnorm(hidden, norm_weight, T, H, norm_eps, bf16, ws + L.xn, ws + L.hdr,
+                                clear_end - L.hdr, s));
+        hidden = ws + L.xn;
+    } else if (clear_end > L.hdr) {
+        MOE_CUDA(launch_clear(ws + L.hdr, clear_end - L.hdr, s));
+    }
     if (path & kPathFusedRoute) {
-        // the error word and the counters start at zero; then one launch: routing,
-        // fc1 + SwiGLU, fc2 and the weighted combine
-        MOE_CUDA(launch_clear(ws + L.hdr, L.tile_counts - L.hdr, s));
+        // one launch: routing, fc1 + SwiGLU, fc2 and the weighted combine
         record(1, s);
         record(2, s);
         DecodeRoutedArgs a{};
@@ -454,8 +484,6 @@ moe_status moe_forward(const void* hidden, const void* router_w, const float* ro
         MOE_CUDA(launch_route_small(a, s));
         record(1, s);
     } else {
-        // the header, the decode FFN's counters and the tile counts start at zero
-        MOE_CUDA(launch_clear(ws + L.hdr, L.logits - L.hdr, s));
         int32_t* tile_counts = reinterpret_cast<int32_t*>(ws + L.tile_counts);
         if (path & kPathTcRouter) {
             // logits on the tensor cores, routing and per-tile bincount in the epilogue

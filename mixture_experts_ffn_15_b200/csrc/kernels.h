@@ -40,6 +40,12 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// ---------------------------------------------------------------- rmsnorm.cu
+// y [T, H] = the pre-FFN RMSNorm of x with weight w [H] (float64, one rounding to the
+// dtype); the same launch zeroes `clear_bytes` (a multiple of 16) at `clear`.
+cudaError_t launch_rmsnorm(const void* x, const void* w, int T, int H, float eps, bool bf16,
+                           void* y, void* clear, size_t clear_bytes, cudaStream_t s);
+
 // ---------------------------------------------------------------- route.cu
 cudaError_t launch_router_logits_simt(const void* hidden, const void* router_w, int T, int H,
                                       int E, bool bf16, float* logits, cudaStream_t s);

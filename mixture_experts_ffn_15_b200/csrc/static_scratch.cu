@@ -44,7 +44,8 @@ moe_status scratch_address(void** out) {
 
 }  // namespace
 
-extern "C" moe_status moe_forward_static(const void* hidden, const void* router_w,
+extern "C" moe_status moe_forward_static(const void* hidden, const void* norm_weight,
+                                         float norm_eps, const void* router_w,
                                          const float* router_bias, const void* fc1,
                                          const void* fc2, const void* fc1_bias,
                                          const void* fc2_bias, int T, int H, int E, int k, int I,
@@ -57,7 +58,8 @@ extern "C" moe_status moe_forward_static(const void* hidden, const void* router_
     void* scratch = nullptr;
     const moe_status st = scratch_address(&scratch);
     if (st != MOE_OK) return st;
-    return moe_forward(hidden, router_w, router_bias, fc1, fc2, fc1_bias, fc2_bias, T, H, E, k, I,
+    return moe_forward(hidden, norm_weight, norm_eps, router_w, router_bias, fc1, fc2, fc1_bias,
+                       fc2_bias, T, H, E, k, I,
                        normalize, act, fc1_layout, dt, out, scratch, static_cast<size_t>(MOE_STATIC_SCRATCH_BYTES),
                        stream);
 }

@@ -81,12 +81,14 @@ def _biases(fc1_bias, fc2_bias, dt, E, I, H):
 
 def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out=None,
             workspace=None, stream=None, swiglu=(1.0, 0.0, float("inf")), fc1_bias=None,
-            fc2_bias=None, fc1_layout="interleaved"):
+            fc2_bias=None, fc1_layout="interleaved", norm_weight=None, norm_eps=1e-6):
     """The fused MoE layer: out[T, H] = sum_j w[t, j] * FFN_{idx[t, j]}(hidden[t]).
 
     swiglu = (alpha, beta, limit) of the op; fc1_layout "interleaved" (rows 2i, 2i+1 =
     gate_i, up_i) or "chunked" (rows i, I+i), read in place either way; fc1_bias
-    [E, 2I] (fc1's layout) and fc2_bias [E, H] are the optional expert biases."""
+    [E, 2I] (fc1's layout) and fc2_bias [E, H] are the optional expert biases.  With
+    norm_weight [H], hidden is the residual activation and the layer runs on its
+    pre-FFN RMSNorm (computed inside the call, see rmsnorm)."""
     _need(hidden, "hidden")
     dt = hidden.dtype
     T, H = hidden.shape
@@ -98,6 +100,8 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
     if router_bias is not None:
         _need(router_bias, "router_bias", torch.float32, (E,))
     _biases(fc1_bias, fc2_bias, dt, E, I, H)
+    if norm_weight is not None:
+        _need(norm_weight, "norm_weight", dt, (H,))
     if out is None:
         out = torch.empty_like(hidden)
     _need(out, "out", dt, (T, H))
@@ -106,12 +110,27 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
         # invalid sizes give 0 bytes; the C call then reports them
         workspace = alloc_workspace(max(need, 256), hidden.device)
     _need(workspace, "workspace", torch.uint8)
-    st = _lib().moe_forward(_ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(fc1), _ptr(fc2),
+    st = _lib().moe_forward(_ptr(hidden), _ptr(norm_weight), float(norm_eps), _ptr(router_w),
+                            _ptr(router_bias), _ptr(fc1), _ptr(fc2),
                             _ptr(fc1_bias), _ptr(fc2_bias), T, H, E, k, I, int(bool(normalize)),
                             _swiglu(*swiglu), _layout(fc1_layout), _dtcode(hidden), _ptr(out),
                             _ptr(workspace),
                             workspace.numel(), _stream(stream))
     check(st, "moe_forward")
+    return out
+
+
+def rmsnorm(x, weight, eps=1e-6, out=None, stream=None):
+    """Pre-FFN RMSNorm: (x / sqrt(mean(x^2) + eps)) * weight per row, float64 inside,
+    rounded once to x's dtype."""
+    _need(x, "x")
+    T, H = x.shape
+    _need(weight, "weight", x.dtype, (H,))
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", x.dtype, (T, H))
+    check(_lib().moe_rmsnorm(_ptr(x), _ptr(weight), T, H, float(eps), _dtcode(x), _ptr(out),
+                             _stream(stream)), "moe_rmsnorm")
     return out
 
 

@@ -38,7 +38,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
-              "convert_chunked_to_interleaved", "moe_workspace_size", "moe_get_error"):
+              "convert_chunked_to_interleaved", "moe_workspace_size", "moe_get_error",
+              "moe_rmsnorm", "moe_forward_static"):
         assert n in names
 
 
@@ -71,10 +72,10 @@ def test_workspace_sizes():
 
 
 def _fwd(lib, T=4, H=128, E=8, k=2, I=64, act=_abi.STANDARD_SWIGLU, dt=_abi.MOE_BF16, ptr=16,
-         layout=_abi.MOE_FC1_INTERLEAVED):
+         layout=_abi.MOE_FC1_INTERLEAVED, norm=None, eps=1e-6):
     p = ctypes.c_void_p(ptr)
-    return lib.moe_forward(p, p, None, p, p, None, None, T, H, E, k, I, 1, act, layout, dt, p,
-                           ctypes.c_void_p(256), 1 << 40, None)
+    return lib.moe_forward(p, norm, eps, p, None, p, p, None, None, T, H, E, k, I, 1, act, layout,
+                           dt, p, ctypes.c_void_p(256), 1 << 40, None)
 
 
 def test_host_validation_before_any_device_work():
@@ -89,6 +90,16 @@ def test_host_validation_before_any_device_work():
     assert _fwd(lib, layout=2) == _abi.MOE_ERR_INVALID_ARG  # no such fc1 layout
     assert _fwd(lib, layout=-1) == _abi.MOE_ERR_INVALID_ARG
     assert _fwd(lib, T=0, layout=_abi.MOE_FC1_CHUNKED) == _abi.MOE_OK
+    q = ctypes.c_void_p(32)
+    assert _fwd(lib, norm=q, eps=-1.0) == _abi.MOE_ERR_INVALID_ARG        # eps < 0
+    assert _fwd(lib, norm=q, eps=float("nan")) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd(lib, norm=ctypes.c_void_p(34)) == _abi.MOE_ERR_INVALID_ARG  # misaligned weight
+    assert _fwd(lib, norm=q, eps=-1.0, T=0) == _abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_rmsnorm(q, q, 4, 64, 1e-6, _abi.MOE_BF16, ctypes.c_void_p(64), None) == \
+        _abi.MOE_ERR_INVALID_ARG                                           # y overlaps x
+    assert lib.moe_rmsnorm(q, q, 4, 60, 1e-6, _abi.MOE_BF16, ctypes.c_void_p(8192), None) == \
+        _abi.MOE_ERR_INVALID_ARG                                           # H % 8
+    assert lib.moe_rmsnorm(q, q, 0, 64, 1e-6, _abi.MOE_BF16, q, None) == _abi.MOE_OK
     assert _fwd(lib, H=72) == _abi.MOE_ERR_UNSUPPORTED      # bf16 needs H % 64 == 0
     assert _fwd(lib, T=0) == _abi.MOE_OK                   # empty batch: nothing to do
     assert _fwd(lib, ptr=18) == _abi.MOE_ERR_INVALID_ARG    # misaligned tensors

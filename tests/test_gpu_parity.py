@@ -12,7 +12,7 @@ import mixture_experts_ffn_15_b200 as moe
 from oracle import moe_oracle as O
 from parity_util import (W_ATOL, assert_close, bf16_storage_bound, device_inputs, from_dev,
                          match_routing, row_scale, sample_tokens, to_dev, tol)
-from synth import Workload, bf16_bits_to_f32, make_inputs
+from synth import Workload, bf16_bits_to_f32, make_inputs, round_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -342,6 +342,116 @@ def test_expert_ffn_reads_chunked_fc1_in_place(dtype):
                              fc2_bias=db2)
         torch.cuda.synchronize()
         assert torch.equal(_bits(y_c), _bits(y_i)), name
+
+
+# ------------------------------------------------------------------ pre-FFN RMSNorm
+# The Llama-style norm in front of the layer ("Contributing Gemma 4 support and ONNX
+# export optimizations", "Key Technical Contributions").  Both sides evaluate it in
+# float64 and round once to the storage dtype; the float64 values differ by a few
+# float64 ulps at most (the order of the sums), which moves a bf16 or float32 rounding
+# only for values within ~1e-15 relative of a rounding boundary: the results are
+# compared bit for bit.
+NORM_SHAPES = [(1, 64, "bf16", 4.0), (37, 2816, "bf16", 4.0), (300, 72, "bf16", 300.0),
+               (64, 256, "bf16", 1e-3), (33, 136, "f32", 4.0), (5, 2816, "f32", 50.0)]
+
+
+def _bits_np(a, dtype):
+    return a.astype(np.float32).view(np.uint32) if dtype == "f32" else \
+        round_to_bf16_bits(a.astype(np.float32))
+
+
+@pytest.mark.parametrize("T,H,dtype,scale", NORM_SHAPES,
+                         ids=[f"T{t}_H{h}_{d}_x{s:g}" for t, h, d, s in NORM_SHAPES])
+def test_rmsnorm_bitexact(T, H, dtype, scale):
+    from synth import make_pre_norm_inputs
+    wl = W("norm", T=T, H=H, dtype=dtype)
+    x, w = make_pre_norm_inputs(wl, scale=scale)
+    eps = float(np.float32(1e-6))
+    xv = bf16_bits_to_f32(x) if dtype == "bf16" else x
+    wv = bf16_bits_to_f32(w) if dtype == "bf16" else w
+    if T > 3:
+        x = x.copy()
+        x[3] = 0                              # an all-zero row: eps keeps it at zero
+        xv = xv.copy()
+        xv[3] = 0
+    got = moe.rmsnorm(to_dev(x, dtype), to_dev(w, dtype), eps)
+    ref = O.pre_ffn_norm(xv, wv, eps, dtype)
+    got_bits = got.cpu().view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else \
+        got.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(got_bits, _bits_np(ref, dtype))
+
+
+NORM_CASES = [
+    W("norm_one_launch", T=4, H=256, E=64, k=4, I=128),
+    W("norm_router_decode", T=100, H=256, E=64, k=4, I=128, router_bias_std=0.5),
+    W("norm_small_decode", T=100, H=256, E=16, k=4, I=128),
+    W("norm_pairs", T=1100, H=256, E=64, k=4, I=192),
+    W("norm_f32", T=70, H=64, E=6, k=3, I=32, dtype="f32"),
+]
+
+
+@pytest.mark.parametrize("wl", NORM_CASES, ids=[c.name for c in NORM_CASES])
+def test_forward_with_pre_norm(wl):
+    """moe_forward(x, norm_weight) on every path: bit-equal to moe_rmsnorm followed by the
+    plain layer, and the oracle's layer on the oracle's norm of x within tolerance."""
+    from synth import make_pre_norm_inputs
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    x, w = make_pre_norm_inputs(wl)
+    dx, dw = to_dev(x, wl.dtype), to_dev(w, wl.dtype)
+    eps = float(np.float32(1e-5))
+    kw = dict(normalize=bool(wl.normalize), router_bias=dev["router_bias"])
+    fused = moe.forward(dx, dev["router_w"], dev["fc1"], dev["fc2"], wl.k, norm_weight=dw,
+                        norm_eps=eps, **kw)
+    xn = moe.rmsnorm(dx, dw, eps)
+    staged = moe.forward(xn, dev["router_w"], dev["fc1"], dev["fc2"], wl.k, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(fused), _bits(staged)), wl.name
+    f = lambda a: bf16_bits_to_f32(a) if a.dtype == np.uint16 else a
+    xn_ref = O.pre_ffn_norm(f(x), f(w), eps, wl.dtype)
+    got_xn = xn.cpu().view(torch.int16).numpy().view(np.uint16) if wl.dtype == "bf16" else \
+        xn.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(got_xn, _bits_np(xn_ref, wl.dtype))
+    # routing of the normalised input, then the layer, against the oracle
+    r = moe.route(xn, dev["router_w"], wl.k, normalize=bool(wl.normalize),
+                  router_bias=dev["router_bias"])
+    torch.cuda.synchronize()
+    L = O.router_logits(xn_ref, inp.values("router_w"), inp["router_bias"])
+    gidx = from_dev(r["idx"]).astype(np.int64)
+    idx, _ = match_routing(L, gidx, wl.k)
+    np.testing.assert_array_equal(gidx, idx)
+    ref = O.moe_forward(xn_ref, inp.values("router_w"), inp["router_bias"],
+                        lambda e: inp.expert_values("fc1", e), lambda e: inp.expert_values("fc2", e),
+                        wl.k, wl.normalize, wl.fc1_layout, idx=idx)["out"]
+    atol, rtol = tol(wl.dtype, ref)
+    if wl.dtype == "bf16":
+        atol = atol * row_scale(ref)
+    assert_close(from_dev(fused), ref, atol, rtol, f"{wl.name} with pre-FFN norm")
+
+
+@pytest.mark.parametrize("name", ["decode_bf16", "prefill_bf16"])
+def test_full_workload_with_pre_norm(name):
+    """The full-size layer with the pre-FFN norm: the norm bit-exact against the oracle
+    on every element, and the fused call bit-equal to the norm followed by the layer
+    (whose parity the full-workload tests establish)."""
+    from synth import WORKLOADS, make_pre_norm_inputs
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    x, w = make_pre_norm_inputs(wl)
+    dx, dw = to_dev(x, wl.dtype), to_dev(w, wl.dtype)
+    eps = float(np.float32(1e-6))
+    xn = moe.rmsnorm(dx, dw, eps)
+    ref = O.pre_ffn_norm(bf16_bits_to_f32(x), bf16_bits_to_f32(w), eps, "bf16")
+    np.testing.assert_array_equal(xn.cpu().view(torch.int16).numpy().view(np.uint16),
+                                  _bits_np(ref, "bf16"))
+    kw = dict(normalize=bool(wl.normalize), router_bias=dev["router_bias"],
+              fc1_layout=wl.fc1_layout)
+    fused = moe.forward(dx, dev["router_w"], dev["fc1"], dev["fc2"], wl.k, norm_weight=dw,
+                        norm_eps=eps, **kw)
+    staged = moe.forward(xn, dev["router_w"], dev["fc1"], dev["fc2"], wl.k, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(fused), _bits(staged))
 
 
 def test_combine_matches_oracle():

@@ -25,7 +25,8 @@ def _static_forward(dev, wl, out):
     lib = _abi.load()
     p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    return lib.moe_forward_static(p(dev["hidden"]), p(dev["router_w"]), p(dev["router_bias"]),
+    return lib.moe_forward_static(p(dev["hidden"]), None, 1e-6, p(dev["router_w"]),
+                                  p(dev["router_bias"]),
                                   p(dev["fc1"]), p(dev["fc2"]), None, None, wl.T, wl.H, wl.E,
                                   wl.k, wl.I,
                                   wl.normalize, _abi.STANDARD_SWIGLU, _abi.MOE_FC1_INTERLEAVED,
