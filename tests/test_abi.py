@@ -43,6 +43,15 @@ def test_header_declares_the_entry_points():
         assert n in names
 
 
+def test_package_exports_every_binding():
+    import mixture_experts_ffn_15_b200 as moe
+    from mixture_experts_ffn_15_b200 import ops
+    public = [n for n, v in vars(ops).items() if callable(v) and not n.startswith("_")
+              and getattr(v, "__module__", "") == ops.__name__]
+    missing = [n for n in public if not hasattr(moe, n)]
+    assert not missing, missing
+
+
 def test_library_exports_every_declared_symbol():
     lib = _lib()
     missing = [n for n in sorted(declared_functions()) if not hasattr(lib, n)]
