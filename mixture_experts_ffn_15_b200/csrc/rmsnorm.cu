@@ -3,16 +3,28 @@
 // Llama-style normed states times the weight, not times 1 + weight; the Rust
 // weight-loader page lists the pre-FFN norm among each layer's four):
 //   y[t, h] = round((x[t, h] / sqrt(mean_h x[t, h]^2 + eps)) * w[h])
-// evaluated in float64 and rounded ONCE to the storage dtype.  The float64 value is
-// within a few float64 ulps of the exact one and a bf16 rounding boundary is never
-// that close in practice, so the layer's input does not depend on the order of the
-// sums: the bits are those of the plain definition.
+// rounded ONCE to the storage dtype from a value within ~1e-14 relative of the exact
+// one.  A rounding boundary is never that close in practice, so the layer's input does
+// not depend on the order of the sums: the bits are those of the plain definition.
 //
-// A row is spread over TPR threads (TPR = 32 .. 256, so that a thread holds at most a
-// few 16-byte vectors of it): every thread issues all its loads before it uses any,
-// the float64 partial sums of squares (every float32 square is exact in float64) are
-// reduced over the row's threads in a fixed order, then each thread scales, multiplies
-// by the weight and stores its vectors (re-read from L1).  The same launch may clear a
+// bf16 rows stay in float32 arithmetic, whose conversions to and from float64 run at a
+// small fraction of the float32 rate: the squares and the products x w of bf16 values
+// are exact in float32; each vector's eight squares are summed with error-free
+// transformations (TwoSum, D. Knuth, The Art of Computer Programming vol. 2, 4.2.2) and
+// only the (sum, error) pair is widened into the float64 row sum; the scale r =
+// 1 / sqrt(mean + eps) is taken in float64 once per row and split into r_hi + r_lo;
+// t = fl(x w r_hi + fl(x w r_lo)) is within 0.51 float32 ulp of x w r, so rounding t
+// to bf16 is right unless t lies within two float32 ulps of a bf16 midpoint (about 1e-4
+// of the values); those take the exact path: x w r as an unevaluated float32 pair (the
+// product's rounding error from an FMA, "TwoProd") rounded through round-to-odd
+// (below).  float32 rows use float64 arithmetic directly.
+//
+// A row is spread over TPR threads (TPR = 32 .. 256, so that a thread holds at most
+// kNormBatch 16-byte vectors of it): every thread issues all its loads before it uses
+// any and keeps them in registers, the float64 partial sums of squares (every float32
+// square is exact in float64) are reduced over the row's threads in a fixed order, then
+// each thread scales its vectors, multiplies them by the weight and stores them.  Rows
+// longer than 256 kNormBatch vectors take several batches (re-read for the second pass).  The same launch may clear a
 // range of the layer's workspace, so that the normalised layer needs no extra launch.
 #include <math.h>
 
@@ -23,16 +35,33 @@ namespace moe {
 namespace {
 
 constexpr int kNormThreads = 256;
-constexpr int kNormBatch = 2;   // vectors per thread loaded before any is used
+constexpr int kNormBatch = 6;   // vectors per thread loaded before any is used
 
-// float64 -> bf16 with a single rounding to nearest, ties to even: round to odd into
-// float32 first (24 >= 8 + 2 bits, so the second rounding cannot double-round; S. Boldo
-// and G. Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
-// using rounding to odd"), then float32 -> bf16 to nearest even.
-__device__ __forceinline__ uint32_t bf16_bits_from_f64(double y) {
-    float f = __double2float_rz(y);
-    if (static_cast<double>(f) != y) f = __uint_as_float(__float_as_uint(f) | 1u);
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+// hi0 + lo0 (|lo0| at most a few float32 ulps of hi0; hi0 = 0 only if lo0 = 0) -> bf16
+// with a single rounding to nearest, ties to even.  The pair is first renormalised with
+// Fast2Sum (exact for |hi0| >= |lo0|; T. J. Dekker, "A floating-point technique for
+// extending the available precision") into hi + lo, hi the float32 nearest to the sum
+// and |lo| at most half an ulp of hi; then rounded to odd into float32 (24 >= 8 + 2 bits,
+// so the second rounding cannot double-round; S. Boldo and G. Melquiond, "Emulation of
+// FMA and correctly rounded sums: proved algorithms using rounding to odd") and from
+// there to bf16, nearest even.  Round to odd: an inexact value goes to whichever of its
+// two float32 neighbours has an odd last bit -- hi itself if odd, else hi's neighbour on
+// lo's side.
+__device__ __forceinline__ uint32_t bf16_bits_of_pair(float hi0, float lo0) {
+    if (hi0 == 0.0f) return __float_as_uint(hi0) >> 16;   // a signed zero keeps its sign
+    const float hi = __fadd_rn(hi0, lo0);
+    const float lo = __fsub_rn(lo0, __fsub_rn(hi, hi0));
+    uint32_t u = __float_as_uint(hi);
+    if (lo != 0.0f && (u & 1u) == 0u) u = ((lo > 0.0f) == (hi > 0.0f)) ? u + 1u : u - 1u;
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(u))));
+}
+
+// a + b = s + e exactly (TwoSum).  The error-free transformations use the _rn
+// intrinsics, which the compiler never contracts into an FMA or reorders.
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+    s = __fadd_rn(a, b);
+    const float bb = __fsub_rn(s, a);
+    e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
 }
 
 __device__ __forceinline__ double warp_sum_f64(double v) {
@@ -53,26 +82,63 @@ __device__ __forceinline__ void load_vec(const uint4& q, float* f) {
     }
 }
 
-// y = round((x r) w) for one 16-byte vector
+// y = round(x r w) for one 16-byte vector; r = r_hi + r_lo (bf16) or rd (float32)
 template <bool BF16>
-__device__ __forceinline__ uint4 norm_vec(const uint4& q, const uint4& g, double r) {
+__device__ __forceinline__ uint4 norm_vec(const uint4& q, const uint4& g, float r_hi, float r_lo,
+                                          double rd) {
     float f[8], gw[8];
     load_vec<BF16>(q, f);
     load_vec<BF16>(g, gw);
     if constexpr (BF16) {
+        float t[8];
+        bool near_mid = false;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float xw = __fmul_rn(f[i], gw[i]);       // exact: 8 x 8 significant bits
+            t[i] = fmaf(xw, r_hi, __fmul_rn(xw, r_lo));
+            const int low = static_cast<int>(__float_as_uint(t[i]) & 0xffffu);
+            near_mid |= abs(low - 0x8000) <= 2;
+        }
+        if (!near_mid) return pack_bf16x8(t);
         uint32_t b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            b[i] = bf16_bits_from_f64((static_cast<double>(f[i]) * r) * static_cast<double>(gw[i]));
+        for (int i = 0; i < 8; ++i) {
+            const float xw = __fmul_rn(f[i], gw[i]);
+            const float p_hi = __fmul_rn(xw, r_hi);
+            const float p_err = fmaf(xw, r_hi, -p_hi);      // the product's rounding error
+            const float p_lo = fmaf(xw, r_lo, p_err);
+            b[i] = bf16_bits_of_pair(p_hi, p_lo);
+        }
         return make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16),
                           b[6] | (b[7] << 16));
     } else {
         float z[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            z[i] = __double2float_rn((static_cast<double>(f[i]) * r) * static_cast<double>(gw[i]));
+            z[i] = __double2float_rn((static_cast<double>(f[i]) * rd) * static_cast<double>(gw[i]));
         return make_uint4(__float_as_uint(z[0]), __float_as_uint(z[1]), __float_as_uint(z[2]),
                           __float_as_uint(z[3]));
+    }
+}
+
+// the sum of squares of one 16-byte vector, added to the float64 row sum
+template <bool BF16>
+__device__ __forceinline__ double add_squares(const uint4& q, double ss) {
+    float f[8];
+    load_vec<BF16>(q, f);
+    if constexpr (BF16) {
+        float hi = __fmul_rn(f[0], f[0]), lo = 0.0f;   // squares of bf16 values are exact
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            float e;
+            two_sum(hi, __fmul_rn(f[i], f[i]), hi, e);
+            lo = __fadd_rn(lo, e);
+        }
+        return ss + (static_cast<double>(hi) + static_cast<double>(lo));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ss = fma(static_cast<double>(f[i]), static_cast<double>(f[i]), ss);
+        return ss;
     }
 }
 
@@ -98,22 +164,16 @@ rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ w, int T, in
         const bool live = t < T;
         const uint4* xr = reinterpret_cast<const uint4*>(x) + static_cast<size_t>(live ? t : 0) * nv;
         double ss = 0.0;
+        uint4 q[kNormBatch];   // the thread's vectors of the row (first batch)
         if (live) {
             for (int base = j; base < nv; base += TPR * kNormBatch) {
-                uint4 q[kNormBatch];
 #pragma unroll
                 for (int b = 0; b < kNormBatch; ++b) {
                     const int v = base + b * TPR;
                     q[b] = v < nv ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
-                for (int b = 0; b < kNormBatch; ++b) {
-                    float f[8];
-                    load_vec<BF16>(q[b], f);
-#pragma unroll
-                    for (int i = 0; i < VEC; ++i)
-                        ss = fma(static_cast<double>(f[i]), static_cast<double>(f[i]), ss);
-                }
+                for (int b = 0; b < kNormBatch; ++b) ss = add_squares<BF16>(q[b], ss);
             }
         }
         ss = warp_sum_f64(ss);
@@ -127,21 +187,24 @@ rmsnorm_kernel(const void* __restrict__ x, const void* __restrict__ w, int T, in
         }
         if (!live) continue;
         const double r = 1.0 / sqrt(ss / static_cast<double>(H) + eps);
+        const float r_hi = static_cast<float>(r);
+        const float r_lo = static_cast<float>(r - static_cast<double>(r_hi));
         uint4* yr = reinterpret_cast<uint4*>(y) + static_cast<size_t>(t) * nv;
+        const bool one_batch = nv <= TPR * kNormBatch;   // q still holds the whole share
         for (int base = j; base < nv; base += TPR * kNormBatch) {
-            uint4 q[kNormBatch], g[kNormBatch];
+            uint4 g[kNormBatch];
 #pragma unroll
             for (int b = 0; b < kNormBatch; ++b) {
                 const int v = base + b * TPR;
                 if (v < nv) {
-                    q[b] = __ldg(xr + v);
+                    if (!one_batch) q[b] = __ldg(xr + v);
                     g[b] = __ldg(wv + v);
                 }
             }
 #pragma unroll
             for (int b = 0; b < kNormBatch; ++b) {
                 const int v = base + b * TPR;
-                if (v < nv) yr[v] = norm_vec<BF16>(q[b], g[b], r);
+                if (v < nv) yr[v] = norm_vec<BF16>(q[b], g[b], r_hi, r_lo, r);
             }
         }
     }
@@ -166,11 +229,15 @@ cudaError_t launch_rmsnorm(const void* x, const void* w, int T, int H, float eps
     if ((clear_bytes & 15) != 0 || (reinterpret_cast<uintptr_t>(clear) & 15) != 0)
         return cudaErrorInvalidValue;
     const long long n_clear = static_cast<long long>(clear_bytes / 16);
-    // threads per row: the smallest of 32 .. 256 that leaves each thread at most two
-    // vectors of the row (rows longer than 512 vectors take more batches)
+    // threads per row: the smallest of 32 .. 256 that leaves each thread at most
+    // kNormBatch vectors of the row (longer rows take more batches), widened while the
+    // batch would not give every SM a block (small batches: spread each row out)
     const int nv = H / (bf16 ? 8 : 4);
     int tpr = 32;
-    while (tpr < kNormThreads && 2 * tpr < nv) tpr *= 2;
+    while (tpr < kNormThreads && kNormBatch * tpr < nv) tpr *= 2;
+    while (tpr < kNormThreads && tpr < nv &&
+           (static_cast<long long>(T) * tpr + kNormThreads - 1) / kNormThreads < device_sm_count())
+        tpr *= 2;
     const int rpb = kNormThreads / tpr;
     // one pass of the row loop per block: the hardware schedules the blocks in waves
     long long blocks = (static_cast<long long>(T) + rpb - 1) / rpb;

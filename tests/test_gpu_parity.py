@@ -372,8 +372,8 @@ def test_rmsnorm_bitexact(T, H, dtype, scale):
     if T > 3:
         x = x.copy()
         x[3] = 0                              # an all-zero row: eps keeps it at zero
-        xv = xv.copy()
-        xv[3] = 0
+        x[2, :5] = 0x8000 if dtype == "bf16" else np.float32(-0.0)   # signed zeros stay signed
+        xv = bf16_bits_to_f32(x) if dtype == "bf16" else x
     got = moe.rmsnorm(to_dev(x, dtype), to_dev(w, dtype), eps)
     ref = O.pre_ffn_norm(xv, wv, eps, dtype)
     got_bits = got.cpu().view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else \

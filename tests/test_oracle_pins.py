@@ -316,6 +316,9 @@ def check_round_to_dtype():
                                   [1.0, 1 + 2 ** -6, -1.0, 1 + 2 ** -7, 2.0, 0.375])
     np.testing.assert_array_equal(O.round_to_dtype(np.array([1 + 2 ** -24, 1 + 3 * 2 ** -24]), "f32"),
                                   [1.0, 1 + 2 ** -22])
+    # a negative zero stays negative (the norm of a -0 input is -0)
+    assert np.signbit(O.round_to_dtype(np.array([-0.0]), "bf16"))[0]
+    assert np.signbit(O.pre_ffn_norm(np.array([[-0.0, 1.0]]), np.ones(2), 0.0, "bf16"))[0, 0]
 
 
 def check_rms_norm_closed_forms():
