@@ -95,7 +95,8 @@ __device__ __forceinline__ uint4 norm_vec(const uint4& q, const uint4& g, float 
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float xw = __fmul_rn(f[i], gw[i]);       // exact: 8 x 8 significant bits
-            t[i] = fmaf(xw, r_hi, __fmul_rn(xw, r_lo));
+            // (a zero keeps its sign: -0 w r is -0, which the FMA's sum would lose)
+            t[i] = xw == 0.0f ? __fmul_rn(xw, r_hi) : fmaf(xw, r_hi, __fmul_rn(xw, r_lo));
             const int low = static_cast<int>(__float_as_uint(t[i]) & 0xffffu);
             near_mid |= abs(low - 0x8000) <= 2;
         }
