@@ -30,6 +30,10 @@ following the pages in their order:
   weight as in Gemma 2); the Rust weight-loader page lists a pre-FFN norm among the
   four norms of each layer.  `rms_norm` is that norm, `pre_ffn_norm` the layer's
   input made from a residual activation by it.
+* "Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", description: the CUDA
+  pull request it cites adds a quantised MoE operator (QMoE); the Rust weight-loader
+  page loads 4-bit MLP weights.  Neither gives a format; `dequantize_rows` is the
+  reading used here for weight-only int8 experts (see below).
 * same forum page, "Key Technical Contributions", ONNX tracing compatibility: inside
   grouped_mm_experts_forward the per-expert token count is a bincount over the
   chosen expert ids, followed by a grouped matmul over experts.
@@ -55,7 +59,10 @@ notes of the repository):
 * the RMSNorm is y = (x / sqrt(mean(x^2) + eps)) * weight evaluated in float64 and
   rounded once to the storage dtype (round to nearest, ties to even): the pages fix
   the formula, not its precision, and one rounding of the exact value is the plain
-  definition; eps is the caller's.
+  definition; eps is the caller's;
+* int8 experts: every weight row r holds int8 values q[r, :] in [-127, 127] and one
+  scale s[r]; its weights are q[r, :] * s[r] (symmetric, one scale per output row);
+  the layer is the same layer on those weights.
 
 Parity pins for every function here live in tests/test_oracle_pins.py.  No
 function in this file is "parity unpinned".
@@ -290,6 +297,11 @@ def combine(y_perm, perm_dst, w, T: int, k: int) -> np.ndarray:
 
 
 # ------------------------------------------------------------------------ pre-FFN norm
+
+def dequantize_rows(q, scale) -> np.ndarray:
+    """Weight-only int8 weights of one expert: w[r, :] = q[r, :] * scale[r], float64."""
+    return np.asarray(q, dtype=F64) * np.asarray(scale, dtype=F64)[:, None]
+
 
 def round_to_dtype(y, dtype: str) -> np.ndarray:
     """float64 values rounded once to the storage dtype, round to nearest, ties to

@@ -39,6 +39,7 @@ import numpy as np
 # Stream identifiers: fixed forever, so that a seed always means the same tensors.
 _S_HIDDEN, _S_ROUTER, _S_BIAS, _S_FC1, _S_FC2, _S_OUTLIER = 1, 2, 3, 4, 5, 6
 _S_FC1_BIAS, _S_FC2_BIAS, _S_NORM_W, _S_RESIDUAL = 7, 8, 9, 10
+_S_Q1, _S_Q2, _S_QS1, _S_QS2 = 11, 12, 13, 14
 
 
 @dataclass(frozen=True)
@@ -195,3 +196,25 @@ def make_pre_norm_inputs(wl: Workload, scale: float = 4.0, seed: Optional[int] =
     x = _normal((s, _S_RESIDUAL), (wl.T, wl.H), scale)
     w = 1.0 + _normal((s, _S_NORM_W), (wl.H,), 0.1)
     return _store(x, wl.dtype), _store(w.astype(np.float32), wl.dtype)
+
+
+def make_q8_experts(wl: Workload, seed: Optional[int] = None):
+    """Weight-only int8 experts for `wl`: per expert, q = round(N(0, 1) * 127 / 4)
+    clipped to [-127, 127] (int8) and one float32 scale per weight row, the layer's
+    weight std (1/sqrt(H) for fc1, 1/sqrt(I) for fc2) * 4 / 127 times U(0.75, 1.25), so
+    that q * scale has about the std of the bf16 weights.  Returns (fc1_q [E, 2I, H]
+    int8 in the workload's fc1 layout, fc1_scale [E, 2I] float32, fc2_q [E, H, I] int8,
+    fc2_scale [E, H] float32), drawn expert by expert."""
+    s = wl.seed if seed is None else seed
+    E, H, I = wl.E, wl.H, wl.I
+    fc1_q = np.empty((E, 2 * I, H), dtype=np.int8)
+    fc2_q = np.empty((E, H, I), dtype=np.int8)
+    for e in range(E):
+        for dst, key, shape in ((fc1_q, _S_Q1, (2 * I, H)), (fc2_q, _S_Q2, (H, I))):
+            z = _normal((s, key, e), shape, 127.0 / 4.0)
+            dst[e] = np.clip(np.rint(z), -127, 127).astype(np.int8)
+    u1 = np.random.default_rng([s, _S_QS1]).uniform(0.75, 1.25, size=(E, 2 * I))
+    u2 = np.random.default_rng([s, _S_QS2]).uniform(0.75, 1.25, size=(E, H))
+    fc1_scale = (u1 * (4.0 / 127.0) / np.sqrt(H)).astype(np.float32)
+    fc2_scale = (u2 * (4.0 / 127.0) / np.sqrt(I)).astype(np.float32)
+    return fc1_q, fc1_scale, fc2_q, fc2_scale

@@ -363,6 +363,34 @@ def check_pre_ffn_norm_rounds_once():
     np.testing.assert_array_equal(O.round_to_dtype(y, "bf16"), y)   # already bf16 values
 
 
+def check_dequantize_rows():
+    # closed forms: unit scales return q itself; scale s multiplies row r only
+    q = np.array([[1, -2, 127], [-127, 0, 5]], dtype=np.int8)
+    np.testing.assert_array_equal(O.dequantize_rows(q, [1.0, 1.0]), q.astype(np.float64))
+    np.testing.assert_array_equal(O.dequantize_rows(q, [0.5, 3.0]),
+                                  [[0.5, -1.0, 63.5], [-381.0, 0.0, 15.0]])
+    # (2q, s/2) is the same weight; an expert FFN on dequantized rows is the FFN of the
+    # float64 weights q * s, and doubling one fc2 row's scale doubles that output column
+    rng = np.random.default_rng(21)
+    q1 = rng.integers(-63, 64, size=(8, 16)).astype(np.int8)
+    s1 = rng.uniform(0.01, 0.02, size=8)
+    np.testing.assert_array_equal(O.dequantize_rows(2 * q1.astype(np.int16), s1 / 2),
+                                  O.dequantize_rows(q1, s1))
+    q2 = rng.integers(-127, 128, size=(16, 4)).astype(np.int8)
+    s2 = rng.uniform(0.01, 0.02, size=16)
+    x = rng.standard_normal((3, 16))
+    y = O.expert_ffn(x, O.dequantize_rows(q1, s1), O.dequantize_rows(q2, s2))
+    s2b = s2.copy()
+    s2b[5] *= 2
+    y2 = O.expert_ffn(x, O.dequantize_rows(q1, s1), O.dequantize_rows(q2, s2b))
+    np.testing.assert_allclose(y2[:, 5], 2 * y[:, 5], rtol=1e-14)
+    np.testing.assert_array_equal(np.delete(y2, 5, axis=1), np.delete(y, 5, axis=1))
+
+
+def test_dequantize_rows():
+    check_dequantize_rows()
+
+
 def test_round_to_dtype():
     check_round_to_dtype()
 
@@ -619,6 +647,12 @@ def _mut_round_truncate(y, dtype):
     return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
 
 
+def _mut_scale_per_column(q, scale):
+    q = np.asarray(q, dtype=np.float64)
+    sc = np.asarray(scale, dtype=np.float64)
+    return q * np.resize(sc, q.shape[1])[None, :]
+
+
 _real_rms_norm = O.rms_norm
 _real_perm = O.stable_permutation
 _real_swiglu = O.swiglu
@@ -642,6 +676,7 @@ MUTATIONS = [
     ("rms_norm", _mut_sum_not_mean),
     ("round_to_dtype", _mut_round_half_up),
     ("round_to_dtype", _mut_round_truncate),
+    ("dequantize_rows", _mut_scale_per_column),
 ]
 
 PIN_CHECKS = [check_golden_values, check_golden_routing, check_topk_brute_force,
@@ -649,7 +684,8 @@ PIN_CHECKS = [check_golden_values, check_golden_routing, check_topk_brute_force,
               check_dense_masked_equals_sparse, check_expert_ffn_scalar_loops,
               check_swiglu_closed_forms, check_swiglu_limit_saturation,
               check_expert_biases_zero_input, check_biased_chunked_equals_interleaved,
-              check_round_to_dtype, check_rms_norm_closed_forms, check_pre_ffn_norm_rounds_once]
+              check_round_to_dtype, check_rms_norm_closed_forms, check_pre_ffn_norm_rounds_once,
+              check_dequantize_rows]
 
 
 @pytest.mark.parametrize("name,mutant", MUTATIONS, ids=[f"{m[0]}-{m[1].__name__}" for m in MUTATIONS])
