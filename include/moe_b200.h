@@ -220,6 +220,35 @@ moe_status moe_forward_static(const void* hidden, const void* norm_weight, float
                               int normalize, moe_swiglu act, moe_fc1_layout fc1_layout,
                               moe_dtype dt, void* out, void* stream);
 
+/* ------------------------------------------------------------ int8 expert weights */
+
+/* Weight-only int8 experts for decode-sized batches.  The pages name quantised MoE
+ * (the QMoE operator of the CUDA pull request they cite) and 4-bit checkpoint weights
+ * without a format; this library's reading: each weight row holds int8 values q in
+ * [-127, 127] and one float32 scale, the weight being q * scale (symmetric, per output
+ * row).  Activations, biases and outputs stay bf16; arithmetic as the bf16 path (q is
+ * exact in bf16, the tensor cores accumulate sum_k q x in float32, the epilogue
+ * multiplies by the row's scale before the bias and the activation).
+ *   fc1_q [E, 2I, H] int8 in fc1_layout, fc1_scale [E, 2I] float32 (same layout)
+ *   fc2_q [E, H, I] int8, fc2_scale [E, H] float32
+ * Everything else as moe_forward / moe_expert_ffn with dt = MOE_BF16.  The int8
+ * weights run in the decode FFN only: sizes where it does not apply (more than 64
+ * routed rows per expert on average, H or 2I not multiples of 128) return
+ * MOE_ERR_UNSUPPORTED; the whole-layer call routes with the staged kernels (the
+ * single-launch decode layer is bf16 only).  moe_workspace_size(T, H, E, k, I,
+ * MOE_BF16) and moe_expert_ffn_workspace_size(rows, I, MOE_BF16) apply. */
+moe_status moe_forward_q8(const void* hidden, const void* norm_weight, float norm_eps,
+                          const void* router_w, const float* router_bias, const int8_t* fc1_q,
+                          const float* fc1_scale, const int8_t* fc2_q, const float* fc2_scale,
+                          const void* fc1_bias, const void* fc2_bias, int T, int H, int E, int k,
+                          int I, int normalize, moe_swiglu act, moe_fc1_layout fc1_layout,
+                          void* out, void* workspace, size_t ws_bytes, void* stream);
+moe_status moe_expert_ffn_q8(const void* x_perm, const int32_t* offsets, const int8_t* fc1_q,
+                             const float* fc1_scale, const int8_t* fc2_q, const float* fc2_scale,
+                             const void* fc1_bias, const void* fc2_bias, int rows, int H, int E,
+                             int I, moe_swiglu act, moe_fc1_layout fc1_layout, void* y_perm,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Layout conversion of fc1 from the Hugging Face chunked layout ("Weight layout":
  * [E, 2*inter, H], the first inter rows gate, the next inter rows up) to the
  * interleaved layout of swiglu_fusion = 1:  dst[e, 2j+s, :] = src[e, s*I + j, :].

@@ -35,6 +35,10 @@ SIGNATURES = {
                          MoeSwiglu, _i, _i, _vp, _vp, _sz, _vp]),
     "moe_forward_static": (_i, [_vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                 _i, MoeSwiglu, _i, _i, _vp, _vp]),
+    "moe_forward_q8": (_i, [_vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                            _i, _i, MoeSwiglu, _i, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn_q8": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, MoeSwiglu,
+                               _i, _vp, _vp, _sz, _vp]),
     "convert_chunked_to_interleaved": (_i, [_vp, _vp, _i, _i, _i, _i, _vp]),
     "moe_get_error": (_i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),

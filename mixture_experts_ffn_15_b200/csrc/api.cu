@@ -161,6 +161,15 @@ int forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
     return path;
 }
 
+// int8 experts: the decode FFN with the staged routing (0: no such path for these sizes)
+int forward_path_q8(int T, int H, int E, int k, int I) {
+    const int rows = T * k;
+    if (!decode_ffn_supported(rows, E, H, I)) return 0;
+    if (T > kRouteSmallTcT && tc_route_supported(H, E, k)) return kPathTcRouter | kPathDecodeFfn;
+    if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) return kPathSmallRoute | kPathDecodeFfn;
+    return kPathDecodeFfn;   // routed by the float32-logit top-k kernels
+}
+
 void record(int i, cudaStream_t s) {
     if (g_events_on) record_event(g_events[i], s);
 }
@@ -367,14 +376,19 @@ moe_status moe_rmsnorm(const void* x, const void* weight, int T, int H, float ep
     return MOE_OK;
 }
 
-moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_eps,
-                       const void* router_w, const float* router_bias,
-                       const void* fc1, const void* fc2, const void* fc1_bias, const void* fc2_bias,
-                       int T, int H, int E, int k, int I, int normalize, moe_swiglu act,
-                       moe_fc1_layout fc1_layout, moe_dtype dt, void* out, void* workspace,
-                       size_t ws_bytes, void* stream) {
+// The layer; with fc1_scale / fc2_scale, fc1 and fc2 hold int8 weights (moe_forward_q8).
+static moe_status forward_impl(const void* hidden, const void* norm_weight, float norm_eps,
+                               const void* router_w, const float* router_bias, const void* fc1,
+                               const void* fc2, const void* fc1_bias, const void* fc2_bias, int T,
+                               int H, int E, int k, int I, int normalize, moe_swiglu act,
+                               moe_fc1_layout fc1_layout, moe_dtype dt, void* out, void* workspace,
+                               size_t ws_bytes, void* stream, const float* fc1_scale,
+                               const float* fc2_scale) {
     if (!valid_sizes(T, H, E, k) || I <= 0 || I % 8 || !valid_dtype(dt) || !valid_swiglu(act) ||
         !valid_layout(fc1_layout) || (norm_weight && !valid_eps(norm_eps)))
+        return MOE_ERR_INVALID_ARG;
+    const bool q8 = fc1_scale != nullptr;
+    if (q8 && (dt != MOE_BF16 || !fc2_scale || !aligned(fc1_scale, 4) || !aligned(fc2_scale, 4)))
         return MOE_ERR_INVALID_ARG;
     if (norm_weight && !aligned(norm_weight, 16)) return MOE_ERR_INVALID_ARG;
     if ((fc1_bias && !aligned(fc1_bias, elem_size(dt))) || (fc2_bias && !aligned(fc2_bias, elem_size(dt))))
@@ -404,8 +418,15 @@ moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_e
     const bool bf16 = dt == MOE_BF16;
     const int rows = T * k;
 
-    const int path = forward_path(T, H, E, k, I, dt);
-    const FfnAttrs ep = make_ffn_attrs(act, fc1_layout, fc1_bias, fc2_bias);
+    int path = forward_path(T, H, E, k, I, dt);
+    FfnAttrs ep = make_ffn_attrs(act, fc1_layout, fc1_bias, fc2_bias);
+    if (q8) {
+        // int8 experts run in the decode FFN only, routed by the staged kernels
+        path = forward_path_q8(T, H, E, k, I);
+        if (path == 0) return MOE_ERR_UNSUPPORTED;
+        ep.fc1_scale = fc1_scale;
+        ep.fc2_scale = fc2_scale;
+    }
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
@@ -545,6 +566,63 @@ moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_e
     record(4, s);
     MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));
     record(5, s);
+    return MOE_OK;
+}
+
+moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_eps,
+                       const void* router_w, const float* router_bias,
+                       const void* fc1, const void* fc2, const void* fc1_bias, const void* fc2_bias,
+                       int T, int H, int E, int k, int I, int normalize, moe_swiglu act,
+                       moe_fc1_layout fc1_layout, moe_dtype dt, void* out, void* workspace,
+                       size_t ws_bytes, void* stream) {
+    return forward_impl(hidden, norm_weight, norm_eps, router_w, router_bias, fc1, fc2, fc1_bias,
+                        fc2_bias, T, H, E, k, I, normalize, act, fc1_layout, dt, out, workspace,
+                        ws_bytes, stream, nullptr, nullptr);
+}
+
+moe_status moe_forward_q8(const void* hidden, const void* norm_weight, float norm_eps,
+                          const void* router_w, const float* router_bias, const int8_t* fc1_q,
+                          const float* fc1_scale, const int8_t* fc2_q, const float* fc2_scale,
+                          const void* fc1_bias, const void* fc2_bias, int T, int H, int E, int k,
+                          int I, int normalize, moe_swiglu act, moe_fc1_layout fc1_layout,
+                          void* out, void* workspace, size_t ws_bytes, void* stream) {
+    if (!fc1_scale || !fc2_scale) return MOE_ERR_INVALID_ARG;
+    return forward_impl(hidden, norm_weight, norm_eps, router_w, router_bias, fc1_q, fc2_q,
+                        fc1_bias, fc2_bias, T, H, E, k, I, normalize, act, fc1_layout, MOE_BF16, out,
+                        workspace, ws_bytes, stream, fc1_scale, fc2_scale);
+}
+
+moe_status moe_expert_ffn_q8(const void* x_perm, const int32_t* offsets, const int8_t* fc1_q,
+                             const float* fc1_scale, const int8_t* fc2_q, const float* fc2_scale,
+                             const void* fc1_bias, const void* fc2_bias, int rows, int H, int E,
+                             int I, moe_swiglu act, moe_fc1_layout fc1_layout, void* y_perm,
+                             void* workspace, size_t ws_bytes, void* stream) {
+    if (rows < 0 || H <= 0 || H % 8 || I <= 0 || I % 8 || E <= 0 || E > kMaxExperts ||
+        !valid_swiglu(act) || !valid_layout(fc1_layout))
+        return MOE_ERR_INVALID_ARG;
+    if ((fc1_bias && !aligned(fc1_bias, 2)) || (fc2_bias && !aligned(fc2_bias, 2)))
+        return MOE_ERR_INVALID_ARG;
+    if (!fc1_scale || !fc2_scale || !aligned(fc1_scale, 4) || !aligned(fc2_scale, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (!decode_ffn_supported(rows, E, H, I)) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!x_perm || !offsets || !fc1_q || !fc2_q || !y_perm || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_perm, 16) || !aligned(fc1_q, 16) || !aligned(fc2_q, 16) || !aligned(y_perm, 16) ||
+        !aligned(workspace, kAlign))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < moe_expert_ffn_workspace_size(rows, I, MOE_BF16)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* err = reinterpret_cast<int32_t*>(ws);
+    void* act_buf = ws + kAlign;
+    int32_t* ctr = reinterpret_cast<int32_t*>(ws + kAlign + align_up(static_cast<size_t>(rows) * I * 2));
+    MOE_CUDA(cudaMemsetAsync(err, 0, 4, s));
+    FfnAttrs ep = make_ffn_attrs(act, fc1_layout, fc1_bias, fc2_bias);
+    ep.fc1_scale = fc1_scale;
+    ep.fc2_scale = fc2_scale;
+    MOE_CUDA(cudaMemsetAsync(ctr, 0, static_cast<size_t>(decode_ffn_counters(rows, E)) * 4, s));
+    MOE_CUDA(launch_ffn_decode(x_perm, nullptr, rows, offsets, fc1_q, fc2_q, rows, H, E, I, act_buf,
+                               y_perm, ctr, err, nullptr, nullptr, 0, nullptr, s, ep));
     return MOE_OK;
 }
 

@@ -175,7 +175,9 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kPWaitNs);
                     if (ok && lead) mbar_arrive_expect_tx(smem_u32(&full[stage]), bytes);
                 }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                // the whole warp leaves together (lane 0 alone saw the wait give up)
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
                 const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);   // the even CTA's
                 const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);

@@ -417,6 +417,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // Every CTA of the grid (at most one per SM) is resident, so the waits always end.
 constexpr int kUnitRing = 4;
 
+// Weight-only int8 experts (Q8): the weights stream from HBM as int8 through a deep ring
+// of their own (kQStages tiles of 128 rows x 64 bytes, loaded by a dedicated producer
+// warp), four converter warps write each tile as bf16 -- exact, |q| <= 127 -- into the
+// 128-byte-swizzled layout of the bf16 path, and the epilogue multiplies each weight
+// row's accumulator by its float32 scale.  The MMA and the token side are unchanged.
+constexpr int kQBytes = BM * BK;   // one int8 tile: 128 weight rows x 64 K
+
+template <bool Q8>
+struct DecodeCfg {
+    using T = Tr<W_PLAIN, 64>;
+    static constexpr int kABytes = T::kABytes;
+    static constexpr int kBBytes = T::kBBytes;
+    static constexpr int kStages = Q8 ? 5 : T::kStages;     // bf16 A + token B ring
+    static constexpr int kQStages = Q8 ? 12 : 0;            // int8 weight ring
+    static constexpr int kThreads = Q8 ? 352 : 192;         // + Q producer + 4 converters
+    static constexpr int kAccStride = T::kAccStride;
+    static constexpr int kTmemCols = T::kTmemCols;
+    static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
+    static constexpr int kMiscBytes = T::kMiscBytes + 2 * kQStages * 8;   // + int8 ring barriers
+    static constexpr int kSmemBytes = 1024 + kDataBytes + kMiscBytes;
+    static_assert(kStages <= T::kStages, "barrier space");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
 struct DecodeParams {
     const int32_t* offsets;   // [E+1]
     const int32_t* perm_src;  // [rows] with GATHER, else nullptr
@@ -436,6 +460,8 @@ struct DecodeParams {
     const __nv_bfloat16* b1;        // [E, 2I] fc1 bias (fc1's layout) or nullptr
     bool fc1_chunked;               // fc1 and b1 in the chunked layout
     const __nv_bfloat16* b2;        // [E, H] fc2 bias or nullptr
+    const float* s1;                // Q8: [E, 2I] fc1 row scales (fc1's layout)
+    const float* s2;                // Q8: [E, H] fc2 row scales
     // ROUTE: the routing runs inside the launch (fields below); offsets, perm_src,
     // perm_dst and topk_w above are then unused (the kernel keeps them in shared memory)
     const void* hidden;       // [T, H]
@@ -517,18 +543,20 @@ __device__ __forceinline__ DUnit decode_dunit(int u, int U1, int MT1, int MT2, i
     return d;
 }
 
-template <bool GATHER, bool ROUTE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GATHER, bool ROUTE, bool Q8>
+__global__ void __launch_bounds__(DecodeCfg<Q8>::kThreads, 1)
 tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmAct,
                      const DecodeParams p) {
-    using C = Tr<W_PLAIN, 64>;
+    using C = DecodeCfg<Q8>;
+    static_assert(!(Q8 && ROUTE), "the int8 path takes its routing from the staged kernels");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + C::kStages * C::kABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+    uint8_t* sQ = sB + C::kStages * C::kBBytes;               // Q8: int8 weight ring
+    uint64_t* full = reinterpret_cast<uint64_t*>(sQ + C::kQStages * kQBytes);
     uint64_t* empty = full + C::kStages;
     uint64_t* tfull = empty + C::kStages;
     uint64_t* tempty = tfull + 2;
@@ -539,8 +567,10 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     int* s_unit = s_pre + (kMaxExperts + 1);                        // [kUnitRing]
     uint64_t* ufull = reinterpret_cast<uint64_t*>(s_unit + 2 * kUnitRing);   // 8-byte aligned
     uint64_t* uempty = ufull + kUnitRing;
+    uint64_t* qfull = uempty + kUnitRing;                    // Q8: [kQStages]
+    uint64_t* qempty = qfull + C::kQStages;
     // ROUTE only: the routing of the whole batch, after the misc block
-    int* s_ridx = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + C::kMiscBytes);
+    int* s_ridx = reinterpret_cast<int*>(smem + C::kDataBytes + C::kMiscBytes);
     float* s_rw = reinterpret_cast<float*>(s_ridx + kFusedRouteMaxRows);
     int* s_pdst = reinterpret_cast<int*>(s_rw + kFusedRouteMaxRows);
     int* s_psrc = s_pdst + kFusedRouteMaxRows;
@@ -553,7 +583,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     const int G = p.E;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
+            // Q8: the token producer's arrival (with its bytes) and the 4 converter warps
+            mbar_init(smem_u32(&full[s]), Q8 ? 5 : 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -562,7 +593,12 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         }
         for (int q = 0; q < kUnitRing; ++q) {
             mbar_init(smem_u32(&ufull[q]), 1);
-            mbar_init(smem_u32(&uempty[q]), 5);   // the MMA thread and 4 epilogue warps
+            // the MMA thread and 4 epilogue warps (Q8: + the int8 producer and 4 converters)
+            mbar_init(smem_u32(&uempty[q]), Q8 ? 10 : 5);
+        }
+        for (int q = 0; q < C::kQStages; ++q) {
+            mbar_init(smem_u32(&qfull[q]), 1);
+            mbar_init(smem_u32(&qempty[q]), 4);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -791,6 +827,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const bool f1 = d.phase == 1;
             const int nk = f1 ? nk1 : nk2;
             // both weight maps are (k, s, i, e) pair views: rows d.mt BM .. of expert d.g
+            // (Q8: the int8 producer warp loads them)
             const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;
             const int nl = (d.nrows + kBoxTok - 1) / kBoxTok;
             uint32_t bbytes = static_cast<uint32_t>(nl * kBoxTok * BK * 2);
@@ -820,13 +857,15 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             for (int kb = 0; kb < nk; ++kb) {
                 if (lane == 0) {
                     ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
-                    if (ok) mbar_arrive_expect_tx(smem_u32(&full[stage]), C::kABytes + bbytes);
+                    if (ok) mbar_arrive_expect_tx(smem_u32(&full[stage]), (Q8 ? 0 : C::kABytes) + bbytes);
                 }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                // the whole warp leaves together (lane 0 alone saw the wait give up)
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
                 const uint32_t fb = smem_u32(&full[stage]);
                 const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
                 const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                if (lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
+                if (!Q8 && lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
                 if (f1 && GATHER) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -904,7 +943,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 if (acc == 0) acc_phase ^= 1u;
             }
         }
-    } else {
+    } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
@@ -931,10 +970,11 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const int wr = d.mt * BM + r;   // weight row inside the expert
             // this lane's weight row's bias (fc1: interleaved row wr in fc1's layout, fc2: h)
             const __nv_bfloat16* bsrc = f1 ? p.b1 : p.b2;
-            const float bias =
-                bsrc ? bf16_at(bsrc, static_cast<size_t>(d.g) * (f1 ? 2 * p.I : p.H) +
-                                         (f1 ? fc1_row(wr, p.I, p.fc1_chunked) : wr))
-                     : 0.f;
+            const size_t wi = static_cast<size_t>(d.g) * (f1 ? 2 * p.I : p.H) +
+                              (f1 ? fc1_row(wr, p.I, p.fc1_chunked) : wr);
+            const float bias = bsrc ? bf16_at(bsrc, wi) : 0.f;
+            // Q8: the row's float32 scale (the accumulator holds sum_k q x)
+            const float scale = Q8 ? (f1 ? p.s1 : p.s2)[wi] : 1.f;
 #pragma unroll 1
             for (int c = 0; c < d.nrows; c += 16) {
                 uint32_t v[16];
@@ -943,7 +983,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int n = c + i;
-                    const float x = f32(v[i]) + bias;
+                    const float x = Q8 ? fmaf(f32(v[i]), scale, bias) : f32(v[i]) + bias;
                     if (f1) {
                         const float up = __shfl_xor_sync(0xffffffffu, x, 1);
                         if (!(lane & 1) && n < d.nrows)
@@ -983,6 +1023,130 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 }
             }
         }
+    } else if constexpr (Q8) {
+        // the unit sequence, as the other roles read it
+        int slot = 0;
+        uint32_t uphase = 0;
+        auto next_unit = [&]() -> int {
+            const bool got = mbar_wait(smem_u32(&ufull[slot]), uphase, abort_flag, kWaitLimitNs);
+            const int u = got ? s_unit[slot] : U;
+            __syncwarp();
+            if (got && lane == 0) mbar_arrive(smem_u32(&uempty[slot]));
+            if (++slot == kUnitRing) {
+                slot = 0;
+                uphase ^= 1u;
+            }
+            return u;
+        };
+        if (warp == 6) {
+            // -------------------------------------------------------- int8 producer
+            int qs = 0;
+            uint32_t qphase = 0;
+            long long qissued = 0;
+            for (;;) {
+                const int u = next_unit();
+                if (u >= U) break;
+                const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
+                const bool f1 = d.phase == 1;
+                const int nk = f1 ? nk1 : nk2;
+                const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;   // one load site, map chosen at run time
+                bool ok = true;
+                if (lane == 0) {
+                    for (int kb = 0; kb < nk; ++kb) {
+                        ok = mbar_wait(smem_u32(&qempty[qs]), qphase ^ 1u, abort_flag, kWaitLimitNs);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(smem_u32(&qfull[qs]), kQBytes);
+                        tma_load_4d(smem_u32(sQ + qs * kQBytes), ma, smem_u32(&qfull[qs]), kb * BK, 0,
+                                    d.mt * (BM / 2), d.g);
+                        ++qissued;
+                        if (++qs == C::kQStages) {
+                            qs = 0;
+                            qphase ^= 1u;
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            }
+            if (lane == 0 && *abort_flag) {
+                // let the int8 tiles in flight land before the CTA exits
+                int dummy = 0;
+                for (int s2 = 0; s2 < C::kQStages; ++s2) {
+                    if (qissued <= s2) break;
+                    const long long fills = (qissued - 1 - s2) / C::kQStages + 1;
+                    mbar_wait(smem_u32(&qfull[s2]), static_cast<uint32_t>((fills - 1) & 1), &dummy,
+                              kWaitLimitNs / 4);
+                }
+            }
+        } else {
+            // -------------------------------------------------------- int8 -> bf16
+            // Warp cw converts weight rows 32 cw .. 32 cw + 31 of each tile: per pass, 8
+            // rows x 64 bytes (512 contiguous bytes: one conflict-free warp load), each
+            // lane 16 int8 of one row -> 16 bf16 = two 16-byte chunks of the row's 128
+            // bytes, stored at the 128-byte swizzle position (chunk ^ (row & 7)).
+            // int8 b -> float32 exactly: the bit pattern 0x4B000000 | (b ^ 0x80) is
+            // 2^23 + 128 + b; subtracting 2^23 + 128 leaves b, whose float32 bits end in
+            // 16 zero bits (|b| <= 128 has at most 8 significant bits), so its top half
+            // is b in bf16.
+            const int cw = warp - 7;
+            int qs = 0, stage = 0;
+            uint32_t qphase = 0, phase = 0;
+            for (;;) {
+                const int u = next_unit();
+                if (u >= U) break;
+                const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
+                const int nk = d.phase == 1 ? nk1 : nk2;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (lane == 0)
+                        ok = mbar_wait(smem_u32(&qfull[qs]), qphase, abort_flag, kWaitLimitNs) &&
+                             mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
+                    // the whole warp leaves together (lane 0 alone saw the wait give up)
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    const uint8_t* q = sQ + qs * kQBytes;
+                    uint8_t* a = sA + stage * C::kABytes;
+#pragma unroll
+                    for (int pass = 0; pass < 4; ++pass) {
+                        const int row = cw * 32 + pass * 8 + (lane >> 2), c = lane & 3;
+                        const uint4 w = *reinterpret_cast<const uint4*>(q + row * BK + c * 16);
+                        const uint32_t wb[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u,
+                                                w.z ^ 0x80808080u, w.w ^ 0x80808080u};
+                        uint32_t h[8];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            float f[4];
+#pragma unroll
+                            for (int b = 0; b < 4; ++b)
+                                f[b] = __uint_as_float(__byte_perm(wb[i], 0x4B000000u, b | 0x7540u)) -
+                                       8388736.0f;   // 2^23 + 128
+                            h[2 * i] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
+                            h[2 * i + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+                        }
+                        uint8_t* rowp = a + (row >> 3) * 1024 + (row & 7) * 128;
+                        *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) =
+                            make_uint4(h[0], h[1], h[2], h[3]);
+                        *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) =
+                            make_uint4(h[4], h[5], h[6], h[7]);
+                    }
+                    // the bf16 tile is read by the tensor cores (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(smem_u32(&qempty[qs]));
+                        mbar_arrive(smem_u32(&full[stage]));
+                    }
+                    if (++qs == C::kQStages) {
+                        qs = 0;
+                        qphase ^= 1u;
+                    }
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+        }
     }
 
     tc_fence_before();
@@ -993,6 +1157,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     }
     if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
 }
+
 
 // ------------------------------------------------------------------------ host side
 
@@ -1026,13 +1191,13 @@ int decode_grid(int rows, int E, int H, int I) {
     return static_cast<int>(units < sms ? units : sms);
 }
 
-template <bool GATHER, bool ROUTE>
+template <bool GATHER, bool ROUTE, bool Q8 = false>
 cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap& w2,
                           const CUtensorMap& a, const DecodeParams& p, int grid, cudaStream_t s) {
-    using C = Tr<W_PLAIN, 64>;
+    using C = DecodeCfg<Q8>;
     constexpr int kSmem = C::kSmemBytes + (ROUTE ? kRouteSmemBytes : 0);
     static_assert(kSmem <= 227 * 1024, "shared memory");
-    auto kern = tc_ffn_decode_kernel<GATHER, ROUTE>;
+    auto kern = tc_ffn_decode_kernel<GATHER, ROUTE, Q8>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -1042,7 +1207,7 @@ cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUt
         attr_set[dev] = true;
     }
     if (grid <= 0) return cudaSuccess;
-    return launch_k(kern, dim3(grid), dim3(kThreads), kSmem, s, w1, x, w2, a, p);
+    return launch_k(kern, dim3(grid), dim3(C::kThreads), kSmem, s, w1, x, w2, a, p);
 }
 
 }  // namespace
@@ -1100,13 +1265,14 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                               cudaStream_t s, const FfnAttrs& ep) {
     if (rows <= 0) return cudaSuccess;
     CUtensorMap w1, x, w2, a;
-    if (!tmap::fc1_pairs(&w1, fc1, E, I, H, BM / 2, ep.fc1_chunked)) return cudaErrorInvalidValue;
+    const bool q8 = ep.q8();
+    if (!tmap::fc1_pairs(&w1, fc1, E, I, H, BM / 2, ep.fc1_chunked, q8)) return cudaErrorInvalidValue;
     if (perm_src) {
         if (!tmap::matrix(&x, tokens, T, H, 1)) return cudaErrorInvalidValue;
     } else {
         if (!tmap::matrix(&x, tokens, rows, H, kBoxTok)) return cudaErrorInvalidValue;
     }
-    if (!tmap::plain_pairs(&w2, fc2, E, H, I, BM / 2)) return cudaErrorInvalidValue;
+    if (!tmap::plain_pairs(&w2, fc2, E, H, I, BM / 2, q8)) return cudaErrorInvalidValue;
     if (!tmap::matrix(&a, act, rows, I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, E);
     DecodeParams p{};
@@ -1131,7 +1297,12 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
     p.b1 = static_cast<const __nv_bfloat16*>(ep.fc1_bias);
     p.fc1_chunked = ep.fc1_chunked;
     p.b2 = static_cast<const __nv_bfloat16*>(ep.fc2_bias);
+    p.s1 = ep.fc1_scale;
+    p.s2 = ep.fc2_scale;
     const int grid = decode_grid(rows, E, H, I);
+    if (q8)
+        return perm_src ? launch_decode<true, false, true>(w1, x, w2, a, p, grid, s)
+                        : launch_decode<false, false, true>(w1, x, w2, a, p, grid, s);
     return perm_src ? launch_decode<true, false>(w1, x, w2, a, p, grid, s)
                     : launch_decode<false, false>(w1, x, w2, a, p, grid, s);
 }
@@ -1139,7 +1310,7 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) {
     const int rows = r.T * r.k;
     if (rows <= 0) return cudaSuccess;
-    if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I)) return cudaErrorInvalidValue;
+    if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I) || r.ep.q8()) return cudaErrorInvalidValue;
     CUtensorMap w1, x, w2, a;
     if (!tmap::fc1_pairs(&w1, r.fc1, r.E, r.I, r.H, BM / 2, r.ep.fc1_chunked))
         return cudaErrorInvalidValue;

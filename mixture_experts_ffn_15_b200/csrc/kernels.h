@@ -115,11 +115,17 @@ cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int 
 // Every kernel reads the chunked layout in place, as if it were interleaved: the
 // bf16 kernels through a 4-D TMA view (H, gate/up, i, e) whose gate/up stride is one
 // row for interleaved weights and I rows for chunked ones.
+// Weight-only int8 experts (fc1_scale != nullptr): fc1 and fc2 hold int8 q and the
+// weights are q * scale of their row (fc1_scale [E, 2I] in fc1's layout, fc2_scale
+// [E, H], float32); the decode FFN kernel only.
 struct FfnAttrs {
     SwigluAttr act{1.0f, 0.0f, INFINITY, 1};
     bool fc1_chunked = false;
     const void* fc1_bias = nullptr;
     const void* fc2_bias = nullptr;
+    const float* fc1_scale = nullptr;
+    const float* fc2_scale = nullptr;
+    bool q8() const { return fc1_scale != nullptr; }
 };
 
 // Row of fc1 (or entry of fc1_bias) inside one expert that holds interleaved row j

@@ -52,11 +52,13 @@ inline bool matrix(CUtensorMap* m, const void* ptr, long long rows, int K, int b
 //   plain [E, n, K] (fc2; fc1 interleaved: row 2i = gate_i, 2i+1 = up_i):
 //       s_stride 1, i_stride 2
 //   fc1 chunked [E, 2I, K] (row i = gate_i, I+i = up_i): s_stride I, i_stride 1
+//   int8 weights (u8 = true): one byte per element, no swizzle (the box is read by
+//       the converting warps, 64 bytes per row)
 inline bool row_pairs(CUtensorMap* m, const void* w, int E, int n_pairs, int K, int box_pairs,
-                      long long s_stride, long long i_stride) {
+                      long long s_stride, long long i_stride, bool u8 = false) {
     EncodeTiledFn enc = encode_fn();
     if (!enc || E <= 0 || n_pairs <= 0) return false;
-    const cuuint64_t row = static_cast<cuuint64_t>(K) * 2;
+    const cuuint64_t row = static_cast<cuuint64_t>(K) * (u8 ? 1 : 2);
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), 2, static_cast<cuuint64_t>(n_pairs),
                           static_cast<cuuint64_t>(E)};
     cuuint64_t strides[3] = {row * static_cast<cuuint64_t>(s_stride),
@@ -64,22 +66,24 @@ inline bool row_pairs(CUtensorMap* m, const void* w, int E, int n_pairs, int K, 
                              row * 2 * static_cast<cuuint64_t>(n_pairs)};
     cuuint32_t box[4] = {static_cast<cuuint32_t>(kBoxK), 2, static_cast<cuuint32_t>(box_pairs), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+               const_cast<void*>(w), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               u8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // fc1 [E, 2I, H] of either layout, read in interleaved row order (gate_i, up_i pairs).
 inline bool fc1_pairs(CUtensorMap* m, const void* fc1, int E, int I, int H, int box_pairs,
-                      bool chunked) {
-    return chunked ? row_pairs(m, fc1, E, I, H, box_pairs, I, 1)
-                   : row_pairs(m, fc1, E, I, H, box_pairs, 1, 2);
+                      bool chunked, bool u8 = false) {
+    return chunked ? row_pairs(m, fc1, E, I, H, box_pairs, I, 1, u8)
+                   : row_pairs(m, fc1, E, I, H, box_pairs, 1, 2, u8);
 }
 
 // A plain [E, n, K] weight tensor (n even) in the same 4-D form, so that one load
 // instruction serves both GEMMs of a kernel.
-inline bool plain_pairs(CUtensorMap* m, const void* w, int E, int n, int K, int box_pairs) {
-    return n % 2 == 0 && row_pairs(m, w, E, n / 2, K, box_pairs, 1, 2);
+inline bool plain_pairs(CUtensorMap* m, const void* w, int E, int n, int K, int box_pairs,
+                        bool u8 = false) {
+    return n % 2 == 0 && row_pairs(m, w, E, n / 2, K, box_pairs, 1, 2, u8);
 }
 
 }  // namespace tmap

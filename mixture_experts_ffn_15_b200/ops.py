@@ -120,6 +120,70 @@ def forward(hidden, router_w, fc1, fc2, k, normalize=True, router_bias=None, out
     return out
 
 
+def _q8(q, scale, name, rows_shape):
+    _need(q, name, torch.int8, rows_shape)
+    _need(scale, name + "_scale", torch.float32, rows_shape[:2])
+
+
+def forward_q8(hidden, router_w, fc1_q, fc1_scale, fc2_q, fc2_scale, k, normalize=True,
+               router_bias=None, out=None, workspace=None, stream=None,
+               swiglu=(1.0, 0.0, float("inf")), fc1_bias=None, fc2_bias=None,
+               fc1_layout="interleaved", norm_weight=None, norm_eps=1e-6):
+    """The layer with weight-only int8 experts: weight = q * scale of its row (fc1_q
+    [E, 2I, H] int8 with fc1_scale [E, 2I] float32, fc2_q [E, H, I] with fc2_scale
+    [E, H]); hidden and the rest bf16, as in forward.  Decode-sized batches only."""
+    _need(hidden, "hidden", torch.bfloat16)
+    T, H = hidden.shape
+    E = router_w.shape[0]
+    I = fc2_q.shape[2]
+    _need(router_w, "router_w", torch.bfloat16, (E, H))
+    _q8(fc1_q, fc1_scale, "fc1", (E, 2 * I, H))
+    _q8(fc2_q, fc2_scale, "fc2", (E, H, I))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    _biases(fc1_bias, fc2_bias, torch.bfloat16, E, I, H)
+    if norm_weight is not None:
+        _need(norm_weight, "norm_weight", torch.bfloat16, (H,))
+    if out is None:
+        out = torch.empty_like(hidden)
+    _need(out, "out", torch.bfloat16, (T, H))
+    need = workspace_size(T, H, E, k, I, torch.bfloat16)
+    if workspace is None:
+        workspace = alloc_workspace(max(need, 256), hidden.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = _lib().moe_forward_q8(_ptr(hidden), _ptr(norm_weight), float(norm_eps), _ptr(router_w),
+                               _ptr(router_bias), _ptr(fc1_q), _ptr(fc1_scale), _ptr(fc2_q),
+                               _ptr(fc2_scale), _ptr(fc1_bias), _ptr(fc2_bias), T, H, E, k, I,
+                               int(bool(normalize)), _swiglu(*swiglu), _layout(fc1_layout),
+                               _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    check(st, "moe_forward_q8")
+    return out
+
+
+def expert_ffn_q8(x_perm, offsets, fc1_q, fc1_scale, fc2_q, fc2_scale, y_perm=None, stream=None,
+                  swiglu=(1.0, 0.0, float("inf")), fc1_bias=None, fc2_bias=None,
+                  fc1_layout="interleaved"):
+    """expert_ffn with weight-only int8 experts (see forward_q8)."""
+    _need(x_perm, "x_perm", torch.bfloat16)
+    rows, H = x_perm.shape
+    E, two_i, _ = fc1_q.shape
+    I = two_i // 2
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _q8(fc1_q, fc1_scale, "fc1", (E, 2 * I, H))
+    _q8(fc2_q, fc2_scale, "fc2", (E, H, I))
+    _biases(fc1_bias, fc2_bias, torch.bfloat16, E, I, H)
+    if y_perm is None:
+        y_perm = torch.zeros_like(x_perm)
+    ws = alloc_workspace(_lib().moe_expert_ffn_workspace_size(rows, I, _DT[torch.bfloat16]),
+                         x_perm.device)
+    st = _lib().moe_expert_ffn_q8(_ptr(x_perm), _ptr(offsets), _ptr(fc1_q), _ptr(fc1_scale),
+                                  _ptr(fc2_q), _ptr(fc2_scale), _ptr(fc1_bias), _ptr(fc2_bias), rows,
+                                  H, E, I, _swiglu(*swiglu), _layout(fc1_layout), _ptr(y_perm),
+                                  _ptr(ws), ws.numel(), _stream(stream))
+    check(st, "moe_expert_ffn_q8")
+    return y_perm
+
+
 def rmsnorm(x, weight, eps=1e-6, out=None, stream=None):
     """Pre-FFN RMSNorm: (x / sqrt(mean(x^2) + eps)) * weight per row, float64 inside,
     rounded once to x's dtype."""

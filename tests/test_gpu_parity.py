@@ -454,6 +454,125 @@ def test_full_workload_with_pre_norm(name):
     assert torch.equal(_bits(fused), _bits(staged))
 
 
+# ------------------------------------------------------------------ int8 experts
+# Weight-only int8 experts (one float32 scale per weight row) in the decode FFN.
+Q8_CASES = [
+    W("q8_decode", T=4, H=256, E=64, k=4, I=128),
+    W("q8_router_tc", T=100, H=256, E=64, k=4, I=192, router_bias_std=0.5),
+    W("q8_small_route", T=40, H=128, E=16, k=4, I=128),
+    W("q8_chunked_norm0", T=20, H=256, E=32, k=6, I=128, normalize=0, fc1_layout="chunked"),
+]
+
+
+def _q8_dev(wl, seed=None):
+    from synth import make_q8_experts
+    q1, s1, q2, s2 = make_q8_experts(wl, seed)
+    dev = [torch.from_numpy(a).cuda() for a in (q1, s1, q2, s2)]
+    return (q1, s1, q2, s2), dev
+
+
+def _q8_oracle(inp, wl, host, idx, act=(1.0, 0.0, float("inf")), b1=None, b2=None):
+    q1, s1, q2, s2 = host
+    return O.moe_forward(inp.values("hidden"), inp.values("router_w"), inp["router_bias"],
+                         lambda e: O.dequantize_rows(q1[e], s1[e]),
+                         lambda e: O.dequantize_rows(q2[e], s2[e]), wl.k, wl.normalize,
+                         wl.fc1_layout, idx=idx, act=act, fc1_bias=b1, fc2_bias=b2)["out"]
+
+
+@pytest.mark.parametrize("wl", Q8_CASES, ids=[c.name for c in Q8_CASES])
+def test_forward_q8(wl):
+    inp = make_inputs(wl, weights=False)
+    dev = device_inputs(inp)
+    host, (q1, s1, q2, s2) = _q8_dev(wl)
+    out = moe.forward_q8(dev["hidden"], dev["router_w"], q1, s1, q2, s2, wl.k,
+                         normalize=bool(wl.normalize), router_bias=dev["router_bias"],
+                         fc1_layout=wl.fc1_layout)
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    ref = _q8_oracle(inp, wl, host, idx)
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, f"{wl.name} int8 experts")
+
+
+def test_forward_q8_attributes_and_biases():
+    from synth import make_expert_biases
+    wl = W("q8_attr", T=8, H=256, E=32, k=4, I=128)
+    inp = make_inputs(wl, weights=False)
+    dev = device_inputs(inp)
+    host, (q1, s1, q2, s2) = _q8_dev(wl)
+    b1, b2 = make_expert_biases(wl, seed=9)
+    act = (1.702, 1.0, 7.0)
+    out = moe.forward_q8(dev["hidden"], dev["router_w"], q1, s1, q2, s2, wl.k, swiglu=act,
+                         fc1_bias=to_dev(b1, "bf16"), fc2_bias=to_dev(b2, "bf16"))
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    ref = _q8_oracle(inp, wl, host, idx, act, bf16_bits_to_f32(b1), bf16_bits_to_f32(b2))
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, "int8 experts, GPT-OSS + biases")
+
+
+@pytest.mark.parametrize("layout", ["interleaved", "chunked"])
+def test_expert_ffn_q8_unit_scales_equal_bf16_kernel(layout):
+    """With every scale 1 the int8 experts are the bf16 experts bf16(q) (exact): the
+    int8 decode FFN must give the bf16 decode FFN's bits, biases included; with real
+    scales, the oracle on q * scale."""
+    from synth import make_expert_biases
+    rows_per_expert = 6
+    wl = W("q8_ffn", T=rows_per_expert * 8, H=256, E=8, k=1, I=192, fc1_layout=layout)
+    inp = make_inputs(wl, weights=False)
+    host, (q1, s1, q2, s2) = _q8_dev(wl, seed=4)
+    b1, b2 = make_expert_biases(wl, seed=7)
+    db1, db2 = to_dev(b1, "bf16"), to_dev(b2, "bf16")
+    x = to_dev(inp["hidden"], "bf16")
+    offsets = torch.from_numpy((np.arange(wl.E + 1) * rows_per_expert).astype(np.int32)).cuda()
+    one1, one2 = torch.ones_like(s1), torch.ones_like(s2)
+    y_q = moe.expert_ffn_q8(x, offsets, q1, one1, q2, one2, fc1_bias=db1, fc2_bias=db2,
+                            fc1_layout=layout)
+    y_b = moe.expert_ffn(x, offsets, q1.to(torch.bfloat16), q2.to(torch.bfloat16), fc1_bias=db1,
+                         fc2_bias=db2, fc1_layout=layout)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(y_q), _bits(y_b))
+    y = moe.expert_ffn_q8(x, offsets, q1, s1, q2, s2, fc1_bias=db1, fc2_bias=db2, fc1_layout=layout)
+    torch.cuda.synchronize()
+    xv = inp.values("hidden")
+    ref = np.zeros((wl.T, wl.H))
+    for e in range(wl.E):
+        a, b = rows_per_expert * e, rows_per_expert * (e + 1)
+        ref[a:b] = O.expert_ffn(xv[a:b], O.dequantize_rows(host[0][e], host[1][e]),
+                                O.dequantize_rows(host[2][e], host[3][e]), layout,
+                                O.STANDARD_SWIGLU, bf16_bits_to_f32(b1[e]), bf16_bits_to_f32(b2[e]))
+    atol, rtol = tol("bf16", ref)
+    assert_close(from_dev(y), ref, atol * row_scale(ref), rtol, f"int8 expert FFN {layout}")
+
+
+def test_full_decode_q8():
+    """decode_bf16 (T=4, H=2816, E=128, k=8, I=704) with int8 experts: every output row
+    against the oracle on the dequantized weights."""
+    from synth import WORKLOADS
+    wl = WORKLOADS["decode_bf16"]
+    inp = make_inputs(wl, weights=False)
+    dev = device_inputs(inp)
+    host, (q1, s1, q2, s2) = _q8_dev(wl)
+    out = moe.forward_q8(dev["hidden"], dev["router_w"], q1, s1, q2, s2, wl.k)
+    r = run_route(dev, wl)
+    torch.cuda.synchronize()
+    L, idx = check_routing(inp, r)
+    ref = _q8_oracle(inp, wl, host, idx)
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, "decode_bf16 int8 experts")
+
+
+def test_q8_refuses_sizes_outside_the_decode_ffn():
+    wl = W("q8_big", T=2048, H=128, E=8, k=2, I=64)      # 512 rows per expert
+    inp = make_inputs(wl, weights=False)
+    dev = device_inputs(inp)
+    _, (q1, s1, q2, s2) = _q8_dev(wl)
+    with pytest.raises(moe.MoEError, match="UNSUPPORTED"):
+        moe.forward_q8(dev["hidden"], dev["router_w"], q1, s1, q2, s2, wl.k)
+
+
 def test_combine_matches_oracle():
     wl = W("comb", T=77, H=136, E=6, k=3, dtype="f32")
     inp = make_inputs(wl)
