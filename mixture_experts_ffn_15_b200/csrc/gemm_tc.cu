@@ -419,8 +419,9 @@ constexpr int kUnitRing = 4;
 
 // Weight-only int8 experts (Q8): the weights stream from HBM as int8 through a deep ring
 // of their own (kQStages tiles of 128 rows x 64 bytes, loaded by a dedicated producer
-// warp), four converter warps write each tile as bf16 -- exact, |q| <= 127 -- into the
-// 128-byte-swizzled layout of the bf16 path, and the epilogue multiplies each weight
+// warp), converter warps write each tile as bf16 -- exact, |q| <= 127 -- into the
+// 128-byte-swizzled layout of the bf16 path (two groups of four warps taking alternate
+// k-steps, so that two tiles convert at once), and the epilogue multiplies each weight
 // row's accumulator by its float32 scale.  The MMA and the token side are unchanged.
 constexpr int kQBytes = BM * BK;   // one int8 tile: 128 weight rows x 64 K
 
@@ -431,7 +432,7 @@ struct DecodeCfg {
     static constexpr int kBBytes = T::kBBytes;
     static constexpr int kStages = Q8 ? 5 : T::kStages;     // bf16 A + token B ring
     static constexpr int kQStages = Q8 ? 12 : 0;            // int8 weight ring
-    static constexpr int kThreads = Q8 ? 352 : 192;         // + Q producer + 4 converters
+    static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
     static constexpr int kAccStride = T::kAccStride;
     static constexpr int kTmemCols = T::kTmemCols;
     static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
@@ -593,8 +594,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         }
         for (int q = 0; q < kUnitRing; ++q) {
             mbar_init(smem_u32(&ufull[q]), 1);
-            // the MMA thread and 4 epilogue warps (Q8: + the int8 producer and 4 converters)
-            mbar_init(smem_u32(&uempty[q]), Q8 ? 10 : 5);
+            // the MMA thread and 4 epilogue warps (Q8: + the int8 producer and 8 converters)
+            mbar_init(smem_u32(&uempty[q]), Q8 ? 14 : 5);
         }
         for (int q = 0; q < C::kQStages; ++q) {
             mbar_init(smem_u32(&qfull[q]), 1);
@@ -1079,7 +1080,9 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             }
         } else {
             // -------------------------------------------------------- int8 -> bf16
-            // Warp cw converts weight rows 32 cw .. 32 cw + 31 of each tile: per pass, 8
+            // Group grp (warps 7-10, 11-14) converts the k-steps n with n % 2 == grp (n
+            // counts every k-step of the launch, as the rings do); its warp cw converts
+            // weight rows 32 cw .. 32 cw + 31 of the tile: per pass, 8
             // rows x 64 bytes (512 contiguous bytes: one conflict-free warp load), each
             // lane 16 int8 of one row -> 16 bf16 = two 16-byte chunks of the row's 128
             // bytes, stored at the 128-byte swizzle position (chunk ^ (row & 7)).
@@ -1087,8 +1090,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             // 2^23 + 128 + b; subtracting 2^23 + 128 leaves b, whose float32 bits end in
             // 16 zero bits (|b| <= 128 has at most 8 significant bits), so its top half
             // is b in bf16.
-            const int cw = warp - 7;
-            int qs = 0, stage = 0;
+            const int cw = (warp - 7) & 3, grp = (warp - 7) >> 2;
+            int qs = 0, stage = 0, n = 0;
             uint32_t qphase = 0, phase = 0;
             for (;;) {
                 const int u = next_unit();
@@ -1096,7 +1099,18 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
                 const int nk = d.phase == 1 ? nk1 : nk2;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb = 0; kb < nk; ++kb, ++n) {
+                    if ((n & 1) != grp) {   // the other group's k-step: only the rings advance
+                        if (++qs == C::kQStages) {
+                            qs = 0;
+                            qphase ^= 1u;
+                        }
+                        if (++stage == C::kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (lane == 0)
                         ok = mbar_wait(smem_u32(&qfull[qs]), qphase, abort_flag, kWaitLimitNs) &&
                              mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
