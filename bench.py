@@ -57,6 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--pre-norm", action="store_true",
                     help="the layer's input is a residual activation normalised by the pre-FFN "
                          "RMSNorm inside the call")
+    ap.add_argument("--q8", action="store_true",
+                    help="weight-only int8 experts (one float32 scale per weight row); "
+                         "decode workloads only")
     ap.add_argument("--fc1-convert", action="store_true",
                     help="convert chunked fc1 to the interleaved layout at set-up instead of "
                          "reading it in place")
@@ -160,7 +163,7 @@ class ClockSampler:
 NORM_EPS = 1e-6
 
 
-def algorithmic(wl, counts, pre_norm=False):
+def algorithmic(wl, counts, pre_norm=False, q8=False):
     """Algorithmic bytes and FLOPs of one step (only the routed work, used experts once;
     with the pre-FFN norm, its read of the residual and the weight and its write)."""
     T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
@@ -176,6 +179,13 @@ def algorithmic(wl, counts, pre_norm=False):
              "flops": float(T) * (6.0 * k * H * I + 2.0 * H * E)}
     if pre_norm:
         layer["bytes"] += 2 * T * H * es + H * es
+    if q8:
+        # int8 weights (1 byte each) and a float32 scale per weight row
+        for d, n_rows, n_cols in ((fc1, 2 * I, H), (fc2, H, I)):
+            d["bytes"] -= used * n_rows * n_cols * (es - 1)
+            d["bytes"] += used * n_rows * 4
+        layer["bytes"] -= used * 3 * H * I * (es - 1)
+        layer["bytes"] += used * (2 * I + H) * 4
     return used, fc1, fc2, layer
 
 
@@ -217,7 +227,14 @@ def device_tensor(a, dev):
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_cost(wl, inp, seconds, pre=None):
+def q8_getters(q8_host):
+    """Oracle weight getters of int8 experts: q * scale of each row, float64."""
+    from oracle import moe_oracle as O
+    q1, s1, q2, s2 = q8_host
+    return (lambda e: O.dequantize_rows(q1[e], s1[e]), lambda e: O.dequantize_rows(q2[e], s2[e]))
+
+
+def oracle_cost(wl, inp, seconds, pre=None, q8_host=None):
     """The CPU oracle, as it stands, on whole tokens of `wl` for about `seconds` (with
     pre = (residual values, norm weight values), each token through the pre-FFN norm
     first).
@@ -233,6 +250,8 @@ def oracle_cost(wl, inp, seconds, pre=None):
     bias = inp["router_bias"]
     fc1 = lambda e: inp.expert_values("fc1", e)
     fc2 = lambda e: inp.expert_values("fc2", e)
+    if q8_host is not None:
+        fc1, fc2 = q8_getters(q8_host)
     t0 = time.perf_counter()
     n = 0
     while True:
@@ -249,7 +268,8 @@ def oracle_cost(wl, inp, seconds, pre=None):
                            f"top-k, {wl.k} expert FFNs, combine in float64), {el:.1f} s")
 
 
-def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None), pre=None):
+def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None), pre=None,
+                     getters=None):
     """One bounded reference step: routing of one token and one of its expert FFNs (with
     pre, the token's pre-FFN norm first)."""
     import numpy as np
@@ -264,8 +284,9 @@ def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None,
     j = state["j"]
     e = int(idx[0, j])
     b1, b2 = biases
-    y = O.expert_ffn(xt, inp.expert_values("fc1", e),
-                     inp.expert_values("fc2", e), wl.fc1_layout, act,
+    g1, g2 = getters if getters is not None else (lambda i: inp.expert_values("fc1", i),
+                                                   lambda i: inp.expert_values("fc2", i))
+    y = O.expert_ffn(xt, g1(e), g2(e), wl.fc1_layout, act,
                      None if b1 is None else b1[e], None if b2 is None else b2[e])
     assert np.isfinite(w[0, j] * y).all()
     state["j"] += 1
@@ -283,10 +304,14 @@ def run_reference(args):
     steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(wl.name, 100)
     from threadpoolctl import threadpool_info
     cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    inp = make_inputs(wl)
+    inp = make_inputs(wl, weights=not args.q8)
     act = SWIGLU_PRESETS[args.swiglu]
     biases = (None, None)
     pre = None
+    getters = None
+    if args.q8:
+        from synth import make_q8_experts
+        getters = q8_getters(make_q8_experts(wl))
     if args.pre_norm:
         from synth import make_pre_norm_inputs
         px, pw = make_pre_norm_inputs(wl)
@@ -299,10 +324,10 @@ def run_reference(args):
         biases = (wide(nb1), wide(nb2))
     state = {"t": 0, "j": 0}
     for _ in range(args.warmup):
-        oracle_pair_step(wl, inp, state, act, biases, pre)
+        oracle_pair_step(wl, inp, state, act, biases, pre, getters)
     t0 = time.perf_counter()
     for _ in range(steps):
-        oracle_pair_step(wl, inp, state, act, biases, pre)
+        oracle_pair_step(wl, inp, state, act, biases, pre, getters)
     el = time.perf_counter() - t0
     value = (steps / wl.k) / el
     sample = (f"each step: router logits + top-k of one token and one of its {wl.k} expert "
@@ -316,6 +341,7 @@ def run_reference(args):
                        parallelism=f"replicas x{args.gpus}",
                        graph_steps=GRAPH_STEPS.get(wl.name, 4), swiglu=list(act),
                        expert_bias=bool(args.expert_bias), pre_norm=bool(args.pre_norm),
+                       q8=bool(args.q8),
                        fc1_layout_read="interleaved" if args.fc1_convert else wl.fc1_layout),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -365,7 +391,9 @@ def run_ours(args):
     warm_reps = max(1, math.ceil(args.warmup / S))
     sets = args.sets if args.sets is not None else (4 if wl.name in HBM_BOUND else 1)
 
-    inp = make_inputs(wl)
+    if args.q8 and wl.name not in HBM_BOUND:
+        raise SystemExit("--q8: the int8 experts run in the decode FFN only (decode workloads)")
+    inp = make_inputs(wl, weights=not args.q8)
     hidden = device_tensor(inp["hidden"], dev)
     norm_kw, pre = {}, None
     if args.pre_norm:
@@ -378,14 +406,27 @@ def run_ours(args):
         pre = (wide(px), wide(pw))
     router_w = device_tensor(inp["router_w"], dev)
     bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).to(dev)
-    fc1 = device_tensor(inp["fc1"], dev)
     layout = wl.fc1_layout
-    if layout == "chunked" and args.fc1_convert:
-        fc1 = moe.convert_chunked_to_interleaved(fc1)      # set-up, as at session load
-        layout = "interleaved"
-    fc2 = device_tensor(inp["fc2"], dev)
-    fc1s = [fc1] + [fc1.clone() for _ in range(sets - 1)]
-    fc2s = [fc2] + [fc2.clone() for _ in range(sets - 1)]
+    q8_host = None
+    if args.q8:
+        from synth import make_q8_experts
+        q8_host = make_q8_experts(wl)
+        q8 = [torch.from_numpy(a).to(dev) for a in q8_host]
+        weight_sets = [q8] + [[t.clone() for t in q8] for _ in range(sets - 1)]
+    else:
+        fc1 = device_tensor(inp["fc1"], dev)
+        if layout == "chunked" and args.fc1_convert:
+            fc1 = moe.convert_chunked_to_interleaved(fc1)      # set-up, as at session load
+            layout = "interleaved"
+        fc2 = device_tensor(inp["fc2"], dev)
+        weight_sets = [[fc1, fc2]] + [[fc1.clone(), fc2.clone()] for _ in range(sets - 1)]
+
+    def run_layer(x, i, **kw):
+        """One call of the layer on input x with the i-th rotating copy of the weights."""
+        w = weight_sets[i % sets]
+        if args.q8:
+            return moe.forward_q8(x, router_w, w[0], w[1], w[2], w[3], wl.k, **kw)
+        return moe.forward(x, router_w, w[0], w[1], wl.k, **kw)
     act = SWIGLU_PRESETS[args.swiglu]
     b1 = b2 = None
     if args.expert_bias:
@@ -401,10 +442,10 @@ def run_ours(args):
     r = moe.route(x_in, router_w, wl.k, normalize=bool(wl.normalize), router_bias=bias)
     p = moe.permute(r["idx"], wl.E)
     counts = p["counts"].cpu().numpy()
-    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts, args.pre_norm)
+    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts, args.pre_norm, args.q8)
 
     stream = torch.cuda.Stream(device=dev)
-    call = lambda i: moe.forward(hidden, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+    call = lambda i: run_layer(hidden, i,
                                  normalize=bool(wl.normalize), router_bias=bias, out=out,
                                  workspace=ws, **ffn_kw)
     with torch.cuda.stream(stream):
@@ -475,6 +516,8 @@ def run_ours(args):
         for a, n in enumerate(stage_names):
             st[n] += events[i][a].elapsed_time(events[i][a + 1]) / S
     path = lib.moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, 1 if wl.dtype == "bf16" else 0)
+    if args.q8:
+        path &= ~32   # int8 experts: the decode FFN after the staged routing kernels
     fused = bool(path & 2)
     # the dominant kernel: the fused decode FFN (fc1 + SwiGLU and fc2 in one launch),
     # else the fc1 + SwiGLU grouped GEMM
@@ -507,6 +550,10 @@ def run_ours(args):
     roof["algorithmic_per_launch"] = dom["bytes"] if hbm else dom["flops"]
     roof["kernel_us"] = round(dom_ms * 1e3, 2)
     roof["traffic"] = kernel_traffic(wl.name, kernel_source(fused))
+    if args.q8:
+        roof["kernel"] = ("tc_ffn_decode_kernel<Q8> (int8 weights converted to bf16 in shared "
+                          "memory, fc1 + SwiGLU, fc2 and combine, weight rows on M)")
+        roof["traffic"] = None   # the committed counters are the bf16 kernel's
 
     layer_s = ms_step * 1e-3
     layer = {"GB/s": layer_work["bytes"] / layer_s / 1e9, "TFLOP/s": layer_work["flops"] / layer_s / 1e12,
@@ -524,7 +571,7 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         for i in range(3):
             d_in.copy_(h_host, non_blocking=True)
-            moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+            run_layer(d_in, i,
                         normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
                         **ffn_kw)
             o_host.copy_(out, non_blocking=True)
@@ -534,7 +581,7 @@ def run_ours(args):
         t0 = time.perf_counter()
         for i in range(n_e2e):
             d_in.copy_(h_host, non_blocking=True)
-            moe.forward(d_in, router_w, fc1s[i % sets], fc2s[i % sets], wl.k,
+            run_layer(d_in, i,
                         normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
                         **ffn_kw)
             o_host.copy_(out, non_blocking=True)
@@ -555,7 +602,7 @@ def run_ours(args):
         "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
         "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
                        graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias),
-                       pre_norm=bool(args.pre_norm), fc1_layout_read=layout),
+                       pre_norm=bool(args.pre_norm), q8=bool(args.q8), fc1_layout_read=layout),
         "roofline": roof, "layer": layer,
         "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
         "stages_note": "second timed region, same steps with stage events between kernels",
@@ -563,7 +610,7 @@ def run_ours(args):
         "gpu_launches": int(round(launches_per_step * steps)),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds, pre)
+        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds, pre, q8_host)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}
     if rank == 0:

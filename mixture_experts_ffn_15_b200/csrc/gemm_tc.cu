@@ -430,8 +430,8 @@ struct DecodeCfg {
     using T = Tr<W_PLAIN, 64>;
     static constexpr int kABytes = T::kABytes;
     static constexpr int kBBytes = T::kBBytes;
-    static constexpr int kStages = Q8 ? 5 : T::kStages;     // bf16 A + token B ring
-    static constexpr int kQStages = Q8 ? 12 : 0;            // int8 weight ring
+    static constexpr int kStages = Q8 ? 7 : T::kStages;     // bf16 A + token B ring
+    static constexpr int kQStages = Q8 ? 6 : 0;             // int8 weight ring
     static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
     static constexpr int kAccStride = T::kAccStride;
     static constexpr int kTmemCols = T::kTmemCols;
