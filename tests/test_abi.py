@@ -120,6 +120,37 @@ def test_host_validation_before_any_device_work():
     assert lib.moe_set_stage_events(None, 0) == _abi.MOE_OK
 
 
+def _fwd_q8(lib, T=4, H=128, E=8, k=2, I=64, s1=32, s2=32, ptr=16):
+    p = ctypes.c_void_p(ptr)
+    sc = lambda v: None if v is None else ctypes.c_void_p(v)
+    return lib.moe_forward_q8(p, None, 1e-6, p, None, p, sc(s1), p, sc(s2), None, None, T, H, E, k,
+                              I, 1, _abi.STANDARD_SWIGLU, _abi.MOE_FC1_INTERLEAVED, p,
+                              ctypes.c_void_p(256), 1 << 40, None)
+
+
+def test_q8_host_validation_before_any_device_work():
+    """The int8-expert entry points refuse bad arguments and sizes outside the decode FFN
+    before anything is enqueued (every call here returns before a launch)."""
+    lib = _lib()
+    assert _fwd_q8(lib, s1=None) == _abi.MOE_ERR_INVALID_ARG           # no scales
+    assert _fwd_q8(lib, s2=None) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd_q8(lib, s1=34) == _abi.MOE_ERR_INVALID_ARG             # misaligned scales
+    assert _fwd_q8(lib, k=9) == _abi.MOE_ERR_INVALID_ARG
+    assert _fwd_q8(lib, H=72) == _abi.MOE_ERR_UNSUPPORTED              # no tensor-core tiling
+    assert _fwd_q8(lib, T=0) == _abi.MOE_OK
+    assert _fwd_q8(lib, T=4096, E=8, k=2) == _abi.MOE_ERR_UNSUPPORTED  # 1024 rows per expert
+    p = ctypes.c_void_p(16)
+    q8 = lambda rows, s1=32, H=128, I=64: lib.moe_expert_ffn_q8(
+        p, p, p, None if s1 is None else ctypes.c_void_p(s1), p, ctypes.c_void_p(32), None, None,
+        rows, H, 8, I, _abi.STANDARD_SWIGLU, _abi.MOE_FC1_INTERLEAVED, p, ctypes.c_void_p(256),
+        1 << 40, None)
+    assert q8(-1) == _abi.MOE_ERR_INVALID_ARG
+    assert q8(16, s1=None) == _abi.MOE_ERR_INVALID_ARG
+    assert q8(8 * 65) == _abi.MOE_ERR_UNSUPPORTED                     # > 64 rows per expert
+    assert q8(16, I=96) == _abi.MOE_ERR_UNSUPPORTED                   # 2I not a multiple of 128
+    assert q8(0) == _abi.MOE_OK
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "_lib", None)
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "absent.so"))
