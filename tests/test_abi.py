@@ -43,6 +43,19 @@ def test_header_declares_the_entry_points():
         assert n in names
 
 
+def test_header_compiles_as_c_and_cxx(tmp_path):
+    """include/moe_b200.h is a plain C header (also valid C++)."""
+    import shutil
+    import subprocess
+    hdr = os.path.join(ROOT, "include", "moe_b200.h")
+    for cc, lang, std in (("gcc", "c", "-std=c99"), ("g++", "c++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not installed")
+        r = subprocess.run([cc, std, "-Wall", "-Werror", "-fsyntax-only", "-x", lang, hdr],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_package_exports_every_binding():
     import mixture_experts_ffn_15_b200 as moe
     from mixture_experts_ffn_15_b200 import ops
