@@ -19,7 +19,8 @@
  *   otherwise.  The library never allocates device memory and never frees any.
  * - Every tensor is dense and row-major.  Weights are [out, in] (y = x W^T).
  * - `dt` gives the storage type of activations AND weights (hidden, router_w, fc1,
- *   fc2, x_perm, act, y_perm, out): MOE_F32 or MOE_BF16.  Router logits, routing
+ *   fc2, x_perm, act, y_perm, out): MOE_F32 or MOE_BF16 (the *_q8 entry points take
+ *   int8 expert weights with float32 row scales and bf16 everything else).  Router logits, routing
  *   weights and the router bias are always float32; indices and counts int32.
  *   Accumulation is float32 in every kernel; the bf16 expert GEMMs run on the
  *   tcgen05 tensor cores, the float32 path on plain FMA (no TF32).
