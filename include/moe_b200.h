@@ -279,12 +279,24 @@ moe_status moe_set_stage_events(void* const* events, int n_events);
 /* Which kernels moe_forward runs for these sizes, as bits: 1 single-CTA routing
  * (T <= 512 and k <= 32), 2 fused decode FFN (fc1 + SwiGLU and fc2 in one launch,
  * weight rows on the MMA's M side), 4 tensor-core router, 8 token-row grouped GEMMs,
- * 16 float32 FMA FFN.  0 for invalid sizes.  Pure host arithmetic. */
+ * 16 float32 FMA FFN, 32 the routing inside the decode FFN's launch (the whole layer
+ * in one cooperative launch, small bf16 batches).  0 for invalid sizes.  Pure host
+ * arithmetic. */
 int moe_forward_path(int T, int H, int E, int k, int I, moe_dtype dt);
 
 /* Number of kernel launches the library has issued in this process (host-side count,
  * all devices).  A launch captured into a CUDA graph counts once, at capture. */
 unsigned long long moe_kernel_launches(void);
+
+/* Testing aid for the device-side failure detection, off by default: the next
+ * moe_forward (or moe_forward_static) call that takes the one-launch path (bit 32 of
+ * moe_forward_path) makes its routing grid barrier wait for one arrival more than its
+ * grid provides, with a 1 ms limit instead of 2 s.  Every block then gives up before it
+ * has issued any bulk copy or MMA, winds down, frees its tensor memory and sets
+ * MOE_DEVERR_TIMEOUT in the call's error word (moe_get_error: MOE_ERR_TIMEOUT); the
+ * call's outputs are not written.  One-shot: the setting is consumed by that call.
+ * Process-wide; no counterpart on the pages. */
+void moe_debug_arm_route_barrier_timeout(void);
 
 /* Library version as major * 10000 + minor * 100 + patch. */
 int moe_version(void);

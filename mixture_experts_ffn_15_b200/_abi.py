@@ -45,6 +45,7 @@ SIGNATURES = {
     "moe_set_stage_events": (_i, [ctypes.POINTER(_vp), _i]),
     "moe_forward_path": (_i, [_i, _i, _i, _i, _i, _i]),
     "moe_kernel_launches": (ctypes.c_ulonglong, []),
+    "moe_debug_arm_route_barrier_timeout": (None, []),
     "moe_version": (_i, []),
 }
 

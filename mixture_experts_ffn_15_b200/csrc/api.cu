@@ -186,7 +186,9 @@ using namespace moe;
 
 extern "C" {
 
-int moe_version(void) { return 210; }
+int moe_version(void) { return 220; }
+
+void moe_debug_arm_route_barrier_timeout(void) { arm_route_timeout_test(); }
 
 unsigned long long moe_kernel_launches(void) { return g_launches.load(); }
 

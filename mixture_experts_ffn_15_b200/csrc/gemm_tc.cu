@@ -27,6 +27,8 @@
 // MOE_DEVERR_TIMEOUT in the error word and still frees its TMEM.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "combine.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -471,6 +473,8 @@ struct DecodeParams {
     int normalize;
     float* logits;            // [T, E] scratch
     int32_t* route_bar;       // grid-barrier arrivals, zero on entry
+    int route_bar_extra;      // arrivals wanted beyond the grid (0; 1 only to test a timeout)
+    uint64_t route_wait_ns;   // limit of the grid-barrier wait
     // the routing as the staged calls would return it, written by CTA 0
     int32_t* r_topk_idx;      // [T, k]
     float* r_topk_w;          // [T, k]
@@ -498,14 +502,15 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-__device__ __forceinline__ bool wait_count(const int32_t* ctr, int target, volatile int* abort) {
+__device__ __forceinline__ bool wait_count(const int32_t* ctr, int target, volatile int* abort,
+                                           uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire(ctr) >= target) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
         __nanosleep(64);
         if (ld_acquire(ctr) >= target) return true;
         if (*abort) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             *abort = 1;
             return false;
         }
@@ -678,13 +683,15 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 __syncthreads();
             }
         }
-        // (2) grid-wide barrier: every CTA of the launch is resident (at most one per
-        //     SM), so the wait ends; it is bounded all the same (abort on expiry).
+        // (2) grid-wide barrier: the launch is cooperative (every CTA resident, at most
+        //     one per SM), so the wait ends; it is bounded all the same (abort on expiry,
+        //     before any bulk copy or MMA of this CTA is in flight).
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();
             atomicAdd(p.route_bar, 1);
-            wait_count(p.route_bar, static_cast<int>(gridDim.x), abort_flag);
+            wait_count(p.route_bar, static_cast<int>(gridDim.x) + p.route_bar_extra, abort_flag,
+                       p.route_wait_ns);
         }
         __syncthreads();
         // (3) every CTA selects, counts and places the whole batch itself (the same
@@ -1221,7 +1228,9 @@ cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUt
         attr_set[dev] = true;
     }
     if (grid <= 0) return cudaSuccess;
-    return launch_k(kern, dim3(grid), dim3(C::kThreads), kSmem, s, w1, x, w2, a, p);
+    // ROUTE: the routing's grid barrier needs every CTA resident at once, which a
+    // cooperative launch guarantees (or refuses: too large a grid is an error, not a wait)
+    return launch_k_coop(kern, dim3(grid), dim3(C::kThreads), kSmem, s, ROUTE, w1, x, w2, a, p);
 }
 
 }  // namespace
@@ -1321,6 +1330,13 @@ cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T
                     : launch_decode<false, false>(w1, x, w2, a, p, grid, s);
 }
 
+namespace {
+std::atomic<int> g_route_timeout_test{0};
+}  // namespace
+
+void arm_route_timeout_test() { g_route_timeout_test.store(1); }
+bool take_route_timeout_test() { return g_route_timeout_test.exchange(0) != 0; }
+
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) {
     const int rows = r.T * r.k;
     if (rows <= 0) return cudaSuccess;
@@ -1344,6 +1360,10 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     p.sched = r.counters + nctr - 3;
     p.fc2_done = r.counters + nctr - 2;
     p.route_bar = r.counters + nctr - 1;
+    // a timeout armed for testing: one arrival more than the grid gives, a 1 ms limit
+    const bool timeout_test = take_route_timeout_test();
+    p.route_bar_extra = timeout_test ? 1 : 0;
+    p.route_wait_ns = timeout_test ? 1000000ull : kWaitLimitNs;
     p.k = r.k;
     p.out = static_cast<__nv_bfloat16*>(r.out);
     p.err = r.err;

@@ -40,6 +40,28 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same launch, optionally cooperative: every block of the grid resident at once
+// (a kernel with a grid-wide barrier); the launch fails rather than waits when they
+// cannot all be resident.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k_coop(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, bool cooperative, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = cooperative ? 2 : 1;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- rmsnorm.cu
 // y [T, H] = the pre-FFN RMSNorm of x with weight w [H] (float64, one rounding to the
 // dtype); the same launch zeroes `clear_bytes` (a multiple of 16) at `clear`.
@@ -192,6 +214,10 @@ struct DecodeRoutedArgs {
     FfnAttrs ep;
 };
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& a, cudaStream_t s);
+// Testing aid: the next launch_ffn_decode_routed waits at its routing grid barrier for
+// one arrival more than its grid provides, with a 1 ms limit (one-shot).
+void arm_route_timeout_test();
+bool take_route_timeout_test();
 
 cudaError_t launch_ffn_decode(const void* tokens, const int32_t* perm_src, int T,
                               const int32_t* offsets, const void* fc1, const void* fc2, int rows,
