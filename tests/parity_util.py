@@ -32,34 +32,29 @@ def tol(dtype, ref=None):
     return F32_ATOL + floor, F32_RTOL
 
 
-def row_scale(ref):
-    """Per-row factor on the absolute term of the bf16 tolerance, shape [rows, 1].
-
-    The absolute term is in units of a typical row's output.  A row whose output
-    RMS is more than twice the median row RMS (an outlier token, whose input was
-    scaled up) gets s_t = rms_t / median: its intermediates are proportionally
-    larger, and bf16 storage of act and y_perm alone leaves errors that scale with
-    them.  Every other row keeps s_t = 1, i.e. exactly the stated tolerance.
-    """
-    ref = np.asarray(ref, dtype=np.float64)
-    rms = np.sqrt(np.mean(np.square(ref), axis=1))
-    med = max(float(np.median(rms)) if rms.size else 1.0, 1e-30)
-    ratio = rms / med
-    return np.where(ratio > 2.0, ratio, 1.0)[:, None]
-
-
-def assert_close(got, ref, atol, rtol, what):
+def assert_close(got, ref, atol, rtol, what, extra=None):
+    """|got - ref| <= atol + rtol |ref| elementwise (atol a scalar or an array that
+    broadcasts).  `extra` (same shape as ref, or None) is an additional per-element
+    allowance; the elements that need it -- beyond the stated bound, within the
+    stated bound plus `extra` -- are counted and printed.  Returns that count."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     d = np.abs(got - ref)
-    lim = atol + rtol * np.abs(ref)
+    stated = atol + rtol * np.abs(ref)
+    lim = stated if extra is None else stated + extra
     bad = d > lim
     if bad.any():
         i = np.unravel_index(np.argmax(d - lim), d.shape)
         raise AssertionError(
             f"{what}: {int(bad.sum())} of {d.size} elements out of tolerance; worst at {i}: "
             f"got {got[i]!r} ref {ref[i]!r} |d|={d[i]:.3e} limit={lim[i]:.3e}")
+    n_extra = 0
+    if extra is not None:
+        n_extra = int(np.count_nonzero(d > stated))
+        print(f"{what}: {n_extra} of {d.size} elements beyond the stated bound and within "
+              f"the bf16 storage allowance; worst |d|/stated = {float(np.max(d / stated)):.3f}")
+    return n_extra
 
 
 def to_dev(a, dtype, device="cuda"):
@@ -147,3 +142,39 @@ def bf16_storage_bound(act, fc2_e, y):
     act [n, I], fc2_e [H, I], y [n, H], all exact (float64)."""
     u = 2.0 ** -9
     return u * (np.abs(act) @ np.abs(fc2_e).T + np.abs(y))
+
+
+def scaled_row_storage_bound(inp, idx, tokens, scaled_rows):
+    """The bf16 storage allowance of the layer's output on the rows the input generator
+    scaled up (the long-prefill workload's x8 outlier rows), zero on every other row.
+
+    For token t and its chosen experts e_j with routing weights w_j (the oracle's, from
+    its float64 logits): sum_j w_j 2^-9 (|a_j| |fc2_e_j|^T + |y_j|), a_j = the oracle's
+    SwiGLU of t under e_j and y_j = a_j fc2_e_j^T -- what bf16 storage of the
+    intermediates act and y_perm may move the output by, to first order.  An x8 input
+    row makes its gate and up values 8 times larger and its act ~64 times larger, so
+    the absolute term of the stated tolerance, sized for ordinary rows, cannot hold
+    there for any kernel that stores act in bf16.
+
+    Returns [len(tokens), H] float64 (standard SwiGLU, no expert biases)."""
+    wl = inp.wl
+    tokens = np.asarray(tokens, dtype=np.int64)
+    scaled = set(int(t) for t in np.asarray(scaled_rows).tolist())
+    out = np.zeros((tokens.size, wl.H))
+    pick = [i for i, t in enumerate(tokens.tolist()) if t in scaled]
+    if not pick:
+        return out
+    x = inp.values("hidden")
+    L = O.router_logits(x[tokens[pick]], inp.values("router_w"), inp["router_bias"])
+    w = O.routing_weights(L, np.asarray(idx)[tokens[pick]], wl.normalize)
+    sub_idx = np.asarray(idx)[tokens[pick]]
+    for e in np.unique(sub_idx):
+        rows, slots = np.nonzero(sub_idx == e)
+        xe = x[tokens[pick][rows]].astype(np.float64)
+        w_gate, w_up = O.fc1_gate_up(inp.expert_values("fc1", int(e)).astype(np.float64),
+                                     wl.fc1_layout)
+        a = O.swiglu(xe @ w_gate.T, xe @ w_up.T)
+        fc2_e = inp.expert_values("fc2", int(e)).astype(np.float64)
+        b = bf16_storage_bound(a, fc2_e, a @ fc2_e.T)
+        np.add.at(out, np.asarray(pick)[rows], w[rows, slots][:, None] * b)
+    return out

@@ -11,7 +11,7 @@ import torch
 import mixture_experts_ffn_15_b200 as moe
 from oracle import moe_oracle as O
 from parity_util import (W_ATOL, assert_close, bf16_storage_bound, device_inputs, from_dev,
-                         match_routing, row_scale, sample_tokens, to_dev, tol)
+                         match_routing, sample_tokens, scaled_row_storage_bound, to_dev, tol)
 from synth import Workload, bf16_bits_to_f32, make_inputs, round_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
@@ -137,8 +137,6 @@ def test_expert_ffn(wl):
         if b > a:
             y_ref[a:b] = O.expert_ffn(xv[a:b], inp.expert_values("fc1", e), inp.expert_values("fc2", e))
     atol, rtol = tol(wl.dtype, y_ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(y_ref)
     assert_close(from_dev(y), y_ref, atol, rtol, "y_perm")
 
 
@@ -172,7 +170,7 @@ def test_expert_ffn_at_tile_edges(scale):
         if b > a:
             y_ref[a:b] = O.expert_ffn(xv[a:b], inp.expert_values("fc1", e), inp.expert_values("fc2", e))
     atol, rtol = tol(wl.dtype, y_ref)
-    assert_close(from_dev(y), y_ref, atol * row_scale(y_ref), rtol, f"y_perm at tile edges (scale {scale})")
+    assert_close(from_dev(y), y_ref, atol, rtol, f"y_perm at tile edges (scale {scale})")
 
 
 @pytest.mark.parametrize("wl", CASES, ids=IDS)
@@ -186,8 +184,6 @@ def test_forward(wl):
     L, idx = check_routing(inp, r)
     ref = oracle_forward(inp, idx)["out"]
     atol, rtol = tol(wl.dtype, ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(ref)
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} output")
 
 
@@ -229,8 +225,6 @@ def test_forward_swiglu_attributes_and_biases(wl, attr, biased):
                         wl.k, wl.normalize, wl.fc1_layout, idx=idx, act=act,
                         fc1_bias=f(b1), fc2_bias=f(b2))["out"]
     atol, rtol = tol(wl.dtype, ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(ref)
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} {attr[0]} biased={biased}")
 
 
@@ -260,10 +254,12 @@ def test_expert_ffn_attributes_and_biases_on_both_bf16_kernels():
             g = xv[a:b].astype(np.float64) @ fc1_e[0::2].T.astype(np.float64) + b1_e[0::2]
             u = xv[a:b].astype(np.float64) @ fc1_e[1::2].T.astype(np.float64) + b1_e[1::2]
             bound[a:b] = bf16_storage_bound(O.swiglu(g, u, *act), fc2_e.astype(np.float64), y_ref[a:b])
-        # the beta on the up branch roughly doubles |act|, and with it the error of
-        # storing act in bf16: the stated tolerance plus that storage bound
+        # y_perm is an intermediate (each row before its routing weight): the beta on
+        # the up branch and the biases roughly double |act|, and with it the error of
+        # storing act in bf16.  The stated tolerance plus that storage bound; the
+        # layer-level tests of the same attributes keep the stated tolerance alone.
         atol, rtol = tol(wl.dtype, y_ref)
-        assert_close(from_dev(y), y_ref, atol * row_scale(y_ref) + bound, rtol, f"y_perm {name}")
+        assert_close(from_dev(y), y_ref, atol, rtol, f"y_perm {name}", extra=bound)
 
 
 # ------------------------------------------- fc1 in the chunked layout, read in place
@@ -316,8 +312,6 @@ def test_forward_reads_chunked_fc1_in_place(wl, biased):
                         wl.k, wl.normalize, "chunked", idx=idx, act=act,
                         fc1_bias=f(b1), fc2_bias=f(b2))["out"]
     atol, rtol = tol(wl.dtype, ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(ref)
     assert_close(from_dev(out_c), ref, atol, rtol, f"{wl.name} chunked biased={biased}")
 
 
@@ -424,8 +418,6 @@ def test_forward_with_pre_norm(wl):
                         lambda e: inp.expert_values("fc1", e), lambda e: inp.expert_values("fc2", e),
                         wl.k, wl.normalize, wl.fc1_layout, idx=idx)["out"]
     atol, rtol = tol(wl.dtype, ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(ref)
     assert_close(from_dev(fused), ref, atol, rtol, f"{wl.name} with pre-FFN norm")
 
 
@@ -492,7 +484,7 @@ def test_forward_q8(wl):
     L, idx = check_routing(inp, r)
     ref = _q8_oracle(inp, wl, host, idx)
     atol, rtol = tol(wl.dtype, ref)
-    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, f"{wl.name} int8 experts")
+    assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} int8 experts")
 
 
 def test_forward_q8_attributes_and_biases():
@@ -510,7 +502,7 @@ def test_forward_q8_attributes_and_biases():
     L, idx = check_routing(inp, r)
     ref = _q8_oracle(inp, wl, host, idx, act, bf16_bits_to_f32(b1), bf16_bits_to_f32(b2))
     atol, rtol = tol(wl.dtype, ref)
-    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, "int8 experts, GPT-OSS + biases")
+    assert_close(from_dev(out), ref, atol, rtol, "int8 experts, GPT-OSS + biases")
 
 
 @pytest.mark.parametrize("layout", ["interleaved", "chunked"])
@@ -544,7 +536,7 @@ def test_expert_ffn_q8_unit_scales_equal_bf16_kernel(layout):
                                 O.dequantize_rows(host[2][e], host[3][e]), layout,
                                 O.STANDARD_SWIGLU, bf16_bits_to_f32(b1[e]), bf16_bits_to_f32(b2[e]))
     atol, rtol = tol("bf16", ref)
-    assert_close(from_dev(y), ref, atol * row_scale(ref), rtol, f"int8 expert FFN {layout}")
+    assert_close(from_dev(y), ref, atol, rtol, f"int8 expert FFN {layout}")
 
 
 def test_full_decode_q8():
@@ -561,7 +553,7 @@ def test_full_decode_q8():
     L, idx = check_routing(inp, r)
     ref = _q8_oracle(inp, wl, host, idx)
     atol, rtol = tol(wl.dtype, ref)
-    assert_close(from_dev(out), ref, atol * row_scale(ref), rtol, "decode_bf16 int8 experts")
+    assert_close(from_dev(out), ref, atol, rtol, "decode_bf16 int8 experts")
 
 
 def test_q8_refuses_sizes_outside_the_decode_ffn():
@@ -696,6 +688,34 @@ def test_invalid_arguments_are_rejected():
                     torch.zeros((E, 72, I), dtype=torch.bfloat16, device="cuda"), 2)
 
 
+def test_routing_barrier_timeout_is_reported_and_the_next_call_is_clean():
+    """Device-side failure detection without a fault: a test-only setting makes the
+    one-launch path's routing grid barrier wait for an arrival that never comes, with a
+    1 ms limit.  Every block gives up before any bulk copy or MMA, winds down and reports
+    MOE_DEVERR_TIMEOUT; the context stays usable, and the next calls -- on the same
+    workspace and on a fresh one -- are bit for bit the normal result."""
+    from mixture_experts_ffn_15_b200 import _abi
+    lib = _abi.load()
+    wl = W("timeout", T=4, H=256, E=64, k=4, I=128)
+    assert lib.moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, _abi.MOE_BF16) & 32
+    dev = device_inputs(make_inputs(wl))
+    args = (dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], wl.k)
+    ref = moe.forward(*args)
+    need = moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, torch.bfloat16)
+    ws = moe.alloc_workspace(need, torch.device("cuda"))
+    lib.moe_debug_arm_route_barrier_timeout()
+    moe.forward(*args, workspace=ws)
+    st, bits = moe.get_error(moe.workspace_error_word(ws))
+    assert st == _abi.MOE_ERR_TIMEOUT and bits & _abi.MOE_DEVERR_TIMEOUT, (st, bits)
+    again = moe.forward(*args, workspace=ws)          # the setting was one-shot
+    st, bits = moe.get_error(moe.workspace_error_word(ws))
+    assert st == _abi.MOE_OK and bits == 0
+    assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+    fresh = moe.forward(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(fresh.view(torch.int16), ref.view(torch.int16))
+
+
 def test_bad_expert_ids_are_reported_and_skipped():
     E, T, k = 8, 40, 2
     idx = np.stack([np.arange(T) % E, (np.arange(T) + 3) % E], axis=1).astype(np.int32)
@@ -746,11 +766,16 @@ def test_full_workload(name):
     # values: every token when the oracle is quick, else a seeded sample that holds
     # the outlier rows and tokens of the least and most loaded experts
     tokens = None
+    scaled = outlier_rows(wl, wl.seed)
     if wl.T > 256:
-        tokens = sample_tokens(wl.T, idx, wl.E, n=192, must=outlier_rows(wl, wl.seed)[:64])
+        tokens = sample_tokens(wl.T, idx, wl.E, n=192, must=scaled[:64])
     ref = oracle_forward(inp, idx, tokens=tokens)["out"]
     got = from_dev(out) if tokens is None else from_dev(out[torch.from_numpy(tokens).cuda()])
     atol, rtol = tol(wl.dtype, ref)
-    if wl.dtype == "bf16":
-        atol = atol * row_scale(ref)
-    assert_close(got, ref, atol, rtol, f"{name} output")
+    # the stated tolerance on every row; the rows the generator scaled x8 (long
+    # prefill) also get the oracle's bound of storing act and y_perm in bf16
+    extra = None
+    if scaled.size and wl.dtype == "bf16":
+        extra = scaled_row_storage_bound(inp, idx, np.arange(wl.T) if tokens is None else tokens,
+                                         scaled)
+    assert_close(got, ref, atol, rtol, f"{name} output", extra=extra)
