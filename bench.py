@@ -5,17 +5,22 @@
 
 A step is one call of the whole layer (route -> permute -> fc1 + SwiGLU -> fc2 ->
 combine) on one batch of synthetic tokens with the inputs resident in HBM.  The
-default workload is decode_bf16 (T=4, H=2816, E=128, k=8, I=704), the configuration
-the layer's headline metric is quoted on; --workload picks another row of
-synth.WORKLOADS.  Steps are replayed from CUDA graphs of S steps each; between
-reuses of a weight set, `--sets` - 1 other copies of the weights are streamed, so
-the touched weights never sit in L2 when a step starts.
+line's workload is long_prefill_bf16 (T=32768, H=4096, E=64, k=4, I=1536, 1% of the
+rows x8), the largest of the five single-GPU workloads of synth.WORKLOADS;
+--workload picks another.  It runs W warm-up steps (eager calls through the public
+API) and then times exactly K steps, replayed from a CUDA graph of S steps (S
+divides K), between two CUDA events on the launching stream.  Each of the other
+four workloads is then measured the same way with its own step counts and reported
+under `per_config` (value, roofline of its dominant kernel, e2e, CPU baseline,
+clocks).  For the weight-streaming workloads `--sets` copies of the weights rotate,
+so that the weights of a step never sit in L2 when it starts; the prefill workloads
+move more than L2 per step.
 
 Prints ONE JSON line (rank 0).  Multi-GPU (torchrun, one rank per GPU) runs
 independent replicas: the layer has no exchange step on one GPU's batch, so there
 is no data-path collective; the barrier and the max-over-ranks timing are the only
-communication.  `--impl reference` times the CPU oracle (the reference arm of this
-build) on the host cores instead.
+communication.  `--impl reference` times the CPU oracle (the reference arm) on the
+host instead.
 """
 import argparse
 import datetime
@@ -32,25 +37,38 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s + TFLOP/s or HBM GB/s as fraction of roofline, 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DEFAULT_STEPS = {"tiny_fp32": 2000, "decode_bf16": 6000, "batched_decode_bf16": 2000,
-                 "prefill_bf16": 400, "long_prefill_bf16": 100}
+ORDER = ["tiny_fp32", "decode_bf16", "batched_decode_bf16", "prefill_bf16", "long_prefill_bf16"]
+DEFAULT_WORKLOAD = "long_prefill_bf16"
+# steps and warm-up steps of a workload when the command line does not set them
+DEFAULT_STEPS = {"tiny_fp32": 10000, "decode_bf16": 4000, "batched_decode_bf16": 1000,
+                 "prefill_bf16": 300, "long_prefill_bf16": 100}
+DEFAULT_WARMUP = {"tiny_fp32": 40, "decode_bf16": 40, "batched_decode_bf16": 20,
+                  "prefill_bf16": 5, "long_prefill_bf16": 3}
+# steps per CUDA graph (at most; the graph size divides the step count)
 GRAPH_STEPS = {"tiny_fp32": 20, "decode_bf16": 20, "batched_decode_bf16": 20,
-               "prefill_bf16": 4, "long_prefill_bf16": 2}
+               "prefill_bf16": 1, "long_prefill_bf16": 1}
 HBM_BOUND = {"decode_bf16", "batched_decode_bf16", "tiny_fp32"}
 SWIGLU_PRESETS = {"standard": (1.0, 0.0, float("inf")), "gpt_oss": (1.702, 1.0, 7.0)}
+NORM_EPS = 1e-6
+CPU_WORKERS_MAX = 32
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode_bf16")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--sets", type=int, default=None, help="rotating weight copies (L2)")
-    ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--e2e-seconds", type=float, default=1.0,
+                    help="about how long the end-to-end measurement of a workload runs")
+    ap.add_argument("--cpu-seconds", type=float, default=6.0,
+                    help="CPU baseline of the line's workload: seconds per timing")
+    ap.add_argument("--per-config-cpu-seconds", type=float, default=2.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure the line's workload only")
     ap.add_argument("--swiglu", choices=list(SWIGLU_PRESETS), default="standard",
                     help="SwiGLU attributes (alpha, beta, limit) of the op")
     ap.add_argument("--expert-bias", action="store_true", help="with fc1/fc2 expert biases")
@@ -64,6 +82,12 @@ def parse_args(argv=None):
                     help="convert chunked fc1 to the interleaved layout at set-up instead of "
                          "reading it in place")
     return ap.parse_args(argv)
+
+
+def variant_flags(args):
+    """True when a flag changes the layer (then only the line's workload is measured)."""
+    return bool(args.q8 or args.pre_norm or args.expert_bias or args.swiglu != "standard"
+                or args.fc1_convert)
 
 
 # --------------------------------------------------------------------------- helpers
@@ -98,33 +122,37 @@ def max_over_ranks(x, world, device=None):
     return float(t.item())
 
 
+def graph_steps(limit, steps):
+    """Steps per CUDA graph: the largest divisor of `steps` not above `limit`."""
+    for s in range(max(1, min(limit, steps)), 0, -1):
+        if steps % s == 0:
+            return s
+    return 1
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms in the background."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms in the background
+    with their timestamps, so that each timed region takes the samples inside it."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.file = None
-        self.t0 = self.t1 = None
+        self.rows = []
 
     def start(self):
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+                 "-i", str(self.gpu), "-lms", "50"], stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(1.0)
-
-    def mark(self, begin):
-        if begin:
-            self.t0 = time.time()
-        else:
-            self.t1 = time.time()
+        time.sleep(0.5)
 
     def stop(self):
         if self.proc is not None:
@@ -135,32 +163,41 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
         self.file.flush()
-        rows = []
         with open(self.file.name) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                self.rows.append((ts, parts[1:]))
         os.unlink(self.file.name)
-        if not rows:
+
+    @staticmethod
+    def _num(s):
+        try:
+            return float(s)
+        except ValueError:
+            return float("nan")
+
+    def summary(self, t0, t1):
+        """Median SM clock and the throttle reasons seen during [t0, t1] (host times)."""
+        inside = [r for ts, r in self.rows if ts is not None and t0 - 0.06 <= ts <= t1 + 0.06]
+        note = "samples inside the timed region"
+        if not inside:
+            after = [(ts, r) for ts, r in self.rows if ts is not None and ts >= t0]
+            inside = [after[0][1]] if after else [r for _, r in self.rows[-1:]]
+            note = "timed region shorter than the sampling period: the next sample"
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        # the rows of the timed region: the busiest (highest power) contiguous half
-        def num(s):
-            try:
-                return float(s)
-            except ValueError:
-                return float("nan")
-        power = [num(r[3]) for r in rows]
-        thr = sorted(power)[len(power) // 2] if len(power) > 2 else -1
-        load = [r for r, p in zip(rows, power) if p >= thr] or rows
-        sm = sorted(num(r[1]) for r in load)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in load for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": num(load[0][2]), "reasons": reasons,
-                "samples": len(load), "power_w_max": max(num(r[3]) for r in load)}
-
-
-NORM_EPS = 1e-6
+        sm = sorted(self._num(r[0]) for r in inside)
+        reasons = sorted({self.NAMES[i] for r in inside for i in range(4)
+                          if r[4 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self._num(inside[0][1]),
+                "reasons": reasons, "samples": len(inside), "note": note,
+                "power_w_max": max(self._num(r[2]) for r in inside)}
 
 
 def algorithmic(wl, counts, pre_norm=False, q8=False):
@@ -189,10 +226,10 @@ def algorithmic(wl, counts, pre_norm=False, q8=False):
     return used, fc1, fc2, layer
 
 
-def kernel_source(one_launch_or_decode):
+def kernel_source(decode_kernel):
     """Source file of the dominant kernel: the decode FFN (gemm_tc.cu) or the CTA-pair
     grouped GEMM (gemm_pair.cu)."""
-    name = "gemm_tc.cu" if one_launch_or_decode else "gemm_pair.cu"
+    name = "gemm_tc.cu" if decode_kernel else "gemm_pair.cu"
     return os.path.join(ROOT, "mixture_experts_ffn_15_b200", "csrc", name)
 
 
@@ -225,68 +262,151 @@ def device_tensor(a, dev):
     return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
 
+def wide(a):
+    from synth import bf16_bits_to_f32
+    return None if a is None else (bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a)
+
+
+# --------------------------------------------------------------------------- host inputs
+
+def host_inputs(names, q8=False):
+    """The synthetic inputs of each workload (CPU arrays).  Expert weights depend only
+    on (seed, E, H, I, dtype), so workloads that share those share one draw."""
+    from synth import WORKLOADS, make_inputs
+    drawn = {}
+    out = {}
+    for n in names:
+        wl = WORKLOADS[n]
+        inp = make_inputs(wl, weights=False)
+        if not q8:
+            key = (wl.seed, wl.E, wl.H, wl.I, wl.dtype)
+            if key not in drawn:
+                full = make_inputs(wl)
+                drawn[key] = (full["fc1"], full["fc2"])
+            inp.arrays["fc1"], inp.arrays["fc2"] = drawn[key]
+        out[n] = inp
+    return out
+
+
+class LayerOptions:
+    """The layer's optional inputs, as host arrays, for the oracle and the device."""
+
+    def __init__(self, args, wl):
+        from synth import make_expert_biases, make_pre_norm_inputs, make_q8_experts
+        self.act = SWIGLU_PRESETS[args.swiglu]
+        self.biases = make_expert_biases(wl) if args.expert_bias else (None, None)
+        self.pre = make_pre_norm_inputs(wl) if args.pre_norm else None
+        self.q8 = make_q8_experts(wl) if args.q8 else None
+
+    def oracle_getters(self, inp):
+        from oracle import moe_oracle as O
+        if self.q8 is not None:
+            q1, s1, q2, s2 = self.q8
+            return (lambda e: O.dequantize_rows(q1[e], s1[e]),
+                    lambda e: O.dequantize_rows(q2[e], s2[e]))
+        return (lambda e: inp.expert_values("fc1", e), lambda e: inp.expert_values("fc2", e))
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
-def q8_getters(q8_host):
-    """Oracle weight getters of int8 experts: q * scale of each row, float64."""
-    from oracle import moe_oracle as O
-    q1, s1, q2, s2 = q8_host
-    return (lambda e: O.dequantize_rows(q1[e], s1[e]), lambda e: O.dequantize_rows(q2[e], s2[e]))
-
-
-def oracle_cost(wl, inp, seconds, pre=None, q8_host=None):
-    """The CPU oracle, as it stands, on whole tokens of `wl` for about `seconds` (with
-    pre = (residual values, norm weight values), each token through the pre-FFN norm
-    first).
-
-    Returns (tokens/s, threads, description of the sample)."""
+def oracle_tokens(wl, inp, opts, seconds, start=0, stride=1):
+    """The CPU oracle, as it stands, on whole tokens start, start + stride, ... of `wl`
+    for about `seconds` (each token routed over all E experts and run through its k
+    experts in float64; with the pre-FFN norm, normalised first).  Returns (tokens, s)."""
     import numpy as np
-    from threadpoolctl import threadpool_info
 
     from oracle import moe_oracle as O
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     x = inp.values("hidden")
     rw = inp.values("router_w")
-    bias = inp["router_bias"]
-    fc1 = lambda e: inp.expert_values("fc1", e)
-    fc2 = lambda e: inp.expert_values("fc2", e)
-    if q8_host is not None:
-        fc1, fc2 = q8_getters(q8_host)
+    fc1, fc2 = opts.oracle_getters(inp)
+    b1, b2 = (wide(b) for b in opts.biases)
     t0 = time.perf_counter()
     n = 0
+    t = start % wl.T
     while True:
-        t = n % wl.T
-        xt = x[t:t + 1] if pre is None else O.pre_ffn_norm(pre[0][t:t + 1], pre[1], NORM_EPS,
-                                                           wl.dtype)
-        r = O.moe_forward(xt, rw, bias, fc1, fc2, wl.k, wl.normalize, wl.fc1_layout)
+        xt = x[t:t + 1] if opts.pre is None else O.pre_ffn_norm(
+            wide(opts.pre[0])[t:t + 1], wide(opts.pre[1]), NORM_EPS, wl.dtype)
+        r = O.moe_forward(xt, rw, inp["router_bias"], fc1, fc2, wl.k, wl.normalize,
+                          wl.fc1_layout, act=opts.act, fc1_bias=b1, fc2_bias=b2)
         assert np.isfinite(r["out"]).all()
         n += 1
+        t = (t + stride) % wl.T
         if time.perf_counter() - t0 >= seconds:
             break
-    el = time.perf_counter() - t0
-    return n / el, cores, (f"{n} whole tokens of the workload, one at a time (router logits, "
-                           f"top-k, {wl.k} expert FFNs, combine in float64), {el:.1f} s")
+    return n, time.perf_counter() - t0
 
 
-def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None, None), pre=None,
-                     getters=None):
+_POOL_STATE = {}
+
+
+def _pool_job(job):
+    """One worker of the all-core CPU baseline: its own token stride, one BLAS thread."""
+    from threadpoolctl import threadpool_limits
+    name, start, stride, seconds = job
+    wl, inp, opts = _POOL_STATE[name]
+    with threadpool_limits(1):
+        return oracle_tokens(wl, inp, opts, seconds, start, stride)
+
+
+class CpuBaseline:
+    """The oracle timed on the host: one thread, and one process per core (up to
+    CPU_WORKERS_MAX) on interleaved tokens.  The worker processes are forked before
+    the first CUDA call, so that they hold the inputs already drawn."""
+
+    def __init__(self, workloads):
+        import multiprocessing as mp
+        _POOL_STATE.update(workloads)
+        self.workers = max(1, min(os.cpu_count() or 1, CPU_WORKERS_MAX))
+        self.pool = mp.get_context("fork").Pool(self.workers) if self.workers > 1 else None
+
+    def measure(self, name, seconds):
+        from threadpoolctl import threadpool_limits
+        wl, inp, opts = _POOL_STATE[name]
+        with threadpool_limits(1):
+            n1, s1 = oracle_tokens(wl, inp, opts, seconds)
+        single = n1 / s1
+        res = {"value": single, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": (f"{n1} whole tokens of the workload, one thread (router logits over "
+                          f"all {wl.E} experts, top-k, {wl.k} expert FFNs, combine in float64), "
+                          f"{s1:.1f} s")}
+        if self.pool is not None:
+            jobs = [(name, i, self.workers, seconds) for i in range(self.workers)]
+            try:
+                got = self.pool.map_async(_pool_job, jobs).get(timeout=seconds * 4 + 60)
+                n = sum(g[0] for g in got)
+                el = max(g[1] for g in got)
+                res = {"value": n / el, "unit": "tokens/s", "cores": self.workers,
+                       "kind": "oracle",
+                       "sample": (f"{n} whole tokens in {el:.1f} s on {self.workers} processes "
+                                  f"(one BLAS thread each, interleaved tokens)"),
+                       "single_thread": res}
+            except Exception as ex:   # a stuck worker: keep the one-thread figure
+                res["all_cores"] = f"unavailable: {type(ex).__name__}"
+        return res
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.terminate()
+            self.pool.join()
+
+
+def oracle_pair_step(wl, inp, opts, state):
     """One bounded reference step: routing of one token and one of its expert FFNs (with
-    pre, the token's pre-FFN norm first)."""
+    the pre-FFN norm, the token's norm first)."""
     import numpy as np
 
     from oracle import moe_oracle as O
     t = state["t"]
-    xt = inp.values("hidden")[t:t + 1] if pre is None else \
-        O.pre_ffn_norm(pre[0][t:t + 1], pre[1], NORM_EPS, wl.dtype)
+    xt = inp.values("hidden")[t:t + 1] if opts.pre is None else \
+        O.pre_ffn_norm(wide(opts.pre[0])[t:t + 1], wide(opts.pre[1]), NORM_EPS, wl.dtype)
     L = O.router_logits(xt, inp.values("router_w"), inp["router_bias"])
     idx = O.select_topk(L, wl.k)
     w = O.routing_weights(L, idx, wl.normalize)
     j = state["j"]
     e = int(idx[0, j])
-    b1, b2 = biases
-    g1, g2 = getters if getters is not None else (lambda i: inp.expert_values("fc1", i),
-                                                   lambda i: inp.expert_values("fc2", i))
-    y = O.expert_ffn(xt, g1(e), g2(e), wl.fc1_layout, act,
+    b1, b2 = (wide(b) for b in opts.biases)
+    g1, g2 = opts.oracle_getters(inp)
+    y = O.expert_ffn(xt, g1(e), g2(e), wl.fc1_layout, opts.act,
                      None if b1 is None else b1[e], None if b2 is None else b2[e])
     assert np.isfinite(w[0, j] * y).all()
     state["j"] += 1
@@ -296,60 +416,51 @@ def oracle_pair_step(wl, inp, state, act=(1.0, 0.0, float("inf")), biases=(None,
 
 
 def run_reference(args):
-    from synth import WORKLOADS, bf16_bits_to_f32, make_inputs
+    from threadpoolctl import threadpool_limits
+
+    from synth import WORKLOADS, make_inputs
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     wl = WORKLOADS[args.workload]
     steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(wl.name, 100)
-    from threadpoolctl import threadpool_info
-    cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    warmup = args.warmup if args.warmup is not None else DEFAULT_WARMUP.get(wl.name, 3)
     inp = make_inputs(wl, weights=not args.q8)
-    act = SWIGLU_PRESETS[args.swiglu]
-    biases = (None, None)
-    pre = None
-    getters = None
-    if args.q8:
-        from synth import make_q8_experts
-        getters = q8_getters(make_q8_experts(wl))
-    if args.pre_norm:
-        from synth import make_pre_norm_inputs
-        px, pw = make_pre_norm_inputs(wl)
-        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
-        pre = (wide(px), wide(pw))
-    if args.expert_bias:
-        from synth import make_expert_biases
-        nb1, nb2 = make_expert_biases(wl)
-        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
-        biases = (wide(nb1), wide(nb2))
+    opts = LayerOptions(args, wl)
     state = {"t": 0, "j": 0}
-    for _ in range(args.warmup):
-        oracle_pair_step(wl, inp, state, act, biases, pre, getters)
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        oracle_pair_step(wl, inp, state, act, biases, pre, getters)
-    el = time.perf_counter() - t0
+    with threadpool_limits(1):
+        for _ in range(warmup):
+            oracle_pair_step(wl, inp, opts, state)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            oracle_pair_step(wl, inp, opts, state)
+        el = time.perf_counter() - t0
     value = (steps / wl.k) / el
     sample = (f"each step: router logits + top-k of one token and one of its {wl.k} expert "
-              f"FFNs (1/{wl.k} token); {steps} steps in {el:.1f} s")
+              f"FFNs (1/{wl.k} token), one thread; {steps} steps in {el:.1f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
         "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(wl, sets=4 if wl.name in HBM_BOUND else 1),
-                       parallelism=f"replicas x{args.gpus}",
-                       graph_steps=GRAPH_STEPS.get(wl.name, 4), swiglu=list(act),
+        "config": dict(workload_config(wl, sets=default_sets(wl, args)),
+                       parallelism=f"replicas x{args.gpus}", swiglu=list(opts.act),
                        expert_bias=bool(args.expert_bias), pre_norm=bool(args.pre_norm),
                        q8=bool(args.q8),
                        fc1_layout_read="interleaved" if args.fc1_convert else wl.fc1_layout),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def default_sets(wl, args):
+    if args.sets is not None:
+        return args.sets
+    return 4 if wl.name in HBM_BOUND else 1
 
 
 def workload_config(wl, sets):
@@ -367,51 +478,29 @@ def workload_config(wl, sets):
 
 # --------------------------------------------------------------------------- our arm
 
-def run_ours(args):
+def measure(wl, inp, opts, args, steps, warmup, world, dev, clocks):
+    """The layer on workload `wl`: W eager warm-up calls, then K steps replayed from a
+    CUDA graph between two events, a second region with stage events, and the end-to-end
+    figure through the public API.  Returns the workload's result row."""
     import numpy as np
     import torch
 
     import mixture_experts_ffn_15_b200 as moe
-    from synth import WORKLOADS, make_inputs
 
-    rank, world, local = dist_env()
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                device_id=dev)
-    wl = WORKLOADS[args.workload]
-    S = GRAPH_STEPS.get(wl.name, 4)
-    steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(wl.name, 100)
-    reps = max(1, math.ceil(steps / S))
-    steps = reps * S
-    warm_reps = max(1, math.ceil(args.warmup / S))
-    sets = args.sets if args.sets is not None else (4 if wl.name in HBM_BOUND else 1)
-
-    if args.q8 and wl.name not in HBM_BOUND:
-        raise SystemExit("--q8: the int8 experts run in the decode FFN only (decode workloads)")
-    inp = make_inputs(wl, weights=not args.q8)
+    sets = default_sets(wl, args)
+    S = graph_steps(GRAPH_STEPS.get(wl.name, 1), steps)
+    reps = steps // S
     hidden = device_tensor(inp["hidden"], dev)
-    norm_kw, pre = {}, None
-    if args.pre_norm:
+    norm_kw = {}
+    if opts.pre is not None:
         # the input is a residual activation; the layer normalises it itself
-        from synth import bf16_bits_to_f32, make_pre_norm_inputs
-        px, pw = make_pre_norm_inputs(wl)
-        hidden = device_tensor(px, dev)
-        norm_kw = dict(norm_weight=device_tensor(pw, dev), norm_eps=NORM_EPS)
-        wide = lambda a: bf16_bits_to_f32(a) if a.dtype.name == "uint16" else a
-        pre = (wide(px), wide(pw))
+        hidden = device_tensor(opts.pre[0], dev)
+        norm_kw = dict(norm_weight=device_tensor(opts.pre[1], dev), norm_eps=NORM_EPS)
     router_w = device_tensor(inp["router_w"], dev)
     bias = None if inp["router_bias"] is None else torch.from_numpy(inp["router_bias"]).to(dev)
     layout = wl.fc1_layout
-    q8_host = None
-    if args.q8:
-        from synth import make_q8_experts
-        q8_host = make_q8_experts(wl)
-        q8 = [torch.from_numpy(a).to(dev) for a in q8_host]
+    if opts.q8 is not None:
+        q8 = [torch.from_numpy(a).to(dev) for a in opts.q8]
         weight_sets = [q8] + [[t.clone() for t in q8] for _ in range(sets - 1)]
     else:
         fc1 = device_tensor(inp["fc1"], dev)
@@ -420,44 +509,42 @@ def run_ours(args):
             layout = "interleaved"
         fc2 = device_tensor(inp["fc2"], dev)
         weight_sets = [[fc1, fc2]] + [[fc1.clone(), fc2.clone()] for _ in range(sets - 1)]
+    b1 = b2 = None
+    if opts.biases[0] is not None:
+        b1, b2 = (device_tensor(b, dev) for b in opts.biases)
+    ffn_kw = dict(swiglu=opts.act, fc1_bias=b1, fc2_bias=b2, fc1_layout=layout, **norm_kw)
+    out = torch.empty_like(hidden)
+    ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
 
     def run_layer(x, i, **kw):
         """One call of the layer on input x with the i-th rotating copy of the weights."""
         w = weight_sets[i % sets]
-        if args.q8:
+        if opts.q8 is not None:
             return moe.forward_q8(x, router_w, w[0], w[1], w[2], w[3], wl.k, **kw)
         return moe.forward(x, router_w, w[0], w[1], wl.k, **kw)
-    act = SWIGLU_PRESETS[args.swiglu]
-    b1 = b2 = None
-    if args.expert_bias:
-        from synth import make_expert_biases
-        nb1, nb2 = make_expert_biases(wl)
-        b1, b2 = device_tensor(nb1, dev), device_tensor(nb2, dev)
-    ffn_kw = dict(swiglu=act, fc1_bias=b1, fc2_bias=b2, fc1_layout=layout, **norm_kw)
-    out = torch.empty_like(hidden)
-    ws = moe.alloc_workspace(moe.workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, hidden.dtype), dev)
 
     # routing outside the timed region, for the byte accounting only
-    x_in = moe.rmsnorm(hidden, norm_kw["norm_weight"], NORM_EPS) if args.pre_norm else hidden
+    x_in = moe.rmsnorm(hidden, norm_kw["norm_weight"], NORM_EPS) if norm_kw else hidden
     r = moe.route(x_in, router_w, wl.k, normalize=bool(wl.normalize), router_bias=bias)
-    p = moe.permute(r["idx"], wl.E)
-    counts = p["counts"].cpu().numpy()
-    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts, args.pre_norm, args.q8)
+    counts = moe.permute(r["idx"], wl.E)["counts"].cpu().numpy()
+    del r, x_in
+    used, fc1_work, fc2_work, layer_work = algorithmic(wl, counts, opts.pre is not None,
+                                                       opts.q8 is not None)
 
     stream = torch.cuda.Stream(device=dev)
-    call = lambda i: run_layer(hidden, i,
-                                 normalize=bool(wl.normalize), router_bias=bias, out=out,
-                                 workspace=ws, **ffn_kw)
+    call = lambda x, i: run_layer(x, i, normalize=bool(wl.normalize), router_bias=bias, out=out,
+                                  workspace=ws, **ffn_kw)
+    # warm-up: W eager steps through the public API (the first call of each weight set
+    # also does the library's once-per-device set-up, which must precede a capture)
     with torch.cuda.stream(stream):
-        for i in range(sets):
-            call(i)
+        for i in range(max(warmup, sets)):
+            call(hidden, i)
     torch.cuda.synchronize(dev)
 
-    # Two graphs of S steps each.  The timed region for `value` replays the plain
-    # graph: consecutive kernels overlap their launch through programmatic
-    # dependencies, which an event node between them would cut.  The stage times
-    # (and the dominant kernel's duration for the roofline) come from a second timed
-    # region that replays the same steps with the 6 stage events of every step.
+    # The timed graph (S steps): consecutive kernels overlap their launch through
+    # programmatic dependencies, which an event between them would cut.  The stage
+    # times (and the dominant kernel's duration) come from a second graph of the same
+    # steps with the 6 stage events of every step, replayed after the timed region.
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(S)]
     for row in events:
         for ev in row:
@@ -468,70 +555,63 @@ def run_ours(args):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(S):
-            call(i)
+            call(hidden, i)
     launches_per_step = (lib.moe_kernel_launches() - n0) / S
     graph_ev = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_ev, stream=stream):
         for i in range(S):
             moe.set_stage_events([ev.cuda_event for ev in events[i]])
-            call(i)
+            call(hidden, i)
         moe.set_stage_events(None)
 
-    with torch.cuda.stream(stream):
-        for _ in range(warm_reps):
-            graph.replay()
-            graph_ev.replay()
-    torch.cuda.synchronize(dev)
-    clocks = ClockSampler(local)
-    clocks.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    clocks.mark(True)
+    h0 = time.time()
     with torch.cuda.stream(stream):
         t_start.record(stream)
         for _ in range(reps):
             graph.replay()
         t_end.record(stream)
     torch.cuda.synchronize(dev)
-    clocks.mark(False)
+    h1 = time.time()
     if world > 1:
         torch.distributed.barrier()
-    # second timed region: the same steps with stage events
+    ms_step = max_over_ranks(t_start.elapsed_time(t_end), world, dev) / steps
+
+    # second region: the same steps with stage events (stage times of the last replay)
     with torch.cuda.stream(stream):
-        for _ in range(max(1, reps // 4)):
+        for _ in range(max(1, min(reps // 4, 8))):
             graph_ev.replay()
     torch.cuda.synchronize(dev)
-    clk = clocks.stop()
-    ms_total = t_start.elapsed_time(t_end)
-    ms_total = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total / steps
-
-    # stage durations of the last replay (inside the timed region)
     stage_names = ["route", "permute", "ffn1", "ffn2", "combine"]
     st = {n: 0.0 for n in stage_names}
     for i in range(S):
         for a, n in enumerate(stage_names):
             st[n] += events[i][a].elapsed_time(events[i][a + 1]) / S
     path = lib.moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, 1 if wl.dtype == "bf16" else 0)
-    if args.q8:
+    if opts.q8 is not None:
         path &= ~32   # int8 experts: the decode FFN after the staged routing kernels
     fused = bool(path & 2)
-    # the dominant kernel: the fused decode FFN (fc1 + SwiGLU and fc2 in one launch),
-    # else the fc1 + SwiGLU grouped GEMM
-    dom_ms = max_over_ranks(st["ffn1"], world, dev)
-    # the fused decode kernel also does the combine: reads y_perm, writes out
-    es = 2 if wl.dtype == "bf16" else 4
-    comb_bytes = wl.T * wl.k * wl.H * es + wl.T * wl.H * es
-    dom = {"bytes": fc1_work["bytes"] + fc2_work["bytes"] + comb_bytes,
-           "flops": fc1_work["flops"] + fc2_work["flops"]} if fused else fc1_work
     one_launch = bool(path & 32)
+    es = 2 if wl.dtype == "bf16" else 4
+    # the dominant kernel: the fused decode FFN (fc1 + SwiGLU, fc2 and the combine in one
+    # launch; one-launch decode: also the routing), else fc1 + SwiGLU
+    dom = fc1_work
+    if fused:
+        comb_bytes = wl.T * wl.k * wl.H * es + wl.T * wl.H * es
+        dom = {"bytes": fc1_work["bytes"] + fc2_work["bytes"] + comb_bytes,
+               "flops": fc1_work["flops"] + fc2_work["flops"]}
     if one_launch:
-        # ... and the routing: router weights and the token rows, the logits
         dom = {"bytes": dom["bytes"] + wl.E * wl.H * es + wl.T * wl.H * es + wl.T * wl.E * 4,
                "flops": dom["flops"] + 2.0 * wl.T * wl.H * wl.E}
+    dom_ms_events = max_over_ranks(st["ffn1"], world, dev)
+    # an event on each side cuts the launch overlap with the neighbouring kernels, so the
+    # bracketed time can exceed the step's share; the kernel never takes longer than the
+    # step it is part of
+    dom_ms = min(dom_ms_events, ms_step)
 
     peaks, peak_kind = load_peaks()
     hbm = wl.name in HBM_BOUND
@@ -540,20 +620,36 @@ def run_ours(args):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
         achieved = dom["flops"] / (dom_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    if not hbm:
+        roof["peak_sustained"] = peaks["bf16_tflops_sustained"]
+        roof["frac_sustained"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
+    if wl.dtype != "bf16":
+        roof["note"] = ("float32 on the FMA pipes, launch-latency bound at this size: neither "
+                        "roofline is reachable; HBM fraction reported for reference")
     roof["kernel"] = ("tc_ffn_decode_kernel<ROUTE> (routing, fc1 + SwiGLU, fc2 and combine, weight rows on M)"
                       if one_launch else
                       "tc_ffn_decode_kernel (fc1 + SwiGLU, fc2 and combine, weight rows on M)" if fused else
-                      "tc_pair_kernel<SWIGLU> (fc1 + SwiGLU on CTA pairs, weight rows on M)")
+                      "tc_pair_kernel<SWIGLU> (fc1 + SwiGLU on CTA pairs, weight rows on M)"
+                      if wl.dtype == "bf16" else "ffn_simt fc1 + SwiGLU (float32 FMA)")
+    if opts.q8 is not None:
+        roof["kernel"] = ("tc_ffn_decode_kernel<Q8> (int8 weights converted to bf16, fc1 + "
+                          "SwiGLU, fc2 and combine, weight rows on M)")
     roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if hbm else 'bf16_tflops, burst'})"
     roof["algorithmic_per_launch"] = dom["bytes"] if hbm else dom["flops"]
     roof["kernel_us"] = round(dom_ms * 1e3, 2)
-    roof["traffic"] = kernel_traffic(wl.name, kernel_source(fused))
-    if args.q8:
-        roof["kernel"] = ("tc_ffn_decode_kernel<Q8> (int8 weights converted to bf16 in shared "
-                          "memory, fc1 + SwiGLU, fc2 and combine, weight rows on M)")
-        roof["traffic"] = None   # the committed counters are the bf16 kernel's
+    roof["kernel_us_events"] = round(dom_ms_events * 1e3, 2)
+    roof["traffic"] = None if opts.q8 is not None or wl.dtype != "bf16" else \
+        kernel_traffic(wl.name, kernel_source(fused))
+    if not fused and wl.dtype == "bf16":
+        # the second grouped GEMM of the prefill path, for reference
+        fc2_ms = max_over_ranks(st["ffn2"], world, dev)
+        roof["fc2"] = {"kernel": "tc_pair_kernel<plain> (fc2 on CTA pairs)",
+                       "achieved": fc2_work["flops"] / (fc2_ms * 1e-3) / 1e12,
+                       "frac": fc2_work["flops"] / (fc2_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                       "kernel_us": round(fc2_ms * 1e3, 2)}
 
     layer_s = ms_step * 1e-3
     layer = {"GB/s": layer_work["bytes"] / layer_s / 1e9, "TFLOP/s": layer_work["flops"] / layer_s / 1e12,
@@ -567,13 +663,13 @@ def run_ours(args):
     h_host.copy_(hidden)
     o_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     d_in = torch.empty_like(hidden)
-    n_e2e = args.e2e_steps
+    io_bytes = 2 * h_host.numel() * h_host.element_size()
+    est_s = layer_s + io_bytes / 25e9
+    n_e2e = int(max(3, min(200, args.e2e_seconds / est_s)))
     with torch.cuda.stream(stream):
-        for i in range(3):
+        for i in range(2):
             d_in.copy_(h_host, non_blocking=True)
-            run_layer(d_in, i,
-                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
-                        **ffn_kw)
+            call(d_in, i)
             o_host.copy_(out, non_blocking=True)
             stream.synchronize()
         if world > 1:
@@ -581,9 +677,7 @@ def run_ours(args):
         t0 = time.perf_counter()
         for i in range(n_e2e):
             d_in.copy_(h_host, non_blocking=True)
-            run_layer(d_in, i,
-                        normalize=bool(wl.normalize), router_bias=bias, out=out, workspace=ws,
-                        **ffn_kw)
+            call(d_in, i)
             o_host.copy_(out, non_blocking=True)
             stream.synchronize()
         e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
@@ -593,29 +687,101 @@ def run_ours(args):
 
     st_err, bits = moe.get_error(moe.workspace_error_word(ws), stream)
     if st_err != 0:
-        raise SystemExit(f"device error word {bits} after the bench")
+        raise SystemExit(f"{wl.name}: device error word {bits} after the bench")
 
-    line = {
-        "metric": METRIC, "value": job_throughput(wl.T, world, ms_step), "unit": "tokens/s",
-        "n_gpus": world, "steps": steps, "warmup": warm_reps * S, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+    row = {
+        "value": job_throughput(wl.T, world, ms_step), "unit": "tokens/s",
+        "steps": steps, "warmup": max(warmup, sets), "ms_per_step": ms_step,
         "config": dict(workload_config(wl, sets), parallelism=f"replicas x{world}",
-                       graph_steps=S, swiglu=list(act), expert_bias=bool(args.expert_bias),
-                       pre_norm=bool(args.pre_norm), q8=bool(args.q8), fc1_layout_read=layout),
+                       graph_steps=S),
         "roofline": roof, "layer": layer,
         "stages_us": {n: round(v * 1e3, 2) for n, v in st.items()},
-        "stages_note": "second timed region, same steps with stage events between kernels",
-        "e2e": e2e, "clocks": clk,
+        "e2e": e2e,
         "gpu_launches": int(round(launches_per_step * steps)),
+        "_timed_host": (h0, h1),
     }
+    del graph, graph_ev, weight_sets, ws, out, hidden, d_in, h_host, o_host
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return row
+
+
+def run_ours(args):
+    from synth import WORKLOADS
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    head = WORKLOADS[args.workload]
+    if args.q8 and head.name not in HBM_BOUND:
+        raise SystemExit("--q8: the int8 experts run in the decode FFN only (decode workloads)")
+    names = [head.name]
+    if not args.no_per_config and not variant_flags(args):
+        names += [n for n in ORDER if n != head.name]
+
+    # host inputs and the CPU baseline's worker processes, before the first CUDA call
+    inputs = host_inputs(names, q8=args.q8)
+    opts = {n: LayerOptions(args, WORKLOADS[n]) for n in names}
+    cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_cost(wl, inp, args.cpu_seconds, pre, q8_host)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+        cpu = CpuBaseline({n: (WORKLOADS[n], inputs[n], opts[n]) for n in names})
+
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    rows = {}
+    try:
+        for n in names:
+            wl = WORKLOADS[n]
+            is_head = n == head.name
+            steps = DEFAULT_STEPS.get(n, 100)
+            warmup = DEFAULT_WARMUP.get(n, 3)
+            if is_head:
+                steps = args.steps if args.steps is not None else steps
+                warmup = args.warmup if args.warmup is not None else warmup
+            rows[n] = measure(wl, inputs[n], opts[n], args, steps, warmup, world, dev, clocks)
+    finally:
+        clocks.stop()
+    for n in names:
+        rows[n]["clocks"] = clocks.summary(*rows[n].pop("_timed_host"))
+    if cpu is not None:
+        try:
+            for n in names:
+                secs = args.cpu_seconds if n == head.name else args.per_config_cpu_seconds
+                rows[n]["cpu_baseline"] = cpu.measure(n, secs)
+        finally:
+            cpu.close()
+
+    h = rows[head.name]
+    line = {
+        "metric": METRIC, "value": h["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": h["steps"], "warmup": h["warmup"], "ms_per_step": h["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if head.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": dict(h["config"], swiglu=list(opts[head.name].act),
+                       expert_bias=bool(args.expert_bias), pre_norm=bool(args.pre_norm),
+                       q8=bool(args.q8), fc1_layout_read=(
+                           "interleaved" if args.fc1_convert else head.fc1_layout)),
+        "roofline": h["roofline"], "layer": h["layer"], "stages_us": h["stages_us"],
+        "stages_note": "second timed region, same steps with stage events between kernels",
+        "e2e": h["e2e"], "clocks": h["clocks"], "gpu_launches": h["gpu_launches"],
+    }
+    if "cpu_baseline" in h:
+        line["cpu_baseline"] = h["cpu_baseline"]
+    if len(names) > 1:
+        line["per_config"] = {
+            n: {k: rows[n][k] for k in ("value", "unit", "ms_per_step", "steps", "warmup",
+                                        "config", "roofline", "layer", "stages_us", "e2e",
+                                        "clocks", "gpu_launches", "cpu_baseline") if k in rows[n]}
+            for n in names[1:]}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_ev
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -65,3 +65,47 @@ def test_algorithmic_bytes_of_the_variants():
     assert fc2["bytes"] - q2["bytes"] == 28 * H * I - 28 * H * 4
     assert layer["bytes"] - q8["bytes"] == 28 * 3 * H * I - 28 * (2 * I + H) * 4
     assert q8["flops"] == layer["flops"]
+
+
+def test_graph_steps_divide_the_step_count():
+    import bench
+    for limit in (1, 2, 20):
+        for steps in (1, 5, 20, 37, 100, 4000):
+            s = bench.graph_steps(limit, steps)
+            assert 1 <= s <= limit and steps % s == 0
+
+
+def test_workloads_with_the_same_expert_shapes_share_one_weight_draw():
+    import numpy as np
+
+    import bench
+    from synth import WORKLOADS, Workload, make_inputs
+    a = Workload("wa", T=8, H=64, E=4, k=2, I=32, dtype="bf16")
+    b = Workload("wb", T=16, H=64, E=4, k=2, I=32, dtype="bf16", fc1_layout="chunked")
+    WORKLOADS.update(wa=a, wb=b)
+    try:
+        got = bench.host_inputs(["wa", "wb"])
+    finally:
+        del WORKLOADS["wa"], WORKLOADS["wb"]
+    assert got["wa"]["fc1"] is got["wb"]["fc1"]
+    np.testing.assert_array_equal(got["wb"]["fc1"], make_inputs(b)["fc1"])
+    np.testing.assert_array_equal(got["wb"]["hidden"], make_inputs(b)["hidden"])
+
+
+def test_cpu_baseline_one_thread_and_all_cores():
+    import argparse
+
+    import bench
+    from synth import WORKLOADS
+    wl = WORKLOADS["tiny_fp32"]
+    args = bench.parse_args([])
+    inputs = bench.host_inputs([wl.name])
+    cpu = bench.CpuBaseline({wl.name: (wl, inputs[wl.name], bench.LayerOptions(args, wl))})
+    try:
+        r = cpu.measure(wl.name, 0.3)
+    finally:
+        cpu.close()
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    if r["cores"] > 1:
+        assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
+    del argparse
