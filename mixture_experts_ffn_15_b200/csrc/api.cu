@@ -58,11 +58,15 @@ struct Carver {
 };
 
 struct FwdLayout {
-    size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, ctr, x_perm,
-        act, y, xn, total;
+    size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, perm_pair,
+        ctr, x_perm, act, y, xn, total;
 };
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+int forward_path(int T, int H, int E, int k, int I, moe_dtype dt);
+constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
+              kPathF32Ffn = 16, kPathFusedRoute = 32;
 
 FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     const size_t es = elem_size(dt);
@@ -83,7 +87,10 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     L.offsets = c.take(static_cast<size_t>(E + 1) * 4);
     L.perm_src = c.take(rows * 4);
     L.perm_dst = c.take(rows * 4);
-    L.x_perm = c.take(rows * H * es);
+    L.perm_pair = c.take(rows * 4);
+    // the bf16 token-row GEMMs gather their rows from hidden: no permuted copy
+    const bool gathers = dt == MOE_BF16 && (forward_path(T, H, E, k, I, dt) & kPathTokenGemm);
+    L.x_perm = c.take(gathers ? 0 : rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
     L.xn = c.take(static_cast<size_t>(T) * H * es);   // the normalised input (pre-FFN norm)
@@ -140,9 +147,8 @@ FfnAttrs make_ffn_attrs(const moe_swiglu& a, moe_fc1_layout layout, const void* 
     return ep;
 }
 
-// Which kernels moe_forward runs for these sizes (bits of moe_forward_path).
-constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
-              kPathF32Ffn = 16, kPathFusedRoute = 32;
+// Which kernels moe_forward runs for these sizes (bits of moe_forward_path, declared
+// above).
 // Up to this many tokens a bf16 batch is routed by the split router + one CTA; above
 // it, by the tensor-core router with the routing in its epilogue.
 constexpr int kRouteSmallTcT = 16;
@@ -414,6 +420,7 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
     int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
     int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
     int32_t* perm_dst = reinterpret_cast<int32_t*>(ws + L.perm_dst);
+    int32_t* perm_pair = reinterpret_cast<int32_t*>(ws + L.perm_pair);
     void* x_perm = ws + L.x_perm;
     void* act_buf = ws + L.act;
     void* y = ws + L.y;
@@ -432,6 +439,9 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
+    // the bf16 token-row GEMMs gather their token rows from hidden and write y in token
+    // order (pair (t, j) at row t k + j), which the combine then reads row block by block
+    const bool pair_gemm_path = bf16 && (path & kPathTokenGemm);
     record(0, s);
     // The first launch zeroes what must start at zero (the error word, the decode-FFN
     // counters, the tile counts; the split router of the small-route path clears the
@@ -500,6 +510,7 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         a.offsets = offsets;
         a.perm_src = perm_src;
         a.perm_dst = perm_dst;
+        if (pair_gemm_path) a.perm_pair = perm_pair;
         if (path & kPathDecodeFfn) {
             a.zero_words = ctr;
             a.n_zero = decode_ffn_counters(rows, E);
@@ -530,7 +541,7 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         }
         record(1, s);
         MOE_CUDA(launch_scatter(idx, tile_counts, T, E, k, counts, offsets, perm_src, perm_dst,
-                                err, s));
+                                err, s, pair_gemm_path ? perm_pair : nullptr));
     }
     if (path & kPathDecodeFfn) {
         // fc1 + SwiGLU and fc2 in one launch.  With at most 4 rows per expert on
@@ -551,22 +562,25 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         record(5, s);
         return MOE_OK;
     } else {
-        MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
-                               static_cast<int>(elem_size(dt)), x_perm, s));
-        record(2, s);
         cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
-        if (bf16)
-            MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
-                                     mid, ep));
-        else
+        if (pair_gemm_path) {
+            // fc1 gathers the token rows from hidden itself (no x_perm)
+            record(2, s);
+            MOE_CUDA(launch_ffn_pair(hidden, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
+                                     mid, ep, perm_src, T, perm_pair));
+        } else {
+            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
+                                   static_cast<int>(elem_size(dt)), x_perm, s));
+            record(2, s);
             MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                          static_cast<const float*>(fc1),
                                          static_cast<const float*>(fc2), rows, H, E, I,
                                          static_cast<float*>(act_buf), static_cast<float*>(y), s,
                                          mid, ep));
+        }
     }
     record(4, s);
-    MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));
+    MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s, pair_gemm_path));
     record(5, s);
     return MOE_OK;
 }

@@ -187,6 +187,33 @@ def test_forward(wl):
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} output")
 
 
+def test_gathering_token_gemms_equal_the_staged_calls_bit_for_bit():
+    """The layer's large-batch path gathers fc1's token rows from hidden (tile::gather4)
+    and writes fc2's rows in token order for the combine; the staged calls run the same
+    GEMM kernels on the permuted copy x_perm and write y in permuted order.  Same
+    routing (the tensor-core router in both), same arithmetic: the same bits.  A skewed
+    router gives experts of every size, so token tiles end at every offset."""
+    from mixture_experts_ffn_15_b200 import _abi
+    wl = W("gather_pairs", T=1500, H=256, E=64, k=4, I=192, router_bias_std=1.0)
+    assert moe.load_library().moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, _abi.MOE_BF16) & 8
+    inp = make_inputs(wl)
+    dev = device_inputs(inp)
+    out = moe.forward(dev["hidden"], dev["router_w"], dev["fc1"], dev["fc2"], wl.k,
+                      router_bias=dev["router_bias"])
+    r = run_route(dev, wl)
+    p = moe.permute(r["idx"], wl.E, hidden=dev["hidden"])
+    y = moe.expert_ffn(p["x_perm"], p["offsets"], dev["fc1"], dev["fc2"])
+    staged = moe.combine(y, p["perm_dst"], r["w"], wl.T, wl.k)
+    torch.cuda.synchronize()
+    counts = from_dev(p["counts"])
+    assert counts.min() < 32 and counts.max() > 256       # ragged tiles of every kind
+    assert torch.equal(out.view(torch.int16), staged.view(torch.int16))
+    L, idx = check_routing(inp, r)
+    ref = oracle_forward(inp, idx)["out"]
+    atol, rtol = tol(wl.dtype, ref)
+    assert_close(from_dev(out), ref, atol, rtol, "gathered token GEMMs")
+
+
 # ------------------------------------------- SwiGLU attributes and expert biases
 # The op's activation_alpha / activation_beta / swiglu_limit ("Attribute set") and its
 # optional fc1/fc2 expert biases, on every path of moe_forward.  limit 1.0 clips most
