@@ -397,6 +397,200 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
 }
 
+// ------------------------------------------------------------------------ split-K router
+// Router logits and routing for a few 128-token tiles (batched decode, mid-sized
+// prefill), where one CTA per tile would stream the whole K range alone.  A cluster of
+// CS CTAs runs one tile: CTA r accumulates the K slices [r nk / CS, (r + 1) nk / CS) on
+// the tensor cores (128 tokens on M, all E experts on N) and stores its partial logits
+// in its own shared memory.  After a cluster barrier, CTA r takes the rows
+// r 128 / CS .. of the tile, sums the CS partials of each logit in rank order 0 .. CS-1
+// through distributed shared memory (a fixed order: the logits do not depend on timing)
+// and routes the row with the warp top-k that the single-CTA router uses.  No global
+// scratch; the host picks this kernel by (T, H, E) alone, for the staged router and the
+// layer alike, so both return the same bits.
+constexpr int kSplitPad = 1;   // partials stored [e][row] with a row stride of 129 floats
+
+template <int E>
+struct SplitCfg {
+    static constexpr int kABytes = BM * BK * 2;                 // 128 token rows x 64 K
+    static constexpr int kBBytes = E * BK * 2;                  // E router rows x 64 K
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kPartBytes = E * (BM + kSplitPad) * 4;
+    static constexpr int kStagesFit = (200 * 1024 - kPartBytes) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
+    static constexpr int kRowBytes = (kThreads / 32) * E * 4;   // one logits row per warp
+    // barriers (full, empty: kStages each; tfull), then the TMEM slot and the abort flag
+    static constexpr int kMiscBytes = (2 * kStages + 1) * 8 + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPartBytes + kRowBytes + kMiscBytes;
+    static constexpr int kTmemCols = E;                         // 64 or 128
+    static_assert(kStages >= 2, "pipeline");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+template <int E, int CS>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const TcParams p, const RouteParams rp) {
+    using C = SplitCfg<E>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::kStages * C::kABytes;
+    float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM + pad]
+    float* rowbuf = part + E * (BM + kSplitPad);                            // [warps][E]
+    uint64_t* full = reinterpret_cast<uint64_t*>(rowbuf + (kThreads / 32) * E);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* tfull = empty + C::kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int tile = static_cast<int>(blockIdx.x) / CS;
+    const int nk = p.K / BK;
+    const int kb0 = nk * rank / CS, kb1 = nk * (rank + 1) / CS;   // CS <= nk: never empty
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        mbar_init(smem_u32(tfull), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    // the prologue above touches no global memory; everything below may
+    pdl_wait();
+    pdl_trigger();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
+                const uint32_t fb = smem_u32(&full[stage]);
+                mbar_arrive_expect_tx(fb, C::kStageBytes);
+                tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * BK, tile * BM);
+                tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * BK, 0);
+                ++issued;
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (*abort_flag) {
+                // let the copies already in flight land before the CTA goes on
+                int dummy = 0;
+                for (int s2 = 0; s2 < C::kStages; ++s2) {
+                    if (issued <= s2) break;
+                    const long long fills = (issued - 1 - s2) / C::kStages + 1;
+                    mbar_wait(smem_u32(&full[s2]), static_cast<uint32_t>((fills - 1) & 1), &dummy,
+                              kWaitLimitNs / 4);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, E);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    umma_bf16(tmem_base, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                              idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                umma_commit(smem_u32(&empty[stage]));
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) umma_commit(smem_u32(tfull));
+        }
+    } else {
+        // ------------------------------------------------------------ partials
+        // warps 2..5: TMEM lane quadrant warp % 4; thread = token row r of the tile
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        if (mbar_wait(smem_u32(tfull), 0, abort_flag, kWaitLimitNs)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < E; c += 32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) part[(c + i) * (BM + kSplitPad) + r] = __uint_as_float(v[i]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();   // every CTA's partials are written and visible to the cluster
+
+    // ---------------------------------------------------------------- reduce and route
+    constexpr int kRowsPerCta = BM / CS;
+    float* mine = rowbuf + warp * E;
+#pragma unroll 1
+    for (int i = warp; i < kRowsPerCta; i += kThreads / 32) {
+        const int r = rank * kRowsPerCta + i;
+        const size_t row = static_cast<size_t>(tile) * BM + r;
+        const bool valid = row < static_cast<size_t>(p.rows);
+#pragma unroll
+        for (int e = lane; e < E; e += 32) {
+            const uint32_t a = smem_u32(&part[e * (BM + kSplitPad) + r]);
+            float sum = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) sum += ld_shared_cluster_f32(mapa_shared(a, q));
+            mine[e] = sum;
+            if (valid && rp.logits) rp.logits[row * E + e] = sum + (rp.bias ? rp.bias[e] : 0.f);
+        }
+        __syncwarp();
+        if (valid) {
+            const WarpTopk res = warp_topk(mine, rp.bias, E, rp.k, rp.normalize, lane);
+            if (lane < rp.k) {
+                rp.topk_idx[row * rp.k + lane] = res.idx;
+                rp.topk_w[row * rp.k + lane] = res.w;
+                if (rp.tile_counts && static_cast<unsigned>(res.idx) < static_cast<unsigned>(E))
+                    atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + res.idx], 1);
+            }
+            if (lane == 0 && rp.near_tie) rp.near_tie[row] = res.flags;
+        }
+        __syncwarp();
+    }
+    cluster_sync();   // no CTA leaves while a peer may still read its partials
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
+}
+
 // ------------------------------------------------------------------------ decode FFN
 // fc1 + SwiGLU and fc2 for batches with few rows per expert, in ONE persistent
 // launch.  Both GEMMs put 128 weight rows on the MMA's M side and the expert's tokens
@@ -1204,6 +1398,49 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParam
     return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p, rp);
 }
 
+// Cluster size of the split-K router for these sizes (1: the one-CTA-per-tile router).
+// A pure function of the sizes (a fixed budget of 148 CTAs, not the device's count), so
+// that the staged router and the layer take the same kernel and give the same bits.
+int route_split_cluster(int T, int H, int E) {
+    if (E != 64 && E != 128) return 1;
+    const int tiles = (T + BM - 1) / BM, nk = H / BK;
+    for (int cs = 8; cs >= 2; cs >>= 1)
+        if (tiles * cs <= 148 && cs <= nk) return cs;
+    return 1;
+}
+
+template <int E, int CS>
+cudaError_t launch_route_split(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p,
+                               const RouteParams& rp, int tiles, cudaStream_t s) {
+    using C = SplitCfg<E>;
+    auto kern = tc_route_split_kernel<E, CS>;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * CS));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, kern, a, b, p, rp);
+}
+
 // Grid of a persistent decode FFN launch: every unit of both GEMMs, at most one CTA per SM.
 int decode_grid(int rows, int E, int H, int I) {
     const long long units =
@@ -1251,6 +1488,16 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
     CUtensorMap ma, mb;
     if (!tmap::matrix(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
     if (!tmap::matrix(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
+    const int cs = route_split_cluster(T, H, E);
+    const int tiles = (T + BM - 1) / BM;
+    if (cs > 1) {
+#define MOE_SPLIT_CASE(EV, CV) \
+    if (E == EV && cs == CV) return launch_route_split<EV, CV>(ma, mb, p, rp, tiles, s);
+        MOE_SPLIT_CASE(64, 2) MOE_SPLIT_CASE(64, 4) MOE_SPLIT_CASE(64, 8)
+        MOE_SPLIT_CASE(128, 2) MOE_SPLIT_CASE(128, 4) MOE_SPLIT_CASE(128, 8)
+#undef MOE_SPLIT_CASE
+        return cudaErrorInvalidValue;
+    }
     const int bound = (T + BM - 1) / BM;
     const bool small_k = k <= 8;
 #define MOE_ROUTE_CASE(EV)                                                                   \
