@@ -64,7 +64,6 @@ struct FwdLayout {
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 
-int forward_path(int T, int H, int E, int k, int I, moe_dtype dt);
 constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
               kPathF32Ffn = 16, kPathFusedRoute = 32;
 
@@ -88,9 +87,9 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     L.perm_src = c.take(rows * 4);
     L.perm_dst = c.take(rows * 4);
     L.perm_pair = c.take(rows * 4);
-    // the bf16 token-row GEMMs gather their rows from hidden: no permuted copy
-    const bool gathers = dt == MOE_BF16 && (forward_path(T, H, E, k, I, dt) & kPathTokenGemm);
-    L.x_perm = c.take(gathers ? 0 : rows * H * es);
+    // every bf16 path gathers its token rows from hidden: only the float32 path keeps a
+    // permuted copy
+    L.x_perm = c.take(dt == MOE_BF16 ? 0 : rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
     L.xn = c.take(static_cast<size_t>(T) * H * es);   // the normalised input (pre-FFN norm)
@@ -544,19 +543,12 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
                                 err, s, pair_gemm_path ? perm_pair : nullptr));
     }
     if (path & kPathDecodeFfn) {
-        // fc1 + SwiGLU and fc2 in one launch.  With at most 4 rows per expert on
-        // average, fc1 gathers its token rows straight from hidden (one TMA row box
-        // each); with more, the rows are gathered once into x_perm and loaded in
-        // 16-row boxes.
-        const bool tma_gather = rows <= 4 * E;
-        if (!tma_gather)
-            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
-                                   static_cast<int>(elem_size(dt)), x_perm, s));
+        // fc1 + SwiGLU and fc2 in one launch; fc1 gathers its token rows straight from
+        // hidden (tile::gather4, four rows per load) ...
         record(2, s);
         // ... and the weighted combine, after every fc2 unit has published its rows
-        MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
-                                   T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err,
-                                   perm_dst, w, k, out, s, ep));
+        MOE_CUDA(launch_ffn_decode(hidden, perm_src, T, offsets, fc1, fc2, rows, H, E, I, act_buf,
+                                   y, ctr, err, perm_dst, w, k, out, s, ep));
         record(3, s);
         record(4, s);
         record(5, s);

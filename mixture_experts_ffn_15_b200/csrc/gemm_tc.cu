@@ -604,8 +604,8 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
 // fence and a release increment of the chunk's counter, and the fc2 producer waits
 // (bounded) for 4 x (fc1 units per chunk) increments with an acquire load before
 // loading the activations with TMA.  The fc2 weights of a unit do not depend on fc1.
-// With GATHER, fc1's token rows come straight from `hidden` through perm_src (one TMA
-// box of one row each); otherwise from contiguous rows of x_perm (16-row boxes).
+// With GATHER, fc1's token rows come straight from `hidden` through perm_src (four rows
+// per tile::gather4 load); otherwise from contiguous rows of x_perm (16-row boxes).
 // With `out`, the kernel also does the weighted combine: once every fc2 unit has
 // published its rows (a grid-wide count, acquire), the epilogue warps of all CTAs
 // split the output vectors among themselves, with the same arithmetic as
@@ -1033,21 +1033,24 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const CUtensorMap* ma = f1 ? &tmW1 : &tmW2;
             const int nl = (d.nrows + kBoxTok - 1) / kBoxTok;
             uint32_t bbytes = static_cast<uint32_t>(nl * kBoxTok * BK * 2);
-            int src[2] = {0, 0};   // this lane's gathered token rows: lane, lane + 32
+            // gathered token rows: lane < nl4 loads rows 4 lane .. 4 lane + 3 of the chunk
+            // (one tile::gather4 load; rows past the chunk repeat its last row)
+            const int nl4 = (d.nrows + 3) / 4;
+            int src[4] = {0, 0, 0, 0};
             if (f1 && GATHER) {
+                if (lane < nl4) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int i = lane + 32 * h;
-                    if (i < d.nrows) {
-                        int t = ROUTE ? s_psrc[d.row0 + i] : p.perm_src[d.row0 + i];
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = d.row0 + min(4 * lane + i, d.nrows - 1);
+                        int t = ROUTE ? s_psrc[r] : p.perm_src[r];
                         if (t < 0 || t >= p.T) {
                             atomicOr(p.err, kErrBadExpert);
                             t = 0;
                         }
-                        src[h] = t;
+                        src[i] = t;
                     }
                 }
-                bbytes = static_cast<uint32_t>(d.nrows * BK * 2);
+                bbytes = static_cast<uint32_t>(nl4 * 4 * BK * 2);
             }
             if (!f1) {
                 bool ok = true;
@@ -1069,11 +1072,9 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
                 if (!Q8 && lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
                 if (f1 && GATHER) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int i = lane + 32 * h;
-                        if (i < d.nrows) tma_load_2d(b_dst + i * BK * 2, &tmX, fb, kb * BK, src[h]);
-                    }
+                    if (lane < nl4)
+                        tma_gather4(b_dst + lane * 4 * BK * 2, &tmX, fb, kb * BK, src[0], src[1],
+                                    src[2], src[3]);
                 } else if (lane < nl) {
                     tma_load_2d(b_dst + lane * kBoxTok * BK * 2, f1 ? &tmX : &tmAct, fb, kb * BK,
                                 d.row0 + lane * kBoxTok);

@@ -82,7 +82,10 @@ def test_status_strings_and_version():
 
 def test_workspace_sizes():
     lib = _lib()
-    assert lib.moe_workspace_size(4, 2816, 128, 8, 704, _abi.MOE_BF16) > 4 * 8 * (2 * 2816 + 704) * 2
+    # bf16: act and y_perm (every bf16 path gathers its token rows from hidden); float32
+    # also keeps the permuted copy x_perm
+    assert lib.moe_workspace_size(4, 2816, 128, 8, 704, _abi.MOE_BF16) > 4 * 8 * (2816 + 704) * 2
+    assert lib.moe_workspace_size(4, 2816, 128, 8, 704, _abi.MOE_F32) > 4 * 8 * (2 * 2816 + 704) * 4
     assert lib.moe_workspace_size(4, 2816, 128, 300, 704, _abi.MOE_BF16) == 0     # k > E
     assert lib.moe_workspace_size(4, 2816, 300, 8, 704, _abi.MOE_BF16) == 0       # E > 256
     assert lib.moe_workspace_size(4, 2817, 128, 8, 704, _abi.MOE_BF16) == 0       # H % 8
