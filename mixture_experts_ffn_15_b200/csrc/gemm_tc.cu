@@ -615,22 +615,26 @@ constexpr int kUnitRing = 4;
 
 // Weight-only int8 experts (Q8): the weights stream from HBM as int8 through a deep ring
 // of their own (kQStages tiles of 128 rows x 64 bytes, loaded by a dedicated producer
-// warp), converter warps write each tile as bf16 -- exact, |q| <= 127 -- into the
-// 128-byte-swizzled layout of the bf16 path (two groups of four warps taking alternate
-// k-steps, so that two tiles convert at once), and the epilogue multiplies each weight
-// row's accumulator by its float32 scale.  The MMA and the token side are unchanged.
+// warp); converter warps turn each tile into bf16 -- exact, |q| <= 127 -- and store it
+// straight into tensor memory, where the MMA reads its A operand (two groups of four
+// warps taking alternate k-steps, so that two tiles convert at once); shared memory
+// carries only int8 weights and token rows.  The epilogue multiplies each weight row's
+// accumulator by its float32 scale.  The token side is the bf16 path's.
 constexpr int kQBytes = BM * BK;   // one int8 tile: 128 weight rows x 64 K
 
 template <bool Q8>
 struct DecodeCfg {
     using T = Tr<W_PLAIN, 64>;
-    static constexpr int kABytes = T::kABytes;
+    static constexpr int kABytes = Q8 ? 0 : T::kABytes;     // Q8: A lives in tensor memory
     static constexpr int kBBytes = T::kBBytes;
-    static constexpr int kStages = Q8 ? 7 : T::kStages;     // bf16 A + token B ring
-    static constexpr int kQStages = Q8 ? 6 : 0;             // int8 weight ring
+    static constexpr int kStages = T::kStages;              // A (smem or TMEM) + token B ring
+    static constexpr int kQStages = Q8 ? 16 : 0;            // int8 weight ring
     static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
     static constexpr int kAccStride = T::kAccStride;
-    static constexpr int kTmemCols = T::kTmemCols;
+    // Q8: two accumulators (2 x 64 columns), then one A stage of 32 columns per ring stage
+    static constexpr int kTmemA = 2 * kAccStride;
+    static constexpr int kTmemCols = Q8 ? 512 : T::kTmemCols;
+    static_assert(!Q8 || kTmemA + kStages * 32 <= kTmemCols, "tensor memory");
     static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
     static constexpr int kMiscBytes = T::kMiscBytes + 2 * kQStages * 8;   // + int8 ring barriers
     static constexpr int kSmemBytes = 1024 + kDataBytes + kMiscBytes;
@@ -1130,10 +1134,19 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
                     const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+                    if constexpr (Q8) {
+                        // A: the converted stage in tensor memory, 8 columns per 16 K
+                        const uint32_t at = tmem_base + static_cast<uint32_t>(C::kTmemA + stage * 32);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                                  idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16_ta(d_tmem, at + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc,
+                                         (kb | kk) != 0);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                      smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                    }
                     umma_commit(smem_u32(&empty[stage]));
                     if (++stage == C::kStages) {
                         stage = 0;
@@ -1283,16 +1296,21 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         } else {
             // -------------------------------------------------------- int8 -> bf16
             // Group grp (warps 7-10, 11-14) converts the k-steps n with n % 2 == grp (n
-            // counts every k-step of the launch, as the rings do); its warp cw converts
-            // weight rows 32 cw .. 32 cw + 31 of the tile: per pass, 8
-            // rows x 64 bytes (512 contiguous bytes: one conflict-free warp load), each
-            // lane 16 int8 of one row -> 16 bf16 = two 16-byte chunks of the row's 128
-            // bytes, stored at the 128-byte swizzle position (chunk ^ (row & 7)).
+            // counts every k-step of the launch, as the rings do).  A warp owns the tensor
+            // memory lane quadrant warp % 4, i.e. weight rows 32 quad .. 32 quad + 31, one
+            // row per lane: the lane reads its row's 64 int8 (the tile lands with the
+            // 64-byte swizzle, logical 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3),
+            // so a warp's 32 rows read without bank conflicts), converts them to bf16 and
+            // writes the 32 packed pairs into the ring stage's A columns in tensor memory
+            // with one tcgen05.st.
             // int8 b -> float32 exactly: the bit pattern 0x4B000000 | (b ^ 0x80) is
             // 2^23 + 128 + b; subtracting 2^23 + 128 leaves b, whose float32 bits end in
             // 16 zero bits (|b| <= 128 has at most 8 significant bits), so its top half
             // is b in bf16.
-            const int cw = (warp - 7) & 3, grp = (warp - 7) >> 2;
+            const int quad = warp & 3, grp = (warp - 7) >> 2;
+            const int row = quad * 32 + lane;
+            const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                    static_cast<uint32_t>(C::kTmemA);
             int qs = 0, stage = 0, n = 0;
             uint32_t qphase = 0, phase = 0;
             for (;;) {
@@ -1319,15 +1337,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                     // the whole warp leaves together (lane 0 alone saw the wait give up)
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
-                    const uint8_t* q = sQ + qs * kQBytes;
-                    uint8_t* a = sA + stage * C::kABytes;
+                    tc_fence_after();   // the MMAs that read this A stage have completed
+                    const uint8_t* q = sQ + qs * kQBytes + row * BK;
+                    uint32_t h[32];
 #pragma unroll
-                    for (int pass = 0; pass < 4; ++pass) {
-                        const int row = cw * 32 + pass * 8 + (lane >> 2), c = lane & 3;
-                        const uint4 w = *reinterpret_cast<const uint4*>(q + row * BK + c * 16);
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(q + ((c ^ ((row >> 1) & 3)) << 4));
                         const uint32_t wb[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u,
                                                 w.z ^ 0x80808080u, w.w ^ 0x80808080u};
-                        uint32_t h[8];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             float f[4];
@@ -1335,17 +1352,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                             for (int b = 0; b < 4; ++b)
                                 f[b] = __uint_as_float(__byte_perm(wb[i], 0x4B000000u, b | 0x7540u)) -
                                        8388736.0f;   // 2^23 + 128
-                            h[2 * i] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
-                            h[2 * i + 1] = __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+                            h[c * 8 + 2 * i] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
+                            h[c * 8 + 2 * i + 1] =
+                                __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
                         }
-                        uint8_t* rowp = a + (row >> 3) * 1024 + (row & 7) * 128;
-                        *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) =
-                            make_uint4(h[0], h[1], h[2], h[3]);
-                        *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) =
-                            make_uint4(h[4], h[5], h[6], h[7]);
                     }
-                    // the bf16 tile is read by the tensor cores (async proxy)
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    tmem_st_32x32b_x32(a_lane + static_cast<uint32_t>(stage * 32), h);
+                    tmem_wait_st();
+                    tc_fence_before();   // ... before the MMA thread learns of it
                     __syncwarp();
                     if (lane == 0) {
                         mbar_arrive(smem_u32(&qempty[qs]));

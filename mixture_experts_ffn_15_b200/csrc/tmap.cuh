@@ -52,8 +52,9 @@ inline bool matrix(CUtensorMap* m, const void* ptr, long long rows, int K, int b
 //   plain [E, n, K] (fc2; fc1 interleaved: row 2i = gate_i, 2i+1 = up_i):
 //       s_stride 1, i_stride 2
 //   fc1 chunked [E, 2I, K] (row i = gate_i, I+i = up_i): s_stride I, i_stride 1
-//   int8 weights (u8 = true): one byte per element, no swizzle (the box is read by
-//       the converting warps, 64 bytes per row)
+//   int8 weights (u8 = true): one byte per element, 64-byte rows stored with the 64-byte
+//       swizzle (logical 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)), so that
+//       the converting warps read one row per lane without bank conflicts
 inline bool row_pairs(CUtensorMap* m, const void* w, int E, int n_pairs, int K, int box_pairs,
                       long long s_stride, long long i_stride, bool u8 = false) {
     EncodeTiledFn enc = encode_fn();
@@ -68,7 +69,7 @@ inline bool row_pairs(CUtensorMap* m, const void* w, int E, int n_pairs, int K, 
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                const_cast<void*>(w), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               u8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+               u8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
