@@ -592,8 +592,6 @@ def measure(wl, inp, opts, args, steps, warmup, world, dev, clocks):
         for a, n in enumerate(stage_names):
             st[n] += events[i][a].elapsed_time(events[i][a + 1]) / S
     path = lib.moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, 1 if wl.dtype == "bf16" else 0)
-    if opts.q8 is not None:
-        path &= ~32   # int8 experts: the decode FFN after the staged routing kernels
     fused = bool(path & 2)
     one_launch = bool(path & 32)
     es = 2 if wl.dtype == "bf16" else 4
@@ -635,8 +633,9 @@ def measure(wl, inp, opts, args, steps, warmup, world, dev, clocks):
                       "tc_pair_kernel<SWIGLU> (fc1 + SwiGLU on CTA pairs, weight rows on M)"
                       if wl.dtype == "bf16" else "ffn_simt fc1 + SwiGLU (float32 FMA)")
     if opts.q8 is not None:
-        roof["kernel"] = ("tc_ffn_decode_kernel<Q8> (int8 weights converted to bf16, fc1 + "
-                          "SwiGLU, fc2 and combine, weight rows on M)")
+        roof["kernel"] = ("tc_ffn_decode_kernel<Q8> (" + ("routing, " if one_launch else "") +
+                          "int8 weights converted to bf16 in tensor memory, fc1 + SwiGLU, fc2 "
+                          "and combine, weight rows on M)")
     roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if hbm else 'bf16_tflops, burst'})"
     roof["algorithmic_per_launch"] = dom["bytes"] if hbm else dom["flops"]
     roof["kernel_us"] = round(dom_ms * 1e3, 2)

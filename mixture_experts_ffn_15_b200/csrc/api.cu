@@ -166,9 +166,11 @@ int forward_path(int T, int H, int E, int k, int I, moe_dtype dt) {
     return path;
 }
 
-// int8 experts: the decode FFN with the staged routing (0: no such path for these sizes)
+// int8 experts: the decode FFN, with the routing inside its launch for small batches,
+// else after the staged routing kernels (0: no such path for these sizes)
 int forward_path_q8(int T, int H, int E, int k, int I) {
     const int rows = T * k;
+    if (fused_route_supported(T, H, E, k, I)) return kPathFusedRoute | kPathDecodeFfn;
     if (!decode_ffn_supported(rows, E, H, I)) return 0;
     if (T > kRouteSmallTcT && tc_route_supported(H, E, k)) return kPathTcRouter | kPathDecodeFfn;
     if (T <= kRouteSmallMaxT && k <= kRouteSmallMaxK) return kPathSmallRoute | kPathDecodeFfn;

@@ -688,7 +688,7 @@ constexpr int kRouteSmemBytes =
     4 * kFusedRouteMaxRows * 4 +                  // ids, weights, perm_dst, perm_src
     kMaxExperts * 4 + (kMaxExperts + 4) * 4 +     // counts, offsets
     kMaxExperts * (kFusedRouteMaxT / 32) * 4 +    // token masks per expert
-    (kThreads / 32) * 8 * 4;                      // partial dot products
+    16 * 8 * 4;                                   // partial dot products (<= 16 warps)
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
     int v;
@@ -753,7 +753,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                      const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmAct,
                      const DecodeParams p) {
     using C = DecodeCfg<Q8>;
-    static_assert(!(Q8 && ROUTE), "the int8 path takes its routing from the staged kernels");
+    static_assert(C::kThreads <= 16 * 32, "partial dot products of the routing");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -841,11 +841,11 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
 #pragma unroll
                 for (int t = 0; t < 8; ++t) acc[t] = 0.f;
 #pragma unroll 1
-                for (int v0 = threadIdx.x; v0 < nv; v0 += kR1Vec * kThreads) {
+                for (int v0 = threadIdx.x; v0 < nv; v0 += kR1Vec * C::kThreads) {
                     uint4 wv[kR1Vec], xv[8][kR1Vec];
 #pragma unroll
                     for (int j = 0; j < kR1Vec; ++j) {
-                        const int v = v0 + j * kThreads;
+                        const int v = v0 + j * C::kThreads;
                         wv[j] = v < nv ? __ldg(w4 + v) : zero4;
 #pragma unroll
                         for (int t = 0; t < 8; ++t)
@@ -875,7 +875,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 if (threadIdx.x < 8 && t0 + static_cast<int>(threadIdx.x) < T) {
                     float sum = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kThreads / 32; ++w) sum += s_red[w * 8 + threadIdx.x];
+                    for (int w = 0; w < C::kThreads / 32; ++w) sum += s_red[w * 8 + threadIdx.x];
                     p.logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = sum;
                 }
                 __syncthreads();
@@ -899,27 +899,27 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         {
             // all loads first, then the shared-memory stores (one L2 latency)
             constexpr int kR3Per = 8;
-            for (int i0 = threadIdx.x; i0 < T * E; i0 += kR3Per * kThreads) {
+            for (int i0 = threadIdx.x; i0 < T * E; i0 += kR3Per * C::kThreads) {
                 float lv[kR3Per];
 #pragma unroll
                 for (int j = 0; j < kR3Per; ++j) {
-                    const int i = i0 + j * kThreads;
+                    const int i = i0 + j * C::kThreads;
                     lv[j] = i < T * E ? __ldcg(p.logits + i) : 0.f;
                 }
 #pragma unroll
                 for (int j = 0; j < kR3Per; ++j) {
-                    const int i = i0 + j * kThreads;
+                    const int i = i0 + j * C::kThreads;
                     if (i < T * E) s_log[i] = lv[j];
                 }
             }
         }
         const int words = (T + 31) / 32;
-        for (int i = threadIdx.x; i < E * words; i += kThreads) s_rmask[i] = 0;
-        for (int e = threadIdx.x; e < E; e += kThreads) s_rcnt[e] = 0;
+        for (int i = threadIdx.x; i < E * words; i += C::kThreads) s_rmask[i] = 0;
+        for (int e = threadIdx.x; e < E; e += C::kThreads) s_rcnt[e] = 0;
         __syncthreads();
         const bool lead = blockIdx.x == 0;
 #pragma unroll 1
-        for (int t = warp; t < T; t += kThreads / 32) {
+        for (int t = warp; t < T; t += C::kThreads / 32) {
             const WarpTopk r = warp_topk(s_log + t * E, p.bias, E, k, p.normalize, lane);
             if (lane < k) {
                 s_ridx[t * k + lane] = r.idx;
@@ -972,7 +972,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         }
         __syncthreads();
         // stable placement: the rank of t among the tokens of its expert
-        for (int q = threadIdx.x; q < T * k; q += kThreads) {
+        for (int q = threadIdx.x; q < T * k; q += C::kThreads) {
             const int e = s_ridx[q], t = q / k;
             int row = -1;
             if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
@@ -1602,12 +1602,13 @@ bool take_route_timeout_test() { return g_route_timeout_test.exchange(0) != 0; }
 cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) {
     const int rows = r.T * r.k;
     if (rows <= 0) return cudaSuccess;
-    if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I) || r.ep.q8()) return cudaErrorInvalidValue;
+    if (!fused_route_supported(r.T, r.H, r.E, r.k, r.I)) return cudaErrorInvalidValue;
+    const bool q8 = r.ep.q8();
     CUtensorMap w1, x, w2, a;
-    if (!tmap::fc1_pairs(&w1, r.fc1, r.E, r.I, r.H, BM / 2, r.ep.fc1_chunked))
+    if (!tmap::fc1_pairs(&w1, r.fc1, r.E, r.I, r.H, BM / 2, r.ep.fc1_chunked, q8))
         return cudaErrorInvalidValue;
     if (!tmap::matrix(&x, r.hidden, r.T, r.H, 1)) return cudaErrorInvalidValue;
-    if (!tmap::plain_pairs(&w2, r.fc2, r.E, r.H, r.I, BM / 2)) return cudaErrorInvalidValue;
+    if (!tmap::plain_pairs(&w2, r.fc2, r.E, r.H, r.I, BM / 2, q8)) return cudaErrorInvalidValue;
     if (!tmap::matrix(&a, r.act, rows, r.I, kBoxTok)) return cudaErrorInvalidValue;
     const int nctr = decode_ffn_counters(rows, r.E);
     DecodeParams p{};
@@ -1633,6 +1634,8 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     p.b1 = static_cast<const __nv_bfloat16*>(r.ep.fc1_bias);
     p.fc1_chunked = r.ep.fc1_chunked;
     p.b2 = static_cast<const __nv_bfloat16*>(r.ep.fc2_bias);
+    p.s1 = r.ep.fc1_scale;
+    p.s2 = r.ep.fc2_scale;
     p.hidden = r.hidden;
     p.router_w = r.router_w;
     p.bias = r.bias;
@@ -1646,7 +1649,8 @@ cudaError_t launch_ffn_decode_routed(const DecodeRoutedArgs& r, cudaStream_t s) 
     p.r_perm_src = r.perm_src;
     p.r_perm_dst = r.perm_dst;
     const int grid = decode_grid(rows, r.E, r.H, r.I);
-    return launch_decode<true, true>(w1, x, w2, a, p, grid, s);
+    return q8 ? launch_decode<true, true, true>(w1, x, w2, a, p, grid, s)
+              : launch_decode<true, true>(w1, x, w2, a, p, grid, s);
 }
 
 }  // namespace moe

@@ -205,8 +205,8 @@ struct DecodeRoutedArgs {
     const void* hidden;        // [T, H] bf16
     const void* router_w;      // [E, H] bf16
     const float* bias;         // [E] or nullptr
-    const void* fc1;           // [E, 2I, H] interleaved
-    const void* fc2;           // [E, H, I]
+    const void* fc1;           // [E, 2I, H] (int8 with ep.fc1_scale)
+    const void* fc2;           // [E, H, I] (int8 with ep.fc2_scale)
     int T, H, E, k, I, normalize;
     float* logits;             // [T, E] scratch
     int32_t* topk_idx;         // [T, k] out

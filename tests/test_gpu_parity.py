@@ -475,11 +475,14 @@ def test_full_workload_with_pre_norm(name):
 
 # ------------------------------------------------------------------ int8 experts
 # Weight-only int8 experts (one float32 scale per weight row) in the decode FFN.
+# The routing inside the launch (T <= 64), after the tensor-core router, after the
+# one-CTA router (an expert count the tensor-core router does not take).
 Q8_CASES = [
     W("q8_decode", T=4, H=256, E=64, k=4, I=128),
     W("q8_router_tc", T=100, H=256, E=64, k=4, I=192, router_bias_std=0.5),
-    W("q8_small_route", T=40, H=128, E=16, k=4, I=128),
+    W("q8_small_route", T=100, H=128, E=16, k=4, I=128),
     W("q8_chunked_norm0", T=20, H=256, E=32, k=6, I=128, normalize=0, fc1_layout="chunked"),
+    W("q8_one_launch_bias", T=48, H=256, E=16, k=4, I=128, router_bias_std=0.5),
 ]
 
 
@@ -500,6 +503,9 @@ def _q8_oracle(inp, wl, host, idx, act=(1.0, 0.0, float("inf")), b1=None, b2=Non
 
 @pytest.mark.parametrize("wl", Q8_CASES, ids=[c.name for c in Q8_CASES])
 def test_forward_q8(wl):
+    lib = moe.load_library()
+    one_launch = bool(lib.moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, 1) & 32)
+    assert one_launch == (wl.T <= 64), wl.name
     inp = make_inputs(wl, weights=False)
     dev = device_inputs(inp)
     host, (q1, s1, q2, s2) = _q8_dev(wl)
