@@ -206,7 +206,7 @@ moe_status moe_forward(const void* hidden, const void* norm_weight, float norm_e
  *   device array of MOE_STATIC_SCRATCH_BYTES inside the library, which every GPU
  *   that loads the library holds until the process exits.  Sizes whose
  *   moe_workspace_size(T, H, E, k, I, dt) exceeds MOE_STATIC_SCRATCH_BYTES (with
- *   E = 128, k = 8, H = 2816, I = 704 in bf16: up to 133 tokens) are rejected with
+ *   E = 128, k = 8, H = 2816, I = 704 in bf16: up to 77 tokens) are rejected with
  *   MOE_ERR_INVALID_ARG before anything is enqueued; nothing is allocated, ever.
  *   The first call on a device looks up the array's device address (with that
  *   device current); make that first call before any stream capture.

@@ -58,14 +58,22 @@ struct Carver {
 };
 
 struct FwdLayout {
-    size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, perm_pair,
-        ctr, x_perm, act, y, xn, total;
+    size_t hdr, logits, idx, w, near, tile_counts, counts, offsets, perm_src, perm_dst, ctr,
+        x_perm, act, y, xn, total;
 };
 
 size_t elem_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
 
 constexpr int kPathSmallRoute = 1, kPathDecodeFfn = 2, kPathTcRouter = 4, kPathTokenGemm = 8,
               kPathF32Ffn = 16, kPathFusedRoute = 32;
+
+// The bf16 decode FFN gathers its token rows from hidden itself (tile::gather4, four rows
+// per load) when each expert has at most 4 rows on average; with more, TMA row gathers
+// cannot keep up and the rows are gathered once into x_perm and loaded in 16-row boxes.
+bool decode_gathers(int T, int H, int E, int k, int I, moe_dtype dt) {
+    const long long rows = static_cast<long long>(T) * k;
+    return dt == MOE_BF16 && rows <= 4LL * E && decode_ffn_supported(static_cast<int>(rows), E, H, I);
+}
 
 FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     const size_t es = elem_size(dt);
@@ -86,10 +94,8 @@ FwdLayout fwd_layout(int T, int H, int E, int k, int I, moe_dtype dt) {
     L.offsets = c.take(static_cast<size_t>(E + 1) * 4);
     L.perm_src = c.take(rows * 4);
     L.perm_dst = c.take(rows * 4);
-    L.perm_pair = c.take(rows * 4);
-    // every bf16 path gathers its token rows from hidden: only the float32 path keeps a
-    // permuted copy
-    L.x_perm = c.take(dt == MOE_BF16 ? 0 : rows * H * es);
+    // the permuted copy of the token rows, unless the decode FFN gathers them itself
+    L.x_perm = c.take(decode_gathers(T, H, E, k, I, dt) ? 0 : rows * H * es);
     L.act = c.take(rows * I * es);
     L.y = c.take(rows * H * es);
     L.xn = c.take(static_cast<size_t>(T) * H * es);   // the normalised input (pre-FFN norm)
@@ -421,7 +427,6 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
     int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
     int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
     int32_t* perm_dst = reinterpret_cast<int32_t*>(ws + L.perm_dst);
-    int32_t* perm_pair = reinterpret_cast<int32_t*>(ws + L.perm_pair);
     void* x_perm = ws + L.x_perm;
     void* act_buf = ws + L.act;
     void* y = ws + L.y;
@@ -440,9 +445,6 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
     int32_t* ctr = reinterpret_cast<int32_t*>(ws + L.ctr);
     int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
     int32_t* near = reinterpret_cast<int32_t*>(ws + L.near);
-    // the bf16 token-row GEMMs gather their token rows from hidden and write y in token
-    // order (pair (t, j) at row t k + j), which the combine then reads row block by block
-    const bool pair_gemm_path = bf16 && (path & kPathTokenGemm);
     record(0, s);
     // The first launch zeroes what must start at zero (the error word, the decode-FFN
     // counters, the tile counts; the split router of the small-route path clears the
@@ -511,7 +513,6 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         a.offsets = offsets;
         a.perm_src = perm_src;
         a.perm_dst = perm_dst;
-        if (pair_gemm_path) a.perm_pair = perm_pair;
         if (path & kPathDecodeFfn) {
             a.zero_words = ctr;
             a.n_zero = decode_ffn_counters(rows, E);
@@ -542,39 +543,43 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         }
         record(1, s);
         MOE_CUDA(launch_scatter(idx, tile_counts, T, E, k, counts, offsets, perm_src, perm_dst,
-                                err, s, pair_gemm_path ? perm_pair : nullptr));
+                                err, s));
     }
     if (path & kPathDecodeFfn) {
-        // fc1 + SwiGLU and fc2 in one launch; fc1 gathers its token rows straight from
-        // hidden (tile::gather4, four rows per load) ...
+        // fc1 + SwiGLU and fc2 in one launch.  With at most 4 rows per expert on
+        // average, fc1 gathers its token rows straight from hidden (tile::gather4, four
+        // rows per load); with more, the rows are gathered once into x_perm and loaded
+        // in 16-row boxes.
+        const bool tma_gather = decode_gathers(T, H, E, k, I, dt);
+        if (!tma_gather)
+            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
+                                   static_cast<int>(elem_size(dt)), x_perm, s));
         record(2, s);
         // ... and the weighted combine, after every fc2 unit has published its rows
-        MOE_CUDA(launch_ffn_decode(hidden, perm_src, T, offsets, fc1, fc2, rows, H, E, I, act_buf,
-                                   y, ctr, err, perm_dst, w, k, out, s, ep));
+        MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
+                                   T, offsets, fc1, fc2, rows, H, E, I, act_buf, y, ctr, err,
+                                   perm_dst, w, k, out, s, ep));
         record(3, s);
         record(4, s);
         record(5, s);
         return MOE_OK;
     } else {
+        MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
+                               static_cast<int>(elem_size(dt)), x_perm, s));
+        record(2, s);
         cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
-        if (pair_gemm_path) {
-            // fc1 gathers the token rows from hidden itself (no x_perm)
-            record(2, s);
-            MOE_CUDA(launch_ffn_pair(hidden, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
-                                     mid, ep, perm_src, T, perm_pair));
-        } else {
-            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
-                                   static_cast<int>(elem_size(dt)), x_perm, s));
-            record(2, s);
+        if (bf16)
+            MOE_CUDA(launch_ffn_pair(x_perm, offsets, fc1, fc2, rows, H, E, I, act_buf, y, err, s,
+                                     mid, ep));
+        else
             MOE_CUDA(launch_ffn_simt_f32(static_cast<const float*>(x_perm), offsets,
                                          static_cast<const float*>(fc1),
                                          static_cast<const float*>(fc2), rows, H, E, I,
                                          static_cast<float*>(act_buf), static_cast<float*>(y), s,
                                          mid, ep));
-        }
     }
     record(4, s);
-    MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s, pair_gemm_path));
+    MOE_CUDA(launch_combine(y, perm_dst, w, T, H, k, bf16, out, s));
     record(5, s);
     return MOE_OK;
 }

@@ -21,7 +21,7 @@ namespace {
 // a token are loaded before they are summed (in slot order), so the loads overlap.
 constexpr int kCombineThreads = 128;
 
-template <bool BF16, int KC, int P, bool TOKEN_ORDER = false>
+template <bool BF16, int KC, int P>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm_dst,
                const float* __restrict__ topk_w, int T, int H, int k, int rows_max,
@@ -40,13 +40,12 @@ combine_kernel(const void* __restrict__ y_perm, const int32_t* __restrict__ perm
         int t = blockIdx.x;
         for (; t + (P - 1) * step < T; t += P * step) {
             uint4 r[P];
-            combine_vecs_bf16<KC, P, TOKEN_ORDER>(y, nvec, perm_dst, topk_w, t, step, k, v, rows_max, r);
+            combine_vecs_bf16<KC, P>(y, nvec, perm_dst, topk_w, t, step, k, v, rows_max, r);
 #pragma unroll
             for (int p = 0; p < P; ++p) o[static_cast<size_t>(t + p * step) * nvec + v] = r[p];
         }
         for (; t < T; t += step)
-            o[static_cast<size_t>(t) * nvec + v] =
-                combine_vec_bf16<TOKEN_ORDER>(y, nvec, perm_dst, topk_w, t, k, v, rows_max);
+            o[static_cast<size_t>(t) * nvec + v] = combine_vec_bf16(y, nvec, perm_dst, topk_w, t, k, v, rows_max);
     } else {
         if (v >= nvec) return;
         for (int t = blockIdx.x; t < T; t += gridDim.x) {
@@ -108,8 +107,7 @@ cudaError_t launch_clear(void* words, size_t bytes, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w,
-                           int T, int H, int k, bool bf16, void* out, cudaStream_t s,
-                           bool token_order) {
+                           int T, int H, int k, bool bf16, void* out, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     const int nvec = H / (bf16 ? 8 : 4);
     const int slabs = (nvec + kCombineThreads - 1) / kCombineThreads;
@@ -120,13 +118,6 @@ cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const fl
     if (!bf16)
         return launch_k(combine_kernel<false, 1, 1>, grid, dim3(kCombineThreads), 0, s, y_perm,
                         perm_dst, topk_w, T, H, k, rows_max, out);
-    if (token_order) {
-        if (k <= 4)
-            return launch_k(combine_kernel<true, 4, 4, true>, grid, dim3(kCombineThreads), 0, s,
-                            y_perm, perm_dst, topk_w, T, H, k, rows_max, out);
-        return launch_k(combine_kernel<true, 8, 2, true>, grid, dim3(kCombineThreads), 0, s, y_perm,
-                        perm_dst, topk_w, T, H, k, rows_max, out);
-    }
     if (k <= 4)
         return launch_k(combine_kernel<true, 4, 4>, grid, dim3(kCombineThreads), 0, s, y_perm,
                         perm_dst, topk_w, T, H, k, rows_max, out);

@@ -14,16 +14,14 @@ constexpr int kCombineUnroll = 8;
 
 // Rows j0 .. j0+KC-1 of token t (16-byte vector v of each): raw bf16 vectors and
 // weights; a slot past k, or a row outside [0, rows_max), holds weight 0 and a zero
-// vector (its fma then adds +0, as for any zero row).  TOKEN_ORDER: the expert outputs
-// are stored in token order, pair (t, j) at row t k + j (perm_dst then only marks the
-// pairs to skip); the arithmetic is the same.
+// vector (its fma then adds +0, as for any zero row).
 template <int KC>
 struct CombineChunk {
     uint4 y[KC];
     float w[KC];
 };
 
-template <int KC, bool TOKEN_ORDER = false>
+template <int KC>
 __device__ __forceinline__ void combine_load(CombineChunk<KC>& c, const uint4* __restrict__ y,
                                              int nvec, const int32_t* __restrict__ perm_dst,
                                              const float* __restrict__ topk_w, int t, int k, int j0,
@@ -42,8 +40,7 @@ __device__ __forceinline__ void combine_load(CombineChunk<KC>& c, const uint4* _
             c.y[jj] = make_uint4(0u, 0u, 0u, 0u);
         } else {
             c.w[jj] = w;
-            const size_t row = TOKEN_ORDER ? static_cast<size_t>(t) * k + j : static_cast<size_t>(r);
-            c.y[jj] = y[row * nvec + v];
+            c.y[jj] = y[static_cast<size_t>(r) * nvec + v];
         }
     }
 }
@@ -64,7 +61,7 @@ __device__ __forceinline__ void combine_accumulate(float* acc, const CombineChun
 // P tokens t0, t0 + step, ... at once (the loads of all of them are in flight
 // together), chunks of KC rows; every token's sum runs over j = 0 .. k-1 in order,
 // so the result does not depend on KC or P.
-template <int KC, int P, bool TOKEN_ORDER = false>
+template <int KC, int P>
 __device__ __forceinline__ void combine_vecs_bf16(const uint4* __restrict__ y, int nvec,
                                                   const int32_t* __restrict__ perm_dst,
                                                   const float* __restrict__ topk_w, int t0, int step,
@@ -78,8 +75,7 @@ __device__ __forceinline__ void combine_vecs_bf16(const uint4* __restrict__ y, i
         CombineChunk<KC> c[P];
 #pragma unroll
         for (int p = 0; p < P; ++p)
-            combine_load<KC, TOKEN_ORDER>(c[p], y, nvec, perm_dst, topk_w, t0 + p * step, k, j0, v,
-                                          rows_max);
+            combine_load<KC>(c[p], y, nvec, perm_dst, topk_w, t0 + p * step, k, j0, v, rows_max);
 #pragma unroll
         for (int p = 0; p < P; ++p) combine_accumulate<KC>(acc[p], c[p], k, j0);
     }
@@ -87,14 +83,12 @@ __device__ __forceinline__ void combine_vecs_bf16(const uint4* __restrict__ y, i
     for (int p = 0; p < P; ++p) o[p] = pack_bf16x8(acc[p]);
 }
 
-template <bool TOKEN_ORDER = false>
 __device__ __forceinline__ uint4 combine_vec_bf16(const uint4* __restrict__ y, int nvec,
                                                   const int32_t* __restrict__ perm_dst,
                                                   const float* __restrict__ topk_w, int t, int k,
                                                   int v, int rows_max) {
     uint4 o;
-    combine_vecs_bf16<kCombineUnroll, 1, TOKEN_ORDER>(y, nvec, perm_dst, topk_w, t, 0, k, v,
-                                                      rows_max, &o);
+    combine_vecs_bf16<kCombineUnroll, 1>(y, nvec, perm_dst, topk_w, t, 0, k, v, rows_max, &o);
     return o;
 }
 

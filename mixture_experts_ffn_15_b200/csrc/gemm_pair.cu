@@ -17,14 +17,9 @@
 // 128 x 256 x 64 multiply-adds -- two thirds of what a single-CTA 128 x 256 tile
 // needs -- and the token side rounds up to 32 rows, not to a 128-row tile.
 //
-// fc2 reads contiguous activation rows in one 128-row TMA box; fc1 reads either
-// contiguous rows of x_perm the same way or -- the layer's path -- gathers its token
-// rows straight from the hidden states through perm_src, four rows per tile::gather4
-// load, so that the permuted copy of the tokens is never written.  The accumulator
-// holds weight rows x tokens, so the epilogue transposes each warp's 32 x 32 block
-// through shared memory and writes every token row with 16-byte stores, to the row
-// the optional output row map names (the layer writes fc2's rows in token order:
-// pair (t, j) at row t k + j, so that the combine reads each token's rows together).
+// Both GEMMs read contiguous token rows (x_perm, act) in one 128-row TMA box.  The
+// accumulator holds weight rows x tokens, so the epilogue transposes each warp's
+// 32 x 32 block through shared memory and writes every token row with 16-byte stores.
 //
 // Per CTA, 10 warps:
 //   warp 0     TMA producer (both CTAs): its CTA's weight and token slices into a
@@ -84,12 +79,6 @@ struct PairParams {
     SwigluAttr act;           // fc1: SwiGLU attributes
     const __nv_bfloat16* bias;   // [E, n_out] bias of the weight rows, or nullptr
     bool fc1_chunked;            // fc1 (SWIGLU): weights and bias in the chunked layout
-    // token rows gathered from x [T, K] through gather_src [rows] (permuted row -> token),
-    // four rows per tile::gather4 load; nullptr: the rows of x are the permuted rows
-    const int32_t* gather_src;
-    int T;
-    // output row of permuted row r: out_rows[r] (nullptr: r)
-    const int32_t* out_rows;
 };
 
 struct PUnit {
@@ -170,7 +159,6 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         // ------------------------------------------------------------ TMA producer
         int stage = 0;
         uint32_t phase = 0;
-        const bool gather = p.gather_src != nullptr;
         for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
             const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
             const int half = d.n / 2;                     // token rows of this CTA
@@ -179,27 +167,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // loaded through the (k, s, i, e) pair view of either weight tensor
             const int w_in = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
             // one box of 128 weight rows and one of 128 token rows per CTA (rows past
-            // the tile are loaded too, and ignored: one TMA instruction each); gathered
-            // token rows: exactly `half` rows, four per lane (half is a multiple of 16)
-            uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
-            int src[4] = {0, 0, 0, 0};
-            if (gather) {
-                bytes = static_cast<uint32_t>(2 * (kPABytes + half * kPBK * 2));
-                const int last = d.row0 + d.nrows - 1;   // rows past the tile repeat it
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = min(trow0 + 4 * lane + i, last);
-                    int t = 0;
-                    if (4 * lane < half) {
-                        t = p.gather_src[r];
-                        if (t < 0 || t >= p.T) {
-                            atomicOr(p.err, kErrBadExpert);
-                            t = 0;
-                        }
-                    }
-                    src[i] = t;
-                }
-            }
+            // the tile are loaded too, and ignored: one TMA instruction each)
+            const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
                 if (lane == 0) {
@@ -214,11 +183,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
                 if (lane == 0) {
                     tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
-                    if (!gather) tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
+                    tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
                 }
-                if (gather && 4 * lane < half)
-                    tma_gather4_pair(b_dst + lane * 4 * kPBK * 2, &tmX, fb, kb * kPBK, src[0],
-                                     src[1], src[2], src[3]);
                 if (++stage == kPStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -319,12 +285,9 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
                     for (int pass = 0; pass < 2; ++pass) {
                         const int tt = pass * 16 + (lane >> 1), q = lane & 1;
-                        if (wvalid && c + tt < d.nrows) {
-                            const int r = d.row0 + c + tt;
-                            const size_t orow = static_cast<size_t>(p.out_rows ? p.out_rows[r] : r);
-                            *reinterpret_cast<uint4*>(p.out + orow * p.ldo + i0 + q * 8) =
+                        if (wvalid && c + tt < d.nrows)
+                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + i0 + q * 8) =
                                 *reinterpret_cast<const uint4*>(scr + tt * 32 + q * 16);
-                        }
                     }
                 } else {
                     // lanes 2j, 2j+1 hold rows 2j, 2j+1.  For tokens (i, i+1) one exchange
@@ -345,12 +308,9 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 #pragma unroll
                     for (int pass = 0; pass < 4; ++pass) {
                         const int tt = pass * 8 + (lane >> 2), q = lane & 3;
-                        if (wvalid && c + tt < d.nrows) {
-                            const int r = d.row0 + c + tt;
-                            const size_t orow = static_cast<size_t>(p.out_rows ? p.out_rows[r] : r);
-                            *reinterpret_cast<uint4*>(p.out + orow * p.ldo + w0 + q * 8) =
+                        if (wvalid && c + tt < d.nrows)
+                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + w0 + q * 8) =
                                 *reinterpret_cast<const uint4*>(scr + tt * 64 + q * 16);
-                        }
                     }
                 }
                 __syncwarp();   // the scratch is rewritten by the next chunk
@@ -426,17 +386,14 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
 // 4-D pair view, which reads chunked fc1 in place).
 cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
                       const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s,
-                      const FfnAttrs& at, const void* bias, const int32_t* gather_src, int T,
-                      const int32_t* out_rows) {
+                      const FfnAttrs& at, const void* bias) {
     CUtensorMap mw, mx;
     const bool ok_w = swiglu ? tmap::fc1_pairs(&mw, w, E, n_out / 2, K, kPWRows / 2, at.fc1_chunked)
                              : tmap::plain_pairs(&mw, w, E, n_out, K, kPWRows / 2);
     if (!ok_w) return cudaErrorInvalidValue;
-    // gathered rows: x is [T, K], read one row per box (four boxes per gather4 load)
-    if (!(gather_src ? tmap::matrix(&mx, x, T, K, 1) : tmap::matrix(&mx, x, rows, K, kPBox)))
-        return cudaErrorInvalidValue;
+    if (!tmap::matrix(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
     PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, at.act,
-                 static_cast<const __nv_bfloat16*>(bias), at.fc1_chunked, gather_src, T, out_rows};
+                 static_cast<const __nv_bfloat16*>(bias), at.fc1_chunked};
     const long long units = (static_cast<long long>((rows + kPTok - 1) / kPTok) + E) *
                             ((n_out + 2 * kPWRows - 1) / (2 * kPWRows));
     return swiglu ? launch_pair<true>(mw, mx, p, units, s) : launch_pair<false>(mw, mx, p, units, s);
@@ -446,17 +403,15 @@ cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w
 
 bool pair_ffn_supported(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0; }
 
-cudaError_t launch_ffn_pair(const void* x, const int32_t* offsets, const void* fc1,
+cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep,
-                            const int32_t* perm_src, int T, const int32_t* y_rows) {
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep) {
     if (rows <= 0) return cudaSuccess;
-    cudaError_t e = pair_gemm(true, x, rows, H, fc1, E, 2 * I, offsets, act, I, err, s, ep,
-                              ep.fc1_bias, perm_src, T, nullptr);
+    cudaError_t e = pair_gemm(true, x_perm, rows, H, fc1, E, 2 * I, offsets, act, I, err, s, ep,
+                              ep.fc1_bias);
     if (e != cudaSuccess) return e;
     if (mid) record_event(mid, s);
-    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s, ep, ep.fc2_bias,
-                     nullptr, 0, y_rows);
+    return pair_gemm(false, act, rows, I, fc2, E, H, offsets, y, H, err, s, ep, ep.fc2_bias);
 }
 
 }  // namespace moe

@@ -106,7 +106,6 @@ struct RouteSmallArgs {
     int32_t* offsets = nullptr;      // [E + 1]
     int32_t* perm_src = nullptr;     // [T * k]
     int32_t* perm_dst = nullptr;     // [T * k]
-    int32_t* perm_pair = nullptr;    // [T * k] or nullptr: the pair t k + j of permuted row r
     int32_t* zero_words = nullptr;   // cleared by the kernel (the decode FFN's counters)
     int n_zero = 0;
 };
@@ -114,11 +113,9 @@ cudaError_t launch_route_small(const RouteSmallArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- permute.cu
 // counts [E], offsets [E+1], perm_src, perm_dst from topk_idx and the per-tile counts
-// perm_pair (optional) [T k]: the pair t k + j that permuted row r holds
 cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, int T, int E,
                            int k, int32_t* counts, int32_t* offsets, int32_t* perm_src,
-                           int32_t* perm_dst, int32_t* err, cudaStream_t s,
-                           int32_t* perm_pair = nullptr);
+                           int32_t* perm_dst, int32_t* err, cudaStream_t s);
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
                           int E, int T, int rows_max, int H, int elem_bytes, void* x_perm,
                           cudaStream_t s);
@@ -127,11 +124,8 @@ cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int
 // Zeroes `bytes` (a multiple of 16, 16-byte aligned) with a kernel, so that the launch
 // overlaps the previous kernel on the stream (a memset node would not).
 cudaError_t launch_clear(void* words, size_t bytes, cudaStream_t s);
-// token_order (bf16): y holds pair (t, j)'s expert output at row t k + j (perm_dst then
-// only marks the pairs to skip, < 0); else at row perm_dst[t k + j].
 cudaError_t launch_combine(const void* y_perm, const int32_t* perm_dst, const float* topk_w,
-                           int T, int H, int k, bool bf16, void* out, cudaStream_t s,
-                           bool token_order = false);
+                           int T, int H, int k, bool bf16, void* out, cudaStream_t s);
 cudaError_t launch_convert(const void* src, void* dst, int E, int I, int H, int elem_bytes,
                            cudaStream_t s);
 
@@ -179,16 +173,12 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
 
 // ---------------------------------------------------------------- gemm_pair.cu
 // fc1 + SwiGLU and fc2 for large batches on CTA pairs (weight rows on M, M = 256 per
-// pair): x [rows, H] -> act [rows, I] -> y [rows, H]; `mid` (optional) is recorded
-// between the two GEMMs.  With perm_src, x is the hidden states [T, H] and fc1 gathers
-// permuted row r from x[perm_src[r]]; with y_rows, permuted row r of y is written at
-// row y_rows[r].
+// pair): x_perm [rows, H] -> act [rows, I] -> y [rows, H]; `mid` (optional) is
+// recorded between the two GEMMs.
 bool pair_ffn_supported(int H, int I);
-cudaError_t launch_ffn_pair(const void* x, const int32_t* offsets, const void* fc1,
+cudaError_t launch_ffn_pair(const void* x_perm, const int32_t* offsets, const void* fc1,
                             const void* fc2, int rows, int H, int E, int I, void* act, void* y,
-                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep,
-                            const int32_t* perm_src = nullptr, int T = 0,
-                            const int32_t* y_rows = nullptr);
+                            int32_t* err, cudaStream_t s, cudaEvent_t mid, const FfnAttrs& ep);
 
 // Decode FFN: fc1 + SwiGLU and fc2 in one persistent launch (weight rows on M).
 bool decode_ffn_supported(int rows, int E, int H, int I);

@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kScatterThreads)
 scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ tile_counts,
                int T, int E, int k, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_dst,
-               int32_t* __restrict__ err, int32_t* __restrict__ perm_pair) {
+               int32_t* __restrict__ err) {
     __shared__ uint32_t s_mask[kMaxExperts * kMaskWords];
     __shared__ int s_tot[kScatterThreads];
     __shared__ int s_before[kScatterThreads];
@@ -121,7 +121,6 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
             for (int q = 0; q < w; ++q) rank += __popc(m[q]);
             row = s_base[e] + rank;
             perm_src[row] = t_begin + tl;
-            if (perm_pair) perm_pair[row] = t_begin * k + p;
         }
         perm_dst[static_cast<size_t>(t_begin) * k + p] = row;
     }
@@ -165,10 +164,10 @@ gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm
 
 cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, int T, int E,
                            int k, int32_t* counts, int32_t* offsets, int32_t* perm_src,
-                           int32_t* perm_dst, int32_t* err, cudaStream_t s, int32_t* perm_pair) {
+                           int32_t* perm_dst, int32_t* err, cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
     return launch_k(scatter_kernel, dim3(num_token_tiles(T)), dim3(kScatterThreads), 0, s, topk_idx,
-                    tile_counts, T, E, k, counts, offsets, perm_src, perm_dst, err, perm_pair);
+                    tile_counts, T, E, k, counts, offsets, perm_src, perm_dst, err);
 }
 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,

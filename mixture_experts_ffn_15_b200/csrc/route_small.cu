@@ -183,7 +183,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1) route_small_kernel(const Rou
                 for (int i = 0; i < w; ++i) rank += __popc(m[i]);
                 row = s_off[e] + rank;
                 a.perm_src[row] = t;
-                if (a.perm_pair) a.perm_pair[row] = t * k + lane;
             }
             a.perm_dst[static_cast<size_t>(t) * k + lane] = row;
         }

@@ -292,20 +292,6 @@ __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
-// Four rows r0..r3 (64 columns from c0) of a 2-D tensor whose map has a one-row box,
-// gathered into this CTA's shared memory at dst, dst + 128, dst + 256, dst + 384 (the
-// 128-byte swizzle applies by address, as for a four-row box), with the completion of
-// tma_load_2d_pair.
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int c0, int r0, int r1, int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-        ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-        "r"(r3)
-        : "memory");
-}
-
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                uint32_t idesc, uint32_t accumulate) {
     asm volatile(

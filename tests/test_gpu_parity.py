@@ -187,14 +187,13 @@ def test_forward(wl):
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} output")
 
 
-def test_gathering_token_gemms_equal_the_staged_calls_bit_for_bit():
-    """The layer's large-batch path gathers fc1's token rows from hidden (tile::gather4)
-    and writes fc2's rows in token order for the combine; the staged calls run the same
-    GEMM kernels on the permuted copy x_perm and write y in permuted order.  Same
-    routing (the tensor-core router in both), same arithmetic: the same bits.  A skewed
-    router gives experts of every size, so token tiles end at every offset."""
+def test_token_gemm_layer_equals_the_staged_calls_bit_for_bit():
+    """The layer's large-batch path (router, scatter, gather, fc1 and fc2 on CTA pairs,
+    combine in one call) against the staged calls on the same inputs: same routing (the
+    tensor-core router in both), same kernels, the same bits.  A skewed router gives
+    experts of every size, so token tiles end at every offset."""
     from mixture_experts_ffn_15_b200 import _abi
-    wl = W("gather_pairs", T=1500, H=256, E=64, k=4, I=192, router_bias_std=1.0)
+    wl = W("token_gemm_skew", T=1500, H=256, E=64, k=4, I=192, router_bias_std=1.0)
     assert moe.load_library().moe_forward_path(wl.T, wl.H, wl.E, wl.k, wl.I, _abi.MOE_BF16) & 8
     inp = make_inputs(wl)
     dev = device_inputs(inp)
@@ -211,7 +210,7 @@ def test_gathering_token_gemms_equal_the_staged_calls_bit_for_bit():
     L, idx = check_routing(inp, r)
     ref = oracle_forward(inp, idx)["out"]
     atol, rtol = tol(wl.dtype, ref)
-    assert_close(from_dev(out), ref, atol, rtol, "gathered token GEMMs")
+    assert_close(from_dev(out), ref, atol, rtol, "token GEMM layer")
 
 
 # ------------------------------------------- SwiGLU attributes and expert biases
