@@ -192,6 +192,16 @@ void record(int i, cudaStream_t s) {
         if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
     } while (0)
 
+// x_perm from hidden: token by token (each hidden row read once) for k <= 32, else row
+// by row through perm_src.
+cudaError_t gather_rows(const void* hidden, const int32_t* perm_src, const int32_t* perm_dst,
+                        const int32_t* offsets, int T, int E, int k, int H, moe_dtype dt,
+                        void* x_perm, cudaStream_t s) {
+    const int es = static_cast<int>(elem_size(dt));
+    if (k <= 32) return launch_gather_by_token(hidden, perm_dst, T, k, T * k, H, es, x_perm, s);
+    return launch_gather(hidden, perm_src, offsets, E, T, T * k, H, es, x_perm, s);
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -552,8 +562,7 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         // in 16-row boxes.
         const bool tma_gather = decode_gathers(T, H, E, k, I, dt);
         if (!tma_gather)
-            MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
-                                   static_cast<int>(elem_size(dt)), x_perm, s));
+            MOE_CUDA(gather_rows(hidden, perm_src, perm_dst, offsets, T, E, k, H, dt, x_perm, s));
         record(2, s);
         // ... and the weighted combine, after every fc2 unit has published its rows
         MOE_CUDA(launch_ffn_decode(tma_gather ? hidden : x_perm, tma_gather ? perm_src : nullptr,
@@ -564,8 +573,7 @@ static moe_status forward_impl(const void* hidden, const void* norm_weight, floa
         record(5, s);
         return MOE_OK;
     } else {
-        MOE_CUDA(launch_gather(hidden, perm_src, offsets, E, T, rows, H,
-                               static_cast<int>(elem_size(dt)), x_perm, s));
+        MOE_CUDA(gather_rows(hidden, perm_src, perm_dst, offsets, T, E, k, H, dt, x_perm, s));
         record(2, s);
         cudaEvent_t mid = g_events_on ? g_events[3] : nullptr;
         if (bf16)

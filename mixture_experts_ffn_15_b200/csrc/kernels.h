@@ -119,6 +119,11 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
                           int E, int T, int rows_max, int H, int elem_bytes, void* x_perm,
                           cudaStream_t s);
+// The same rows written token by token: x_perm[perm_dst[t k + j]] = hidden[t] (k <= 32;
+// every row of hidden read once).
+cudaError_t launch_gather_by_token(const void* hidden, const int32_t* perm_dst, int T, int k,
+                                  int rows_max, int H, int elem_bytes, void* x_perm,
+                                  cudaStream_t s);
 
 // ---------------------------------------------------------------- combine.cu
 // Zeroes `bytes` (a multiple of 16, 16-byte aligned) with a kernel, so that the launch

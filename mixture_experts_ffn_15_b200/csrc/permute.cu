@@ -126,6 +126,48 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
     }
 }
 
+// x_perm[perm_dst[t k + j]] = hidden[t] for every pair (t, j); one warp per token,
+// 16-byte vectors.  Walking the tokens (not the permuted rows) reads every row of
+// hidden once, in order, and writes its k copies: by permuted row, a row would be read
+// k times from far-apart places, i.e. from HBM each time once hidden exceeds L2.  Pairs
+// whose row is outside [0, rows_max) (an id that was out of range) are skipped; rows
+// that no pair names are not written.
+__global__ void __launch_bounds__(256)
+gather_by_token_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm_dst,
+                       int T, int k, int rows_max, int vec_per_row, uint4* __restrict__ x_perm) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int kKMax = 32;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        // the token's destination rows: lane j holds row j (k <= 32)
+        int dst = -1;
+        if (lane < k) {
+            const int r = perm_dst[static_cast<size_t>(t) * k + lane];
+            dst = (r >= 0 && r < rows_max) ? r : -1;
+        }
+        const uint4* s = hidden + static_cast<size_t>(t) * vec_per_row;
+        // 8 loads in flight per lane before the stores
+        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (v0 + 32 * q < vec_per_row) buf[q] = __ldcs(s + v0 + 32 * q);
+#pragma unroll 1
+            for (int j = 0; j < k && j < kKMax; ++j) {
+                const int r = __shfl_sync(0xffffffffu, dst, j);
+                if (r < 0) continue;
+                uint4* d = x_perm + static_cast<size_t>(r) * vec_per_row;
+                // streaming stores: x_perm is read back once, by the grouped GEMM
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (v0 + 32 * q < vec_per_row) __stcs(d + v0 + 32 * q, buf[q]);
+            }
+        }
+    }
+}
+
 // x_perm[r] = hidden[perm_src[r]] for r < offsets[E]; one warp per row, 16-byte
 // vectors.  A source index outside [0, T) (possible only after bad ids in the
 // staged API) writes a zero row instead of reading out of bounds.
@@ -168,6 +210,19 @@ cudaError_t launch_scatter(const int32_t* topk_idx, const int32_t* tile_counts, 
     if (T <= 0) return cudaSuccess;
     return launch_k(scatter_kernel, dim3(num_token_tiles(T)), dim3(kScatterThreads), 0, s, topk_idx,
                     tile_counts, T, E, k, counts, offsets, perm_src, perm_dst, err);
+}
+
+cudaError_t launch_gather_by_token(const void* hidden, const int32_t* perm_dst, int T, int k,
+                                  int rows_max, int H, int elem_bytes, void* x_perm,
+                                  cudaStream_t s) {
+    if (T <= 0 || k > 32) return T <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+    const int vec = H * elem_bytes / 16;
+    int blocks = (T + 7) / 8;
+    const int cap = device_sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    return launch_k(gather_by_token_kernel, dim3(blocks), dim3(256), 0, s,
+                    static_cast<const uint4*>(hidden), perm_dst, T, k, rows_max, vec,
+                    static_cast<uint4*>(x_perm));
 }
 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,

@@ -45,6 +45,8 @@ CASES = [
       router_bias_std=0.5),
     W("bf16_onelaunch_E256_k16", T=8, H=128, E=256, k=16, I=64),
     W("bf16_k1", T=130, H=128, E=8, k=1, I=64),
+    # k > 32: the float32-logit top-k, and the row-by-row gather into x_perm
+    W("bf16_k40", T=40, H=128, E=64, k=40, I=64),
     W("bf16_k_eq_E", T=20, H=128, E=4, k=4, I=64),
     W("bf16_T1", T=1, H=128, E=8, k=2, I=64),
     W("bf16_normalize_off", T=90, H=128, E=8, k=3, I=64, normalize=0),
