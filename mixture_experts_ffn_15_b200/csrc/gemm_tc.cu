@@ -402,28 +402,31 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // prefill), where one CTA per tile would stream the whole K range alone.  A cluster of
 // CS CTAs runs one tile: CTA r accumulates the K slices [r nk / CS, (r + 1) nk / CS) on
 // the tensor cores (128 tokens on M, all E experts on N) and stores its partial logits
-// in its own shared memory.  After a cluster barrier, CTA r takes the rows
-// r 128 / CS .. of the tile, sums the CS partials of each logit in rank order 0 .. CS-1
-// through distributed shared memory (a fixed order: the logits do not depend on timing)
-// and routes the row with the warp top-k that the single-CTA router uses.  No global
-// scratch; the host picks this kernel by (T, H, E) alone, for the staged router and the
-// layer alike, so both return the same bits.
-constexpr int kSplitPad = 1;   // partials stored [e][row] with a row stride of 129 floats
-
-template <int E>
+// in its own shared memory, [e][row].  After a cluster barrier, CTA r takes the rows
+// r 128 / CS .. of the tile: its threads fetch the CS partials of those rows through
+// distributed shared memory, 16-byte loads along the rows, all CS (and two or more row
+// groups) issued before the first is used, sum them in rank order 0 .. CS-1 (a fixed
+// order: the logits do not depend on timing) into a [row][e] block, and warps route the
+// rows with the warp top-k of the single-CTA router.  No global scratch; the host picks
+// this kernel by (T, H, E) alone, for the staged router and the layer alike, so both
+// return the same bits.
+template <int E, int CS>
 struct SplitCfg {
+    static constexpr int kRows = BM / CS;                       // rows reduced and routed per CTA
     static constexpr int kABytes = BM * BK * 2;                 // 128 token rows x 64 K
     static constexpr int kBBytes = E * BK * 2;                  // E router rows x 64 K
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kPartBytes = E * (BM + kSplitPad) * 4;
-    static constexpr int kStagesFit = (200 * 1024 - kPartBytes) / kStageBytes;
+    static constexpr int kPartBytes = E * BM * 4;               // partials [e][row]
+    static constexpr int kRedBytes = kRows * (E + 1) * 4;       // sums [row][e], padded
+    static constexpr int kStagesFit = (210 * 1024 - kPartBytes - kRedBytes) / kStageBytes;
     static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
-    static constexpr int kRowBytes = (kThreads / 32) * E * 4;   // one logits row per warp
     // barriers (full, empty: kStages each; tfull), then the TMEM slot and the abort flag
     static constexpr int kMiscBytes = (2 * kStages + 1) * 8 + 16;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPartBytes + kRowBytes + kMiscBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPartBytes + kRedBytes + kMiscBytes;
     static constexpr int kTmemCols = E;                         // 64 or 128
+    static constexpr int kGroupsPerPass = 16 / CS;              // 16 loads in flight a thread
     static_assert(kStages >= 2, "pipeline");
+    static_assert(kRows % 4 == 0, "16-byte row groups");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -431,15 +434,15 @@ template <int E, int CS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const TcParams p, const RouteParams rp) {
-    using C = SplitCfg<E>;
+    using C = SplitCfg<E, CS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + C::kStages * C::kABytes;
-    float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM + pad]
-    float* rowbuf = part + E * (BM + kSplitPad);                            // [warps][E]
-    uint64_t* full = reinterpret_cast<uint64_t*>(rowbuf + (kThreads / 32) * E);
+    float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM]
+    float* red = part + E * BM;                                             // [kRows][E + 1]
+    uint64_t* full = reinterpret_cast<uint64_t*>(red + C::kRows * (E + 1));
     uint64_t* empty = full + C::kStages;
     uint64_t* tfull = empty + C::kStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
@@ -545,7 +548,7 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) part[(c + i) * (BM + kSplitPad) + r] = __uint_as_float(v[i]);
+                for (int i = 0; i < 32; ++i) part[(c + i) * BM + r] = __uint_as_float(v[i]);
             }
         }
     }
@@ -554,34 +557,59 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     cluster_sync();   // every CTA's partials are written and visible to the cluster
 
     // ---------------------------------------------------------------- reduce and route
-    constexpr int kRowsPerCta = BM / CS;
-    float* mine = rowbuf + warp * E;
+    // position i = (e, row group of 4): the float4 at part[e][row0 + 4 g] of every rank
+    constexpr int kGroups = C::kRows / 4;
+    constexpr int kPos = E * kGroups;
+    const int row0 = rank * C::kRows;
 #pragma unroll 1
-    for (int i = warp; i < kRowsPerCta; i += kThreads / 32) {
-        const int r = rank * kRowsPerCta + i;
-        const size_t row = static_cast<size_t>(tile) * BM + r;
-        const bool valid = row < static_cast<size_t>(p.rows);
+    for (int i0 = threadIdx.x; i0 < kPos; i0 += kThreads * C::kGroupsPerPass) {
+        float4 v[C::kGroupsPerPass][CS];
 #pragma unroll
-        for (int e = lane; e < E; e += 32) {
-            const uint32_t a = smem_u32(&part[e * (BM + kSplitPad) + r]);
-            float sum = 0.f;
+        for (int j = 0; j < C::kGroupsPerPass; ++j) {
+            const int i = i0 + j * kThreads;
+            if (i < kPos) {
+                const int e = i / kGroups, g = i - e * kGroups;
+                const uint32_t a = smem_u32(&part[e * BM + row0 + 4 * g]);
 #pragma unroll
-            for (int q = 0; q < CS; ++q) sum += ld_shared_cluster_f32(mapa_shared(a, q));
-            mine[e] = sum;
-            if (valid && rp.logits) rp.logits[row * E + e] = sum + (rp.bias ? rp.bias[e] : 0.f);
-        }
-        __syncwarp();
-        if (valid) {
-            const WarpTopk res = warp_topk(mine, rp.bias, E, rp.k, rp.normalize, lane);
-            if (lane < rp.k) {
-                rp.topk_idx[row * rp.k + lane] = res.idx;
-                rp.topk_w[row * rp.k + lane] = res.w;
-                if (rp.tile_counts && static_cast<unsigned>(res.idx) < static_cast<unsigned>(E))
-                    atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + res.idx], 1);
+                for (int q = 0; q < CS; ++q) v[j][q] = ld_shared_cluster_v4(mapa_shared(a, q));
             }
-            if (lane == 0 && rp.near_tie) rp.near_tie[row] = res.flags;
         }
-        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < C::kGroupsPerPass; ++j) {
+            const int i = i0 + j * kThreads;
+            if (i < kPos) {
+                const int e = i / kGroups, g = i - e * kGroups;
+                float4 sum = v[j][0];
+#pragma unroll
+                for (int q = 1; q < CS; ++q) {
+                    sum.x += v[j][q].x;
+                    sum.y += v[j][q].y;
+                    sum.z += v[j][q].z;
+                    sum.w += v[j][q].w;
+                }
+                red[(4 * g + 0) * (E + 1) + e] = sum.x;
+                red[(4 * g + 1) * (E + 1) + e] = sum.y;
+                red[(4 * g + 2) * (E + 1) + e] = sum.z;
+                red[(4 * g + 3) * (E + 1) + e] = sum.w;
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int i = warp; i < C::kRows; i += kThreads / 32) {
+        const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
+        if (row >= static_cast<size_t>(p.rows)) continue;
+        const float* mine = red + i * (E + 1);
+        if (rp.logits)
+            for (int e = lane; e < E; e += 32) rp.logits[row * E + e] = mine[e] + (rp.bias ? rp.bias[e] : 0.f);
+        const WarpTopk res = warp_topk(mine, rp.bias, E, rp.k, rp.normalize, lane);
+        if (lane < rp.k) {
+            rp.topk_idx[row * rp.k + lane] = res.idx;
+            rp.topk_w[row * rp.k + lane] = res.w;
+            if (rp.tile_counts && static_cast<unsigned>(res.idx) < static_cast<unsigned>(E))
+                atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + res.idx], 1);
+        }
+        if (lane == 0 && rp.near_tie) rp.near_tie[row] = res.flags;
     }
     cluster_sync();   // no CTA leaves while a peer may still read its partials
     if (warp == 1) {
@@ -630,11 +658,21 @@ struct DecodeCfg {
     static constexpr int kStages = T::kStages;              // A (smem or TMEM) + token B ring
     static constexpr int kQStages = Q8 ? 16 : 0;            // int8 weight ring
     static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
+    // Accumulators.  A stage's four 16-wide K steps accumulate into four separate
+    // accumulators (64 columns each: at most 64 tokens), summed in a fixed order in the
+    // epilogue: with N <= 64 an MMA takes a few cycles of math but a long pipeline
+    // latency, and MMAs into one accumulator wait for each other, so a single chain of
+    // 4 MMAs per stage bounds the stage rate (measured: the int8 path, with half the
+    // bytes, ran no faster than bf16).  bf16: two buffers of 4 x 64 columns (the epilogue
+    // of one unit overlaps the next).  Q8: one buffer, then one A stage of 32 columns per
+    // ring stage.
     static constexpr int kAccStride = T::kAccStride;
-    // Q8: two accumulators (2 x 64 columns), then one A stage of 32 columns per ring stage
-    static constexpr int kTmemA = 2 * kAccStride;
-    static constexpr int kTmemCols = Q8 ? 512 : T::kTmemCols;
-    static_assert(!Q8 || kTmemA + kStages * 32 <= kTmemCols, "tensor memory");
+    static constexpr int kKSplit = BK / 16;
+    static constexpr int kSlots = Q8 ? 1 : 2;
+    static constexpr int kBufCols = kKSplit * kAccStride;
+    static constexpr int kTmemA = kSlots * kBufCols;
+    static constexpr int kTmemCols = 512;
+    static_assert(kTmemA + (Q8 ? kStages * 32 : 0) <= kTmemCols, "tensor memory");
     static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
     static constexpr int kMiscBytes = T::kMiscBytes + 2 * kQStages * 8;   // + int8 ring barriers
     static constexpr int kSmemBytes = 1024 + kDataBytes + kMiscBytes;
@@ -1124,7 +1162,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const uint32_t idesc = idesc_bf16_f32(BM, ((d.nrows + 15) / 16) * 16);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
+                // K step kk of every stage accumulates into accumulator kk of the buffer
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kBufCols);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
@@ -1138,14 +1177,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                         // A: the converted stage in tensor memory, 8 columns per 16 K
                         const uint32_t at = tmem_base + static_cast<uint32_t>(C::kTmemA + stage * 32);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16_ta(d_tmem, at + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc,
-                                         (kb | kk) != 0);
+                        for (int kk = 0; kk < C::kKSplit; ++kk)
+                            umma_bf16_ta(d_tmem + kk * C::kAccStride, at + kk * 8,
+                                         smem_desc_sw128(b0 + kk * 32), idesc, kb != 0);
                     } else {
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32),
-                                      smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < C::kKSplit; ++kk)
+                            umma_bf16(d_tmem + kk * C::kAccStride, smem_desc_sw128(a0 + kk * 32),
+                                      smem_desc_sw128(b0 + kk * 32), idesc, kb != 0);
                     }
                     umma_commit(smem_u32(&empty[stage]));
                     if (++stage == C::kStages) {
@@ -1155,8 +1194,10 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 }
                 if (!ok) break;
                 umma_commit(smem_u32(&tfull[acc]));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
+                if (++acc == C::kSlots) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
             }
         }
     } else if (warp < 6) {
@@ -1182,7 +1223,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                static_cast<uint32_t>(acc * C::kAccStride);
+                                static_cast<uint32_t>(acc * C::kBufCols);
             const int wr = d.mt * BM + r;   // weight row inside the expert
             // this lane's weight row's bias (fc1: interleaved row wr in fc1's layout, fc2: h)
             const __nv_bfloat16* bsrc = f1 ? p.b1 : p.b2;
@@ -1193,13 +1234,18 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const float scale = Q8 ? (f1 ? p.s1 : p.s2)[wi] : 1.f;
 #pragma unroll 1
             for (int c = 0; c < d.nrows; c += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(tb + c, v);
+                // the four accumulators of the buffer, summed in order 0, 1, 2, 3
+                uint32_t v[C::kKSplit][16];
+#pragma unroll
+                for (int a = 0; a < C::kKSplit; ++a) tmem_ld_32x32b_x16(tb + a * C::kAccStride + c, v[a]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int n = c + i;
-                    const float x = Q8 ? fmaf(f32(v[i]), scale, bias) : f32(v[i]) + bias;
+                    float sum = f32(v[0][i]);
+#pragma unroll
+                    for (int a = 1; a < C::kKSplit; ++a) sum += f32(v[a][i]);
+                    const float x = Q8 ? fmaf(sum, scale, bias) : sum + bias;
                     if (f1) {
                         const float up = __shfl_xor_sync(0xffffffffu, x, 1);
                         if (!(lane & 1) && n < d.nrows)
@@ -1218,8 +1264,10 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 __threadfence();
                 atomicAdd(f1 ? &p.done[d.chunk] : p.fc2_done, 1);
             }
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            if (++acc == C::kSlots) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
         }
         if (p.out != nullptr) {
             // ------------------------------------------------------------ combine
@@ -1427,7 +1475,7 @@ int route_split_cluster(int T, int H, int E) {
 template <int E, int CS>
 cudaError_t launch_route_split(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p,
                                const RouteParams& rp, int tiles, cudaStream_t s) {
-    using C = SplitCfg<E>;
+    using C = SplitCfg<E, CS>;
     auto kern = tc_route_split_kernel<E, CS>;
     static bool attr_set[64] = {false};
     int dev = 0;
