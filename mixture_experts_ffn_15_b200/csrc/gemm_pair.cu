@@ -51,33 +51,21 @@ constexpr int kPThreads = 320;                // producer, MMA, 8 epilogue warps
 constexpr int kPWRows = 128;                  // weight rows per CTA (256 per pair)
 constexpr int kPBK = 64;                      // K per stage: one 128-byte row of bf16
 static_assert(kPBK == tmap::kBoxK, "TMA box width");
-constexpr int kPSub = 256;                    // tokens per MMA (<= 128 per CTA)
+constexpr int kPTok = 256;                    // tokens per pair tile (<= 128 per CTA)
+constexpr int kPStages = 6;
 constexpr int kPABytes = kPWRows * kPBK * 2;  // 16 KB
-constexpr int kPBox = kPSub / 2;              // token rows per TMA box: a CTA's half of an MMA
-constexpr int kPSubBytes = kPBox * kPBK * 2;  // 16 KB
+constexpr int kPBBytes = (kPTok / 2) * kPBK * 2;   // 16 KB
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPAccCols = 256;                // one accumulator: 256 fp32 columns
 constexpr int kPTmemCols = 512;
+constexpr int kPBox = kPTok / 2;              // token rows per TMA box: a CTA's whole half
 constexpr uint64_t kPWaitNs = 2000000000ull;
+constexpr int kPMiscBytes =
+    (2 * kPStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 64;
 constexpr int kPEpiWarpBytes = 32 * 64;      // per epilogue warp: 32 tokens x 32 rows bf16
 constexpr int kPEpiBytes = 8 * kPEpiWarpBytes;
-
-// NW token sub-tiles of 256 per unit.  NW = 1: one MMA of N <= 256 per K slice, two
-// accumulators of 256 columns in tensor memory, so the epilogue of one unit overlaps the
-// next unit's main loop.  NW = 2: two MMAs per K slice on the same weight tile (a unit
-// covers 512 tokens: 48 KB per CTA and K slice for twice the work of 32 KB), one
-// accumulator pair filling the 512 columns, so the epilogue does not overlap.
-template <int NW>
-struct PairCfg {
-    static constexpr int kTok = kPSub * NW;
-    static constexpr int kBBytes = NW * kPSubBytes;
-    static constexpr int kStageBytes = kPABytes + kBBytes;
-    static constexpr int kStages = NW == 1 ? 6 : 4;
-    static constexpr int kSlots = NW == 1 ? 2 : 1;   // accumulator buffers
-    static constexpr int kMiscBytes =
-        (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 64;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPEpiBytes + kMiscBytes;
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-    static_assert(kSlots * NW * kPSub <= kPTmemCols, "tensor memory");
-};
+constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kPEpiBytes + kPMiscBytes;
+static_assert(kPSmemBytes <= 227 * 1024, "shared memory");
 
 struct PairParams {
     const int32_t* offsets;   // [E+1] device
@@ -94,41 +82,33 @@ struct PairParams {
 };
 
 struct PUnit {
-    int g, row0, nrows, mt;   // expert, first token row, valid tokens, weight tile
+    int g, row0, nrows, n, mt;   // expert, first token row, valid tokens, MMA N, weight tile
 };
 
-template <int NW>
 __device__ __forceinline__ PUnit pair_unit(int u, int MT, int G, const int* s_off, const int* s_pre) {
     PUnit d;
     const int tile = u / MT;
     d.mt = u - tile * MT;
     d.g = tile_group(tile, G, s_pre);
-    d.row0 = s_off[d.g] + (tile - s_pre[d.g]) * PairCfg<NW>::kTok;
-    d.nrows = min(PairCfg<NW>::kTok, s_off[d.g + 1] - d.row0);
+    d.row0 = s_off[d.g] + (tile - s_pre[d.g]) * kPTok;
+    d.nrows = min(kPTok, s_off[d.g + 1] - d.row0);
+    d.n = ((d.nrows + 31) / 32) * 32;   // each CTA's half: a multiple of 16 rows (TMA boxes)
     return d;
 }
 
-// Valid tokens of sub-tile h of a unit (0 .. 256) and its MMA N: a multiple of 32, so
-// that each CTA's half is a multiple of 16 rows.
-__device__ __forceinline__ int sub_rows(const PUnit& d, int h) {
-    return max(0, min(kPSub, d.nrows - h * kPSub));
-}
-__device__ __forceinline__ int sub_n(int rows) { return ((rows + 31) / 32) * 32; }
-
-template <bool SWIGLU, int NW>
+template <bool SWIGLU>
 __global__ void __launch_bounds__(kPThreads, 1)
 tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                const PairParams p) {
-    using C = PairCfg<NW>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + C::kStages * kPABytes;
-    uint8_t* sEpi = sB + C::kStages * C::kBBytes;   // [8 warps][32 tokens][64 bytes]
+    uint8_t* sB = smem + kPStages * kPABytes;
+    uint8_t* sEpi = sB + kPStages * kPBBytes;   // [8 warps][32 tokens][64 bytes]
     uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kPEpiBytes);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* tfull = empty + C::kStages;
+    uint64_t* empty = full + kPStages;
+    uint64_t* tfull = empty + kPStages;
     uint64_t* tempty = tfull + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -141,7 +121,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     const int G = p.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < kPStages; ++s) {
             mbar_init(smem_u32(&full[s]), 1);    // the even CTA's producer (expect_tx)
             mbar_init(smem_u32(&empty[s]), 1);   // the pair MMA's commit
         }
@@ -163,7 +143,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     // the prologue above touches no global memory; everything below may
     pdl_wait();
     pdl_trigger();
-    if (warp == 2) build_group_tiles(p.offsets, p.rows, p.err, G, C::kTok, s_off, s_pre, lane);
+    if (warp == 2) build_group_tiles(p.offsets, p.rows, p.err, G, kPTok, s_off, s_pre, lane);
     tc_fence_before();
     __syncthreads();
     cluster_sync();   // both CTAs' barriers and tensor memory exist before any signal
@@ -180,22 +160,15 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         int stage = 0;
         uint32_t phase = 0;
         for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
-            const PUnit d = pair_unit<NW>(u, MT, G, s_off, s_pre);
+            const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
+            const int half = d.n / 2;                     // token rows of this CTA
+            const int trow0 = d.row0 + static_cast<int>(rank) * half;
             // first weight row of this CTA inside the expert (fc1: in interleaved order),
             // loaded through the (k, s, i, e) pair view of either weight tensor
             const int w_in = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
-            // one box of 128 weight rows and, per non-empty sub-tile, one of 128 token rows
-            // per CTA (rows past the tile are loaded too, and ignored: one TMA
-            // instruction each); sub-tile h's rows of this CTA start at trow[h]
-            int trow[NW];
-            int nsub = 0;
-#pragma unroll
-            for (int h = 0; h < NW; ++h) {
-                const int n = sub_n(sub_rows(d, h));
-                trow[h] = d.row0 + h * kPSub + static_cast<int>(rank) * (n / 2);
-                nsub += n > 0 ? 1 : 0;
-            }
-            const uint32_t bytes = static_cast<uint32_t>(2 * (kPABytes + nsub * kPSubBytes));
+            // one box of 128 weight rows and one of 128 token rows per CTA (rows past
+            // the tile are loaded too, and ignored: one TMA instruction each)
+            const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
                 if (lane == 0) {
@@ -207,14 +180,12 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 if (!ok) break;
                 const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);   // the even CTA's
                 const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
-                const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
+                const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
                 if (lane == 0) {
                     tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
-#pragma unroll
-                    for (int h = 0; h < NW; ++h)
-                        if (h < nsub) tma_load_2d_pair(b_dst + h * kPSubBytes, &tmX, fb, kb * kPBK, trow[h]);
+                    tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
                 }
-                if (++stage == C::kStages) {
+                if (++stage == kPStages) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -229,19 +200,11 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
-                const PUnit d = pair_unit<NW>(u, MT, G, s_off, s_pre);
-                uint32_t idesc[NW];
-                int nsub = 0;
-#pragma unroll
-                for (int h = 0; h < NW; ++h) {
-                    const int n = sub_n(sub_rows(d, h));
-                    idesc[h] = idesc_bf16_f32(2 * kPWRows, n > 0 ? n : 32);
-                    nsub += n > 0 ? 1 : 0;
-                }
+                const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
+                const uint32_t idesc = idesc_bf16_f32(2 * kPWRows, d.n);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kPWaitNs)) break;
                 tc_fence_after();
-                // accumulator of sub-tile h: columns (acc NW + h) 256 ..
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NW * kPSub);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPAccCols);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kPWaitNs)) {
@@ -250,28 +213,21 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * kPABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+                    const uint32_t b0 = smem_u32(sB + stage * kPBBytes);
 #pragma unroll
-                    for (int h = 0; h < NW; ++h) {
-                        if (h >= nsub) break;
-#pragma unroll
-                        for (int kk = 0; kk < kPBK / 16; ++kk)
-                            umma_bf16_pair(d_tmem + h * kPSub, smem_desc_sw128(a0 + kk * 32),
-                                           smem_desc_sw128(b0 + h * kPSubBytes + kk * 32), idesc[h],
-                                           (kb | kk) != 0);
-                    }
+                    for (int kk = 0; kk < kPBK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                       smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
                     umma_commit_pair(smem_u32(&empty[stage]), 0x3);
-                    if (++stage == C::kStages) {
+                    if (++stage == kPStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
                 umma_commit_pair(smem_u32(&tfull[acc]), 0x3);
-                if (++acc == C::kSlots) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
             }
         }
     } else {
@@ -284,13 +240,11 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
         uint32_t acc_phase = 0;
         uint8_t* scr = sEpi + (warp - 2) * kPEpiWarpBytes;
         for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
-            const PUnit d = pair_unit<NW>(u, MT, G, s_off, s_pre);
+            const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kPWaitNs)) break;
             tc_fence_after();
-            // columns c of the unit's tokens: sub-tile c / 256, column c % 256 of its
-            // accumulator, i.e. (acc NW) 256 + c
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                static_cast<uint32_t>(acc * NW * kPSub);
+                                static_cast<uint32_t>(acc * kPAccCols);
             // this warp's 32 weight rows inside the expert: w0 .. w0+31 (all valid or none:
             // n_out is a multiple of 32)
             const int w0 = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows + quad * 32;
@@ -364,10 +318,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
-            if (++acc == C::kSlots) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
         }
     }
 
@@ -388,11 +340,10 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 
 // ------------------------------------------------------------------------ host side
 
-template <bool SWIGLU, int NW>
+template <bool SWIGLU>
 cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairParams& p,
                         long long units, cudaStream_t s) {
-    using C = PairCfg<NW>;
-    auto kern = tc_pair_kernel<SWIGLU, NW>;
+    auto kern = tc_pair_kernel<SWIGLU>;
     // once per device (outside any stream capture: the first call of every path runs
     // eagerly before a graph is captured): the shared-memory limit and the number of
     // pairs that fit on the GPU at once
@@ -408,12 +359,12 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kPThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.dynamicSmemBytes = kPSmemBytes;
     cfg.stream = s;
     cfg.attrs = attr;
     if (max_pairs[dev] == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
+                                             kPSmemBytes);
         if (e != cudaSuccess) return e;
         cfg.gridDim = dim3(2 * (device_sm_count() / 2));
         cfg.numAttrs = 1;
@@ -430,14 +381,6 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
     return cudaLaunchKernelEx(&cfg, kern, w, x, p);
 }
 
-// Token sub-tiles per unit (see PairCfg).
-int pair_width(int rows, int E, int K) {
-    (void)rows;
-    (void)E;
-    (void)K;
-    return 1;
-}
-
 // One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
 // the experts' blocks) and the weights w [E, n_out, K] of E experts (both through the
 // 4-D pair view, which reads chunked fc1 in place).
@@ -451,14 +394,9 @@ cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w
     if (!tmap::matrix(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
     PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, at.act,
                  static_cast<const __nv_bfloat16*>(bias), at.fc1_chunked};
-    const int nw = pair_width(rows, E, K);
-    const int tok = kPSub * nw;
-    const long long units = (static_cast<long long>((rows + tok - 1) / tok) + E) *
+    const long long units = (static_cast<long long>((rows + kPTok - 1) / kPTok) + E) *
                             ((n_out + 2 * kPWRows - 1) / (2 * kPWRows));
-    if (nw == 2)
-        return swiglu ? launch_pair<true, 2>(mw, mx, p, units, s)
-                      : launch_pair<false, 2>(mw, mx, p, units, s);
-    return swiglu ? launch_pair<true, 1>(mw, mx, p, units, s) : launch_pair<false, 1>(mw, mx, p, units, s);
+    return swiglu ? launch_pair<true>(mw, mx, p, units, s) : launch_pair<false>(mw, mx, p, units, s);
 }
 
 }  // namespace

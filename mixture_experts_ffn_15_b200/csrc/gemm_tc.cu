@@ -397,6 +397,67 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
 }
 
+// Routing of one token row from its E raw logits in shared memory (one thread): the
+// KS = k+1 (or more) largest biased logits in a register list sorted descending,
+// experts inserted in index order so that equal logits keep the lower index first;
+// softmax weights over the chosen k (normalize) or over all E, near-tie flags, and the
+// row's k counts added to the tile's bincount.
+template <int E, int KS>
+__device__ __forceinline__ void route_row(const float* logit, const float* s_bias, size_t row,
+                                          int tile, const RouteParams& rp) {
+    const int k = rp.k;
+    float vals[KS];
+    int ids[KS];
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        vals[j] = -INFINITY;
+        ids[j] = -1;
+    }
+#pragma unroll 4
+    for (int e = 0; e < E; ++e) {
+        const float xv = logit[e] + s_bias[e];
+        if (xv > vals[KS - 1]) {
+#pragma unroll
+            for (int j = KS - 1; j >= 0; --j) {
+                if (vals[j] < xv) {
+                    if (j == 0 || vals[j - 1] >= xv) {
+                        vals[j] = xv;
+                        ids[j] = e;
+                    } else {
+                        vals[j] = vals[j - 1];
+                        ids[j] = ids[j - 1];
+                    }
+                }
+            }
+        }
+    }
+    const float vmax = vals[0];
+    float den = 0.f;
+    if (rp.normalize) {
+#pragma unroll
+        for (int j = 0; j < KS; ++j)
+            if (j < k) den += expf(vals[j] - vmax);
+    } else {
+#pragma unroll 4
+        for (int e = 0; e < E; ++e) den += expf(logit[e] + s_bias[e] - vmax);
+    }
+    int flags = 0;
+    float kth = 0.f, next = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+        if (j < k) {
+            rp.topk_idx[row * k + j] = ids[j];
+            rp.topk_w[row * k + j] = expf(vals[j] - vmax) / den;
+            if (rp.tile_counts) atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + ids[j]], 1);
+            if (j + 1 < k && vals[j] - vals[j + 1] < kNearTieGap) flags |= 2;
+        }
+        if (j == k - 1) kth = vals[j];
+        if (j == k) next = vals[j];
+    }
+    if (k < E && kth - next < kNearTieGap) flags |= 1;
+    if (rp.near_tie) rp.near_tie[row] = flags;
+}
+
 // ------------------------------------------------------------------------ split-K router
 // Router logits and routing for a few 128-token tiles (batched decode, mid-sized
 // prefill), where one CTA per tile would stream the whole K range alone.  A cluster of
@@ -406,8 +467,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // r 128 / CS .. of the tile: its threads fetch the CS partials of those rows through
 // distributed shared memory, 16-byte loads along the rows, all CS (and two or more row
 // groups) issued before the first is used, sum them in rank order 0 .. CS-1 (a fixed
-// order: the logits do not depend on timing) into a [row][e] block, and warps route the
-// rows with the warp top-k of the single-CTA router.  No global scratch; the host picks
+// order: the logits do not depend on timing) into a [row][e] block, and one thread per
+// row routes it (a warp per row, with its k + 1 rounds of warp reductions, took 1.3 us a
+// row).  No global scratch; the host picks
 // this kernel by (T, H, E) alone, for the staged router and the layer alike, so both
 // return the same bits.
 template <int E, int CS>
@@ -417,7 +479,7 @@ struct SplitCfg {
     static constexpr int kBBytes = E * BK * 2;                  // E router rows x 64 K
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kPartBytes = E * BM * 4;               // partials [e][row]
-    static constexpr int kRedBytes = kRows * (E + 1) * 4;       // sums [row][e], padded
+    static constexpr int kRedBytes = kRows * (E + 1) * 4 + E * 4;   // sums [row][e], padded; bias
     static constexpr int kStagesFit = (210 * 1024 - kPartBytes - kRedBytes) / kStageBytes;
     static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
     // barriers (full, empty: kStages each; tfull), then the TMEM slot and the abort flag
@@ -430,7 +492,7 @@ struct SplitCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
-template <int E, int CS>
+template <int E, int CS, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const TcParams p, const RouteParams rp) {
@@ -442,7 +504,8 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     uint8_t* sB = smem + C::kStages * C::kABytes;
     float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM]
     float* red = part + E * BM;                                             // [kRows][E + 1]
-    uint64_t* full = reinterpret_cast<uint64_t*>(red + C::kRows * (E + 1));
+    float* s_bias = red + C::kRows * (E + 1);                               // [E]
+    uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + E);
     uint64_t* empty = full + C::kStages;
     uint64_t* tfull = empty + C::kStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
@@ -474,6 +537,7 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // the prologue above touches no global memory; everything below may
     pdl_wait();
     pdl_trigger();
+    for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = rp.bias ? rp.bias[e] : 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -595,21 +659,20 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         }
     }
     __syncthreads();
+    if (rp.logits) {   // the staged router returns the logits it selected on
 #pragma unroll 1
-    for (int i = warp; i < C::kRows; i += kThreads / 32) {
-        const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
-        if (row >= static_cast<size_t>(p.rows)) continue;
-        const float* mine = red + i * (E + 1);
-        if (rp.logits)
-            for (int e = lane; e < E; e += 32) rp.logits[row * E + e] = mine[e] + (rp.bias ? rp.bias[e] : 0.f);
-        const WarpTopk res = warp_topk(mine, rp.bias, E, rp.k, rp.normalize, lane);
-        if (lane < rp.k) {
-            rp.topk_idx[row * rp.k + lane] = res.idx;
-            rp.topk_w[row * rp.k + lane] = res.w;
-            if (rp.tile_counts && static_cast<unsigned>(res.idx) < static_cast<unsigned>(E))
-                atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + res.idx], 1);
+        for (int i = warp; i < C::kRows; i += kThreads / 32) {
+            const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
+            if (row < static_cast<size_t>(p.rows))
+                for (int e = lane; e < E; e += 32) rp.logits[row * E + e] = red[i * (E + 1) + e] + s_bias[e];
         }
-        if (lane == 0 && rp.near_tie) rp.near_tie[row] = res.flags;
+    }
+    // one thread per row: the k + 1 (or more) largest biased logits in a descending
+    // register list, as in the one-CTA-per-tile router's epilogue
+    if (threadIdx.x < C::kRows) {
+        const int i = threadIdx.x;
+        const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
+        if (row < static_cast<size_t>(p.rows)) route_row<E, KS>(red + i * (E + 1), s_bias, row, tile, rp);
     }
     cluster_sync();   // no CTA leaves while a peer may still read its partials
     if (warp == 1) {
@@ -658,21 +721,11 @@ struct DecodeCfg {
     static constexpr int kStages = T::kStages;              // A (smem or TMEM) + token B ring
     static constexpr int kQStages = Q8 ? 16 : 0;            // int8 weight ring
     static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
-    // Accumulators.  A stage's four 16-wide K steps accumulate into four separate
-    // accumulators (64 columns each: at most 64 tokens), summed in a fixed order in the
-    // epilogue: with N <= 64 an MMA takes a few cycles of math but a long pipeline
-    // latency, and MMAs into one accumulator wait for each other, so a single chain of
-    // 4 MMAs per stage bounds the stage rate (measured: the int8 path, with half the
-    // bytes, ran no faster than bf16).  bf16: two buffers of 4 x 64 columns (the epilogue
-    // of one unit overlaps the next).  Q8: one buffer, then one A stage of 32 columns per
-    // ring stage.
     static constexpr int kAccStride = T::kAccStride;
-    static constexpr int kKSplit = BK / 16;
-    static constexpr int kSlots = Q8 ? 1 : 2;
-    static constexpr int kBufCols = kKSplit * kAccStride;
-    static constexpr int kTmemA = kSlots * kBufCols;
-    static constexpr int kTmemCols = 512;
-    static_assert(kTmemA + (Q8 ? kStages * 32 : 0) <= kTmemCols, "tensor memory");
+    // Q8: two accumulators (2 x 64 columns), then one A stage of 32 columns per ring stage
+    static constexpr int kTmemA = 2 * kAccStride;
+    static constexpr int kTmemCols = Q8 ? 512 : T::kTmemCols;
+    static_assert(!Q8 || kTmemA + kStages * 32 <= kTmemCols, "tensor memory");
     static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
     static constexpr int kMiscBytes = T::kMiscBytes + 2 * kQStages * 8;   // + int8 ring barriers
     static constexpr int kSmemBytes = 1024 + kDataBytes + kMiscBytes;
@@ -1162,8 +1215,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 const uint32_t idesc = idesc_bf16_f32(BM, ((d.nrows + 15) / 16) * 16);
                 if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                 tc_fence_after();
-                // K step kk of every stage accumulates into accumulator kk of the buffer
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kBufCols);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
@@ -1177,14 +1229,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                         // A: the converted stage in tensor memory, 8 columns per 16 K
                         const uint32_t at = tmem_base + static_cast<uint32_t>(C::kTmemA + stage * 32);
 #pragma unroll
-                        for (int kk = 0; kk < C::kKSplit; ++kk)
-                            umma_bf16_ta(d_tmem + kk * C::kAccStride, at + kk * 8,
-                                         smem_desc_sw128(b0 + kk * 32), idesc, kb != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16_ta(d_tmem, at + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc,
+                                         (kb | kk) != 0);
                     } else {
 #pragma unroll
-                        for (int kk = 0; kk < C::kKSplit; ++kk)
-                            umma_bf16(d_tmem + kk * C::kAccStride, smem_desc_sw128(a0 + kk * 32),
-                                      smem_desc_sw128(b0 + kk * 32), idesc, kb != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                      smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
                     }
                     umma_commit(smem_u32(&empty[stage]));
                     if (++stage == C::kStages) {
@@ -1194,10 +1246,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 }
                 if (!ok) break;
                 umma_commit(smem_u32(&tfull[acc]));
-                if (++acc == C::kSlots) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
             }
         }
     } else if (warp < 6) {
@@ -1223,7 +1273,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                static_cast<uint32_t>(acc * C::kBufCols);
+                                static_cast<uint32_t>(acc * C::kAccStride);
             const int wr = d.mt * BM + r;   // weight row inside the expert
             // this lane's weight row's bias (fc1: interleaved row wr in fc1's layout, fc2: h)
             const __nv_bfloat16* bsrc = f1 ? p.b1 : p.b2;
@@ -1234,18 +1284,13 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             const float scale = Q8 ? (f1 ? p.s1 : p.s2)[wi] : 1.f;
 #pragma unroll 1
             for (int c = 0; c < d.nrows; c += 16) {
-                // the four accumulators of the buffer, summed in order 0, 1, 2, 3
-                uint32_t v[C::kKSplit][16];
-#pragma unroll
-                for (int a = 0; a < C::kKSplit; ++a) tmem_ld_32x32b_x16(tb + a * C::kAccStride + c, v[a]);
+                uint32_t v[16];
+                tmem_ld_32x32b_x16(tb + c, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int n = c + i;
-                    float sum = f32(v[0][i]);
-#pragma unroll
-                    for (int a = 1; a < C::kKSplit; ++a) sum += f32(v[a][i]);
-                    const float x = Q8 ? fmaf(sum, scale, bias) : sum + bias;
+                    const float x = Q8 ? fmaf(f32(v[i]), scale, bias) : f32(v[i]) + bias;
                     if (f1) {
                         const float up = __shfl_xor_sync(0xffffffffu, x, 1);
                         if (!(lane & 1) && n < d.nrows)
@@ -1264,10 +1309,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 __threadfence();
                 atomicAdd(f1 ? &p.done[d.chunk] : p.fc2_done, 1);
             }
-            if (++acc == C::kSlots) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
         }
         if (p.out != nullptr) {
             // ------------------------------------------------------------ combine
@@ -1472,11 +1515,11 @@ int route_split_cluster(int T, int H, int E) {
     return 1;
 }
 
-template <int E, int CS>
+template <int E, int CS, int KS>
 cudaError_t launch_route_split(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p,
                                const RouteParams& rp, int tiles, cudaStream_t s) {
     using C = SplitCfg<E, CS>;
-    auto kern = tc_route_split_kernel<E, CS>;
+    auto kern = tc_route_split_kernel<E, CS, KS>;
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -1554,8 +1597,10 @@ cudaError_t launch_route_tc(const void* hidden, const void* router_w, const floa
     const int cs = route_split_cluster(T, H, E);
     const int tiles = (T + BM - 1) / BM;
     if (cs > 1) {
-#define MOE_SPLIT_CASE(EV, CV) \
-    if (E == EV && cs == CV) return launch_route_split<EV, CV>(ma, mb, p, rp, tiles, s);
+#define MOE_SPLIT_CASE(EV, CV)                                                            \
+    if (E == EV && cs == CV)                                                              \
+        return k <= 8 ? launch_route_split<EV, CV, 9>(ma, mb, p, rp, tiles, s)             \
+                      : launch_route_split<EV, CV, 33>(ma, mb, p, rp, tiles, s);
         MOE_SPLIT_CASE(64, 2) MOE_SPLIT_CASE(64, 4) MOE_SPLIT_CASE(64, 8)
         MOE_SPLIT_CASE(128, 2) MOE_SPLIT_CASE(128, 4) MOE_SPLIT_CASE(128, 8)
 #undef MOE_SPLIT_CASE
