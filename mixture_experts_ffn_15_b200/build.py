@@ -21,9 +21,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["api.cu", "route.cu", "route_small.cu", "permute.cu", "combine.cu", "ffn_simt.cu",
-           "gemm_tc.cu", "gemm_pair.cu", "static_scratch.cu", "rmsnorm.cu"]
+           "gemm_tc.cu", "route_tc.cu", "gemm_pair.cu", "static_scratch.cu", "rmsnorm.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h", "combine.cuh", "topk_warp.cuh", "tile_map.cuh",
-           "tmap.cuh"]
+           "tmap.cuh", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,13 +1,4 @@
-// Single-CTA tcgen05 kernels (sm_100a): the router GEMM with the routing in its
-// epilogue, and the decode FFN.
-//
-// Router ("Gemma 4 MoE: re-enable fused com.microsoft::MoE op - #326", "Attribute
-// set": k = top_k, normalize_routing_weights): logits[t, e] = hidden[t] . router_w[e]
-// (+ bias) for 128-token tiles on M and all E experts on N; the epilogue selects,
-// weighs and counts (per-tile bincount of "Contributing Gemma 4 support and ONNX
-// export optimizations", "Key Technical Contributions").
-//
-// Decode FFN: the grouped matmul of grouped_mm_experts_forward for batches with few
+// Decode FFN on the tensor cores (sm_100a): the grouped matmul of grouped_mm_experts_forward for batches with few
 // rows per expert, fc1 + SwiGLU and fc2 (standard SwiGLU, interleaved fc1) in one
 // persistent launch with 128 weight rows on M and the expert's tokens on N, so that
 // every weight byte streams from HBM once; optionally with the routing and the
@@ -33,6 +24,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 #include "tile_map.cuh"
 #include "tmap.cuh"
 #include "topk_warp.cuh"
@@ -41,646 +33,7 @@ namespace moe {
 namespace {
 
 using namespace sm100;
-
-constexpr int BM = 128;              // rows of A per tile (MMA M)
-constexpr int BK = 64;               // K per stage: one 128-byte row of bf16
-static_assert(BK == tmap::kBoxK, "TMA box width");
-constexpr int kThreads = 192;
-constexpr int kTokChunk = 64;        // weight-M: tokens per unit
-constexpr int kBoxTok = 16;          // weight-M: token rows per TMA box
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-// TOK_ROUTE: router logits with the routing itself in the epilogue (top-k, softmax,
-// near-tie flags, per-tile bincount).
-enum Mode : int { W_PLAIN = 4, TOK_ROUTE = 5 };
-
-template <int MODE, int BN>
-struct Tr {
-    static constexpr bool kWeightM = (MODE == W_PLAIN);
-    static constexpr int kBRows = kWeightM ? kTokChunk : BN;
-    static constexpr int kABytes = BM * BK * 2;
-    static constexpr int kBBytes = kBRows * BK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
-    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-    static constexpr int kAccStride = kWeightM ? kTokChunk : 256;
-    static constexpr int kTmemCols = kWeightM ? 128 : 512;
-    // barriers, tmem slot + abort flag, offsets, prefix, gather rows of one chunk
-    static constexpr int kMiscBytes =
-        (2 * kStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 16 * 8 + 64 +
-        (MODE == TOK_ROUTE ? 5 * kMaxExperts * 4 : 0);   // bias [E], counts [4][E]
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kMiscBytes;
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-    static_assert(kWeightM || (BN % 16 == 0 && BN >= 16 && BN <= 256), "UMMA N");
-};
-
-struct TcParams {
-    const int32_t* offsets;   // [E+1] device, or nullptr: one group of `rows` rows
-    int E;
-    int rows;                 // rows of the token matrix
-    int K;                    // reduction length (multiple of 64)
-    int n_out;                // weight rows per expert
-    void* out;
-    int ldo;                  // output row stride, elements
-    int32_t* err;
-};
-
-// The routing half of TOK_ROUTE (n_out = number of experts).
-struct RouteParams {
-    const float* bias;        // [E] or nullptr
-    int k, normalize;
-    int32_t* topk_idx;        // [T, k]
-    float* topk_w;            // [T, k]
-    int32_t* near_tie;        // [T] or nullptr
-    float* logits;            // [T, E] or nullptr (logits + bias)
-    int32_t* tile_counts;     // [ceil(T / 128), E]
-};
-
-struct Unit {
-    int g;      // expert
-    int row0;   // first token row
-    int nrows;  // valid token rows (<= kUnitRows)
-    int sub;    // column tile (token-M) or weight row tile (weight-M) inside the expert
-};
-
-__device__ __forceinline__ void build_tile_map(const TcParams& p, int G, int unit_rows, int* s_off,
-                                               int* s_pre, int lane) {
-    build_group_tiles(p.offsets, p.rows, p.err, G, unit_rows, s_off, s_pre, lane);
-}
-
-__device__ __forceinline__ Unit decode_unit(int u, int per_unit, int G, int unit_rows,
-                                            const int* s_off, const int* s_pre) {
-    const int tile = u / per_unit;
-    Unit t;
-    t.sub = u - tile * per_unit;
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    t.g = lo;
-    t.row0 = s_off[lo] + (tile - s_pre[lo]) * unit_rows;
-    t.nrows = min(unit_rows, s_off[lo + 1] - t.row0);
-    return t;
-}
-
-__device__ __forceinline__ float f32(uint32_t x) { return __uint_as_float(x); }
-
-// Routing of one 128-token tile from its logits in TMEM (columns 0..E-1, thread =
-// token row).  Each thread keeps the KS = k+1 (or more) largest biased logits in a
-// register list sorted descending, inserting the experts in index order so that equal
-// logits keep the lower index first; then the softmax weights over the chosen k (or,
-// normalize = 0, over all E), the near-tie flags, and the tile's bincount: per warp in
-// shared memory (s_cnt is this warp's [E] slice), then added to tile_counts.
-template <int E, int KS>
-__device__ __forceinline__ void route_epilogue(uint32_t tb, bool valid, size_t row, int tile,
-                                               const RouteParams& rp, const float* s_bias,
-                                               int* s_cnt, int lane) {
-    const int k = rp.k;
-    float vals[KS];
-    int ids[KS];
-#pragma unroll
-    for (int j = 0; j < KS; ++j) {
-        vals[j] = -INFINITY;
-        ids[j] = -1;
-    }
-#pragma unroll 1
-    for (int c = 0; c < E; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tb + c, v);
-        tmem_wait_ld();
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = f32(v[i]) + s_bias[c + i];
-        if (valid && rp.logits) {
-            uint4* dst = reinterpret_cast<uint4*>(rp.logits + row * E + c);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                dst[q] = make_uint4(__float_as_uint(x[4 * q]), __float_as_uint(x[4 * q + 1]),
-                                    __float_as_uint(x[4 * q + 2]), __float_as_uint(x[4 * q + 3]));
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float xv = x[i];
-            if (xv > vals[KS - 1]) {
-                const int e = c + i;
-#pragma unroll
-                for (int j = KS - 1; j >= 0; --j) {
-                    if (vals[j] < xv) {
-                        if (j == 0 || vals[j - 1] >= xv) {
-                            vals[j] = xv;
-                            ids[j] = e;
-                        } else {
-                            vals[j] = vals[j - 1];
-                            ids[j] = ids[j - 1];
-                        }
-                    }
-                }
-            }
-        }
-    }
-    // rows past the batch hold bias-only logits (their A rows were zero-filled): finite
-    const float vmax = vals[0];
-    float den = 0.f;
-    if (rp.normalize) {
-#pragma unroll
-        for (int j = 0; j < KS; ++j)
-            if (j < k) den += expf(vals[j] - vmax);
-    } else {
-        // softmax over all E: a second, warp-uniform pass over the logits in TMEM
-#pragma unroll 1
-        for (int c = 0; c < E; c += 32) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tb + c, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) den += expf(f32(v[i]) + s_bias[c + i] - vmax);
-        }
-    }
-    if (valid) {
-        int flags = 0;
-        float kth = 0.f, next = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < KS; ++j) {
-            if (j < k) {
-                rp.topk_idx[row * k + j] = ids[j];
-                rp.topk_w[row * k + j] = expf(vals[j] - vmax) / den;
-                atomicAdd(&s_cnt[ids[j]], 1);
-                if (j + 1 < k && vals[j] - vals[j + 1] < kNearTieGap) flags |= 2;
-            }
-            if (j == k - 1) kth = vals[j];
-            if (j == k) next = vals[j];
-        }
-        if (k < E && kth - next < kNearTieGap) flags |= 1;
-        if (rp.near_tie) rp.near_tie[row] = flags;
-    }
-    // this warp's 32 rows: add its counts to the tile's (zeroed before the launch) and
-    // clear them for the next tile; warp-local, so a warp that gave up on a wait never
-    // holds the others at a barrier
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) {
-        const int c = s_cnt[e];
-        if (c) {
-            if (rp.tile_counts) atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + e], c);
-            s_cnt[e] = 0;
-        }
-    }
-    __syncwarp();
-}
-
-template <int MODE, int BN, int KS = 1>
-__global__ void __launch_bounds__(kThreads, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const TcParams p, const RouteParams rp) {
-    using C = Tr<MODE, BN>;
-    static_assert(!C::kWeightM, "weight rows on M run in tc_ffn_decode_kernel");
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + C::kStages * C::kABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* tfull = empty + C::kStages;
-    uint64_t* tempty = tfull + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
-    int* s_pre = s_off + (kMaxExperts + 1);
-    float* s_bias = reinterpret_cast<float*>(s_pre + (kMaxExperts + 1));   // TOK_ROUTE
-    int* s_cnt = reinterpret_cast<int*>(s_bias + kMaxExperts);            // TOK_ROUTE
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = p.offsets ? p.E : 1;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 4);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-        tmem_relinquish();
-    }
-    // the prologue above touches no global memory; everything below may
-    pdl_wait();
-    pdl_trigger();
-    if (warp == 2) build_tile_map(p, G, BM, s_off, s_pre, lane);
-    if constexpr (MODE == TOK_ROUTE) {
-        for (int e = threadIdx.x; e < BN; e += kThreads) s_bias[e] = rp.bias ? rp.bias[e] : 0.f;
-        for (int e = threadIdx.x; e < 4 * BN; e += kThreads) s_cnt[e] = 0;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    const int per_unit = p.n_out / BN;
-    const int num_units = s_pre[G] * per_unit;
-    const int nk = p.K / BK;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            long long issued = 0;
-            for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-                const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
-                const uint32_t bytes = C::kStageBytes;
-                const int wrow = t.g * p.n_out + t.sub * BN;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
-                    const uint32_t fb = smem_u32(&full[stage]);
-                    mbar_arrive_expect_tx(fb, bytes);
-                    const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
-                    const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                    tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
-                    tma_load_2d(b_dst, &tmB, fb, kb * BK, wrow);
-                    ++issued;
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            if (*abort_flag) {
-                // let the copies already in flight land before the CTA exits
-                int dummy = 0;
-                for (int s = 0; s < C::kStages; ++s) {
-                    if (issued <= s) break;
-                    const long long fills = (issued - 1 - s) / C::kStages + 1;
-                    mbar_wait(smem_u32(&full[s]), static_cast<uint32_t>((fills - 1) & 1),
-                              &dummy, kWaitLimitNs / 4);
-                }
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
-            for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-                const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
-                const uint32_t idesc = idesc_bf16_f32(BM, BN);
-                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
-                bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                                  idesc, (kb | kk) != 0);
-                    umma_commit(smem_u32(&empty[stage]));
-                    if (++stage == C::kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (!ok) break;
-                umma_commit(smem_u32(&tfull[acc]));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1u;
-            }
-        }
-    } else {
-        // ------------------------------------------------------------ epilogue
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;   // TMEM lane = row of the accumulator
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        for (int u = blockIdx.x; u < num_units && !*abort_flag; u += gridDim.x) {
-            const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
-            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kWaitLimitNs)) break;
-            tc_fence_after();
-            const uint32_t tb =
-                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * C::kAccStride);
-            const bool valid = r < t.nrows;
-            const size_t orow = static_cast<size_t>(t.row0 + r);
-            route_epilogue<BN, KS>(tb, valid, orow, t.row0 / BM, rp, s_bias,
-                                   s_cnt + quad * BN, lane);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
-    }
-    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
-}
-
-// Routing of one token row from its E raw logits in shared memory (one thread): the
-// KS = k+1 (or more) largest biased logits in a register list sorted descending,
-// experts inserted in index order so that equal logits keep the lower index first;
-// softmax weights over the chosen k (normalize) or over all E, near-tie flags, and the
-// row's k counts added to the tile's bincount.
-template <int E, int KS>
-__device__ __forceinline__ void route_row(const float* logit, const float* s_bias, size_t row,
-                                          int tile, const RouteParams& rp) {
-    const int k = rp.k;
-    float vals[KS];
-    int ids[KS];
-#pragma unroll
-    for (int j = 0; j < KS; ++j) {
-        vals[j] = -INFINITY;
-        ids[j] = -1;
-    }
-#pragma unroll 4
-    for (int e = 0; e < E; ++e) {
-        const float xv = logit[e] + s_bias[e];
-        if (xv > vals[KS - 1]) {
-#pragma unroll
-            for (int j = KS - 1; j >= 0; --j) {
-                if (vals[j] < xv) {
-                    if (j == 0 || vals[j - 1] >= xv) {
-                        vals[j] = xv;
-                        ids[j] = e;
-                    } else {
-                        vals[j] = vals[j - 1];
-                        ids[j] = ids[j - 1];
-                    }
-                }
-            }
-        }
-    }
-    const float vmax = vals[0];
-    float den = 0.f;
-    if (rp.normalize) {
-#pragma unroll
-        for (int j = 0; j < KS; ++j)
-            if (j < k) den += expf(vals[j] - vmax);
-    } else {
-#pragma unroll 4
-        for (int e = 0; e < E; ++e) den += expf(logit[e] + s_bias[e] - vmax);
-    }
-    int flags = 0;
-    float kth = 0.f, next = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < KS; ++j) {
-        if (j < k) {
-            rp.topk_idx[row * k + j] = ids[j];
-            rp.topk_w[row * k + j] = expf(vals[j] - vmax) / den;
-            if (rp.tile_counts) atomicAdd(&rp.tile_counts[static_cast<size_t>(tile) * E + ids[j]], 1);
-            if (j + 1 < k && vals[j] - vals[j + 1] < kNearTieGap) flags |= 2;
-        }
-        if (j == k - 1) kth = vals[j];
-        if (j == k) next = vals[j];
-    }
-    if (k < E && kth - next < kNearTieGap) flags |= 1;
-    if (rp.near_tie) rp.near_tie[row] = flags;
-}
-
-// ------------------------------------------------------------------------ split-K router
-// Router logits and routing for a few 128-token tiles (batched decode, mid-sized
-// prefill), where one CTA per tile would stream the whole K range alone.  A cluster of
-// CS CTAs runs one tile: CTA r accumulates the K slices [r nk / CS, (r + 1) nk / CS) on
-// the tensor cores (128 tokens on M, all E experts on N) and stores its partial logits
-// in its own shared memory, [e][row].  After a cluster barrier, CTA r takes the rows
-// r 128 / CS .. of the tile: its threads fetch the CS partials of those rows through
-// distributed shared memory, 16-byte loads along the rows, all CS (and two or more row
-// groups) issued before the first is used, sum them in rank order 0 .. CS-1 (a fixed
-// order: the logits do not depend on timing) into a [row][e] block, and one thread per
-// row routes it (a warp per row, with its k + 1 rounds of warp reductions, took 1.3 us a
-// row).  No global scratch; the host picks
-// this kernel by (T, H, E) alone, for the staged router and the layer alike, so both
-// return the same bits.
-template <int E, int CS>
-struct SplitCfg {
-    static constexpr int kRows = BM / CS;                       // rows reduced and routed per CTA
-    static constexpr int kABytes = BM * BK * 2;                 // 128 token rows x 64 K
-    static constexpr int kBBytes = E * BK * 2;                  // E router rows x 64 K
-    static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kPartBytes = E * BM * 4;               // partials [e][row]
-    static constexpr int kRedBytes = kRows * (E + 1) * 4 + E * 4;   // sums [row][e], padded; bias
-    static constexpr int kStagesFit = (210 * 1024 - kPartBytes - kRedBytes) / kStageBytes;
-    static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
-    // barriers (full, empty: kStages each; tfull), then the TMEM slot and the abort flag
-    static constexpr int kMiscBytes = (2 * kStages + 1) * 8 + 16;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPartBytes + kRedBytes + kMiscBytes;
-    static constexpr int kTmemCols = E;                         // 64 or 128
-    static constexpr int kGroupsPerPass = 16 / CS;              // 16 loads in flight a thread
-    static_assert(kStages >= 2, "pipeline");
-    static_assert(kRows % 4 == 0, "16-byte row groups");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-};
-
-template <int E, int CS, int KS>
-__global__ void __launch_bounds__(kThreads, 1)
-tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const TcParams p, const RouteParams rp) {
-    using C = SplitCfg<E, CS>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + C::kStages * C::kABytes;
-    float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM]
-    float* red = part + E * BM;                                             // [kRows][E + 1]
-    float* s_bias = red + C::kRows * (E + 1);                               // [E]
-    uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + E);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* tfull = empty + C::kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int tile = static_cast<int>(blockIdx.x) / CS;
-    const int nk = p.K / BK;
-    const int kb0 = nk * rank / CS, kb1 = nk * (rank + 1) / CS;   // CS <= nk: never empty
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), 1);
-        }
-        mbar_init(smem_u32(tfull), 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
-        tmem_relinquish();
-    }
-    // the prologue above touches no global memory; everything below may
-    pdl_wait();
-    pdl_trigger();
-    for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = rp.bias ? rp.bias[e] : 0.f;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            long long issued = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
-                const uint32_t fb = smem_u32(&full[stage]);
-                mbar_arrive_expect_tx(fb, C::kStageBytes);
-                tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * BK, tile * BM);
-                tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * BK, 0);
-                ++issued;
-                if (++stage == C::kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (*abort_flag) {
-                // let the copies already in flight land before the CTA goes on
-                int dummy = 0;
-                for (int s2 = 0; s2 < C::kStages; ++s2) {
-                    if (issued <= s2) break;
-                    const long long fills = (issued - 1 - s2) / C::kStages + 1;
-                    mbar_wait(smem_u32(&full[s2]), static_cast<uint32_t>((fills - 1) & 1), &dummy,
-                              kWaitLimitNs / 4);
-                }
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(BM, E);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb) {
-                if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-                const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
-#pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    umma_bf16(tmem_base, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                              idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
-                umma_commit(smem_u32(&empty[stage]));
-                if (++stage == C::kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (ok) umma_commit(smem_u32(tfull));
-        }
-    } else {
-        // ------------------------------------------------------------ partials
-        // warps 2..5: TMEM lane quadrant warp % 4; thread = token row r of the tile
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;
-        if (mbar_wait(smem_u32(tfull), 0, abort_flag, kWaitLimitNs)) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < E; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) part[(c + i) * BM + r] = __uint_as_float(v[i]);
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();   // every CTA's partials are written and visible to the cluster
-
-    // ---------------------------------------------------------------- reduce and route
-    // position i = (e, row group of 4): the float4 at part[e][row0 + 4 g] of every rank
-    constexpr int kGroups = C::kRows / 4;
-    constexpr int kPos = E * kGroups;
-    const int row0 = rank * C::kRows;
-#pragma unroll 1
-    for (int i0 = threadIdx.x; i0 < kPos; i0 += kThreads * C::kGroupsPerPass) {
-        float4 v[C::kGroupsPerPass][CS];
-#pragma unroll
-        for (int j = 0; j < C::kGroupsPerPass; ++j) {
-            const int i = i0 + j * kThreads;
-            if (i < kPos) {
-                const int e = i / kGroups, g = i - e * kGroups;
-                const uint32_t a = smem_u32(&part[e * BM + row0 + 4 * g]);
-#pragma unroll
-                for (int q = 0; q < CS; ++q) v[j][q] = ld_shared_cluster_v4(mapa_shared(a, q));
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < C::kGroupsPerPass; ++j) {
-            const int i = i0 + j * kThreads;
-            if (i < kPos) {
-                const int e = i / kGroups, g = i - e * kGroups;
-                float4 sum = v[j][0];
-#pragma unroll
-                for (int q = 1; q < CS; ++q) {
-                    sum.x += v[j][q].x;
-                    sum.y += v[j][q].y;
-                    sum.z += v[j][q].z;
-                    sum.w += v[j][q].w;
-                }
-                red[(4 * g + 0) * (E + 1) + e] = sum.x;
-                red[(4 * g + 1) * (E + 1) + e] = sum.y;
-                red[(4 * g + 2) * (E + 1) + e] = sum.z;
-                red[(4 * g + 3) * (E + 1) + e] = sum.w;
-            }
-        }
-    }
-    __syncthreads();
-    if (rp.logits) {   // the staged router returns the logits it selected on
-#pragma unroll 1
-        for (int i = warp; i < C::kRows; i += kThreads / 32) {
-            const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
-            if (row < static_cast<size_t>(p.rows))
-                for (int e = lane; e < E; e += 32) rp.logits[row * E + e] = red[i * (E + 1) + e] + s_bias[e];
-        }
-    }
-    // one thread per row: the k + 1 (or more) largest biased logits in a descending
-    // register list, as in the one-CTA-per-tile router's epilogue
-    if (threadIdx.x < C::kRows) {
-        const int i = threadIdx.x;
-        const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
-        if (row < static_cast<size_t>(p.rows)) route_row<E, KS>(red + i * (E + 1), s_bias, row, tile, rp);
-    }
-    cluster_sync();   // no CTA leaves while a peer may still read its partials
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
-    }
-    if (threadIdx.x == 0 && *abort_flag && p.err) atomicOr(p.err, kErrTimeout);
-}
+using namespace tc;
 
 // ------------------------------------------------------------------------ decode FFN
 // fc1 + SwiGLU and fc2 for batches with few rows per expert, in ONE persistent
@@ -1482,71 +835,6 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
 
 // ------------------------------------------------------------------------ host side
 
-template <int MODE, int BN, int KS = 1>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p, int bound,
-                       cudaStream_t s, const RouteParams& rp = RouteParams{}) {
-    using C = Tr<MODE, BN>;
-    auto kern = tc_gemm_kernel<MODE, BN, KS>;
-    // once per device (outside any stream capture: the first call of every path
-    // runs eagerly before a graph is captured)
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
-    int grid = device_sm_count();
-    if (bound < grid) grid = bound;
-    if (grid <= 0) return cudaSuccess;
-    return launch_k(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, s, a, b, p, rp);
-}
-
-// Cluster size of the split-K router for these sizes (1: the one-CTA-per-tile router).
-// A pure function of the sizes (a fixed budget of 148 CTAs, not the device's count), so
-// that the staged router and the layer take the same kernel and give the same bits.
-int route_split_cluster(int T, int H, int E) {
-    if (E != 64 && E != 128) return 1;
-    const int tiles = (T + BM - 1) / BM, nk = H / BK;
-    for (int cs = 8; cs >= 2; cs >>= 1)
-        if (tiles * cs <= 148 && cs <= nk) return cs;
-    return 1;
-}
-
-template <int E, int CS, int KS>
-cudaError_t launch_route_split(const CUtensorMap& a, const CUtensorMap& b, const TcParams& p,
-                               const RouteParams& rp, int tiles, cudaStream_t s) {
-    using C = SplitCfg<E, CS>;
-    auto kern = tc_route_split_kernel<E, CS, KS>;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles * CS));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    count_launch();
-    return cudaLaunchKernelEx(&cfg, kern, a, b, p, rp);
-}
-
 // Grid of a persistent decode FFN launch: every unit of both GEMMs, at most one CTA per SM.
 int decode_grid(int rows, int E, int H, int I) {
     const long long units =
@@ -1579,48 +867,6 @@ cudaError_t launch_decode(const CUtensorMap& w1, const CUtensorMap& x, const CUt
 }  // namespace
 
 bool tc_ffn_supported(int H, int I) { return H % 64 == 0 && I % 64 == 0 && H > 0 && I > 0; }
-
-bool tc_route_supported(int H, int E, int k) {
-    return H % 64 == 0 && (E == 64 || E == 128 || E == 256) && k >= 1 && k <= 32;
-}
-
-cudaError_t launch_route_tc(const void* hidden, const void* router_w, const float* bias, int T,
-                            int H, int E, int k, int normalize, int32_t* topk_idx, float* topk_w,
-                            int32_t* near_tie, float* logits, int32_t* tile_counts, int32_t* err,
-                            cudaStream_t s) {
-    if (T <= 0) return cudaSuccess;
-    TcParams p{nullptr, 1, T, H, E, nullptr, E, err};
-    RouteParams rp{bias, k, normalize ? 1 : 0, topk_idx, topk_w, near_tie, logits, tile_counts};
-    CUtensorMap ma, mb;
-    if (!tmap::matrix(&ma, hidden, T, H, BM)) return cudaErrorInvalidValue;
-    if (!tmap::matrix(&mb, router_w, E, H, E)) return cudaErrorInvalidValue;
-    const int cs = route_split_cluster(T, H, E);
-    const int tiles = (T + BM - 1) / BM;
-    if (cs > 1) {
-#define MOE_SPLIT_CASE(EV, CV)                                                            \
-    if (E == EV && cs == CV)                                                              \
-        return k <= 8 ? launch_route_split<EV, CV, 9>(ma, mb, p, rp, tiles, s)             \
-                      : launch_route_split<EV, CV, 33>(ma, mb, p, rp, tiles, s);
-        MOE_SPLIT_CASE(64, 2) MOE_SPLIT_CASE(64, 4) MOE_SPLIT_CASE(64, 8)
-        MOE_SPLIT_CASE(128, 2) MOE_SPLIT_CASE(128, 4) MOE_SPLIT_CASE(128, 8)
-#undef MOE_SPLIT_CASE
-        return cudaErrorInvalidValue;
-    }
-    const int bound = (T + BM - 1) / BM;
-    const bool small_k = k <= 8;
-#define MOE_ROUTE_CASE(EV)                                                                   \
-    case EV:                                                                                 \
-        return small_k ? launch_one<TOK_ROUTE, EV, 9>(ma, mb, p, bound, s, rp)               \
-                       : launch_one<TOK_ROUTE, EV, 33>(ma, mb, p, bound, s, rp);
-    switch (E) {
-        MOE_ROUTE_CASE(64)
-        MOE_ROUTE_CASE(128)
-        MOE_ROUTE_CASE(256)
-        default:
-            return cudaErrorInvalidValue;
-    }
-#undef MOE_ROUTE_CASE
-}
 
 bool decode_ffn_supported(int rows, int E, int H, int I) {
     return tc_ffn_supported(H, I) && (2 * I) % BM == 0 && H % BM == 0 &&
