@@ -41,8 +41,9 @@ using namespace tc;
 // (a chunk of at most 64 permuted rows) on N, so every weight byte streams from HBM
 // once.  The unit list holds every fc1 unit (chunk x 128 rows of fc1) and then every
 // fc2 unit (chunk x 128 rows of fc2).  CTAs claim units in that order from a global
-// counter (the producer warp claims, a 4-slot ring in shared memory hands the unit to
-// the MMA and epilogue warps), so the large fc1 units go first and the small fc2 units
+// counter (the producer warp claims -- with int8 experts the int8 producer, which runs
+// furthest ahead -- and a 4-slot ring in shared memory hands the unit to the other
+// warps), so the large fc1 units go first and the small fc2 units
 // even out the end; every fc1 unit is claimed before any fc2 unit.  An fc2 unit needs the
 // activations of its chunk: each fc1 epilogue warp publishes its stores with a proxy
 // fence and a release increment of the chunk's counter, and the fc2 producer waits
@@ -61,7 +62,7 @@ constexpr int kUnitRing = 4;
 // of their own (kQStages tiles of 128 rows x 64 bytes, loaded by a dedicated producer
 // warp); converter warps turn each tile into bf16 -- exact, |q| <= 127 -- and store it
 // straight into tensor memory, where the MMA reads its A operand (two groups of four
-// warps taking alternate k-steps, so that two tiles convert at once); shared memory
+// warps taking alternate stages, so that two stages convert at once); shared memory
 // carries only int8 weights and token rows.  The epilogue multiplies each weight row's
 // accumulator by its float32 scale.  The token side is the bf16 path's.
 constexpr int kQBytes = BM * BK;   // one int8 tile: 128 weight rows x 64 K
@@ -71,15 +72,23 @@ struct DecodeCfg {
     using T = Tr<W_PLAIN, 64>;
     static constexpr int kABytes = Q8 ? 0 : T::kABytes;     // Q8: A lives in tensor memory
     static constexpr int kBBytes = T::kBBytes;
-    static constexpr int kStages = T::kStages;              // A (smem or TMEM) + token B ring
+    // The ring holds kSlots 64-K slots (A in shared or tensor memory + token B); the
+    // barriers work on stages of kSub consecutive slots, so that every wait and commit
+    // of the MMA thread covers 4 kSub MMAs: a wait on an mbarrier costs the issuing
+    // thread ~160 cycles even when the phase has completed, and a commit ~90, against
+    // ~60 for an M = 128, N <= 64, K = 16 MMA.
+    static constexpr int kSlots = T::kStages;
+    static constexpr int kSub = 2;
+    static constexpr int kStages = kSlots / kSub;
+    static_assert(kStages * kSub == kSlots, "whole stages");
     static constexpr int kQStages = Q8 ? 16 : 0;            // int8 weight ring
     static constexpr int kThreads = Q8 ? 480 : 192;         // + Q producer + 2 x 4 converters
     static constexpr int kAccStride = T::kAccStride;
     // Q8: two accumulators (2 x 64 columns), then one A stage of 32 columns per ring stage
     static constexpr int kTmemA = 2 * kAccStride;
     static constexpr int kTmemCols = Q8 ? 512 : T::kTmemCols;
-    static_assert(!Q8 || kTmemA + kStages * 32 <= kTmemCols, "tensor memory");
-    static constexpr int kDataBytes = kStages * (kABytes + kBBytes) + kQStages * kQBytes;
+    static_assert(!Q8 || kTmemA + kSlots * 32 <= kTmemCols, "tensor memory");
+    static constexpr int kDataBytes = kSlots * (kABytes + kBBytes) + kQStages * kQBytes;
     static constexpr int kMiscBytes = T::kMiscBytes + 2 * kQStages * 8;   // + int8 ring barriers
     static constexpr int kSmemBytes = 1024 + kDataBytes + kMiscBytes;
     static_assert(kStages <= T::kStages, "barrier space");
@@ -202,8 +211,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + C::kStages * C::kABytes;
-    uint8_t* sQ = sB + C::kStages * C::kBBytes;               // Q8: int8 weight ring
+    uint8_t* sB = smem + C::kSlots * C::kABytes;
+    uint8_t* sQ = sB + C::kSlots * C::kBBytes;                // Q8: int8 weight ring
     uint64_t* full = reinterpret_cast<uint64_t*>(sQ + C::kQStages * kQBytes);
     uint64_t* empty = full + C::kStages;
     uint64_t* tfull = empty + C::kStages;
@@ -241,7 +250,8 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         }
         for (int q = 0; q < kUnitRing; ++q) {
             mbar_init(smem_u32(&ufull[q]), 1);
-            // the MMA thread and 4 epilogue warps (Q8: + the int8 producer and 8 converters)
+            // the MMA thread and 4 epilogue warps (Q8: + the token producer and 8 converters;
+            // the int8 producer claims)
             mbar_init(smem_u32(&uempty[q]), Q8 ? 14 : 5);
         }
         for (int q = 0; q < C::kQStages; ++q) {
@@ -462,10 +472,18 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         for (;;) {
             int u = U;
             if (lane == 0) {
-                if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
-                    u = *abort_flag ? U : atomicAdd(p.sched, 1);
-                s_unit[slot] = u;
-                mbar_arrive(smem_u32(&ufull[slot]));
+                if constexpr (Q8) {
+                    // the int8 producer claims; this warp reads the ring like the others
+                    if (mbar_wait(smem_u32(&ufull[slot]), uphase, abort_flag, kWaitLimitNs)) {
+                        u = s_unit[slot];
+                        mbar_arrive(smem_u32(&uempty[slot]));
+                    }
+                } else {
+                    if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
+                        u = *abort_flag ? U : atomicAdd(p.sched, 1);
+                    s_unit[slot] = u;
+                    mbar_arrive(smem_u32(&ufull[slot]));
+                }
             }
             u = __shfl_sync(0xffffffffu, u, 0);
             if (++slot == kUnitRing) {
@@ -507,25 +525,31 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 fence_proxy_async_global();
             }
             bool ok = true;
-            for (int kb = 0; kb < nk; ++kb) {
+            for (int kb0 = 0; kb0 < nk; kb0 += C::kSub) {
+                const int ns = min(C::kSub, nk - kb0);   // slots of this stage (the last may be short)
                 if (lane == 0) {
                     ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
-                    if (ok) mbar_arrive_expect_tx(smem_u32(&full[stage]), (Q8 ? 0 : C::kABytes) + bbytes);
+                    if (ok)
+                        mbar_arrive_expect_tx(smem_u32(&full[stage]),
+                                              static_cast<uint32_t>(ns) * ((Q8 ? 0 : C::kABytes) + bbytes));
                 }
                 // the whole warp leaves together (lane 0 alone saw the wait give up)
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 const uint32_t fb = smem_u32(&full[stage]);
-                const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
-                const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                if (!Q8 && lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
-                if (f1 && GATHER) {
-                    if (lane < nl4)
-                        tma_gather4(b_dst + lane * 4 * BK * 2, &tmX, fb, kb * BK, src[0], src[1],
-                                    src[2], src[3]);
-                } else if (lane < nl) {
-                    tma_load_2d(b_dst + lane * kBoxTok * BK * 2, f1 ? &tmX : &tmAct, fb, kb * BK,
-                                d.row0 + lane * kBoxTok);
+                for (int j = 0; j < ns; ++j) {
+                    const int kb = kb0 + j, sl = stage * C::kSub + j;
+                    const uint32_t a_dst = smem_u32(sA + sl * C::kABytes);
+                    const uint32_t b_dst = smem_u32(sB + sl * C::kBBytes);
+                    if (!Q8 && lane == 0) tma_load_4d(a_dst, ma, fb, kb * BK, 0, d.mt * (BM / 2), d.g);
+                    if (f1 && GATHER) {
+                        if (lane < nl4)
+                            tma_gather4(b_dst + lane * 4 * BK * 2, &tmX, fb, kb * BK, src[0], src[1],
+                                        src[2], src[3]);
+                    } else if (lane < nl) {
+                        tma_load_2d(b_dst + lane * kBoxTok * BK * 2, f1 ? &tmX : &tmAct, fb, kb * BK,
+                                    d.row0 + lane * kBoxTok);
+                    }
                 }
                 ++issued;
                 if (++stage == C::kStages) {
@@ -570,26 +594,30 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb0 = 0; kb0 < nk; kb0 += C::kSub) {
+                    const int ns = min(C::kSub, nk - kb0);
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
-                    if constexpr (Q8) {
-                        // A: the converted stage in tensor memory, 8 columns per 16 K
-                        const uint32_t at = tmem_base + static_cast<uint32_t>(C::kTmemA + stage * 32);
+                    for (int j = 0; j < ns; ++j) {
+                        const int kb = kb0 + j, sl = stage * C::kSub + j;
+                        const uint32_t a0 = smem_u32(sA + sl * C::kABytes);
+                        const uint32_t b0 = smem_u32(sB + sl * C::kBBytes);
+                        if constexpr (Q8) {
+                            // A: the converted slot in tensor memory, 8 columns per 16 K
+                            const uint32_t at = tmem_base + static_cast<uint32_t>(C::kTmemA + sl * 32);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16_ta(d_tmem, at + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc,
-                                         (kb | kk) != 0);
-                    } else {
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                umma_bf16_ta(d_tmem, at + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc,
+                                             (kb | kk) != 0);
+                        } else {
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32),
-                                      smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                          smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        }
                     }
                     umma_commit(smem_u32(&empty[stage]));
                     if (++stage == C::kStages) {
@@ -700,11 +728,29 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         };
         if (warp == 6) {
             // -------------------------------------------------------- int8 producer
+            // It claims the units: its ring is the deepest (kQStages tiles), so the int8
+            // stream runs ahead across unit boundaries instead of waiting for the token
+            // producer, which can run only kSlots k-steps ahead of the MMA.
+            auto claim_unit = [&]() -> int {
+                int u = U;
+                if (lane == 0) {
+                    if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
+                        u = *abort_flag ? U : atomicAdd(p.sched, 1);
+                    s_unit[slot] = u;
+                    mbar_arrive(smem_u32(&ufull[slot]));
+                }
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (++slot == kUnitRing) {
+                    slot = 0;
+                    uphase ^= 1u;
+                }
+                return u;
+            };
             int qs = 0;
             uint32_t qphase = 0;
             long long qissued = 0;
             for (;;) {
-                const int u = next_unit();
+                const int u = claim_unit();
                 if (u >= U) break;
                 const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
                 const bool f1 = d.phase == 1;
@@ -739,14 +785,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             }
         } else {
             // -------------------------------------------------------- int8 -> bf16
-            // Group grp (warps 7-10, 11-14) converts the k-steps n with n % 2 == grp (n
-            // counts every k-step of the launch, as the rings do).  A warp owns the tensor
+            // Group grp (warps 7-10, 11-14) converts the stages n with n % 2 == grp (n
+            // counts every stage of the launch, as the rings do).  A warp owns the tensor
             // memory lane quadrant warp % 4, i.e. weight rows 32 quad .. 32 quad + 31, one
-            // row per lane: the lane reads its row's 64 int8 (the tile lands with the
-            // 64-byte swizzle, logical 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3),
-            // so a warp's 32 rows read without bank conflicts), converts them to bf16 and
-            // writes the 32 packed pairs into the ring stage's A columns in tensor memory
-            // with one tcgen05.st.
+            // row per lane: for each 64-K slot of the stage the lane reads its row's 64
+            // int8 (the tile lands with the 64-byte swizzle, logical 16-byte chunk c of
+            // row r at chunk c ^ ((r >> 1) & 3), so a warp's 32 rows read without bank
+            // conflicts), converts them to bf16 and writes the 32 packed pairs into the
+            // slot's A columns in tensor memory with one tcgen05.st.
             // int8 b -> float32 exactly: the bit pattern 0x4B000000 | (b ^ 0x80) is
             // 2^23 + 128 + b; subtracting 2^23 + 128 leaves b, whose float32 bits end in
             // 16 zero bits (|b| <= 128 has at most 8 significant bits), so its top half
@@ -757,61 +803,67 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                                     static_cast<uint32_t>(C::kTmemA);
             int qs = 0, stage = 0, n = 0;
             uint32_t qphase = 0, phase = 0;
+            auto next_q = [&]() {
+                if (++qs == C::kQStages) {
+                    qs = 0;
+                    qphase ^= 1u;
+                }
+            };
             for (;;) {
                 const int u = next_unit();
                 if (u >= U) break;
                 const DUnit d = decode_dunit(u, U1, MT1, MT2, G, s_off, s_pre);
                 const int nk = d.phase == 1 ? nk1 : nk2;
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb, ++n) {
-                    if ((n & 1) != grp) {   // the other group's k-step: only the rings advance
-                        if (++qs == C::kQStages) {
-                            qs = 0;
-                            qphase ^= 1u;
-                        }
-                        if (++stage == C::kStages) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                        continue;
-                    }
-                    if (lane == 0)
-                        ok = mbar_wait(smem_u32(&qfull[qs]), qphase, abort_flag, kWaitLimitNs) &&
-                             mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
-                    // the whole warp leaves together (lane 0 alone saw the wait give up)
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    tc_fence_after();   // the MMAs that read this A stage have completed
-                    const uint8_t* q = sQ + qs * kQBytes + row * BK;
-                    uint32_t h[32];
+                for (int kb0 = 0; kb0 < nk; kb0 += C::kSub, ++n) {
+                    const int ns = min(C::kSub, nk - kb0);
+                    if ((n & 1) == grp) {
+                        if (lane == 0)
+                            ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs);
+                        // the whole warp leaves together (lane 0 alone saw the wait give up)
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        tc_fence_after();   // the MMAs that read this stage's A slots have completed
+                        const int qs0 = qs;
+                        for (int j = 0; j < ns; ++j) {
+                            if (lane == 0) ok = mbar_wait(smem_u32(&qfull[qs]), qphase, abort_flag, kWaitLimitNs);
+                            ok = __shfl_sync(0xffffffffu, ok, 0);
+                            if (!ok) break;
+                            const uint8_t* q = sQ + qs * kQBytes + row * BK;
+                            uint32_t h[32];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(q + ((c ^ ((row >> 1) & 3)) << 4));
-                        const uint32_t wb[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u,
-                                                w.z ^ 0x80808080u, w.w ^ 0x80808080u};
+                            for (int c = 0; c < 4; ++c) {
+                                const uint4 w = *reinterpret_cast<const uint4*>(q + ((c ^ ((row >> 1) & 3)) << 4));
+                                const uint32_t wb[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u,
+                                                        w.z ^ 0x80808080u, w.w ^ 0x80808080u};
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            float f[4];
+                                for (int i = 0; i < 4; ++i) {
+                                    float f[4];
 #pragma unroll
-                            for (int b = 0; b < 4; ++b)
-                                f[b] = __uint_as_float(__byte_perm(wb[i], 0x4B000000u, b | 0x7540u)) -
-                                       8388736.0f;   // 2^23 + 128
-                            h[c * 8 + 2 * i] = __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
-                            h[c * 8 + 2 * i + 1] =
-                                __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+                                    for (int b = 0; b < 4; ++b)
+                                        f[b] = __uint_as_float(__byte_perm(wb[i], 0x4B000000u, b | 0x7540u)) -
+                                               8388736.0f;   // 2^23 + 128
+                                    h[c * 8 + 2 * i] =
+                                        __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
+                                    h[c * 8 + 2 * i + 1] =
+                                        __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+                                }
+                            }
+                            tmem_st_32x32b_x32(a_lane + static_cast<uint32_t>((stage * C::kSub + j) * 32), h);
+                            next_q();
                         }
-                    }
-                    tmem_st_32x32b_x32(a_lane + static_cast<uint32_t>(stage * 32), h);
-                    tmem_wait_st();
-                    tc_fence_before();   // ... before the MMA thread learns of it
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(smem_u32(&qempty[qs]));
-                        mbar_arrive(smem_u32(&full[stage]));
-                    }
-                    if (++qs == C::kQStages) {
-                        qs = 0;
-                        qphase ^= 1u;
+                        tmem_wait_st();   // also on a failed wait: no store outlives the warp
+                        if (!ok) break;
+                        tc_fence_before();   // ... before the MMA thread learns of it
+                        __syncwarp();
+                        if (lane == 0) {
+                            for (int j = 0; j < ns; ++j)
+                                mbar_arrive(smem_u32(&qempty[(qs0 + j) % C::kQStages]));
+                            mbar_arrive(smem_u32(&full[stage]));
+                        }
+                    } else {
+                        // the other group's stage: only the rings advance
+                        for (int j = 0; j < ns; ++j) next_q();
                     }
                     if (++stage == C::kStages) {
                         stage = 0;
