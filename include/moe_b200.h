@@ -235,9 +235,10 @@ moe_status moe_forward_static(const void* hidden, const void* norm_weight, float
  * Everything else as moe_forward / moe_expert_ffn with dt = MOE_BF16.  The int8
  * weights run in the decode FFN only: sizes where it does not apply (more than 64
  * routed rows per expert on average, H or 2I not multiples of 128) return
- * MOE_ERR_UNSUPPORTED; the whole-layer call routes with the staged kernels (the
- * single-launch decode layer is bf16 only).  moe_workspace_size(T, H, E, k, I,
- * MOE_BF16) and moe_expert_ffn_workspace_size(rows, I, MOE_BF16) apply. */
+ * MOE_ERR_UNSUPPORTED.  Batches of at most 64 tokens run the whole layer in one
+ * cooperative launch (bit 32 of moe_forward_path, as for bf16 weights); larger ones
+ * route with the staged kernels first.  moe_workspace_size(T, H, E, k, I, MOE_BF16)
+ * and moe_expert_ffn_workspace_size(rows, I, MOE_BF16) apply. */
 moe_status moe_forward_q8(const void* hidden, const void* norm_weight, float norm_eps,
                           const void* router_w, const float* router_bias, const int8_t* fc1_q,
                           const float* fc1_scale, const int8_t* fc2_q, const float* fc2_scale,

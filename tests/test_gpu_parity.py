@@ -484,6 +484,14 @@ Q8_CASES = [
     W("q8_small_route", T=100, H=128, E=16, k=4, I=128),
     W("q8_chunked_norm0", T=20, H=256, E=32, k=6, I=128, normalize=0, fc1_layout="chunked"),
     W("q8_one_launch_bias", T=48, H=256, E=16, k=4, I=128, router_bias_std=0.5),
+    # decode batches of 1 to 4 tokens: 1 to 4 rows per expert, wide H and I
+    W("q8_one_token", T=1, H=512, E=64, k=8, I=192),
+    W("q8_every_expert_all_rows", T=4, H=256, E=4, k=4, I=128),
+    W("q8_shared_experts", T=4, H=384, E=8, k=4, I=128, router_bias_std=1.0),
+    W("q8_three_tokens_chunked_norm0", T=3, H=384, E=32, k=6, I=192, normalize=0,
+      fc1_layout="chunked"),
+    W("q8_wide", T=2, H=4096, E=4, k=2, I=1536),
+    W("q8_wider_h", T=4, H=4224, E=8, k=2, I=128),
 ]
 
 
@@ -521,9 +529,11 @@ def test_forward_q8(wl):
     assert_close(from_dev(out), ref, atol, rtol, f"{wl.name} int8 experts")
 
 
-def test_forward_q8_attributes_and_biases():
+@pytest.mark.parametrize("T", [8, 3])
+def test_forward_q8_attributes_and_biases(T):
+    """The op's SwiGLU attributes and both expert biases, at 8 and at 3 tokens."""
     from synth import make_expert_biases
-    wl = W("q8_attr", T=8, H=256, E=32, k=4, I=128)
+    wl = W("q8_attr", T=T, H=256, E=32, k=4, I=128)
     inp = make_inputs(wl, weights=False)
     dev = device_inputs(inp)
     host, (q1, s1, q2, s2) = _q8_dev(wl)
@@ -588,6 +598,38 @@ def test_full_decode_q8():
     ref = _q8_oracle(inp, wl, host, idx)
     atol, rtol = tol(wl.dtype, ref)
     assert_close(from_dev(out), ref, atol, rtol, "decode_bf16 int8 experts")
+
+
+@pytest.mark.parametrize("T", [4, 9])
+def test_forward_q8_with_pre_norm(T):
+    """forward_q8(x, norm_weight): bit-equal to rmsnorm then forward_q8 (the same
+    kernels after the norm), and the oracle's layer on the oracle's norm of x."""
+    from synth import make_pre_norm_inputs
+    wl = W("q8_norm", T=T, H=512, E=16, k=4, I=128)
+    inp = make_inputs(wl, weights=False)
+    dev = device_inputs(inp)
+    host, (q1, s1, q2, s2) = _q8_dev(wl)
+    x, w = make_pre_norm_inputs(wl)
+    dx, dw = to_dev(x, "bf16"), to_dev(w, "bf16")
+    eps = float(np.float32(1e-5))
+    fused = moe.forward_q8(dx, dev["router_w"], q1, s1, q2, s2, wl.k, norm_weight=dw, norm_eps=eps)
+    xn = moe.rmsnorm(dx, dw, eps)
+    staged = moe.forward_q8(xn, dev["router_w"], q1, s1, q2, s2, wl.k)
+    r = moe.route(xn, dev["router_w"], wl.k)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(fused), _bits(staged))
+    xn_ref = O.pre_ffn_norm(bf16_bits_to_f32(x), bf16_bits_to_f32(w), eps, "bf16")
+    L = O.router_logits(xn_ref, inp.values("router_w"), inp["router_bias"])
+    gidx = from_dev(r["idx"]).astype(np.int64)
+    idx, _ = match_routing(L, gidx, wl.k)
+    np.testing.assert_array_equal(gidx, idx)
+    q1h, s1h, q2h, s2h = host
+    ref = O.moe_forward(xn_ref, inp.values("router_w"), inp["router_bias"],
+                        lambda e: O.dequantize_rows(q1h[e], s1h[e]),
+                        lambda e: O.dequantize_rows(q2h[e], s2h[e]), wl.k, wl.normalize,
+                        wl.fc1_layout, idx=idx)["out"]
+    atol, rtol = tol("bf16", ref)
+    assert_close(from_dev(fused), ref, atol, rtol, f"int8 experts with pre-FFN norm, T={T}")
 
 
 def test_q8_refuses_sizes_outside_the_decode_ffn():
