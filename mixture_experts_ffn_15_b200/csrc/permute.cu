@@ -126,21 +126,28 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__
     }
 }
 
-// x_perm[perm_dst[t k + j]] = hidden[t] for every pair (t, j); one warp per token,
-// 16-byte vectors.  Walking the tokens (not the permuted rows) reads every row of
-// hidden once, in order, and writes its k copies: by permuted row, a row would be read
-// k times from far-apart places, i.e. from HBM each time once hidden exceeds L2.  Pairs
-// whose row is outside [0, rows_max) (an id that was out of range) are skipped; rows
-// that no pair names are not written.
+// x_perm[perm_dst[t k + j]] = hidden[t] for every pair (t, j); one warp per (token,
+// chunk of chunk_vecs 16-byte vectors).  Walking the tokens (not the permuted rows)
+// reads every row of hidden once, in order, and writes its k copies: by permuted row, a
+// row would be read k times from far-apart places, i.e. from HBM each time once hidden
+// exceeds L2.  Large batches take a whole row per warp; small ones split rows so that
+// every SM gets warps.  Pairs whose row is outside [0, rows_max) (an id that was out of
+// range) are skipped; rows that no pair names are not written.
 __global__ void __launch_bounds__(256)
 gather_by_token_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm_dst,
-                       int T, int k, int rows_max, int vec_per_row, uint4* __restrict__ x_perm) {
+                       int T, int k, int rows_max, int vec_per_row, int chunk_vecs,
+                       uint4* __restrict__ x_perm) {
     pdl_wait();
     pdl_trigger();
     constexpr int kKMax = 32;
     const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+    const int nchunks = (vec_per_row + chunk_vecs - 1) / chunk_vecs;
+    const long long items = static_cast<long long>(T) * nchunks;
+    for (long long it = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         it < items; it += warps) {
+        const int t = static_cast<int>(it / nchunks);
+        const int c = static_cast<int>(it - static_cast<long long>(t) * nchunks);
         // the token's destination rows: lane j holds row j (k <= 32)
         int dst = -1;
         if (lane < k) {
@@ -148,12 +155,13 @@ gather_by_token_kernel(const uint4* __restrict__ hidden, const int32_t* __restri
             dst = (r >= 0 && r < rows_max) ? r : -1;
         }
         const uint4* s = hidden + static_cast<size_t>(t) * vec_per_row;
+        const int v_end = min(vec_per_row, (c + 1) * chunk_vecs);
         // 8 loads in flight per lane before the stores
-        for (int v0 = lane; v0 < vec_per_row; v0 += 32 * 8) {
+        for (int v0 = c * chunk_vecs + lane; v0 < v_end; v0 += 32 * 8) {
             uint4 buf[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                if (v0 + 32 * q < vec_per_row) buf[q] = __ldcs(s + v0 + 32 * q);
+                if (v0 + 32 * q < v_end) buf[q] = __ldcs(s + v0 + 32 * q);
 #pragma unroll 1
             for (int j = 0; j < k && j < kKMax; ++j) {
                 const int r = __shfl_sync(0xffffffffu, dst, j);
@@ -162,7 +170,7 @@ gather_by_token_kernel(const uint4* __restrict__ hidden, const int32_t* __restri
                 // streaming stores: x_perm is read back once, by the grouped GEMM
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    if (v0 + 32 * q < vec_per_row) __stcs(d + v0 + 32 * q, buf[q]);
+                    if (v0 + 32 * q < v_end) __stcs(d + v0 + 32 * q, buf[q]);
             }
         }
     }
@@ -217,12 +225,22 @@ cudaError_t launch_gather_by_token(const void* hidden, const int32_t* perm_dst, 
                                   cudaStream_t s) {
     if (T <= 0 || k > 32) return T <= 0 ? cudaSuccess : cudaErrorInvalidValue;
     const int vec = H * elem_bytes / 16;
-    int blocks = (T + 7) / 8;
-    const int cap = device_sm_count() * 8;
+    const int sms = device_sm_count();
+    // batches of fewer than 16 tokens per SM split their rows into chunks (a multiple of
+    // 32 vectors) until there are about 16 warps per SM; larger ones take whole rows
+    const long long want = 16LL * sms;
+    int nchunks = static_cast<int>((want + T - 1) / T);
+    const int max_chunks = (vec + 31) / 32;
+    if (nchunks > max_chunks) nchunks = max_chunks;
+    if (nchunks < 1) nchunks = 1;
+    const int chunk = ((vec + nchunks - 1) / nchunks + 31) / 32 * 32;
+    const long long items = static_cast<long long>(T) * ((vec + chunk - 1) / chunk);
+    long long blocks = (items + 7) / 8;
+    const long long cap = static_cast<long long>(sms) * 8;
     if (blocks > cap) blocks = cap;
-    return launch_k(gather_by_token_kernel, dim3(blocks), dim3(256), 0, s,
+    return launch_k(gather_by_token_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
                     static_cast<const uint4*>(hidden), perm_dst, T, k, rows_max, vec,
-                    static_cast<uint4*>(x_perm));
+                    chunk, static_cast<uint4*>(x_perm));
 }
 
 cudaError_t launch_gather(const void* hidden, const int32_t* perm_src, const int32_t* offsets,
