@@ -23,7 +23,8 @@
 //
 // Per CTA, 10 warps:
 //   warp 0     TMA producer (both CTAs): its CTA's weight and token slices into a
-//              6-stage ring; completion counted on the even CTA's barrier;
+//              ring of six 64-K slots, signalled in stages of two; completion counted on
+//              the even CTA's barrier;
 //   warp 1     MMA issuer (even CTA only): tcgen05.mma.cta_group::2 into one of two
 //              accumulators; commits free the ring stage in both CTAs and publish
 //              the accumulator to both epilogues;
@@ -52,7 +53,15 @@ constexpr int kPWRows = 128;                  // weight rows per CTA (256 per pa
 constexpr int kPBK = 64;                      // K per stage: one 128-byte row of bf16
 static_assert(kPBK == tmap::kBoxK, "TMA box width");
 constexpr int kPTok = 256;                    // tokens per pair tile (<= 128 per CTA)
-constexpr int kPStages = 6;
+constexpr int kPStages = 6;                   // 64-K slots in the ring
+// The barriers work on stages of kPSub consecutive slots: the MMA thread waits and
+// commits once per 128 K.  A wait costs the issuing thread ~160 cycles even on a
+// completed phase and a commit ~90, so with one stage per 64 K the four M = 256,
+// N = 256 MMAs of a slot (~515 cycles of tensor work) took ~610 cycles; with 128-K
+// stages they run back to back (measured stand-alone on a ring of six slots).
+constexpr int kPSub = 2;
+constexpr int kPBars = kPStages / kPSub;
+static_assert(kPBars * kPSub == kPStages, "whole stages");
 constexpr int kPABytes = kPWRows * kPBK * 2;  // 16 KB
 constexpr int kPBBytes = (kPTok / 2) * kPBK * 2;   // 16 KB
 constexpr int kPStageBytes = kPABytes + kPBBytes;
@@ -121,7 +130,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     const int G = p.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kPStages; ++s) {
+        for (int s = 0; s < kPBars; ++s) {
             mbar_init(smem_u32(&full[s]), 1);    // the even CTA's producer (expect_tx)
             mbar_init(smem_u32(&empty[s]), 1);   // the pair MMA's commit
         }
@@ -170,22 +179,24 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             // the tile are loaded too, and ignored: one TMA instruction each)
             const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
             bool ok = true;
-            for (int kb = 0; kb < nk; ++kb) {
+            for (int kb0 = 0; kb0 < nk; kb0 += kPSub) {
+                const int ns = min(kPSub, nk - kb0);   // slots of this stage (the last may be short)
                 if (lane == 0) {
                     ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kPWaitNs);
-                    if (ok && lead) mbar_arrive_expect_tx(smem_u32(&full[stage]), bytes);
+                    if (ok && lead) mbar_arrive_expect_tx(smem_u32(&full[stage]), static_cast<uint32_t>(ns) * bytes);
                 }
                 // the whole warp leaves together (lane 0 alone saw the wait give up)
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);   // the even CTA's
-                const uint32_t a_dst = smem_u32(sA + stage * kPABytes);
-                const uint32_t b_dst = smem_u32(sB + stage * kPBBytes);
                 if (lane == 0) {
-                    tma_load_4d_pair(a_dst, &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
-                    tma_load_2d_pair(b_dst, &tmX, fb, kb * kPBK, trow0);
+                    for (int j = 0; j < ns; ++j) {
+                        const int sl = stage * kPSub + j, kb = kb0 + j;
+                        tma_load_4d_pair(smem_u32(sA + sl * kPABytes), &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
+                        tma_load_2d_pair(smem_u32(sB + sl * kPBBytes), &tmX, fb, kb * kPBK, trow0);
+                    }
                 }
-                if (++stage == kPStages) {
+                if (++stage == kPBars) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -206,20 +217,24 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPAccCols);
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int kb0 = 0; kb0 < nk; kb0 += kPSub) {
+                    const int ns = min(kPSub, nk - kb0);
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kPWaitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * kPABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * kPBBytes);
+                    for (int j = 0; j < ns; ++j) {
+                        const int sl = stage * kPSub + j, kb = kb0 + j;
+                        const uint32_t a0 = smem_u32(sA + sl * kPABytes);
+                        const uint32_t b0 = smem_u32(sB + sl * kPBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kPBK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * 32),
-                                       smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < kPBK / 16; ++kk)
+                            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + kk * 32),
+                                           smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                    }
                     umma_commit_pair(smem_u32(&empty[stage]), 0x3);
-                    if (++stage == kPStages) {
+                    if (++stage == kPBars) {
                         stage = 0;
                         phase ^= 1u;
                     }
