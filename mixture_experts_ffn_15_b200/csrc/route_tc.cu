@@ -127,12 +127,19 @@ __device__ __forceinline__ void route_epilogue(uint32_t tb, bool valid, size_t r
     __syncwarp();
 }
 
+// Both router kernels signal their ring in stages of kRSub consecutive 64-K slots: a
+// wait on an mbarrier costs the MMA thread ~160 cycles even on a completed phase and a
+// commit ~90, more than the four N = 64 MMAs of one slot take on the tensor cores.
+constexpr int kRSub = 2;
+
 template <int MODE, int BN, int KS = 1>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcParams p, const RouteParams rp) {
     using C = Tr<MODE, BN>;
     static_assert(!C::kWeightM, "weight rows on M run in tc_ffn_decode_kernel");
+    constexpr int kBars = C::kStages / kRSub;   // barrier stages of the slot ring
+    static_assert(kBars * kRSub == C::kStages && kBars >= 2, "whole stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -153,7 +160,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int G = p.offsets ? p.E : 1;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < kBars; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -199,16 +206,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 const Unit t = decode_unit(u, per_unit, G, BM, s_off, s_pre);
                 const uint32_t bytes = C::kStageBytes;
                 const int wrow = t.g * p.n_out + t.sub * BN;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int k0 = 0; k0 < nk; k0 += kRSub) {
+                    const int ns = min(kRSub, nk - k0);   // slots of this stage (the last may be short)
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                     const uint32_t fb = smem_u32(&full[stage]);
-                    mbar_arrive_expect_tx(fb, bytes);
-                    const uint32_t a_dst = smem_u32(sA + stage * C::kABytes);
-                    const uint32_t b_dst = smem_u32(sB + stage * C::kBBytes);
-                    tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
-                    tma_load_2d(b_dst, &tmB, fb, kb * BK, wrow);
+                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(ns) * bytes);
+                    for (int j = 0; j < ns; ++j) {
+                        const int sl = stage * kRSub + j, kb = k0 + j;
+                        tma_load_2d(smem_u32(sA + sl * C::kABytes), &tmA, fb, kb * BK, t.row0);
+                        tma_load_2d(smem_u32(sB + sl * C::kBBytes), &tmB, fb, kb * BK, wrow);
+                    }
                     ++issued;
-                    if (++stage == C::kStages) {
+                    if (++stage == kBars) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -217,9 +226,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (*abort_flag) {
                 // let the copies already in flight land before the CTA exits
                 int dummy = 0;
-                for (int s = 0; s < C::kStages; ++s) {
+                for (int s = 0; s < kBars; ++s) {
                     if (issued <= s) break;
-                    const long long fills = (issued - 1 - s) / C::kStages + 1;
+                    const long long fills = (issued - 1 - s) / kBars + 1;
                     mbar_wait(smem_u32(&full[s]), static_cast<uint32_t>((fills - 1) & 1),
                               &dummy, kWaitLimitNs / 4);
                 }
@@ -239,20 +248,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::kAccStride);
                 bool ok = true;
-                for (int kb = 0; kb < nk; ++kb) {
+                for (int k0 = 0; k0 < nk; k0 += kRSub) {
+                    const int ns = min(kRSub, nk - k0);
                     if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+                    for (int j = 0; j < ns; ++j) {
+                        const int sl = stage * kRSub + j, kb = k0 + j;
+                        const uint32_t a0 = smem_u32(sA + sl * C::kABytes);
+                        const uint32_t b0 = smem_u32(sB + sl * C::kBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                                  idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_bf16(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                                      idesc, (kb | kk) != 0);
+                    }
                     umma_commit(smem_u32(&empty[stage]));
-                    if (++stage == C::kStages) {
+                    if (++stage == kBars) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -412,6 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const TcParams p, const RouteParams rp) {
     using C = SplitCfg<E, CS>;
+    // slots per barrier stage: two where the ring holds an even number of at least 4
+    constexpr int kSub = (C::kStages % 2 == 0 && C::kStages >= 4) ? kRSub : 1;
+    constexpr int kBars = C::kStages / kSub;
+    static_assert(kBars * kSub == C::kStages && kBars >= 2, "whole stages");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -433,7 +450,7 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     const int kb0 = nk * rank / CS, kb1 = nk * (rank + 1) / CS;   // CS <= nk: never empty
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
+        for (int s = 0; s < kBars; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
@@ -464,14 +481,18 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int k0 = kb0; k0 < kb1; k0 += kSub) {
+                const int ns = min(kSub, kb1 - k0);
                 if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, kWaitLimitNs)) break;
                 const uint32_t fb = smem_u32(&full[stage]);
-                mbar_arrive_expect_tx(fb, C::kStageBytes);
-                tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, fb, kb * BK, tile * BM);
-                tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, fb, kb * BK, 0);
+                mbar_arrive_expect_tx(fb, static_cast<uint32_t>(ns) * C::kStageBytes);
+                for (int j = 0; j < ns; ++j) {
+                    const int sl = stage * kSub + j, kb = k0 + j;
+                    tma_load_2d(smem_u32(sA + sl * C::kABytes), &tmA, fb, kb * BK, tile * BM);
+                    tma_load_2d(smem_u32(sB + sl * C::kBBytes), &tmB, fb, kb * BK, 0);
+                }
                 ++issued;
-                if (++stage == C::kStages) {
+                if (++stage == kBars) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -479,9 +500,9 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             if (*abort_flag) {
                 // let the copies already in flight land before the CTA goes on
                 int dummy = 0;
-                for (int s2 = 0; s2 < C::kStages; ++s2) {
+                for (int s2 = 0; s2 < kBars; ++s2) {
                     if (issued <= s2) break;
-                    const long long fills = (issued - 1 - s2) / C::kStages + 1;
+                    const long long fills = (issued - 1 - s2) / kBars + 1;
                     mbar_wait(smem_u32(&full[s2]), static_cast<uint32_t>((fills - 1) & 1), &dummy,
                               kWaitLimitNs / 4);
                 }
@@ -494,20 +515,24 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int k0 = kb0; k0 < kb1; k0 += kSub) {
+                const int ns = min(kSub, kb1 - k0);
                 if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
-                const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+                for (int j = 0; j < ns; ++j) {
+                    const int sl = stage * kSub + j, kb = k0 + j;
+                    const uint32_t a0 = smem_u32(sA + sl * C::kABytes);
+                    const uint32_t b0 = smem_u32(sB + sl * C::kBBytes);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    umma_bf16(tmem_base, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                              idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16(tmem_base, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
+                                  idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                }
                 umma_commit(smem_u32(&empty[stage]));
-                if (++stage == C::kStages) {
+                if (++stage == kBars) {
                     stage = 0;
                     phase ^= 1u;
                 }
