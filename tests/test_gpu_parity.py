@@ -32,6 +32,9 @@ CASES = [
     W("bf16_tokenM_bn192", T=300, H=256, E=16, k=4, I=192),
     W("bf16_tokenM_bn176", T=300, H=128, E=8, k=2, I=704),
     W("bf16_tokenM_bias", T=520, H=192, E=8, k=2, I=64, router_bias_std=1.0),
+    # CTA pairs with more units than pairs and an odd number of 64-K slices in both
+    # GEMMs (23 and 3): the slot ring wraps after short last stages
+    W("bf16_tokenM_odd_k_wrap", T=6144, H=1472, E=8, k=2, I=192),
     W("bf16_weightM", T=40, H=256, E=16, k=4, I=192),
     W("bf16_weightM_skew", T=100, H=256, E=8, k=2, I=128, router_bias_std=1.0),
     W("bf16_router_tc", T=600, H=256, E=64, k=4, I=128),
