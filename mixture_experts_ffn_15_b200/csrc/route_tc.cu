@@ -390,23 +390,26 @@ __device__ __forceinline__ void route_row(const float* logit, const float* s_bia
 // Router logits and routing for a few 128-token tiles (batched decode, mid-sized
 // prefill), where one CTA per tile would stream the whole K range alone.  A cluster of
 // CS CTAs runs one tile: CTA r accumulates the K slices [r nk / CS, (r + 1) nk / CS) on
-// the tensor cores (128 tokens on M, all E experts on N) and stores its partial logits
-// in its own shared memory, [e][row].  After a cluster barrier, CTA r takes the rows
-// r 128 / CS .. of the tile: its threads fetch the CS partials of those rows through
-// distributed shared memory, 16-byte loads along the rows, all CS (and two or more row
-// groups) issued before the first is used, sum them in rank order 0 .. CS-1 (a fixed
-// order: the logits do not depend on timing) into a [row][e] block, and one thread per
-// row routes it (a warp per row, with its k + 1 rounds of warp reductions, took 1.3 us a
-// row).  No global scratch; the host picks
-// this kernel by (T, H, E) alone, for the staged router and the layer alike, so both
-// return the same bits.
+// the tensor cores (128 tokens on M, all E experts on N).  CTA q reduces and routes rows
+// q 128 / CS .. of the tile: every CTA stores each of its partial rows straight from
+// tensor memory into the shared memory of the CTA that reduces it (16-byte stores
+// through the cluster, one block per source rank), and one cluster barrier publishes
+// them all.  CTA q then sums the CS partials of its rows in rank order 0 .. CS-1 (a
+// fixed order: the logits do not depend on timing) into a [row][e] block and one thread
+// per row routes it (a warp per row, with its k + 1 rounds of warp reductions, took
+// 1.3 us a row).  After the barrier no CTA touches another's shared memory, so none
+// waits for the others before leaving.  No global scratch; the host picks this kernel
+// by (T, H, E) alone, for the staged router and the layer alike, so both return the
+// same bits.
 template <int E, int CS>
 struct SplitCfg {
     static constexpr int kRows = BM / CS;                       // rows reduced and routed per CTA
     static constexpr int kABytes = BM * BK * 2;                 // 128 token rows x 64 K
     static constexpr int kBBytes = E * BK * 2;                  // E router rows x 64 K
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kPartBytes = E * BM * 4;               // partials [e][row]
+    static constexpr int kRecvLd = E + 4;                       // floats a received row (padded)
+    // received partials [CS source ranks][kRows rows][kRecvLd]: CS * kRows = BM rows
+    static constexpr int kPartBytes = BM * kRecvLd * 4;
     static constexpr int kRedBytes = kRows * (E + 1) * 4 + E * 4;   // sums [row][e], padded; bias
     static constexpr int kStagesFit = (210 * 1024 - kPartBytes - kRedBytes) / kStageBytes;
     static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
@@ -414,7 +417,6 @@ struct SplitCfg {
     static constexpr int kMiscBytes = (2 * kStages + 1) * 8 + 16;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPartBytes + kRedBytes + kMiscBytes;
     static constexpr int kTmemCols = E;                         // 64 or 128
-    static constexpr int kGroupsPerPass = 16 / CS;              // 16 loads in flight a thread
     static_assert(kStages >= 2, "pipeline");
     static_assert(kRows % 4 == 0, "16-byte row groups");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -434,8 +436,8 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + C::kStages * C::kABytes;
-    float* part = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [E][BM]
-    float* red = part + E * BM;                                             // [kRows][E + 1]
+    float* recv = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes);   // [CS][kRows][kRecvLd]
+    float* red = recv + BM * C::kRecvLd;                                    // [kRows][E + 1]
     float* s_bias = red + C::kRows * (E + 1);                               // [E]
     uint64_t* full = reinterpret_cast<uint64_t*>(s_bias + E);
     uint64_t* empty = full + C::kStages;
@@ -541,9 +543,14 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         }
     } else {
         // ------------------------------------------------------------ partials
-        // warps 2..5: TMEM lane quadrant warp % 4; thread = token row r of the tile
+        // warps 2..5: TMEM lane quadrant warp % 4; thread = token row r of the tile.  The
+        // row goes straight into the shared memory of the CTA that reduces it (rank
+        // r / kRows), at recv[this rank][r % kRows]: 16-byte stores through the cluster.
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
+        const int owner = r / C::kRows, ri = r - owner * C::kRows;
+        const uint32_t dst = mapa_shared(smem_u32(recv + (rank * C::kRows + ri) * C::kRecvLd),
+                                         static_cast<uint32_t>(owner));
         if (mbar_wait(smem_u32(tfull), 0, abort_flag, kWaitLimitNs)) {
             tc_fence_after();
 #pragma unroll 1
@@ -552,51 +559,38 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                 tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) part[(c + i) * BM + r] = __uint_as_float(v[i]);
+                for (int i = 0; i < 32; i += 4)
+                    st_shared_cluster_v4(dst + (c + i) * 4, __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();   // every CTA's partials are written and visible to the cluster
+    // every CTA's partials have landed where they are reduced: after this barrier no CTA
+    // touches another's shared memory, so none waits for the others again before leaving
+    cluster_sync();
 
     // ---------------------------------------------------------------- reduce and route
-    // position i = (e, row group of 4): the float4 at part[e][row0 + 4 g] of every rank
-    constexpr int kGroups = C::kRows / 4;
-    constexpr int kPos = E * kGroups;
+    // row i, experts 4 q .. 4 q + 3: the CS received partials summed in rank order 0 ..
+    // CS-1 (a fixed order: the logits do not depend on timing)
     const int row0 = rank * C::kRows;
 #pragma unroll 1
-    for (int i0 = threadIdx.x; i0 < kPos; i0 += kThreads * C::kGroupsPerPass) {
-        float4 v[C::kGroupsPerPass][CS];
+    for (int pos = threadIdx.x; pos < C::kRows * (E / 4); pos += kThreads) {
+        const int i = pos / (E / 4), e = 4 * (pos - i * (E / 4));
+        float4 sum = *reinterpret_cast<const float4*>(recv + i * C::kRecvLd + e);
 #pragma unroll
-        for (int j = 0; j < C::kGroupsPerPass; ++j) {
-            const int i = i0 + j * kThreads;
-            if (i < kPos) {
-                const int e = i / kGroups, g = i - e * kGroups;
-                const uint32_t a = smem_u32(&part[e * BM + row0 + 4 * g]);
-#pragma unroll
-                for (int q = 0; q < CS; ++q) v[j][q] = ld_shared_cluster_v4(mapa_shared(a, q));
-            }
+        for (int q = 1; q < CS; ++q) {
+            const float4 v = *reinterpret_cast<const float4*>(recv + (q * C::kRows + i) * C::kRecvLd + e);
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
         }
-#pragma unroll
-        for (int j = 0; j < C::kGroupsPerPass; ++j) {
-            const int i = i0 + j * kThreads;
-            if (i < kPos) {
-                const int e = i / kGroups, g = i - e * kGroups;
-                float4 sum = v[j][0];
-#pragma unroll
-                for (int q = 1; q < CS; ++q) {
-                    sum.x += v[j][q].x;
-                    sum.y += v[j][q].y;
-                    sum.z += v[j][q].z;
-                    sum.w += v[j][q].w;
-                }
-                red[(4 * g + 0) * (E + 1) + e] = sum.x;
-                red[(4 * g + 1) * (E + 1) + e] = sum.y;
-                red[(4 * g + 2) * (E + 1) + e] = sum.z;
-                red[(4 * g + 3) * (E + 1) + e] = sum.w;
-            }
-        }
+        red[i * (E + 1) + e + 0] = sum.x;
+        red[i * (E + 1) + e + 1] = sum.y;
+        red[i * (E + 1) + e + 2] = sum.z;
+        red[i * (E + 1) + e + 3] = sum.w;
     }
     __syncthreads();
     if (rp.logits) {   // the staged router returns the logits it selected on
@@ -614,7 +608,6 @@ tc_route_split_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
         const size_t row = static_cast<size_t>(tile) * BM + row0 + i;
         if (row < static_cast<size_t>(p.rows)) route_row<E, KS>(red + i * (E + 1), s_bias, row, tile, rp);
     }
-    cluster_sync();   // no CTA leaves while a peer may still read its partials
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::kTmemCols);
