@@ -12,6 +12,7 @@ namespace moe {
 namespace {
 
 constexpr int SBM = 32, SBN = 64, SBK = 32;
+static_assert(SBM * SBK % 256 == 0 && SBN * SBK % 256 == 0, "whole slices per thread");
 
 // out[r, n] = A[r, :] . W[e, n, :] for the rows of each expert, 32 x 64 output tile
 // per unit; with SWIGLU the adjacent (gate, up) columns are fused into one act value
@@ -60,18 +61,37 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
         const int nrows = min(SBM, s_off[e + 1] - row0);
         const float* We = W + static_cast<size_t>(e) * n_w * K;
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        for (int k0 = 0; k0 < K; k0 += SBK) {
-            for (int i = tid; i < SBM * SBK; i += 256) {
-                const int r = i / SBK, c = i - (i / SBK) * SBK;
-                sA[r][c] = (r < nrows && k0 + c < K) ? A[static_cast<size_t>(row0 + r) * lda + k0 + c] : 0.f;
+        // the next K slice is loaded into registers while the current one is multiplied
+        constexpr int kAPer = SBM * SBK / 256, kWPer = SBN * SBK / 256;
+        float ra[kAPer], rw[kWPer];
+        auto fetch = [&](int k0) {
+#pragma unroll
+            for (int j = 0; j < kAPer; ++j) {
+                const int i = tid + j * 256, r = i / SBK, c = i - (i / SBK) * SBK;
+                ra[j] = (r < nrows && k0 + c < K) ? A[static_cast<size_t>(row0 + r) * lda + k0 + c] : 0.f;
             }
-            for (int i = tid; i < SBN * SBK; i += 256) {
-                const int n = i / SBK, c = i - (i / SBK) * SBK;
+#pragma unroll
+            for (int j = 0; j < kWPer; ++j) {
+                const int i = tid + j * 256, n = i / SBK, c = i - (i / SBK) * SBK;
                 const int wn = nt * SBN + n;
                 const int wr = SWIGLU ? fc1_row(wn, n_w / 2, chunked) : wn;
-                sW[n][c] = (wn < n_w && k0 + c < K) ? We[static_cast<size_t>(wr) * K + k0 + c] : 0.f;
+                rw[j] = (wn < n_w && k0 + c < K) ? We[static_cast<size_t>(wr) * K + k0 + c] : 0.f;
+            }
+        };
+        fetch(0);
+        for (int k0 = 0; k0 < K; k0 += SBK) {
+#pragma unroll
+            for (int j = 0; j < kAPer; ++j) {
+                const int i = tid + j * 256;
+                sA[i / SBK][i - (i / SBK) * SBK] = ra[j];
+            }
+#pragma unroll
+            for (int j = 0; j < kWPer; ++j) {
+                const int i = tid + j * 256;
+                sW[i / SBK][i - (i / SBK) * SBK] = rw[j];
             }
             __syncthreads();
+            if (k0 + SBK < K) fetch(k0 + SBK);
 #pragma unroll 8
             for (int c = 0; c < SBK; ++c) {
                 const float a0 = sA[ty * 2][c], a1 = sA[ty * 2 + 1][c];
