@@ -7,6 +7,7 @@
 // fc1 rows of either layout ("Weight layout": interleaved 2i / 2i+1, or chunked i / I+i).
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_map.cuh"
 
 namespace moe {
 namespace {
@@ -31,20 +32,9 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
     const int tid = threadIdx.x;
     pdl_wait();
     pdl_trigger();
-    if (tid == 0) {
-        int prev = 0, pre = 0;
-        for (int e = 0; e <= E; ++e) {
-            int o = offsets[e];
-            o = o < prev ? prev : (o > rows ? rows : o);
-            s_off[e] = o;
-            prev = o;
-        }
-        for (int e = 0; e < E; ++e) {
-            s_pre[e] = pre;
-            pre += (s_off[e + 1] - s_off[e] + SBM - 1) / SBM;
-        }
-        s_pre[E] = pre;
-    }
+    // the tile map (offsets clamped to [0, rows] and made non-decreasing, tiles of SBM
+    // rows per expert), built by one warp with all its loads in flight at once
+    if (tid < 32) build_group_tiles(offsets, rows, nullptr, E, SBM, s_off, s_pre, tid);
     __syncthreads();
     const int NT = (n_w + SBN - 1) / SBN;
     const int total = s_pre[E] * NT;
