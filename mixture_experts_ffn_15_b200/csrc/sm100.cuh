@@ -257,23 +257,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     return r;
 }
 
-// 32-bit load from shared memory of any CTA of the cluster (a mapa_shared address).
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-    return v;
-}
-
-// 16-byte load from shared memory of any CTA of the cluster (a mapa_shared address).
-__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr)
-                 : "memory");
-    return v;
-}
-
 // 16-byte store to shared memory of any CTA of the cluster (a mapa_shared address).
 __device__ __forceinline__ void st_shared_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
                                                      float d) {
