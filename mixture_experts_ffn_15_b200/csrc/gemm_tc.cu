@@ -153,6 +153,20 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Two int8 weights held as float32 bit patterns 0x4B000000 | (b ^ 0x80) = 2^23 + 128 + b:
+// subtract 2^23 + 128 from both with one packed add.rn.f32x2 (exact, the differences are
+// the integers b) and pack the two upper halves -- b in bf16, exact for |b| <= 128 -- into
+// one bf16x2 word, the first weight in the lower half.
+__device__ __forceinline__ uint32_t sub_magic_f32x2(uint32_t a, uint32_t b) {
+    uint64_t d;
+    asm("{\n\t.reg .b64 x;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "add.rn.f32x2 %0, x, %3;\n\t}"
+        : "=l"(d)
+        : "r"(a), "r"(b), "l"(0xCB000080CB000080ull));   // -(2^23 + 128) in both halves
+    return __byte_perm(static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32), 0x7632u);
+}
+
 __device__ __forceinline__ bool wait_count(const int32_t* ctr, int target, volatile int* abort,
                                            uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire(ctr) >= target) return true;
@@ -838,15 +852,16 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                                                         w.z ^ 0x80808080u, w.w ^ 0x80808080u};
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
-                                    float f[4];
-#pragma unroll
-                                    for (int b = 0; b < 4; ++b)
-                                        f[b] = __uint_as_float(__byte_perm(wb[i], 0x4B000000u, b | 0x7540u)) -
-                                               8388736.0f;   // 2^23 + 128
-                                    h[c * 8 + 2 * i] =
-                                        __byte_perm(__float_as_uint(f[0]), __float_as_uint(f[1]), 0x7632u);
-                                    h[c * 8 + 2 * i + 1] =
-                                        __byte_perm(__float_as_uint(f[2]), __float_as_uint(f[3]), 0x7632u);
+                                    // bytes (0, 1) and (2, 3), two float32 subtractions per
+                                    // packed add.rn.f32x2 (exact: the differences are integers)
+                                    const uint32_t lo = sub_magic_f32x2(
+                                        __byte_perm(wb[i], 0x4B000000u, 0x7540u),
+                                        __byte_perm(wb[i], 0x4B000000u, 0x7541u));
+                                    const uint32_t hi = sub_magic_f32x2(
+                                        __byte_perm(wb[i], 0x4B000000u, 0x7542u),
+                                        __byte_perm(wb[i], 0x4B000000u, 0x7543u));
+                                    h[c * 8 + 2 * i] = lo;
+                                    h[c * 8 + 2 * i + 1] = hi;
                                 }
                             }
                             tmem_st_32x32b_x32(a_lane + static_cast<uint32_t>((stage * C::kSub + j) * 32), h);
