@@ -18,8 +18,12 @@
 // needs -- and the token side rounds up to 32 rows, not to a 128-row tile.
 //
 // Both GEMMs read contiguous token rows (x_perm, act) in one 128-row TMA box.  The
-// accumulator holds weight rows x tokens, so the epilogue transposes each warp's
-// 32 x 32 block through shared memory and writes every token row with 16-byte stores.
+// accumulator holds weight rows x tokens; the weight rows are loaded in fragment order
+// (a 5-D view: lane 8 q + j of each 32-lane quadrant holds the quadrant's weight row
+// 4 j + q), so that the 16x256b accumulator fragments give a thread four consecutive
+// weight rows of two tokens, and every token's outputs leave straight from registers
+// (fc2: 8 bytes of one token row per store, fc1 + SwiGLU: 4), a warp's store covering
+// four tokens x 64 (32) contiguous bytes, whole 32-byte sectors.
 //
 // Per CTA, 10 warps:
 //   warp 0     TMA producer (both CTAs): its CTA's weight and token slices into a
@@ -28,10 +32,9 @@
 //   warp 1     MMA issuer (even CTA only): tcgen05.mma.cta_group::2 into one of two
 //              accumulators; commits free the ring stage in both CTAs and publish
 //              the accumulator to both epilogues;
-//   warps 2-9  epilogue (both CTAs): tcgen05.ld of their 128 weight rows x the
-//              tokens, SwiGLU (fc1) or plain (fc2), a warp-private transpose in
-//              shared memory, 16-byte stores of token rows, then release the
-//              accumulator on the even CTA's barrier.
+//   warps 2-9  epilogue (both CTAs): tcgen05.ld (16x256b) of their 128 weight rows
+//              x the tokens, SwiGLU (fc1) or plain (fc2), stores of token rows from
+//              registers, then release the accumulator on the even CTA's barrier.
 // Units are statically strided over the pairs (both CTAs walk the same list), so no
 // cluster ever waits on another.  Every wait is bounded (2 s) and reports
 // MOE_DEVERR_TIMEOUT; both CTAs always reach the final cluster barrier.
@@ -71,9 +74,7 @@ constexpr int kPBox = kPTok / 2;              // token rows per TMA box: a CTA's
 constexpr uint64_t kPWaitNs = 2000000000ull;
 constexpr int kPMiscBytes =
     (2 * kPStages + 4) * 8 + 16 + 2 * (kMaxExperts + 1) * 4 + 64;
-constexpr int kPEpiWarpBytes = 32 * 64;      // per epilogue warp: 32 tokens x 32 rows bf16
-constexpr int kPEpiBytes = 8 * kPEpiWarpBytes;
-constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kPEpiBytes + kPMiscBytes;
+constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kPMiscBytes;
 static_assert(kPSmemBytes <= 227 * 1024, "shared memory");
 
 struct PairParams {
@@ -114,8 +115,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kPStages * kPABytes;
-    uint8_t* sEpi = sB + kPStages * kPBBytes;   // [8 warps][32 tokens][64 bytes]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kPEpiBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPStages * kPBBytes);
     uint64_t* empty = full + kPStages;
     uint64_t* tfull = empty + kPStages;
     uint64_t* tempty = tfull + 2;
@@ -173,8 +173,13 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const int half = d.n / 2;                     // token rows of this CTA
             const int trow0 = d.row0 + static_cast<int>(rank) * half;
             // first weight row of this CTA inside the expert (fc1: in interleaved order),
-            // loaded through the (k, s, i, e) pair view of either weight tensor
+            // loaded in fragment order through the 5-D view of the weight tensor: plain
+            // rows (k, j, q, Q, e) at (k, 0, 0, w_in / 32, g), chunked fc1 (k, j, s, qq, X)
+            // at (k, 0, 0, 0, g I / 8 + w_in / 32)
             const int w_in = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows;
+            const bool chunked = SWIGLU && p.fc1_chunked;
+            const int wc3 = chunked ? 0 : w_in / 32;
+            const int wc4 = chunked ? d.g * (p.n_out / 16) + w_in / 32 : d.g;
             // one box of 128 weight rows and one of 128 token rows per CTA (rows past
             // the tile are loaded too, and ignored: one TMA instruction each)
             const uint32_t bytes = static_cast<uint32_t>(2 * kPStageBytes);
@@ -192,7 +197,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
                 if (lane == 0) {
                     for (int j = 0; j < ns; ++j) {
                         const int sl = stage * kPSub + j, kb = kb0 + j;
-                        tma_load_4d_pair(smem_u32(sA + sl * kPABytes), &tmW, fb, kb * kPBK, 0, w_in / 2, d.g);
+                        tma_load_5d_pair(smem_u32(sA + sl * kPABytes), &tmW, fb, kb * kPBK, 0, 0, wc3, wc4);
                         tma_load_2d_pair(smem_u32(sB + sl * kPBBytes), &tmX, fb, kb * kPBK, trow0);
                     }
                 }
@@ -248,12 +253,15 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------ epilogue
         // warps 2..9: TMEM lane quadrant warp % 4 (hardware rule), and every other
-        // 32-token chunk of the tile
+        // 32-token chunk of the tile.  Thread (fj, ft) = (lane / 4, lane % 4) of the
+        // 16x256b fragments holds lanes fj, fj + 8 (first load) and fj + 16, fj + 24
+        // (second) of the quadrant -- its weight rows 4 fj .. 4 fj + 3 in fragment
+        // order -- for tokens 8 m + 2 ft + e of the chunk (m = 0..3, e = 0, 1).
         const int quad = warp & 3;
         const int part = (warp - 2) >> 2;
+        const int fj = lane >> 2, ft = lane & 3;
         int acc = 0;
         uint32_t acc_phase = 0;
-        uint8_t* scr = sEpi + (warp - 2) * kPEpiWarpBytes;
         for (int u = pair; u < num_units && !*abort_flag; u += npairs) {
             const PUnit d = pair_unit(u, MT, G, s_off, s_pre);
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, kPWaitNs)) break;
@@ -261,74 +269,48 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                 static_cast<uint32_t>(acc * kPAccCols);
             // this warp's 32 weight rows inside the expert: w0 .. w0+31 (all valid or none:
-            // n_out is a multiple of 32)
+            // n_out is a multiple of 32); this thread's: wr .. wr + 3 (fc1: interleaved,
+            // i.e. gate and up of outputs wr / 2 and wr / 2 + 1)
             const int w0 = d.mt * 2 * kPWRows + static_cast<int>(rank) * kPWRows + quad * 32;
             const bool wvalid = w0 < p.n_out;
-            // this lane's weight row's bias (fc1: interleaved row w0 + lane in fc1's
-            // layout, fc2: h)
-            const int brow = SWIGLU ? fc1_row(w0 + lane, p.n_out / 2, p.fc1_chunked) : w0 + lane;
-            const float bias = (p.bias && wvalid)
-                                   ? bf16_at(p.bias, static_cast<size_t>(d.g) * p.n_out + brow)
-                                   : 0.f;
+            const int wr = w0 + 4 * fj;
+            float bias[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                // fc1: the bias of interleaved row wr + q in fc1's layout; fc2: of h
+                const int brow = SWIGLU ? fc1_row(wr + q, p.n_out / 2, p.fc1_chunked) : wr + q;
+                bias[q] = (p.bias && wvalid)
+                              ? bf16_at(p.bias, static_cast<size_t>(d.g) * p.n_out + brow)
+                              : 0.f;
+            }
 #pragma unroll 1
             for (int c = part * 32; c < d.nrows; c += 64) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tb + c, v);
+                uint32_t lo[16], hi[16];
+                tmem_ld_16x256b_x4(tb + c, lo);                  // rows 4 fj, 4 fj + 1
+                tmem_ld_16x256b_x4(tb + (16u << 16) + c, hi);    // rows 4 fj + 2, 4 fj + 3
                 tmem_wait_ld();
-                // lane = weight row w0 + lane, v[i] = token c + i.  Transpose through the
-                // warp's scratch (row i = token c + i's outputs), then store whole token
-                // rows: each store instruction writes full 32-byte sectors.
-                if constexpr (SWIGLU) {
-                    // rows come in (gate, up) pairs: lanes 2j, 2j+1 hold gate_j, up_j.  For
-                    // tokens (i, i+1) one exchange gives the even lane (gate, up) of token i
-                    // and the odd lane those of token i+1: every lane computes one output.
-                    const bool odd = lane & 1;
-                    const int j = lane >> 1;   // output 0..15 of this warp: 32 bytes a token
+                if (!wvalid) continue;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float mine_g = __uint_as_float(v[i]) + bias;
-                        const float mine_u = __uint_as_float(v[i + 1]) + bias;
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? mine_g : mine_u, 1);
-                        const float g = odd ? other : mine_g;          // gate of token i + odd
-                        const float u = odd ? mine_u : other;          // up of token i + odd
-                        const int tok = i + (odd ? 1 : 0);
-                        *reinterpret_cast<__nv_bfloat16*>(scr + tok * 32 + j * 2) =
-                            __float2bfloat16_rn(swiglu_attr_fast(g, u, p.act));
-                    }
-                    __syncwarp();
-                    const int i0 = w0 >> 1;   // first output column of this warp
+                for (int m = 0; m < 4; ++m) {
 #pragma unroll
-                    for (int pass = 0; pass < 2; ++pass) {
-                        const int tt = pass * 16 + (lane >> 1), q = lane & 1;
-                        if (wvalid && c + tt < d.nrows)
-                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + i0 + q * 8) =
-                                *reinterpret_cast<const uint4*>(scr + tt * 32 + q * 16);
-                    }
-                } else {
-                    // lanes 2j, 2j+1 hold rows 2j, 2j+1.  For tokens (i, i+1) one exchange
-                    // gives the even lane both rows of token i and the odd lane both rows
-                    // of token i+1: one 4-byte store each, a full 128-byte wavefront.
-                    const bool odd = lane & 1;
-                    const int j = lane >> 1;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float a0 = __uint_as_float(v[i]) + bias, a1 = __uint_as_float(v[i + 1]) + bias;
-                        const float other = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
-                        const float lo = odd ? other : a0;    // row 2j of token i + odd
-                        const float hi = odd ? a1 : other;    // row 2j+1 of token i + odd
-                        const int tok = i + (odd ? 1 : 0);
-                        *reinterpret_cast<uint32_t*>(scr + tok * 64 + j * 4) = pack_bf16x2(lo, hi);
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int pass = 0; pass < 4; ++pass) {
-                        const int tt = pass * 8 + (lane >> 2), q = lane & 3;
-                        if (wvalid && c + tt < d.nrows)
-                            *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(d.row0 + c + tt) * p.ldo + w0 + q * 8) =
-                                *reinterpret_cast<const uint4*>(scr + tt * 64 + q * 16);
+                    for (int e = 0; e < 2; ++e) {
+                        const int tok = c + 8 * m + 2 * ft + e;
+                        const float x0 = __uint_as_float(lo[4 * m + e]) + bias[0];
+                        const float x1 = __uint_as_float(lo[4 * m + 2 + e]) + bias[1];
+                        const float x2 = __uint_as_float(hi[4 * m + e]) + bias[2];
+                        const float x3 = __uint_as_float(hi[4 * m + 2 + e]) + bias[3];
+                        if (tok < d.nrows) {
+                            __nv_bfloat16* orow = p.out + static_cast<size_t>(d.row0 + tok) * p.ldo;
+                            if constexpr (SWIGLU)
+                                *reinterpret_cast<uint32_t*>(orow + (wr >> 1)) =
+                                    pack_bf16x2(swiglu_attr_fast(x0, x1, p.act),
+                                                swiglu_attr_fast(x2, x3, p.act));
+                            else
+                                *reinterpret_cast<uint2*>(orow + wr) =
+                                    make_uint2(pack_bf16x2(x0, x1), pack_bf16x2(x2, x3));
+                        }
                     }
                 }
-                __syncwarp();   // the scratch is rewritten by the next chunk
             }
             tc_fence_before();
             __syncwarp();
@@ -398,13 +380,13 @@ cudaError_t launch_pair(const CUtensorMap& w, const CUtensorMap& x, const PairPa
 
 // One grouped GEMM on CTA pairs: out [rows, ldo] from x [rows, K] (contiguous rows of
 // the experts' blocks) and the weights w [E, n_out, K] of E experts (both through the
-// 4-D pair view, which reads chunked fc1 in place).
+// 5-D fragment-order views, the chunked one reading fc1 in place).
 cudaError_t pair_gemm(bool swiglu, const void* x, int rows, int K, const void* w, int E, int n_out,
                       const int32_t* offsets, void* out, int ldo, int32_t* err, cudaStream_t s,
                       const FfnAttrs& at, const void* bias) {
     CUtensorMap mw, mx;
-    const bool ok_w = swiglu ? tmap::fc1_pairs(&mw, w, E, n_out / 2, K, kPWRows / 2, at.fc1_chunked)
-                             : tmap::plain_pairs(&mw, w, E, n_out, K, kPWRows / 2);
+    const bool ok_w = (swiglu && at.fc1_chunked) ? tmap::fc1_quad_rows_chunked(&mw, w, E, n_out / 2, K)
+                                                 : tmap::quad_rows(&mw, w, E, n_out, K);
     if (!ok_w) return cudaErrorInvalidValue;
     if (!tmap::matrix(&mx, x, rows, K, kPBox)) return cudaErrorInvalidValue;
     PairParams p{offsets, E, rows, K, n_out, static_cast<__nv_bfloat16*>(out), ldo, err, at.act,

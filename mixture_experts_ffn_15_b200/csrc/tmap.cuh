@@ -87,5 +87,49 @@ inline bool plain_pairs(CUtensorMap* m, const void* w, int E, int n, int K, int 
     return n % 2 == 0 && row_pairs(m, w, E, n / 2, K, box_pairs, 1, 2, u8);
 }
 
+// bf16 weights in "fragment order" for an accumulator that the epilogue reads in 16x256b
+// fragments (a thread holds lanes j, j + 8, j + 16, j + 24 of a 32-lane quadrant): a box
+// of 128 weight rows from row r0 (a multiple of 32) of an expert lands in shared memory
+// so that box row 32 Q + 8 q + j (Q, q = 0..3, j = 0..7) holds weight row
+// r0 + 32 Q + 4 j + q, i.e. such a thread holds four consecutive weight rows.
+//   plain [E, n, K] (fc2; fc1 interleaved, n = 2I): the 5-D tensor (k, j, q, Q, e) with
+//       row strides (4, 1, 32, n); coordinates (k0, 0, 0, r0 / 32, e).  Rows past n of
+//       the last expert read as zeros.
+inline bool quad_rows(CUtensorMap* m, const void* w, int E, int n, int K) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || E <= 0 || n <= 0 || n % 32 != 0) return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(K) * 2;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(K), 8, 4, static_cast<cuuint64_t>(n / 32),
+                          static_cast<cuuint64_t>(E)};
+    cuuint64_t strides[4] = {row * 4, row, row * 32, row * static_cast<cuuint64_t>(n)};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(kBoxK), 8, 4, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(w), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+//   fc1 chunked [E, 2I, K] (row i = gate_i, I + i = up_i) in the same order over its
+//       interleaved rows 2i + s: with q = 2 qq + s, interleaved row 32 Q + 4 j + 2 qq + s
+//       of expert e is chunked row 2I e + s I + 16 Q + 2 j + qq.  The expert folds into
+//       the last coordinate, X = e I / 8 + Q (16 X = 2I e + 16 Q): the 5-D tensor
+//       (k, j, s, qq, X) with row strides (2, I, 1, 16); coordinates
+//       (k0, 0, 0, 0, e I / 8 + r0 / 32).  X < (2E - 1) I / 16 keeps every element of
+//       the tensor inside the weights; boxes past an expert's rows read another
+//       expert's (or zeros past the last), whose outputs the kernel drops.
+inline bool fc1_quad_rows_chunked(CUtensorMap* m, const void* fc1, int E, int I, int K) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || E <= 0 || I <= 0 || I % 16 != 0) return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(K) * 2;
+    cuuint64_t dims[5] = {static_cast<cuuint64_t>(K), 8, 2, 2,
+                          static_cast<cuuint64_t>(2 * E - 1) * static_cast<cuuint64_t>(I / 16)};
+    cuuint64_t strides[4] = {row * 2, row * static_cast<cuuint64_t>(I), row, row * 16};
+    cuuint32_t box[5] = {static_cast<cuuint32_t>(kBoxK), 8, 2, 2, 4};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(fc1), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tmap
 }  // namespace moe
