@@ -40,11 +40,13 @@ using namespace tc;
 // launch.  Both GEMMs put 128 weight rows on the MMA's M side and the expert's tokens
 // (a chunk of at most 64 permuted rows) on N, so every weight byte streams from HBM
 // once.  The unit list holds every fc1 unit (chunk x 128 rows of fc1) and then every
-// fc2 unit (chunk x 128 rows of fc2).  CTAs claim units in that order from a global
-// counter (the producer warp claims -- with int8 experts the int8 producer, which runs
-// furthest ahead -- and a 4-slot ring in shared memory hands the unit to the other
-// warps), so the large fc1 units go first and the small fc2 units
-// even out the end; every fc1 unit is claimed before any fc2 unit.  An fc2 unit needs the
+// fc2 unit (chunk x 128 rows of fc2).  A CTA's first unit is unit blockIdx.x; later
+// ones come in list order from a global counter starting at gridDim.x (the producer
+// warp claims -- with int8 experts the int8 producer, which runs furthest ahead -- and
+// a 4-slot ring in shared memory hands the unit to the other warps), so the large fc1
+// units go first and the small fc2 units even out the end, and no CTA waits on the
+// counter's atomic before its first load.  An fc2 unit is handed out only after every
+// fc1 unit is some running CTA's (first units are taken before any wait).  An fc2 unit needs the
 // activations of its chunk: each fc1 epilogue warp publishes its stores with a proxy
 // fence and a release increment of the chunk's counter, and the fc2 producer waits
 // (bounded) for 4 x (fc1 units per chunk) increments with an acquire load before
@@ -102,7 +104,7 @@ struct DecodeParams {
     __nv_bfloat16* act;       // [rows, I]
     __nv_bfloat16* y;         // [rows, H]
     int32_t* done;            // one counter per chunk, zero on entry
-    int32_t* sched;           // next unit to claim, zero on entry
+    int32_t* sched;           // units claimed past the first gridDim.x, zero on entry
     int32_t* fc2_done;        // published fc2 units (x 4 warps), zero on entry
     // fused combine (out != nullptr): out[t] = sum_j topk_w[t, j] y[perm_dst[t*k + j]]
     const int32_t* perm_dst;
@@ -483,6 +485,7 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         long long issued = 0;
         int slot = 0;
         uint32_t uphase = 0;
+        int claims = 0;   // bf16: units this producer has claimed
         for (;;) {
             int u = U;
             if (lane == 0) {
@@ -494,7 +497,9 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
                     }
                 } else {
                     if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
-                        u = *abort_flag ? U : atomicAdd(p.sched, 1);
+                        u = *abort_flag ? U
+                            : claims++ == 0 ? static_cast<int>(blockIdx.x)
+                                            : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
                     s_unit[slot] = u;
                     mbar_arrive(smem_u32(&ufull[slot]));
                 }
@@ -745,11 +750,14 @@ tc_ffn_decode_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
             // It claims the units: its ring is the deepest (kQStages tiles), so the int8
             // stream runs ahead across unit boundaries instead of waiting for the token
             // producer, which can run only kSlots k-steps ahead of the MMA.
+            int claims = 0;
             auto claim_unit = [&]() -> int {
                 int u = U;
                 if (lane == 0) {
                     if (mbar_wait(smem_u32(&uempty[slot]), uphase ^ 1u, abort_flag, kWaitLimitNs))
-                        u = *abort_flag ? U : atomicAdd(p.sched, 1);
+                        u = *abort_flag ? U
+                            : claims++ == 0 ? static_cast<int>(blockIdx.x)
+                                            : static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1);
                     s_unit[slot] = u;
                     mbar_arrive(smem_u32(&ufull[slot]));
                 }
