@@ -195,7 +195,12 @@ cudaError_t launch_router_logits_split(const void* hidden, const void* router_w,
                                        int E, bool bf16, float* logits, int32_t* clear_words,
                                        cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    const bool small = T <= kSplitTokens;
+    // four experts a block share every token vector they read; one expert a block when
+    // four would leave most SMs idle (small batches: more, shorter blocks in flight, and
+    // a kernel body a quarter the size, which a cold instruction cache fetches sooner).
+    // The logits are the same bits either way: every sum runs in the same order.
+    const long long tblocks = (T + kSplitTokens - 1) / kSplitTokens;
+    const bool small = (E + 3) / 4 * tblocks < device_sm_count();
     const int epb = small ? 1 : 4;
     dim3 grid((E + epb - 1) / epb, (T + kSplitTokens - 1) / kSplitTokens);
     const dim3 block(kSplitThreads);
