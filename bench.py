@@ -681,13 +681,12 @@ def measure(wl, inp, opts, args, steps, warmup, world, dev, clocks):
                     s_in.wait_event(done[b])          # step i-2's layer has read d_in[b]
                 d_in[b].copy_(h_host, non_blocking=True)
                 in_done[b].record(s_in)
-            with torch.cuda.stream(stream):
-                stream.wait_event(in_done[b])
-                if i >= 2:
-                    stream.wait_event(out_done[b])    # step i-2's output has left d_out[b]
-                run_layer(d_in[b], i, normalize=bool(wl.normalize), router_bias=bias,
-                          out=d_out[b], workspace=ws, **ffn_kw)
-                done[b].record(stream)
+            stream.wait_event(in_done[b])
+            if i >= 2:
+                stream.wait_event(out_done[b])        # step i-2's output has left d_out[b]
+            run_layer(d_in[b], i, normalize=bool(wl.normalize), router_bias=bias,
+                      out=d_out[b], workspace=ws, stream=stream, **ffn_kw)
+            done[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done[b])
                 o_host[b].copy_(d_out[b], non_blocking=True)
