@@ -195,6 +195,29 @@ def test_permutation_properties():
     check_permutation()
 
 
+def test_exclusive_offsets_by_hand():
+    # expert blocks start where the earlier experts' rows end; an empty expert's block
+    # is empty and starts where the next one does
+    np.testing.assert_array_equal(O.exclusive_offsets(np.array([3, 0, 2, 1])), [0, 3, 3, 5, 6])
+    np.testing.assert_array_equal(O.exclusive_offsets(np.array([0, 0])), [0, 0, 0])
+    np.testing.assert_array_equal(O.exclusive_offsets(np.array([], dtype=np.int64)), [0])
+
+
+def test_fc1_gate_up_row_orders_by_hand():
+    # rows labelled by their index: interleaved fc1 puts gate_i in row 2i and up_i in
+    # row 2i + 1; the chunked (Hugging Face) layout puts gate_i in row i, up_i in I + i
+    I, H = 3, 2
+    fc1 = np.repeat(np.arange(2 * I, dtype=np.float64)[:, None], H, axis=1)
+    g, u = O.fc1_gate_up(fc1, "interleaved")
+    np.testing.assert_array_equal(g[:, 0], [0, 2, 4])
+    np.testing.assert_array_equal(u[:, 0], [1, 3, 5])
+    g, u = O.fc1_gate_up(fc1, "chunked")
+    np.testing.assert_array_equal(g[:, 0], [0, 1, 2])
+    np.testing.assert_array_equal(u[:, 0], [3, 4, 5])
+    with pytest.raises(ValueError):
+        O.fc1_gate_up(fc1, "gate_up_pairs")
+
+
 def test_combine_of_permuted_rows_equals_layer():
     inp = small(T=20, E=5, k=2)
     r = fwd(inp)
