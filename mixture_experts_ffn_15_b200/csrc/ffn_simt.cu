@@ -26,7 +26,9 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
                          float* __restrict__ out, int ldo, const float* __restrict__ bias,
                          SwigluAttr act, bool chunked) {
     __shared__ float sA[SBM][SBK + 1];
-    __shared__ float sW[SBN][SBK + 1];
+    // W transposed, k-major: a thread's four output columns at one k are one 16-byte
+    // load (rows padded to a multiple of 16 bytes)
+    __shared__ __align__(16) float sW[SBK][SBN + 4];
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_pre[kMaxExperts + 1];
     const int tid = threadIdx.x;
@@ -78,18 +80,19 @@ simt_grouped_gemm_kernel(const float* __restrict__ A, int lda, const float* __re
 #pragma unroll
             for (int j = 0; j < kWPer; ++j) {
                 const int i = tid + j * 256;
-                sW[i / SBK][i - (i / SBK) * SBK] = rw[j];
+                sW[i - (i / SBK) * SBK][i / SBK] = rw[j];
             }
             __syncthreads();
             if (k0 + SBK < K) fetch(k0 + SBK);
 #pragma unroll 8
             for (int c = 0; c < SBK; ++c) {
                 const float a0 = sA[ty * 2][c], a1 = sA[ty * 2 + 1][c];
+                const float4 w4 = *reinterpret_cast<const float4*>(&sW[c][tx * 4]);
+                const float w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float w = sW[tx * 4 + q][c];
-                    acc[0][q] = fmaf(a0, w, acc[0][q]);
-                    acc[1][q] = fmaf(a1, w, acc[1][q]);
+                    acc[0][q] = fmaf(a0, w[q], acc[0][q]);
+                    acc[1][q] = fmaf(a1, w[q], acc[1][q]);
                 }
             }
             __syncthreads();
